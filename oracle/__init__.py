@@ -1,0 +1,168 @@
+"""Double-precision CPU oracle for the bidirectional Mamba-2 mixer core.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package.  The product
+library never loads it and shares no code with it.
+
+The arithmetic lives in ``bimamba_oracle.c`` (plain C, double precision,
+sequential recurrence, OpenMP only across independent (batch, head) pairs).
+This module compiles it with gcc on first use and marshals numpy arrays.
+Inputs given in a narrower type (bf16, fp32) are widened exactly to float64
+first, so input quantisation never counts as error.
+
+Parity status: every function here is pinned by the tests in
+``tests/test_oracle_pins.py`` (brute-force quadratic form, closed forms,
+flip identities, split/resume, hand-derived golden values).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bimamba_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into oracle/liboracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        cmd = ["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c99",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            dp = ctypes.POINTER(ctypes.c_double)
+            i = ctypes.c_int
+            lib.oracle_num_threads.restype = i
+            lib.oracle_conv.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, dp]
+            lib.oracle_scan.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, dp, dp]
+            lib.oracle_bimamba.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp,
+                                           i, i, i, i, i, i, i, dp, dp, dp, dp]
+            lib.oracle_block_decode.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp,
+                                                i, i, i, i, i, i, i, dp, dp, dp]
+            _lib = lib
+    return _lib
+
+
+def _f64(a):
+    """Exact widening to a contiguous float64 numpy array (None passes through).
+
+    torch tensors (including bfloat16) are widened through float32, which is
+    exact for bf16 and fp32 values.
+    """
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor
+        import torch
+        a = a.detach().to("cpu")
+        if a.dtype in (torch.bfloat16, torch.float16):
+            a = a.float()
+        a = a.double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def conv(u, w, bias=None, tail=None, reverse=False, silu=True):
+    """Depthwise causal (or mirrored) conv1d + optional SiLU.
+
+    u: (batch, len, ch); w: (ch, K); bias: (ch); tail: (batch, K, ch).
+    """
+    lib = _load()
+    u, w, bias, tail = _f64(u), _f64(w), _f64(bias), _f64(tail)
+    bsz, L, ch = u.shape
+    K = w.shape[1]
+    out = np.empty_like(u)
+    lib.oracle_conv(_ptr(u), _ptr(w), _ptr(bias), _ptr(tail), bsz, L, ch, K,
+                    int(bool(reverse)), int(bool(silu)), _ptr(out))
+    return out
+
+
+def scan(x, B, C, dt, A, D, init=None, reverse=False, want_final=False):
+    """One direction of the selective scan (sequential recurrence).
+
+    x: (batch, len, H, P); B, C: (batch, len, G, N); dt: (batch, len, H);
+    A, D: (H); init: (batch, H, P, N).  Returns y (and the final state).
+    """
+    lib = _load()
+    x, B, C, dt, A, D, init = map(_f64, (x, B, C, dt, A, D, init))
+    bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.empty_like(x)
+    fin = np.empty((bsz, H, P, N)) if want_final else None
+    lib.oracle_scan(_ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(D),
+                    _ptr(init), bsz, L, H, P, N, G, int(bool(reverse)),
+                    _ptr(y), _ptr(fin))
+    return (y, fin) if want_final else y
+
+
+def bimamba(xbc, dt, A, D, conv_w=None, conv_b=None, *, heads, headdim, d_state,
+            ngroups=1, tail=None, init=None, want_final=False, want_dirs=False):
+    """Full bidirectional mixer core: conv+SiLU per direction, scan both ways, sum.
+
+    xbc: (batch, len, H*P + 2*G*N) raw; dt: (batch, len, H).
+    Returns y (batch, len, H*P) [, final_state] [, (y_fwd, y_rev)].
+    """
+    lib = _load()
+    xbc, dt, A, D, conv_w, conv_b, tail, init = map(
+        _f64, (xbc, dt, A, D, conv_w, conv_b, tail, init))
+    bsz, L, ch = xbc.shape
+    H, P, N, G = heads, headdim, d_state, ngroups
+    assert ch == H * P + 2 * G * N
+    K = conv_w.shape[1] if conv_w is not None else 4
+    y = np.empty((bsz, L, H * P))
+    fin = np.empty((bsz, H, P, N)) if want_final else None
+    yf = np.empty_like(y) if want_dirs else None
+    yr = np.empty_like(y) if want_dirs else None
+    lib.oracle_bimamba(_ptr(xbc), _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w),
+                       _ptr(conv_b), _ptr(tail), _ptr(init), bsz, L, H, P, N, G,
+                       K, _ptr(y), _ptr(fin), _ptr(yf), _ptr(yr))
+    out = [y]
+    if want_final:
+        out.append(fin)
+    if want_dirs:
+        out.append((yf, yr))
+    return out[0] if len(out) == 1 else tuple(out)
+
+
+def block_decode(block, dt, A, D, conv_w, conv_b, state, tail, *, heads, headdim,
+                 d_state, ngroups=1, want_commit=False):
+    """Cached block decode: forward resumes from (state, tail); reverse covers
+    the block only.  Returns y [, state_out, tail_out]."""
+    lib = _load()
+    block, dt, A, D, conv_w, conv_b, state, tail = map(
+        _f64, (block, dt, A, D, conv_w, conv_b, state, tail))
+    S, L, ch = block.shape
+    H, P, N, G = heads, headdim, d_state, ngroups
+    K = conv_w.shape[1]
+    y = np.empty((S, L, H * P))
+    so = np.empty((S, H, P, N)) if want_commit else None
+    to = np.empty((S, K, ch)) if want_commit else None
+    lib.oracle_block_decode(_ptr(block), _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w),
+                            _ptr(conv_b), _ptr(state), _ptr(tail), S, L, H, P, N,
+                            G, K, _ptr(y), _ptr(so), _ptr(to))
+    return (y, so, to) if want_commit else y

@@ -1,0 +1,263 @@
+/*
+ * bimamba_oracle.c -- plain, slow, double-precision CPU oracle for the
+ * bidirectional Mamba-2 mixer core.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file; only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or helper with the CUDA
+ * library.
+ *
+ * What it computes (sources, by page title and section):
+ *  - "DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone"
+ *    (gist.science, Japanese technical summary, section 2 "Proposed method"):
+ *    every mixer is a bidirectional Mamba-2 mixer; a forward and a reversed
+ *    stream are combined by addition.  The Portuguese summary of the same
+ *    paper (section 2 "Metodologia") says the same: two directions, fused.
+ *  - The blog post "DiffuMamba" (metaphor-xennon), network-architecture
+ *    listing: d_state = 128, d_conv = 4, expand = 2.
+ *  - The Mamba-2 (SSD) recurrence, which the pages name but never print, is
+ *    taken in its standard form:
+ *        h_t = exp(dt_t * A) * h_{t-1} + dt_t * x_t B_t^T      (P x N per head)
+ *        y_t = h_t C_t + D * x_t
+ *    with A a negative scalar per head, dt per (token, head), and B, C shared
+ *    by all heads of a group.
+ *  - "Fixed state, long reach: constant-size caches in large-scale block
+ *    diffusion" (bittide, abstract and section 1): a finished block is
+ *    summarised by the forward SSM state (O(1) memory); the reverse scan is
+ *    restricted to the active block; training on the block-causal objective
+ *    makes cached decoding exactly equal to recomputation.
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *  - conv: depthwise, causal, tap j multiplies u[t-(K-1)+j]; zero padding
+ *    before the sequence start (or the cached tail in decode).  The reversed
+ *    stream uses the mirror image: tap j multiplies u[t+(K-1)-j], zero past
+ *    the end.  This is exactly flip(conv(flip(u))).
+ *  - the conv covers all xBC channels (x, B and C), then SiLU.
+ *  - the reverse scan is the forward recurrence run from t = L-1 down to 0,
+ *    i.e. flip(scan(flip(.))); its initial state is zero.
+ *  - the two directions share every parameter (A, D, conv weights, dt).
+ *  - the D skip term is added in each direction.
+ *
+ * Every function works on plain double arrays, row-major, contiguous.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double silu(double v) { return v / (1.0 + exp(-v)); }
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Depthwise conv1d with K taps, then optional SiLU.
+ *   u    : (batch, len, ch)
+ *   w    : (ch, K)
+ *   bias : (ch) or NULL
+ *   tail : (batch, K, ch) or NULL -- the K raw tokens before t = 0, oldest
+ *          first (forward direction only; ignored when reverse != 0)
+ *   out  : (batch, len, ch)
+ * Forward:  pre[t,c] = bias[c] + sum_j w[c,j] * u[t-(K-1)+j, c]
+ *           u at negative positions = tail (if given) else 0.
+ * Reverse:  pre[t,c] = bias[c] + sum_j w[c,j] * u[t+(K-1)-j, c]
+ *           u at positions >= len = 0.
+ */
+void oracle_conv(const double *u, const double *w, const double *bias,
+                 const double *tail, int batch, int len, int ch, int K,
+                 int reverse, int apply_silu, double *out)
+{
+    for (int b = 0; b < batch; ++b) {
+        for (int t = 0; t < len; ++t) {
+            for (int c = 0; c < ch; ++c) {
+                double acc = bias ? bias[c] : 0.0;
+                for (int j = 0; j < K; ++j) {
+                    long src = reverse ? (long)t + (K - 1) - j
+                                       : (long)t - (K - 1) + j;
+                    double v;
+                    if (src >= 0 && src < len) {
+                        v = u[((size_t)b * len + src) * ch + c];
+                    } else if (!reverse && src < 0 && tail) {
+                        /* tail holds positions -K .. -1 */
+                        v = tail[((size_t)b * K + (size_t)(K + src)) * ch + c];
+                    } else {
+                        v = 0.0;
+                    }
+                    acc += w[(size_t)c * K + j] * v;
+                }
+                out[((size_t)b * len + t) * ch + c] = apply_silu ? silu(acc) : acc;
+            }
+        }
+    }
+}
+
+/*
+ * One direction of the selective scan, sequential in t.
+ *   x    : (batch, len, H, P)
+ *   Bm   : (batch, len, G, N)
+ *   Cm   : (batch, len, G, N)
+ *   dt   : (batch, len, H)        already positive (post-softplus)
+ *   A    : (H)                    negative
+ *   D    : (H)
+ *   init : (batch, H, P, N) or NULL (zero state)
+ *   y    : (batch, len, H, P)     written (not accumulated)
+ *   fin  : (batch, H, P, N) or NULL -- state after the last processed token
+ * Head h reads group h / (H / G).
+ * reverse != 0 walks t = len-1 .. 0 with the same update.
+ */
+void oracle_scan(const double *x, const double *Bm, const double *Cm,
+                 const double *dt, const double *A, const double *D,
+                 const double *init, int batch, int len, int H, int P, int N,
+                 int G, int reverse, double *y, double *fin)
+{
+    int hpg = H / G;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < batch; ++b) {
+        for (int h = 0; h < H; ++h) {
+            int g = h / hpg;
+            double *hs = (double *)malloc(sizeof(double) * (size_t)P * N);
+            if (init)
+                memcpy(hs, init + ((size_t)b * H + h) * P * N,
+                       sizeof(double) * (size_t)P * N);
+            else
+                memset(hs, 0, sizeof(double) * (size_t)P * N);
+            for (int step = 0; step < len; ++step) {
+                int t = reverse ? len - 1 - step : step;
+                double d = dt[((size_t)b * len + t) * H + h];
+                double a = exp(d * A[h]);
+                const double *xt = x + (((size_t)b * len + t) * H + h) * P;
+                const double *bt = Bm + (((size_t)b * len + t) * G + g) * N;
+                const double *ct = Cm + (((size_t)b * len + t) * G + g) * N;
+                double *yt = y + (((size_t)b * len + t) * H + h) * P;
+                for (int p = 0; p < P; ++p) {
+                    double *row = hs + (size_t)p * N;
+                    double dx = d * xt[p];
+                    double acc = 0.0;
+                    for (int n = 0; n < N; ++n) {
+                        row[n] = a * row[n] + dx * bt[n];
+                        acc += row[n] * ct[n];
+                    }
+                    yt[p] = acc + D[h] * xt[p];
+                }
+            }
+            if (fin)
+                memcpy(fin + ((size_t)b * H + h) * P * N, hs,
+                       sizeof(double) * (size_t)P * N);
+            free(hs);
+        }
+    }
+}
+
+/* Split activated xBC (batch, len, ch = H*P + 2*G*N) into x, B, C. */
+static void split_xbc(const double *u, int batch, int len, int H, int P,
+                      int N, int G, double *x, double *Bm, double *Cm)
+{
+    int ch = H * P + 2 * G * N;
+    for (size_t r = 0; r < (size_t)batch * len; ++r) {
+        const double *src = u + r * ch;
+        memcpy(x + r * H * P, src, sizeof(double) * (size_t)H * P);
+        memcpy(Bm + r * G * N, src + H * P, sizeof(double) * (size_t)G * N);
+        memcpy(Cm + r * G * N, src + H * P + G * N, sizeof(double) * (size_t)G * N);
+    }
+}
+
+/*
+ * Whole bidirectional mixer core.
+ *   xbc    : (batch, len, ch) raw (pre-conv) when conv_w != NULL, otherwise
+ *            already activated; ch = H*P + 2*G*N, channel order [x | B | C]
+ *   conv_w : (ch, K) or NULL (no conv, no SiLU)
+ *   conv_b : (ch) or NULL
+ *   tail   : (batch, K, ch) or NULL -- forward conv history (decode)
+ *   init   : (batch, H, P, N) or NULL -- forward initial state
+ *   y      : (batch, len, H*P) = forward stream + reverse stream
+ *   fin    : (batch, H, P, N) or NULL -- forward final state
+ *   yf, yr : optional (batch, len, H*P) per-direction outputs (may be NULL)
+ */
+void oracle_bimamba(const double *xbc, const double *dt, const double *A,
+                    const double *D, const double *conv_w, const double *conv_b,
+                    const double *tail, const double *init, int batch, int len,
+                    int H, int P, int N, int G, int K, double *y, double *fin,
+                    double *yf, double *yr)
+{
+    int ch = H * P + 2 * G * N;
+    size_t nt = (size_t)batch * len;
+    double *act = (double *)malloc(sizeof(double) * nt * ch);
+    double *x = (double *)malloc(sizeof(double) * nt * H * P);
+    double *Bm = (double *)malloc(sizeof(double) * nt * G * N);
+    double *Cm = (double *)malloc(sizeof(double) * nt * G * N);
+    double *of = (double *)malloc(sizeof(double) * nt * H * P);
+    double *orv = (double *)malloc(sizeof(double) * nt * H * P);
+
+    /* forward stream */
+    if (conv_w)
+        oracle_conv(xbc, conv_w, conv_b, tail, batch, len, ch, K, 0, 1, act);
+    else
+        memcpy(act, xbc, sizeof(double) * nt * ch);
+    split_xbc(act, batch, len, H, P, N, G, x, Bm, Cm);
+    oracle_scan(x, Bm, Cm, dt, A, D, init, batch, len, H, P, N, G, 0, of, fin);
+
+    /* reverse stream: mirrored conv, zero padding past the end, zero state */
+    if (conv_w)
+        oracle_conv(xbc, conv_w, conv_b, NULL, batch, len, ch, K, 1, 1, act);
+    else
+        memcpy(act, xbc, sizeof(double) * nt * ch);
+    split_xbc(act, batch, len, H, P, N, G, x, Bm, Cm);
+    oracle_scan(x, Bm, Cm, dt, A, D, NULL, batch, len, H, P, N, G, 1, orv, NULL);
+
+    for (size_t i = 0; i < nt * H * P; ++i)
+        y[i] = of[i] + orv[i];
+    if (yf) memcpy(yf, of, sizeof(double) * nt * H * P);
+    if (yr) memcpy(yr, orv, sizeof(double) * nt * H * P);
+    free(act); free(x); free(Bm); free(Cm); free(of); free(orv);
+}
+
+/*
+ * Cached block decode for block diffusion.  For each stream, the forward
+ * stream resumes from the cached state with the cached conv tail; the reverse
+ * stream covers the active block only, from a zero state, with zero padding
+ * past the block end.  The result is the sum.
+ *   block     : (streams, len, ch) raw xBC of the active block
+ *   state     : (streams, H, P, N) forward state after the prefix
+ *   tail      : (streams, K, ch) last K raw tokens of the prefix, oldest first
+ *   y         : (streams, len, H*P)
+ *   state_out : (streams, H, P, N) or NULL -- forward state after the block
+ *   tail_out  : (streams, K, ch) or NULL   -- last K raw tokens of
+ *               prefix + block, oldest first
+ * This is oracle_bimamba with tail and init on the forward stream, so it
+ * reuses that definition directly.
+ */
+void oracle_block_decode(const double *block, const double *dt, const double *A,
+                         const double *D, const double *conv_w,
+                         const double *conv_b, const double *state,
+                         const double *tail, int streams, int len, int H, int P,
+                         int N, int G, int K, double *y, double *state_out,
+                         double *tail_out)
+{
+    oracle_bimamba(block, dt, A, D, conv_w, conv_b, tail, state, streams, len,
+                   H, P, N, G, K, y, state_out, NULL, NULL);
+    if (tail_out) {
+        int ch = H * P + 2 * G * N;
+        for (int s = 0; s < streams; ++s) {
+            for (int k = 0; k < K; ++k) {
+                /* position len - K + k of the concatenation tail | block */
+                long pos = (long)len - K + k;
+                const double *src;
+                if (pos >= 0)
+                    src = block + ((size_t)s * len + pos) * ch;
+                else
+                    src = tail + ((size_t)s * K + (size_t)(K + pos)) * ch;
+                memcpy(tail_out + ((size_t)s * K + k) * ch, src,
+                       sizeof(double) * ch);
+            }
+        }
+    }
+}

@@ -1,0 +1,304 @@
+"""Pins for the CPU oracle: each check compares it with something other than
+itself -- a brute-force materialised quadratic form, closed forms, library
+routines (numpy cumsum / convolve), hand-derived values under tests/golden,
+and invariants (flip identity, split/resume, decode == recompute).
+
+Each pin is chosen so that a plausible mistake in the oracle (a dropped term,
+a wrong sign or index, a transposed operand, an off-by-one in the decay
+window or the conv taps) fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, *v = line.split()
+            vals[k] = np.array([float(t) for t in v])
+    return vals
+
+
+def _rand(rng, bsz, L, H, P, N, G=1, a_lo=1.0, a_hi=16.0):
+    x = rng.standard_normal((bsz, L, H, P))
+    B = rng.standard_normal((bsz, L, G, N))
+    C = rng.standard_normal((bsz, L, G, N))
+    dt = np.log1p(np.exp(rng.normal(-2.0, math.sqrt(0.5), (bsz, L, H))))
+    A = -np.exp(rng.uniform(math.log(a_lo), math.log(a_hi), H))
+    D = rng.standard_normal(H)
+    return x, B, C, dt, A, D
+
+
+def _xbc(x, B, C):
+    bsz, L, H, P = x.shape
+    return np.concatenate([x.reshape(bsz, L, H * P), B.reshape(bsz, L, -1),
+                           C.reshape(bsz, L, -1)], axis=-1)
+
+
+def _brute_force(x, B, C, dt, A, D):
+    """Materialised quadratic (semiseparable) form of both directions.
+
+    M_f[t,s] = (C_t . B_s) exp(A sum_{r=s+1..t} dt_r) dt_s      (s <= t)
+    M_r[t,s] = (C_t . B_s) exp(A sum_{r=t..s-1} dt_r) dt_s      (s >= t)
+    y = (M_f + M_r) x + 2 D x
+    Built with explicit double loops over (t, s); independent of the
+    sequential recurrence.
+    """
+    bsz, L, H, P = x.shape
+    G = B.shape[2]
+    hpg = H // G
+    y = np.zeros_like(x)
+    for b in range(bsz):
+        for h in range(H):
+            g = h // hpg
+            CB = C[b, :, g, :] @ B[b, :, g, :].T          # (t, s)
+            M = np.zeros((L, L))
+            for t in range(L):
+                for s in range(L):
+                    if s <= t:
+                        seg = dt[b, s + 1:t + 1, h].sum()
+                        M[t, s] += CB[t, s] * math.exp(A[h] * seg) * dt[b, s, h]
+                    if s >= t:
+                        seg = dt[b, t:s, h].sum()
+                        M[t, s] += CB[t, s] * math.exp(A[h] * seg) * dt[b, s, h]
+            y[b, :, h, :] = M @ x[b, :, h, :] + 2.0 * D[h] * x[b, :, h, :]
+    return y
+
+
+@pytest.mark.parametrize("L,H,P,N,G", [(1, 1, 1, 1, 1), (7, 2, 3, 4, 1),
+                                       (33, 4, 2, 5, 2), (64, 2, 4, 8, 1)])
+@pytest.mark.parametrize("memory", ["short", "long"])
+def test_bidirectional_equals_quadratic_form(L, H, P, N, G, memory):
+    rng = np.random.default_rng(L * 1000 + H * 10 + N)
+    a = (1.0, 16.0) if memory == "short" else (1e-3, 1e-2)
+    x, B, C, dt, A, D = _rand(rng, 2, L, H, P, N, G, *a)
+    y = oracle.bimamba(_xbc(x, B, C), dt, A, D, heads=H, headdim=P, d_state=N, ngroups=G)
+    ref = _brute_force(x, B, C, dt, A, D).reshape(2, L, H * P)
+    assert np.max(np.abs(y - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_golden_hand_scalar():
+    g = _golden("scan_hand.txt")
+    x = np.array([1.0, 2.0, 3.0]).reshape(1, 3, 1, 1)
+    one = np.ones((1, 3, 1, 1))
+    dt = np.ones((1, 3, 1))
+    A = np.array([-math.log(2.0)])
+    for D, key in ((0.0, "case1_y_D0"), (0.5, "case1_y_D05")):
+        y, fin = oracle.bimamba(_xbc(x, one, one), dt, A, np.array([D]), heads=1,
+                                headdim=1, d_state=1, want_final=True)
+        np.testing.assert_allclose(y.ravel(), g[key], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(fin.ravel(), g["case1_final"], rtol=0, atol=1e-14)
+
+
+def test_golden_hand_matrix_orientation():
+    g = _golden("scan_hand.txt")
+    x = np.array([[1.0, 0.0], [0.0, 1.0]]).reshape(1, 2, 1, 2)
+    B = np.array([[1.0, 0.0], [0.0, 2.0]]).reshape(1, 2, 1, 2)
+    C = np.array([[1.0, 1.0], [3.0, 0.0]]).reshape(1, 2, 1, 2)
+    dt = np.ones((1, 2, 1))
+    y, fin = oracle.bimamba(_xbc(x, B, C), dt, np.array([-math.log(2.0)]),
+                            np.array([0.0]), heads=1, headdim=2, d_state=2,
+                            want_final=True)
+    np.testing.assert_allclose(y.ravel(), g["case2_y"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(fin.ravel(), g["case2_final"], rtol=0, atol=1e-14)
+
+
+def test_golden_hand_conv():
+    g = _golden("conv_hand.txt")
+    u = g["u"].reshape(1, 4, 1)
+    cases = [((1, 0, 0, 0), "w_shift_fwd", "w_shift_rev"),
+             ((1, 2, 3, 4), "w_1234_fwd", "w_1234_rev")]
+    for w, kf, kr in cases:
+        w = np.array(w, dtype=float).reshape(1, 4)
+        f = oracle.conv(u, w, reverse=False, silu=False).ravel()
+        r = oracle.conv(u, w, reverse=True, silu=False).ravel()
+        np.testing.assert_array_equal(f, g[kf])
+        np.testing.assert_array_equal(r, g[kr])
+    ident = oracle.conv(u, np.array([[0, 0, 0, 1.0]]), silu=False).ravel()
+    np.testing.assert_array_equal(ident, g["u"])
+    tail = g["tail"].reshape(1, 4, 1)
+    f = oracle.conv(u, np.array([[1, 2, 3, 4.0]]), tail=tail, silu=False).ravel()
+    np.testing.assert_array_equal(f, g["w_1234_fwd_tail"])
+
+
+def test_conv_matches_numpy_convolve_and_silu():
+    rng = np.random.default_rng(5)
+    bsz, L, ch, K = 2, 37, 6, 4
+    u = rng.standard_normal((bsz, L, ch))
+    w = rng.standard_normal((ch, K))
+    bias = rng.standard_normal(ch)
+    tail = rng.standard_normal((bsz, K, ch))
+    f = oracle.conv(u, w, bias, tail=tail, reverse=False, silu=True)
+    r = oracle.conv(u, w, bias, reverse=True, silu=True)
+    for b in range(bsz):
+        for c in range(ch):
+            full = np.concatenate([tail[b, :, c], u[b, :, c]])
+            pre_f = np.convolve(full, w[c, ::-1])[K:K + L] + bias[c]
+            pre_r = np.convolve(u[b, ::-1, c], w[c, ::-1])[:L][::-1] + bias[c]
+            np.testing.assert_allclose(f[b, :, c], pre_f / (1 + np.exp(-pre_f)), rtol=1e-13, atol=1e-13)
+            np.testing.assert_allclose(r[b, :, c], pre_r / (1 + np.exp(-pre_r)), rtol=1e-13, atol=1e-13)
+
+
+def test_a_zero_is_prefix_sum():
+    """A = 0: every decay is 1; with B = C = e_0 the forward stream is the
+    running sum of dt*x (numpy cumsum), the reverse stream the suffix sum."""
+    rng = np.random.default_rng(7)
+    bsz, L, H, P, N = 2, 50, 3, 4, 5
+    x = rng.standard_normal((bsz, L, H, P))
+    dt = rng.uniform(0.01, 1.0, (bsz, L, H))
+    B = np.zeros((bsz, L, 1, N)); B[..., 0] = 1.0
+    C = B.copy()
+    A = np.zeros(H)
+    D = rng.standard_normal(H)
+    y, (yf, yr) = oracle.bimamba(_xbc(x, B, C), dt, A, D, heads=H, headdim=P,
+                                 d_state=N, want_dirs=True)
+    dx = dt[..., None] * x
+    pre = np.cumsum(dx, axis=1) + D[None, None, :, None] * x
+    suf = np.cumsum(dx[:, ::-1], axis=1)[:, ::-1] + D[None, None, :, None] * x
+    np.testing.assert_allclose(yf, pre.reshape(yf.shape), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(yr, suf.reshape(yr.shape), rtol=1e-12, atol=1e-12)
+
+
+def test_length_one_closed_form():
+    rng = np.random.default_rng(11)
+    H, P, N = 3, 4, 6
+    x, B, C, dt, A, D = _rand(rng, 1, 1, H, P, N)
+    h0 = rng.standard_normal((1, H, P, N))
+    y = oracle.bimamba(_xbc(x, B, C), dt, A, D, heads=H, headdim=P, d_state=N, init=h0)
+    cb = float(C[0, 0, 0] @ B[0, 0, 0])
+    for h in range(H):
+        d = dt[0, 0, h]
+        xv = x[0, 0, h]
+        fwd = math.exp(d * A[h]) * (h0[0, h] @ C[0, 0, 0]) + cb * d * xv + D[h] * xv
+        rev = cb * d * xv + D[h] * xv
+        np.testing.assert_allclose(y[0, 0, h * P:(h + 1) * P], fwd + rev, rtol=1e-13, atol=1e-13)
+
+
+def test_scalar_geometric_closed_form():
+    """P = N = 1, constant dt, A, x and B = C = 1: the forward stream is a
+    geometric series dt*x*(1-a^(t+1))/(1-a) + D x, the reverse one mirrors it."""
+    L = 40
+    dt, A, xv, D = 0.3, -0.7, 1.25, 0.4
+    a = math.exp(dt * A)
+    x = np.full((1, L, 1, 1), xv)
+    one = np.ones((1, L, 1, 1))
+    y = oracle.bimamba(_xbc(x, one, one), np.full((1, L, 1), dt), np.array([A]),
+                       np.array([D]), heads=1, headdim=1, d_state=1).ravel()
+    t = np.arange(L)
+    fwd = dt * xv * (1 - a ** (t + 1)) / (1 - a) + D * xv
+    rev = dt * xv * (1 - a ** (L - t)) / (1 - a) + D * xv
+    np.testing.assert_allclose(y, fwd + rev, rtol=1e-13)
+
+
+def test_infinite_decay_keeps_only_the_diagonal():
+    rng = np.random.default_rng(13)
+    H, P, N, L = 2, 3, 4, 9
+    x, B, C, dt, _, D = _rand(rng, 1, L, H, P, N)
+    A = np.full(H, -1e30)
+    y = oracle.bimamba(_xbc(x, B, C), dt, A, D, heads=H, headdim=P, d_state=N)
+    cb = np.einsum("tn,tn->t", C[0, :, 0], B[0, :, 0])
+    want = 2 * (cb[:, None, None] * dt[0, :, :, None] * x[0] + D[None, :, None] * x[0])
+    np.testing.assert_allclose(y[0], want.reshape(L, H * P), rtol=1e-13, atol=1e-13)
+
+
+def test_flip_identities():
+    """reverse stream == flip(forward(flip(input))), for the conv and the
+    scan separately, and the tied bidirectional output is flip-equivariant."""
+    rng = np.random.default_rng(17)
+    bsz, L, H, P, N = 2, 29, 2, 3, 4
+    x, B, C, dt, A, D = _rand(rng, bsz, L, H, P, N)
+    ch = H * P + 2 * N
+    u = rng.standard_normal((bsz, L, ch))
+    w = rng.standard_normal((ch, 4))
+    r = oracle.conv(u, w, reverse=True)
+    f = oracle.conv(u[:, ::-1], w, reverse=False)[:, ::-1]
+    np.testing.assert_allclose(r, f, rtol=0, atol=1e-14)
+    yr = oracle.scan(x, B, C, dt, A, D, reverse=True)
+    yf = oracle.scan(x[:, ::-1], B[:, ::-1], C[:, ::-1], dt[:, ::-1], A, D)[:, ::-1]
+    np.testing.assert_allclose(yr, yf, rtol=1e-13, atol=1e-13)
+    y = oracle.bimamba(u, dt, A, D, w, heads=H, headdim=P, d_state=N)
+    yflip = oracle.bimamba(u[:, ::-1], dt[:, ::-1], A, D, w, heads=H, headdim=P, d_state=N)
+    np.testing.assert_allclose(y, yflip[:, ::-1], rtol=1e-12, atol=1e-12)
+
+
+def test_linearity_in_x():
+    rng = np.random.default_rng(19)
+    x, B, C, dt, A, D = _rand(rng, 1, 21, 2, 3, 4)
+    x2 = rng.standard_normal(x.shape)
+    y1 = oracle.scan(x, B, C, dt, A, D)
+    y2 = oracle.scan(x2, B, C, dt, A, D)
+    y12 = oracle.scan(2.0 * x - 3.0 * x2, B, C, dt, A, D)
+    np.testing.assert_allclose(y12, 2.0 * y1 - 3.0 * y2, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("split", [1, 5, 16, 30])
+def test_split_resume(split):
+    """scan(0..L) == scan(l..L | final_state(0..l)) for the forward stream."""
+    rng = np.random.default_rng(23)
+    x, B, C, dt, A, D = _rand(rng, 2, 31, 2, 3, 5, 1, 1e-3, 1e-2)
+    y, fin = oracle.scan(x, B, C, dt, A, D, want_final=True)
+    y1, s1 = oracle.scan(x[:, :split], B[:, :split], C[:, :split], dt[:, :split], A, D, want_final=True)
+    y2, s2 = oracle.scan(x[:, split:], B[:, split:], C[:, split:], dt[:, split:], A, D, init=s1, want_final=True)
+    np.testing.assert_allclose(np.concatenate([y1, y2], axis=1), y, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(s2, fin, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("prefix", [0, 2, 3, 17])
+def test_block_decode_equals_recompute(prefix):
+    """Cached decode of a block == the forward stream of a full recompute over
+    prefix + block at the block positions, plus the reverse stream of the
+    block alone (block-causal reading of the cached-decode pages)."""
+    rng = np.random.default_rng(29 + prefix)
+    S, blk, H, P, N, K = 2, 11, 2, 3, 4, 4
+    ch = H * P + 2 * N
+    u = rng.standard_normal((S, prefix + blk, ch))
+    dt = np.log1p(np.exp(rng.normal(-2.0, 0.7, (S, prefix + blk, H))))
+    A = -np.exp(rng.uniform(math.log(1e-3), math.log(1.0), H))
+    D = rng.standard_normal(H)
+    w = rng.standard_normal((ch, K)) * 0.5
+    bias = rng.standard_normal(ch) * 0.1
+    # prefix summary produced by the oracle itself: state after the prefix and
+    # its last K raw tokens (zeros where the prefix is shorter than K)
+    if prefix:
+        _, state = oracle.bimamba(u[:, :prefix], dt[:, :prefix], A, D, w, bias,
+                                  heads=H, headdim=P, d_state=N, want_final=True)
+    else:
+        state = np.zeros((S, H, P, N))
+    tail = np.zeros((S, K, ch))
+    take = min(prefix, K)
+    if take:
+        tail[:, K - take:] = u[:, prefix - take:prefix]
+    y, so, to = oracle.block_decode(u[:, prefix:], dt[:, prefix:], A, D, w, bias,
+                                    state, tail, heads=H, headdim=P, d_state=N,
+                                    want_commit=True)
+    _, fin, (yf_full, _) = oracle.bimamba(u, dt, A, D, w, bias, heads=H, headdim=P,
+                                          d_state=N, want_final=True, want_dirs=True)
+    _, (_, yr_blk) = oracle.bimamba(u[:, prefix:], dt[:, prefix:], A, D, w, bias,
+                                    heads=H, headdim=P, d_state=N, want_dirs=True)
+    np.testing.assert_allclose(y, yf_full[:, prefix:] + yr_blk, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(so, fin, rtol=1e-12, atol=1e-12)
+    full_tail = np.concatenate([np.zeros((S, K, ch)), u], axis=1)[:, -K:]
+    np.testing.assert_array_equal(to, full_tail)
+
+
+def test_decode_golden_scalar():
+    """Case 1 of scan_hand.txt split as prefix (1,2) + block (3): the forward
+    state after the prefix is 2.5; the block output is 0.5*2.5+3 (forward,
+    resumed) + 3 (reverse over the block alone) = 7.25, which equals the full
+    bidirectional output at the last position."""
+    one = np.ones((1, 1, 1))
+    u = np.array([[[3.0, 1.0, 1.0]]])          # x=3, B=1, C=1, no conv
+    y = oracle.bimamba(u, one, np.array([-math.log(2.0)]), np.array([0.0]),
+                       heads=1, headdim=1, d_state=1, init=np.full((1, 1, 1, 1), 2.5))
+    assert abs(y.ravel()[0] - 7.25) < 1e-14
