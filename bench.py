@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Throughput of the bidirectional Mamba-2 mixer core on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload layer1p3b|long131k|decode] [--no-cpu-baseline]
+
+One step = one bimamba_ssd_fwd_rev call over one batch of the workload
+(conv+SiLU both ways, forward and reverse SSD scans, summed output), inputs
+resident in HBM.  Default workload: b8 x L4096, 64 heads x headdim 64,
+d_state 128, bf16 activations, fp32 state (one 1.3B-model mixer layer).
+Every rank runs its own copy of the workload (independent sequences, no
+data-path collective): scaling is weak, value = all ranks' tokens / the
+slowest rank's time.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the double-precision sequential
+recurrence under oracle/) on the host cores, a bounded sample per step, and
+prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BiMamba-2 scan tokens/s (fwd+rev) on 1 B200; % of HBM/tensor roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["layer1p3b", "long131k", "decode"], default="layer1p3b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- workloads
+def workload_spec(name):
+    from bidirectional_mamba_ssm_b200 import inputs as I
+    if name == "layer1p3b":
+        return I.LAYER_1P3B, I.LAYER_1P3B.batch, I.LAYER_1P3B.seqlen
+    if name == "long131k":
+        return I.LONG_131K, 1, I.LONG_131K.seqlen
+    if name == "decode":
+        return I.LAYER_1P3B, I.DECODE_STREAMS, I.DECODE_BLOCK
+    raise ValueError(name)
+
+
+def algorithmic(w, batch, seqlen, decode=False):
+    """Algorithmic bytes and flops of one step (definitions in the design doc).
+
+    bytes/token = raw xBC in (H*P + 2N) + dt (H) + y out (H*P), in the
+    activation dtype; decode adds the fp32 state read (H*P*N*4 per stream)
+    and the conv tail (4 tokens of xBC) per stream.
+    flops/token = 2*(2*Q*N + H*(Q*P + 4*P*N)) with Q = 64 fixed.
+    """
+    esz = 2 if w.dtype == "bf16" else 4
+    H, P, N = w.heads, w.headdim, w.d_state
+    per_tok = esz * ((H * P + 2 * N) + H + H * P)
+    tokens = batch * seqlen
+    nbytes = per_tok * tokens
+    if decode:
+        nbytes += batch * (H * P * N * 4 + 4 * (H * P + 2 * N) * esz)
+    Q = 64
+    flops = 2 * (2 * Q * N + H * (Q * P + 4 * P * N)) * tokens
+    return nbytes, flops
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_traffic(kernel_file):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel (sha256 recorded there); else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    src = os.path.join(ROOT, "bidirectional_mamba_ssm_b200", "csrc", kernel_file)
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        for line in open(path):
+            parts = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+            if parts.get("file") == kernel_file and parts.get("sha") == sha:
+                return float(parts["dram_bytes_per_launch"])
+    except OSError:
+        pass
+    return None
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from bidirectional_mamba_ssm_b200 import _lib as lib
+    from bidirectional_mamba_ssm_b200 import inputs as I
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    decode = args.workload == "decode"
+    w, batch, seqlen = workload_spec(args.workload)
+    H, P, N = w.heads, w.headdim, w.d_state
+
+    # ---- inputs, generated on the device (seeded per rank)
+    g = I.make_inputs(w, seed=rank, device=dev, seqlen=seqlen, batch=batch,
+                      conv_bias=decode)
+    y = torch.empty((batch, seqlen, H * P), dtype=torch.bfloat16, device=dev)
+    dims = lib.make_dims(batch, seqlen, H, P, N, torch.bfloat16)
+    ws = lib.new_workspace(dims, device=dev)
+    if decode:
+        # cached state from a forward scan over a seeded 65536-token prefix
+        state = torch.empty((batch, H, P, N), device=dev)
+        tail = torch.empty((batch, 4, w.channels), dtype=torch.bfloat16, device=dev)
+        pdims = lib.make_dims(1, I.DECODE_PREFIX, H, P, N, torch.bfloat16)
+        pws = lib.new_workspace(pdims, device=dev)
+        py = torch.empty((1, I.DECODE_PREFIX, H * P), dtype=torch.bfloat16, device=dev)
+        for s in range(batch):
+            pre = I.make_inputs(w, seed=1000 + batch * rank + s, device=dev,
+                                seqlen=I.DECODE_PREFIX, batch=1)
+            lib.bimamba_ssd_fwd_rev(pre["xbc"], pre["dt"], g["A"], g["D"], g["conv_w"], g["conv_b"],
+                                    None, state[s:s + 1], py, pws, heads=H, headdim=P, d_state=N)
+            tail[s] = pre["xbc"][0, -4:]
+        del pre, py, pws
+
+        def step():
+            lib.bimamba_block_decode(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], g["conv_b"],
+                                     state, tail, y, None, None, ws, heads=H, headdim=P, d_state=N)
+    else:
+        def step():
+            lib.bimamba_ssd_fwd_rev(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], None, None,
+                                    None, y, ws, heads=H, headdim=P, d_state=N)
+
+    torch.cuda.synchronize()
+    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    sampler = ClockSampler(gpu_id)
+
+    # ---- warm-up: at least W steps and at least ~1 s of load for the sampler
+    t0 = time.time()
+    n = 0
+    while n < args.warmup or time.time() - t0 < 1.0:
+        step()
+        n += 1
+        if n % 10 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches0 = lib.bimamba_launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = lib.bimamba_launch_count() - launches0
+    clocks = sampler.stop()
+    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+    ms_total = start.elapsed_time(end)
+    per_call_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        t = torch.tensor([ms_total, per_call_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, per_call_ms = float(t[0]), float(t[1])
+        lt = torch.tensor([launches], device=dev, dtype=torch.float64)
+        dist.all_reduce(lt)
+        launches = int(lt.item())
+    ms_step = ms_total / args.steps
+    tokens = batch * seqlen
+    value = tokens * world / (ms_step / 1e3)
+
+    # ---- roofline of the dominant kernel (one launch per step on this path)
+    peaks, peak_kind = load_peaks()
+    nbytes, flops = algorithmic(w, batch, seqlen, decode)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    kernel_s = per_call_ms / 1e3
+    kernel_file = "scan_seq.cu"
+    traffic = kernel_traffic(kernel_file)
+    if decode or t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": nbytes / kernel_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / kernel_s / 1e12,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic
+    roof["peak_source"] = f"{peak_kind} ({'sustained' if roof['bound'] == 'tensor' else 'copy'})"
+    roof["kernel"] = kernel_file
+    hbm_ctx = {"achieved_gbs": nbytes / kernel_s / 1e9, "peak_gbs": peaks["hbm_gbs"],
+               "frac": nbytes / kernel_s / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
+               "algorithmic_flops": flops, "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6}
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, locals().get("state"),
+                  locals().get("tail"), dev, world)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name if not decode else
+                   f"cached block decode: {batch} streams x {seqlen}-token block, "
+                   f"H64x64 N128 bf16, 65536-token prefix state",
+                   "batch_per_gpu": batch, "seqlen": seqlen, "heads": H, "headdim": P,
+                   "d_state": N, "state_dtype": "f32",
+                   "l2": "inputs larger than L2 (xbc + y per step > 126 MB)" if not decode
+                   else "state (64 MiB) + block inputs larger than L2 reuse window",
+                   "parallelism": f"independent replicas x{world} (no data-path collective)"},
+        "roofline": roof, "roofline_hbm_context": hbm_ctx,
+        "e2e": e2e, "clocks": clocks, "gpu_launches": launches,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.workload)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, world):
+    """Same metric through the public API from pinned HOST buffers: each step
+    copies the step's inputs host->device, runs the call, and copies y back."""
+    import torch
+    H, P, N = w.heads, w.headdim, w.d_state
+    hx = g["xbc"].cpu().pin_memory()
+    hdt = g["dt"].cpu().pin_memory()
+    hy = torch.empty((batch, seqlen, H * P), dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(g["xbc"])
+    ddt = torch.empty_like(g["dt"])
+    dy = torch.empty((batch, seqlen, H * P), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dx.copy_(hx, non_blocking=True)
+        ddt.copy_(hdt, non_blocking=True)
+        if decode:
+            lib.bimamba_block_decode(dx, ddt, g["A"], g["D"], g["conv_w"], g["conv_b"], state, tail,
+                                     dy, None, None, ws, heads=H, headdim=P, d_state=N)
+        else:
+            lib.bimamba_ssd_fwd_rev(dx, ddt, g["A"], g["D"], g["conv_w"], None, None, None, dy, ws,
+                                    heads=H, headdim=P, d_state=N)
+        hy.copy_(dy, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.e2e_steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+    h2d = hx.numel() * hx.element_size() + hdt.numel() * hdt.element_size()
+    d2h = hy.numel() * hy.element_size()
+    return {"value": batch * seqlen * world / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_sample_step(w, workload, seq_tokens, seed=0):
+    """Run the oracle once on one sequence prefix of `seq_tokens` tokens of
+    the workload (all heads, both directions, conv fused); return seconds."""
+    import numpy as np
+    import oracle
+    from bidirectional_mamba_ssm_b200 import inputs as I
+    decode = workload == "decode"
+    cpu = I.make_inputs(w, seed=seed, seqlen=seq_tokens, batch=1, conv_bias=decode)
+    n = {k: (None if v is None else v.float().double().numpy()) for k, v in cpu.items()}
+    kw = dict(heads=w.heads, headdim=w.headdim, d_state=w.d_state)
+    t0 = time.perf_counter()
+    if decode:
+        state = np.zeros((1, w.heads, w.headdim, w.d_state))
+        tail = np.zeros((1, 4, w.channels))
+        oracle.block_decode(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], n["conv_b"], state,
+                            tail, **kw)
+    else:
+        oracle.bimamba(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], None, **kw)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, workload):
+    """The oracle, as it stands, on host cores: whole sequences of the
+    workload's length (capped at 4096 tokens) until ~10 s of CPU time."""
+    import oracle
+    seq = 64 if workload == "decode" else 1024
+    tokens, secs, reps = 0, 0.0, 0
+    while secs < 10.0 and reps < 64:
+        secs += oracle_sample_step(w, workload, seq, seed=reps)
+        tokens += seq
+        reps += 1
+    return {"value": tokens / secs, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} sequence(s) x {seq} tokens of the workload, all {w.heads} heads, "
+                      f"both directions, conv fused; double precision; {secs:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w, batch, seqlen = workload_spec(args.workload)
+    seq = 64 if args.workload == "decode" else 256
+    for i in range(args.warmup):
+        oracle_sample_step(w, args.workload, seq, seed=i)
+    total = 0.0
+    for i in range(args.steps):
+        total += oracle_sample_step(w, args.workload, seq, seed=100 + i)
+    ms = total / args.steps * 1e3
+    value = seq / (ms / 1e3)
+    cores = oracle.num_threads()
+    sample = (f"one sequence x {seq} tokens of the workload per step (all {w.heads} heads, both "
+              f"directions, conv fused), double precision")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name if args.workload != "decode" else "cached block decode",
+                   "batch_per_gpu": batch, "seqlen": seqlen, "heads": w.heads,
+                   "headdim": w.headdim, "d_state": w.d_state},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+"""Thin ctypes binding of libbimamba.so (the C ABI in include/bimamba.h).
+
+Argument marshalling only: tensors are passed as device pointers, the stream
+is torch's current CUDA stream unless one is given, and a non-OK status is
+raised as BimambaError.  All computation happens in the library's kernels;
+there is no fallback of any kind -- if the shared library is missing or
+cannot be loaded, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbimamba.so")
+
+BIMAMBA_OK = 0
+BIMAMBA_ERR_INVALID = 1
+BIMAMBA_ERR_UNSUPPORTED = 2
+BIMAMBA_ERR_CUDA = 3
+BIMAMBA_ERR_TIMEOUT = 4
+BIMAMBA_ERR_WORKSPACE = 5
+BIMAMBA_F32 = 0
+BIMAMBA_BF16 = 1
+
+# every symbol include/bimamba.h declares
+EXPORTED = (
+    "bimamba_version",
+    "bimamba_launch_count",
+    "bimamba_strerror",
+    "bimamba_get_error",
+    "bimamba_conv_silu",
+    "bimamba_workspace_bytes",
+    "bimamba_ssd_fwd_rev",
+    "bimamba_block_decode",
+)
+
+
+class BimambaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {strerror(status)} (status {status})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("len", ctypes.c_int), ("heads", ctypes.c_int),
+                ("headdim", ctypes.c_int), ("d_state", ctypes.c_int), ("ngroups", ctypes.c_int),
+                ("d_conv", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "`python -m bidirectional_mamba_ssm_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    dp = ctypes.POINTER(Dims)
+    lib.bimamba_version.restype = i
+    lib.bimamba_version.argtypes = []
+    lib.bimamba_launch_count.restype = ctypes.c_ulonglong
+    lib.bimamba_launch_count.argtypes = []
+    lib.bimamba_strerror.restype = ctypes.c_char_p
+    lib.bimamba_strerror.argtypes = [i]
+    lib.bimamba_get_error.restype = i
+    lib.bimamba_get_error.argtypes = [vp]
+    lib.bimamba_conv_silu.restype = i
+    lib.bimamba_conv_silu.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.bimamba_workspace_bytes.restype = sz
+    lib.bimamba_workspace_bytes.argtypes = [dp]
+    lib.bimamba_ssd_fwd_rev.restype = i
+    lib.bimamba_ssd_fwd_rev.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.bimamba_block_decode.restype = i
+    lib.bimamba_block_decode.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return BIMAMBA_F32
+    if t.dtype == torch.bfloat16:
+        return BIMAMBA_BF16
+    raise BimambaError(BIMAMBA_ERR_UNSUPPORTED, f"dtype {t.dtype}")
+
+
+def _check(status: int, where: str):
+    if status != BIMAMBA_OK:
+        raise BimambaError(status, where)
+
+
+def bimamba_version() -> int:
+    return _lib.bimamba_version()
+
+
+def bimamba_launch_count() -> int:
+    """Kernels this library has launched in this process so far."""
+    return int(_lib.bimamba_launch_count())
+
+
+def strerror(status: int) -> str:
+    return _lib.bimamba_strerror(status).decode()
+
+
+bimamba_strerror = strerror
+
+
+def bimamba_get_error(stream=None) -> int:
+    """Synchronise `stream`, then read and clear the device status word."""
+    return _lib.bimamba_get_error(_stream(stream))
+
+
+def make_dims(batch, seqlen, heads, headdim, d_state, dtype, ngroups=1, d_conv=4) -> Dims:
+    code = dtype if isinstance(dtype, int) else (
+        BIMAMBA_F32 if dtype in (torch.float32, "f32") else BIMAMBA_BF16)
+    return Dims(batch, seqlen, heads, headdim, d_state, ngroups, d_conv, code)
+
+
+def bimamba_workspace_bytes(dims: Dims) -> int:
+    return int(_lib.bimamba_workspace_bytes(ctypes.byref(dims)))
+
+
+def new_workspace(dims: Dims, device=None) -> torch.Tensor:
+    """Zero-filled workspace of the size the library asks for (>= 256 bytes)."""
+    n = max(256, bimamba_workspace_bytes(dims))
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def bimamba_conv_silu(u, out, w, bias=None, tail=None, reverse=False, silu=True, stream=None):
+    """out = SiLU(depthwise conv(u)) (or the pre-activation with silu=False)."""
+    bsz, L, ch = u.shape
+    st = _lib.bimamba_conv_silu(_ptr(u), _ptr(out), _ptr(w), _ptr(bias), _ptr(tail), bsz, L, ch,
+                                w.shape[1], int(bool(reverse)), int(bool(silu)), _dtype_code(u),
+                                _stream(stream))
+    _check(st, "bimamba_conv_silu")
+    return out
+
+
+def bimamba_ssd_fwd_rev(xbc, dt, A, D, conv_w, conv_b, init_state, final_state, y, workspace,
+                        *, heads, headdim, d_state, ngroups=1, stream=None, dims=None):
+    """y = forward stream + reverse stream of the conv+SiLU'd selective scan."""
+    if dims is None:
+        bsz, L, _ = xbc.shape
+        dims = make_dims(bsz, L, heads, headdim, d_state, _dtype_code(xbc), ngroups)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.bimamba_ssd_fwd_rev(ctypes.byref(dims), _ptr(xbc), _ptr(dt), _ptr(A), _ptr(D),
+                                  _ptr(conv_w), _ptr(conv_b), _ptr(init_state), _ptr(final_state),
+                                  _ptr(y), _ptr(workspace), wsz, _stream(stream))
+    _check(st, "bimamba_ssd_fwd_rev")
+    return y
+
+
+def bimamba_block_decode(xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, y, state_out,
+                         tail_out, workspace, *, heads, headdim, d_state, ngroups=1, stream=None):
+    """Cached block decode: forward resumes from (state, tail); reverse covers the block."""
+    S, L, _ = xbc_block.shape
+    dims = make_dims(S, L, heads, headdim, d_state, _dtype_code(xbc_block), ngroups)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.bimamba_block_decode(ctypes.byref(dims), _ptr(xbc_block), _ptr(dt_block), _ptr(A),
+                                   _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(state), _ptr(tail),
+                                   _ptr(y), _ptr(state_out), _ptr(tail_out), _ptr(workspace), wsz,
+                                   _stream(stream))
+    _check(st, "bimamba_block_decode")
+    return y

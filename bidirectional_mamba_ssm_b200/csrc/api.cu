@@ -1,0 +1,216 @@
+// api.cu -- host side of the C ABI declared in include/bimamba.h: argument
+// validation (nothing is launched when it fails), workspace sizing, the
+// per-device status word, and dispatch to the sm_100a kernels.
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "dispatch.h"
+
+namespace bimamba {
+
+__device__ int g_status;
+
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+int *device_status_word()
+{
+    // one address per device; resolved with that device current
+    static std::mutex mu;
+    static int *addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(p);
+    }
+    return addr[dev];
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool pow2_in(int v, int lo, int hi)
+{
+    return v >= lo && v <= hi && (v & (v - 1)) == 0;
+}
+
+// Shape/dtype checks common to every entry point; returns BIMAMBA_OK or an error.
+static int check_dims(const bimamba_dims *d)
+{
+    if (!d) return BIMAMBA_ERR_INVALID;
+    if (d->batch < 0 || d->len < 0 || d->heads <= 0 || d->headdim <= 0 || d->d_state <= 0 ||
+        d->ngroups <= 0 || d->d_conv <= 0)
+        return BIMAMBA_ERR_INVALID;
+    if (d->dtype != BIMAMBA_F32 && d->dtype != BIMAMBA_BF16) return BIMAMBA_ERR_INVALID;
+    if (d->heads % d->ngroups != 0) return BIMAMBA_ERR_INVALID;
+    if (d->ngroups != 1 || d->d_conv != 4) return BIMAMBA_ERR_UNSUPPORTED;
+    if (d->headdim % 8 != 0 || d->headdim > 128) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!pow2_in(d->d_state, 8, 256)) return BIMAMBA_ERR_UNSUPPORTED;
+    // sizes must fit the kernels' 32-bit token indexing and 64-bit offsets
+    const int64_t ch = (int64_t)d->heads * d->headdim + 2LL * d->ngroups * d->d_state;
+    if (ch > (1 << 20) || (int64_t)d->batch * d->len > (int64_t)1 << 40) return BIMAMBA_ERR_UNSUPPORTED;
+    if ((int64_t)d->batch > 65535 || d->heads > 65535) return BIMAMBA_ERR_UNSUPPORTED;
+    return BIMAMBA_OK;
+}
+
+static int cuda_status(cudaError_t e) { return e == cudaSuccess ? BIMAMBA_OK : BIMAMBA_ERR_CUDA; }
+
+}  // namespace bimamba
+
+using namespace bimamba;
+
+extern "C" {
+
+int bimamba_version(void) { return (1 << 16) | 0; }
+
+unsigned long long bimamba_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *bimamba_strerror(int status)
+{
+    switch (status) {
+    case BIMAMBA_OK: return "ok";
+    case BIMAMBA_ERR_INVALID: return "invalid argument";
+    case BIMAMBA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case BIMAMBA_ERR_CUDA: return "CUDA runtime error";
+    case BIMAMBA_ERR_TIMEOUT: return "a kernel's bounded wait timed out";
+    case BIMAMBA_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+    }
+}
+
+int bimamba_get_error(bimamba_stream_t stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    int *w = device_status_word();
+    if (!w) return BIMAMBA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    if (v) {
+        const int zero = 0;
+        if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return BIMAMBA_ERR_CUDA;
+    }
+    if (v & kStatusTimeout) return BIMAMBA_ERR_TIMEOUT;
+    return BIMAMBA_OK;
+}
+
+int bimamba_conv_silu(const void *u, void *out, const float *w, const float *bias,
+                      const void *tail, int batch, int len, int ch, int d_conv, int reverse,
+                      int silu, int dtype, bimamba_stream_t stream)
+{
+    if (batch < 0 || len < 0 || ch <= 0) return BIMAMBA_ERR_INVALID;
+    if (dtype != BIMAMBA_F32 && dtype != BIMAMBA_BF16) return BIMAMBA_ERR_INVALID;
+    if (d_conv != 4 || ch % 8 != 0) return BIMAMBA_ERR_UNSUPPORTED;
+    if (batch > 65535 || (len + 63) / 64 > 65535) return BIMAMBA_ERR_UNSUPPORTED;
+    if (batch == 0 || len == 0) return BIMAMBA_OK;
+    if (!u || !out || !w) return BIMAMBA_ERR_INVALID;
+    if (reverse && tail) return BIMAMBA_ERR_INVALID;
+    if (!aligned16(u) || !aligned16(out) || !aligned16(w) || (tail && !aligned16(tail)))
+        return BIMAMBA_ERR_INVALID;
+    const size_t esz = dtype == BIMAMBA_F32 ? 4 : 2;
+    const char *ub = static_cast<const char *>(u), *ob = static_cast<const char *>(out);
+    const size_t bytes = (size_t)batch * len * ch * esz;
+    if (ub < ob + bytes && ob < ub + bytes) return BIMAMBA_ERR_INVALID;  // overlap
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = dtype == BIMAMBA_F32
+                        ? launch_conv_silu<float>(u, out, w, bias, tail, batch, len, ch, reverse, silu, s)
+                        : launch_conv_silu<__nv_bfloat16>(u, out, w, bias, tail, batch, len, ch,
+                                                          reverse, silu, s);
+    return cuda_status(e);
+}
+
+size_t bimamba_workspace_bytes(const bimamba_dims *d)
+{
+    if (check_dims(d) != BIMAMBA_OK) return 0;
+    return workspace_bytes_for(*d);
+}
+
+// Shared by the full scan and the cached block decode.
+static int run_bimamba(const bimamba_dims *d, const void *xbc, const void *dt, const float *A,
+                       const float *D, const float *conv_w, const float *conv_b,
+                       const void *tail, const float *init, float *fin, void *y,
+                       void *workspace, size_t workspace_bytes, cudaStream_t s)
+{
+    const size_t need = workspace_bytes_for(*d);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+        return BIMAMBA_ERR_WORKSPACE;
+    Problem pr{};
+    pr.dims = *d;
+    pr.xbc = xbc; pr.dt = dt; pr.A = A; pr.D = D;
+    pr.conv_w = conv_w; pr.conv_b = conv_b; pr.tail = tail;
+    pr.init = init; pr.fin = fin; pr.y = y;
+    pr.workspace = workspace; pr.workspace_bytes = workspace_bytes;
+    pr.status = device_status_word();
+    return cuda_status(launch_bimamba(pr, s));
+}
+
+int bimamba_ssd_fwd_rev(const bimamba_dims *d, const void *xbc, const void *dt, const float *A,
+                        const float *D, const float *conv_w, const float *conv_b,
+                        const float *init_state, float *final_state, void *y, void *workspace,
+                        size_t workspace_bytes, bimamba_stream_t stream)
+{
+    int st = check_dims(d);
+    if (st != BIMAMBA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t state_bytes = sizeof(float) * (size_t)d->batch * d->heads * d->headdim * d->d_state;
+    if (d->batch == 0) return BIMAMBA_OK;
+    if (d->len == 0) {
+        // empty sequence: y is empty; the forward state passes through
+        if (!final_state) return BIMAMBA_OK;
+        if (init_state == final_state) return BIMAMBA_OK;
+        cudaError_t e = init_state
+                            ? cudaMemcpyAsync(final_state, init_state, state_bytes,
+                                              cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(final_state, 0, state_bytes, s);
+        return cuda_status(e);
+    }
+    if (!xbc || !dt || !A || !D || !y) return BIMAMBA_ERR_INVALID;
+    if (conv_b && !conv_w) return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {xbc, dt, A, D, y, conv_w, conv_b, init_state, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
+    return run_bimamba(d, xbc, dt, A, D, conv_w, conv_b, nullptr, init_state, final_state, y,
+                       workspace, workspace_bytes, s);
+}
+
+int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block, const void *dt_block,
+                         const float *A, const float *D, const float *conv_w,
+                         const float *conv_b, const float *state, const void *tail, void *y,
+                         float *state_out, void *tail_out, void *workspace,
+                         size_t workspace_bytes, bimamba_stream_t stream)
+{
+    int st = check_dims(d);
+    if (st != BIMAMBA_OK) return st;
+    if (d->batch == 0 || d->len == 0) return d->len == 0 && d->batch > 0 ? BIMAMBA_ERR_INVALID : BIMAMBA_OK;
+    if (!xbc_block || !dt_block || !A || !D || !conv_w || !state || !tail || !y)
+        return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, y, state_out, tail_out};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
+    const size_t esz = d->dtype == BIMAMBA_F32 ? 4 : 2;
+    const int ch = d->heads * d->headdim + 2 * d->ngroups * d->d_state;
+    const size_t tail_bytes = (size_t)d->batch * 4 * ch * esz;
+    if (tail_out) {
+        const char *a = static_cast<const char *>(tail), *b = static_cast<const char *>(tail_out);
+        if (a < b + tail_bytes && b < a + tail_bytes) return BIMAMBA_ERR_INVALID;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = run_bimamba(d, xbc_block, dt_block, A, D, conv_w, conv_b, tail, state, state_out, y,
+                     workspace, workspace_bytes, s);
+    if (st != BIMAMBA_OK || !tail_out) return st;
+    cudaError_t e = d->dtype == BIMAMBA_F32
+                        ? launch_tail_commit<float>(xbc_block, tail, tail_out, d->batch, d->len, ch, s)
+                        : launch_tail_commit<__nv_bfloat16>(xbc_block, tail, tail_out, d->batch,
+                                                            d->len, ch, s);
+    return cuda_status(e);
+}
+
+}  // extern "C"

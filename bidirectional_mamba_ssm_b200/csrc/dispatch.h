@@ -1,0 +1,48 @@
+// dispatch.h -- internal launcher declarations of the mixer library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/bimamba.h"
+
+namespace bimamba {
+
+// One validated call of the bidirectional mixer core (full scan or decode).
+struct Problem {
+    bimamba_dims dims;
+    const void *xbc;
+    const void *dt;
+    const float *A;
+    const float *D;
+    const float *conv_w;   // null: xbc already activated
+    const float *conv_b;
+    const void *tail;      // forward conv history (decode) or null
+    const float *init;     // forward initial state or null
+    float *fin;            // forward final state or null
+    void *y;
+    void *workspace;
+    size_t workspace_bytes;
+    int *status;           // device status word
+};
+
+size_t workspace_bytes_for(const bimamba_dims &d);
+cudaError_t launch_bimamba(const Problem &p, cudaStream_t stream);
+
+template <typename T>
+cudaError_t launch_conv_silu(const void *u, void *out, const float *w, const float *bias,
+                             const void *tail, int batch, int len, int ch, int rev, int silu,
+                             cudaStream_t stream);
+
+template <typename T>
+cudaError_t launch_scan_seq(const void *xbc, const void *dt, const float *A, const float *D,
+                            const float *conv_w, const float *conv_b, const void *tail,
+                            const float *init, float *fin, void *y, int batch, int len, int H,
+                            int P, int N, cudaStream_t stream);
+
+template <typename T>
+cudaError_t launch_tail_commit(const void *block, const void *tail, void *tail_out, int streams,
+                               int len, int ch, cudaStream_t stream);
+
+}  // namespace bimamba

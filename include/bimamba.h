@@ -1,0 +1,175 @@
+/*
+ * bimamba.h -- C ABI of the B200 (sm_100a) bidirectional Mamba-2 mixer core.
+ *
+ * The operation (sources by page title and section):
+ *  - "DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone"
+ *    (Japanese technical summary, section 2 "Proposed method"; Portuguese
+ *    technical summary, section 2 "Metodologia"): each mixer is a
+ *    bidirectional Mamba-2 mixer whose forward and reverse streams are
+ *    combined by addition.
+ *  - "DiffuMamba" blog post, network-architecture listing: d_state = 128,
+ *    d_conv = 4, expand = 2.
+ *  - Mamba-2 selective state space recurrence, per head h (A_h < 0 scalar):
+ *        h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t B_t^T     (P x N state)
+ *        y_t = h_t C_t + D_h x_t
+ *    preceded by a depthwise causal conv1d (K = 4 taps) + SiLU over the
+ *    x, B and C channels.  The reverse stream is the same computation on the
+ *    reversed sequence (mirrored conv taps, zero padding past the end, zero
+ *    initial state), flipped back.  y = forward stream + reverse stream.
+ *  - "Fixed state, long reach: constant-size caches in large-scale block
+ *    diffusion" (abstract, section 1): a finished prefix is cached as the
+ *    forward SSM state (O(1) in the context length) plus the conv history;
+ *    the reverse scan covers only the active block.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  Nothing is
+ *    allocated or freed inside the library.  Every call is asynchronous on
+ *    `stream` (the handle is a cudaStream_t; NULL = legacy default stream).
+ *  - Tensors are dense, row-major (last index fastest), and 16-byte aligned.
+ *  - Activations (xbc, dt, y, conv tails) have the element type `dtype`
+ *    (BIMAMBA_F32 or BIMAMBA_BF16).  A, D, conv weights/bias and SSM states
+ *    are always fp32.  Internal accumulation is fp32.
+ *  - xbc channel order per token is [x (H*P, head-major) | B (G*N) | C (G*N)],
+ *    ch = H*P + 2*G*N.
+ *  - Return value: BIMAMBA_OK, or an error code.  Argument errors are found
+ *    on the host before anything is launched (nothing is written).  Errors a
+ *    kernel detects (a bounded wait that gave up) are recorded in a per-device
+ *    status word; read and clear it with bimamba_get_error after the stream
+ *    has been synchronised.  No C++ exception crosses this boundary.
+ *  - Supported shapes: ngroups = 1, d_conv = 4, headdim a multiple of 8 up
+ *    to 128, d_state a power of two from 8 to 256, batch <= 65535.  Others
+ *    return BIMAMBA_ERR_UNSUPPORTED.
+ */
+#ifndef BIMAMBA_H
+#define BIMAMBA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *bimamba_stream_t; /* == cudaStream_t */
+
+typedef enum {
+    BIMAMBA_OK = 0,
+    BIMAMBA_ERR_INVALID = 1,      /* null pointer, bad size, misaligned      */
+    BIMAMBA_ERR_UNSUPPORTED = 2,  /* valid but not implemented shape/dtype   */
+    BIMAMBA_ERR_CUDA = 3,         /* a CUDA runtime call failed              */
+    BIMAMBA_ERR_TIMEOUT = 4,      /* a kernel's bounded wait gave up         */
+    BIMAMBA_ERR_WORKSPACE = 5     /* workspace missing or too small          */
+} bimamba_status;
+
+typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype;
+
+typedef struct {
+    int batch;    /* independent sequences (decode: streams)                */
+    int len;      /* tokens per sequence (decode: active block length)      */
+    int heads;    /* H                                                      */
+    int headdim;  /* P                                                      */
+    int d_state;  /* N                                                      */
+    int ngroups;  /* G, B/C groups shared by H/G heads each (must be 1)     */
+    int d_conv;   /* K, conv taps (must be 4)                               */
+    int dtype;    /* bimamba_dtype of xbc, dt, y and conv tails             */
+} bimamba_dims;
+
+/* Library version, (major << 16) | minor. */
+int bimamba_version(void);
+
+/* Number of kernels this library has launched in this process so far
+ * (host-side counter, all devices and streams).  For accounting only. */
+unsigned long long bimamba_launch_count(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bimamba_strerror(int status);
+
+/*
+ * Reads and clears this device's kernel status word (the current device).
+ * Synchronises `stream` first.  Returns BIMAMBA_OK when no kernel recorded
+ * an error since the last call, BIMAMBA_ERR_TIMEOUT when a bounded wait gave
+ * up, BIMAMBA_ERR_CUDA when the runtime reports an error.
+ */
+int bimamba_get_error(bimamba_stream_t stream);
+
+/*
+ * Depthwise conv1d with `d_conv` taps followed by SiLU (silu != 0) or the
+ * identity (silu == 0).  Step "conv + SiLU" of the mixer.
+ *   u    : (batch, len, ch)    input, dtype
+ *   out  : (batch, len, ch)    output, dtype; must not overlap u
+ *   w    : (ch, d_conv) fp32   tap j of channel c
+ *   bias : (ch) fp32 or NULL
+ *   tail : (batch, d_conv, ch) dtype or NULL -- the d_conv raw tokens that
+ *          precede t = 0, oldest first (forward only; must be NULL when
+ *          reverse != 0).  NULL means zeros.
+ * Forward (reverse == 0): pre[t,c] = bias[c] + sum_j w[c,j] u[t-(K-1)+j, c]
+ * Reverse (reverse != 0): pre[t,c] = bias[c] + sum_j w[c,j] u[t+(K-1)-j, c],
+ *                         u past the end = 0   (= flip(conv(flip(u)))).
+ * Requires ch % 8 == 0.  Sums are formed in fp32 in tap order j = 0..K-1.
+ */
+int bimamba_conv_silu(const void *u, void *out, const float *w, const float *bias,
+                      const void *tail, int batch, int len, int ch, int d_conv,
+                      int reverse, int silu, int dtype, bimamba_stream_t stream);
+
+/*
+ * Bytes of scratch workspace bimamba_ssd_fwd_rev / bimamba_block_decode need
+ * for dims `d`.  The caller allocates it once (device memory, 256-byte
+ * aligned), zero-fills it before first use, and may reuse it for any later
+ * call whose workspace size is not larger.  The kernels leave it zeroed.
+ * Calls that share one workspace must not run concurrently.
+ * Returns 0 for invalid dims.
+ */
+size_t bimamba_workspace_bytes(const bimamba_dims *d);
+
+/*
+ * Full bidirectional mixer core (steps: load, conv+SiLU both ways, decay,
+ * intra-chunk contraction, chunk states, state passing, off-diagonal term,
+ * fused forward+reverse sum).
+ *   xbc         : (batch, len, ch) raw xBC, dtype.  If conv_w == NULL the
+ *                 conv and SiLU are skipped and xbc is taken as activated.
+ *   dt          : (batch, len, H) dtype, already positive (post-softplus)
+ *   A, D        : (H) fp32
+ *   conv_w      : (ch, 4) fp32 or NULL;  conv_b : (ch) fp32 or NULL
+ *   init_state  : (batch, H, P, N) fp32 or NULL -- forward initial state
+ *   final_state : (batch, H, P, N) fp32 or NULL -- forward state after the
+ *                 last token (written); may alias init_state
+ *   y           : (batch, len, H*P) dtype, written (not accumulated)
+ *   workspace   : bimamba_workspace_bytes(d) bytes, see above
+ */
+int bimamba_ssd_fwd_rev(const bimamba_dims *d, const void *xbc, const void *dt,
+                        const float *A, const float *D, const float *conv_w,
+                        const float *conv_b, const float *init_state,
+                        float *final_state, void *y, void *workspace,
+                        size_t workspace_bytes, bimamba_stream_t stream);
+
+/*
+ * Cached block decode for block diffusion: d->batch independent streams,
+ * each with an active block of d->len tokens.  The forward stream resumes
+ * from `state` with the conv history `tail`; the reverse stream covers the
+ * block only (zero padding past the block end, zero state).  y = sum.
+ * Result equals a full recompute over prefix + block (forward stream at the
+ * block positions) plus the reverse stream over the block alone.
+ *   xbc_block : (streams, len, ch) raw xBC of the active block, dtype
+ *   dt_block  : (streams, len, H) dtype
+ *   A, D, conv_w (required), conv_b (nullable): as above
+ *   state     : (streams, H, P, N) fp32 forward state after the prefix
+ *   tail      : (streams, 4, ch) dtype, last 4 raw prefix tokens, oldest
+ *               first (zeros where the prefix is shorter)
+ *   y         : (streams, len, H*P) dtype
+ *   state_out : (streams, H, P, N) fp32 or NULL -- commit: forward state
+ *               after the block; may alias `state`
+ *   tail_out  : (streams, 4, ch) dtype or NULL -- commit: last 4 raw tokens
+ *               of prefix + block; must not overlap `tail`
+ *   workspace : bimamba_workspace_bytes(d) bytes
+ */
+int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block,
+                         const void *dt_block, const float *A, const float *D,
+                         const float *conv_w, const float *conv_b,
+                         const float *state, const void *tail, void *y,
+                         float *state_out, void *tail_out, void *workspace,
+                         size_t workspace_bytes, bimamba_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BIMAMBA_H */

@@ -1,0 +1,94 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/bimamba.h declares, and rejects bad arguments on
+the host (before any CUDA call) with the documented status codes."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bidirectional_mamba_ssm_b200 import build
+    build.build()
+    from bidirectional_mamba_ssm_b200 import _lib
+    return _lib
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bimamba.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bimamba_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert set(names) == set(lib.EXPORTED)
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in names:
+        assert hasattr(so, n), n
+
+
+def test_version_and_strerror(lib):
+    assert lib.bimamba_version() >> 16 == 1
+    for code in range(6):
+        assert lib.strerror(code) and lib.strerror(code) != "unknown status"
+    assert lib.strerror(99) == "unknown status"
+
+
+def _call_scan(lib, dims, **ptrs):
+    L = lib.library()
+    p = dict(xbc=16, dt=16, A=16, D=16, conv_w=None, conv_b=None, init=None, fin=None, y=16,
+             ws=None, wsz=0)
+    p.update(ptrs)
+    return L.bimamba_ssd_fwd_rev(ctypes.byref(dims), p["xbc"], p["dt"], p["A"], p["D"],
+                                 p["conv_w"], p["conv_b"], p["init"], p["fin"], p["y"], p["ws"],
+                                 p["wsz"], None)
+
+
+def test_host_validation_codes(lib):
+    ok = dict(batch=1, seqlen=8, heads=2, headdim=8, d_state=16, dtype=0)
+    d = lib.make_dims(**ok)
+    # shape errors (checked before anything touches the device)
+    for bad, code in [(dict(heads=0), lib.BIMAMBA_ERR_INVALID),
+                      (dict(headdim=-8), lib.BIMAMBA_ERR_INVALID),
+                      (dict(batch=-1), lib.BIMAMBA_ERR_INVALID),
+                      (dict(headdim=12), lib.BIMAMBA_ERR_UNSUPPORTED),
+                      (dict(headdim=136), lib.BIMAMBA_ERR_UNSUPPORTED),
+                      (dict(d_state=24), lib.BIMAMBA_ERR_UNSUPPORTED),
+                      (dict(d_state=512), lib.BIMAMBA_ERR_UNSUPPORTED),
+                      (dict(ngroups=2), lib.BIMAMBA_ERR_UNSUPPORTED),
+                      (dict(d_conv=3), lib.BIMAMBA_ERR_UNSUPPORTED),
+                      (dict(dtype=7), lib.BIMAMBA_ERR_INVALID)]:
+        args = dict(ok)
+        args.update(bad)
+        assert _call_scan(lib, lib.make_dims(**args)) == code, bad
+        assert lib.bimamba_workspace_bytes(lib.make_dims(**args)) == 0
+    # pointer errors
+    assert _call_scan(lib, d, xbc=None) == lib.BIMAMBA_ERR_INVALID
+    assert _call_scan(lib, d, y=None) == lib.BIMAMBA_ERR_INVALID
+    assert _call_scan(lib, d, xbc=18) == lib.BIMAMBA_ERR_INVALID          # misaligned
+    assert _call_scan(lib, d, conv_b=16) == lib.BIMAMBA_ERR_INVALID       # bias without weights
+    # empty batch is a no-op
+    assert _call_scan(lib, lib.make_dims(**dict(ok, batch=0))) == lib.BIMAMBA_OK
+    L = lib.library()
+    # conv entry point
+    assert L.bimamba_conv_silu(16, 16 + 4096, 16, None, None, 1, 8, 12, 4, 0, 1, 0, None) \
+        == lib.BIMAMBA_ERR_UNSUPPORTED                                      # ch % 8
+    assert L.bimamba_conv_silu(16, 32, 16, None, None, 1, 8, 8, 4, 0, 1, 0, None) \
+        == lib.BIMAMBA_ERR_INVALID                                          # overlap
+    assert L.bimamba_conv_silu(16, 1 << 20, 16, None, 16, 1, 8, 8, 4, 1, 1, 0, None) \
+        == lib.BIMAMBA_ERR_INVALID                                          # tail + reverse
+    # decode entry point: conv weights, state and tail are required
+    r = L.bimamba_block_decode(ctypes.byref(d), 16, 16, 16, 16, None, None, 16, 16, 16, None,
+                               None, None, 0, None)
+    assert r == lib.BIMAMBA_ERR_INVALID
+
+
+def test_workspace_size_is_monotone(lib):
+    a = lib.bimamba_workspace_bytes(lib.make_dims(8, 4096, 64, 64, 128, 1))
+    b = lib.bimamba_workspace_bytes(lib.make_dims(8, 8192, 64, 64, 128, 1))
+    assert 0 <= a <= b
