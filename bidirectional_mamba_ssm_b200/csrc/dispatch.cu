@@ -6,13 +6,16 @@ namespace bimamba {
 
 size_t workspace_bytes_for(const bimamba_dims &d)
 {
-    (void)d;
-    return 0;
+    return tc_path_supported(d) ? tc_workspace_bytes(d) : 0;
 }
 
 cudaError_t launch_bimamba(const Problem &p, cudaStream_t stream)
 {
     const bimamba_dims &d = p.dims;
+    // bf16 at the model's head shape runs on the tensor cores; fp32 (which
+    // needs a 1e-4 bound that bf16 operands cannot hold) and other head
+    // shapes run on the sequential fp32 kernel.
+    if (tc_path_supported(d)) return launch_ssd_tc(p, stream);
     if (d.dtype == BIMAMBA_F32)
         return launch_scan_seq<float>(p.xbc, p.dt, p.A, p.D, p.conv_w, p.conv_b, p.tail, p.init,
                                       p.fin, p.y, d.batch, d.len, d.heads, d.headdim, d.d_state,

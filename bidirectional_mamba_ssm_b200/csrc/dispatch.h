@@ -30,6 +30,11 @@ struct Problem {
 size_t workspace_bytes_for(const bimamba_dims &d);
 cudaError_t launch_bimamba(const Problem &p, cudaStream_t stream);
 
+// chunked tensor-core path (bf16, headdim 64, d_state 128)
+bool tc_path_supported(const bimamba_dims &d);
+size_t tc_workspace_bytes(const bimamba_dims &d);
+cudaError_t launch_ssd_tc(const Problem &p, cudaStream_t stream);
+
 template <typename T>
 cudaError_t launch_conv_silu(const void *u, void *out, const float *w, const float *bias,
                              const void *tail, int batch, int len, int ch, int rev, int silu,
