@@ -6,7 +6,7 @@ binding with the same entry-point names as include/bimamba.h.  The binding
 is loaded on first attribute access so that ``inputs`` can be used without
 the shared library.
 """
-__all__ = ["bimamba_version", "bimamba_launch_count", "bimamba_strerror", "bimamba_get_error", "bimamba_conv_silu",
+__all__ = ["bimamba_version", "bimamba_launch_count", "bimamba_set_timing_events", "bimamba_strerror", "bimamba_get_error", "bimamba_conv_silu",
            "bimamba_workspace_bytes", "bimamba_ssd_fwd_rev", "bimamba_block_decode",
            "make_dims", "new_workspace", "BimambaError"]
 

@@ -29,6 +29,7 @@ BIMAMBA_BF16 = 1
 EXPORTED = (
     "bimamba_version",
     "bimamba_launch_count",
+    "bimamba_set_timing_events",
     "bimamba_strerror",
     "bimamba_get_error",
     "bimamba_conv_silu",
@@ -61,6 +62,8 @@ def _load() -> ctypes.CDLL:
     lib.bimamba_version.argtypes = []
     lib.bimamba_launch_count.restype = ctypes.c_ulonglong
     lib.bimamba_launch_count.argtypes = []
+    lib.bimamba_set_timing_events.restype = i
+    lib.bimamba_set_timing_events.argtypes = [vp, vp]
     lib.bimamba_strerror.restype = ctypes.c_char_p
     lib.bimamba_strerror.argtypes = [i]
     lib.bimamba_get_error.restype = i
@@ -119,6 +122,14 @@ def bimamba_version() -> int:
 def bimamba_launch_count() -> int:
     """Kernels this library has launched in this process so far."""
     return int(_lib.bimamba_launch_count())
+
+
+def bimamba_set_timing_events(start=None, stop=None):
+    """Record torch.cuda.Event `start`/`stop` around the main scan kernel of
+    every later call on this thread (None, None switches it off)."""
+    st = _lib.bimamba_set_timing_events(None if start is None else start.cuda_event,
+                                        None if stop is None else stop.cuda_event)
+    _check(st, "bimamba_set_timing_events")
 
 
 def strerror(status: int) -> str:

@@ -18,6 +18,10 @@ static std::atomic<unsigned long long> g_launches{0};
 
 void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
+static thread_local TimingEvents t_events{nullptr, nullptr};
+
+TimingEvents timing_events() { return t_events; }
+
 int *device_status_word()
 {
     // one address per device; resolved with that device current
@@ -71,6 +75,14 @@ extern "C" {
 int bimamba_version(void) { return (1 << 16) | 0; }
 
 unsigned long long bimamba_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int bimamba_set_timing_events(void *start, void *stop)
+{
+    if ((start == nullptr) != (stop == nullptr)) return BIMAMBA_ERR_INVALID;
+    t_events.start = static_cast<cudaEvent_t>(start);
+    t_events.stop = static_cast<cudaEvent_t>(stop);
+    return BIMAMBA_OK;
+}
 
 const char *bimamba_strerror(int status)
 {

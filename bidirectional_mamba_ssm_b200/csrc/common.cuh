@@ -26,6 +26,14 @@ int *device_status_word();
 // Host-side count of kernels this library has launched (defined in api.cu).
 void count_launch(int n = 1);
 
+// Caller-provided timing events around the main scan kernel (or null); see
+// bimamba_set_timing_events.
+struct TimingEvents {
+    cudaEvent_t start;
+    cudaEvent_t stop;
+};
+TimingEvents timing_events();
+
 // ---- element loads / stores in the activation dtype -------------------------
 template <typename T> struct Elem;
 

@@ -160,9 +160,13 @@ static cudaError_t launch_seq_t(const SeqParams &p, int batch, cudaStream_t stre
     cudaError_t e = cudaFuncSetAttribute(scan_seq_kernel<T, NPT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    const TimingEvents ev = timing_events();
+    if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
     scan_seq_kernel<T, NPT><<<dim3(p.H, batch), threads, smem, stream>>>(p);
     cudaError_t err = cudaGetLastError();
-    if (err == cudaSuccess) count_launch();
+    if (err != cudaSuccess) return err;
+    count_launch();
+    if (ev.stop) err = cudaEventRecord(ev.stop, stream);
     return err;
 }
 

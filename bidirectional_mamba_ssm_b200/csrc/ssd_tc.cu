@@ -42,6 +42,9 @@
 #include "dispatch.h"
 #include "tc_ptx.cuh"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 namespace bimamba {
 
 namespace {
@@ -50,27 +53,29 @@ constexpr int kQ = 128;  // chunk length
 constexpr int kP = 64;   // headdim of this kernel
 constexpr int kN = 128;  // d_state of this kernel
 constexpr int kThreads = 256;
-constexpr int kLocalCh = kP + 2 * kN;  // channels one CTA reads: x of its head, B, C
+constexpr int kBC = 2 * kN;            // B and C channels
+constexpr int kRawRows = kQ + 3;       // raw x rows per chunk: 128 slots + 3-token conv halo
 constexpr uint32_t kTmemCols = 256;
 
 // shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t kOffC = 0;        // C      [t][n]   2 x 16 KB blocks
-constexpr uint32_t kOffB = 32768;    // B      [s][n]   2 x 16 KB
+constexpr uint32_t kOffC = 0;        // C      [t][n]   2 x 16 KB blocks (TMA, swizzled)
+constexpr uint32_t kOffB = 32768;    // B      [s][n]   2 x 16 KB        (TMA, swizzled)
 constexpr uint32_t kOffM = 65536;    // M      [t][s]   2 x 16 KB
 constexpr uint32_t kOffX = 98304;    // X      [s][p]   16 KB
 constexpr uint32_t kOffXw = 114688;  // wX     [s][p]   16 KB
-constexpr uint32_t kOffS = 131072;   // S^T    [n][p]   16 KB (bf16 copy)
-constexpr uint32_t kOffCum = 147456;            // f32[128] prefix sums of dt*A
+constexpr uint32_t kOffS = 131072;   // S^T    [n][p]   16 KB (bf16 copy of the state)
+constexpr uint32_t kOffRaw = 147456; // raw x  [131][64] bf16, row-major (TMA)
+constexpr uint32_t kRawBytes = kRawRows * kP * 2;   // 16768
+constexpr uint32_t kOffCum = kOffRaw + 17408;   // f32[128] prefix sums of dt*A
 constexpr uint32_t kOffDt = kOffCum + 512;      // f32[128] dt
-constexpr uint32_t kOffW = kOffDt + 512;        // f32[128] exp(c_last - c_s) dt_s
-constexpr uint32_t kOffConvW = kOffW + 512;     // float4[320] conv taps
-constexpr uint32_t kOffConvB = kOffConvW + 16 * kLocalCh;  // f32[320]
-constexpr uint32_t kOffWsum = kOffConvB + 4 * kLocalCh;     // f32[8] warp sums
-constexpr uint32_t kOffMbar = kOffWsum + 64;    // u64 mbarrier
-constexpr uint32_t kOffTmem = kOffMbar + 8;     // u32 TMEM base
+constexpr uint32_t kOffConvW = kOffDt + 512;    // float4[64] conv taps of x
+constexpr uint32_t kOffConvB = kOffConvW + 16 * kP;   // f32[64]
+constexpr uint32_t kOffMbar = kOffConvB + 4 * kP;     // u64 x3: MMA, raw-x TMA, B/C TMA
+constexpr uint32_t kOffTmem = kOffMbar + 24;    // u32 TMEM base
 constexpr uint32_t kOffFlag = kOffTmem + 4;     // i32 handshake result
 constexpr uint32_t kSmemUsed = kOffFlag + 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
+constexpr uint32_t kBCBytes = 4 * kQ * 64 * 2;     // four 128 x 64 bf16 boxes
 
 constexpr uint32_t kColG = 0;
 constexpr uint32_t kColYd = 0;
@@ -92,7 +97,7 @@ struct TcParams {
     __nv_bfloat16 *y;
     int *flags;   // [batch][H][nchunks][2]: arrivals, partial-ready
     int *status;
-    int len, H, ch, nchunks;
+    int len, H, ch, nchunks, batch;
 };
 
 __device__ __forceinline__ int ld_acquire(const int *p)
@@ -100,6 +105,13 @@ __device__ __forceinline__ int ld_acquire(const int *p)
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Release store at GPU scope.  Issued by one thread after a CTA barrier, it
+// publishes every write the CTA made before that barrier.
+__device__ __forceinline__ void st_release(int *p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void unpack8(uint4 r, float (&v)[8])
@@ -125,7 +137,76 @@ __device__ __forceinline__ uint4 pack8(const float *v)
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) ssd_tc_kernel(const TcParams p)
+// Prepass: conv+SiLU of the B and C channels, once per (sequence, direction),
+// written in walk order: act[(dir * batch + b) * len + s][n], s = walk step
+// (token s forward, token len-1-s reverse).  Without conv weights the raw
+// values are copied.  One thread: 8 channels x 8 walk steps, 3-step window in
+// registers; a warp covers one token's 256 channels (512 contiguous bytes).
+__global__ void __launch_bounds__(128)
+bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc, const __nv_bfloat16 *__restrict__ tail,
+                  const float *__restrict__ conv_w, const float *__restrict__ conv_b,
+                  __nv_bfloat16 *__restrict__ act, int len, int ch, int cbase, int batch)
+{
+    const int g = threadIdx.x & 31, sub = threadIdx.x >> 5;
+    const int b = blockIdx.y;
+    const bool rev = blockIdx.z != 0;
+    const int s_begin = blockIdx.x * 32 + sub * 8;
+    if (s_begin >= len) return;
+    const int s_end = min(s_begin + 8, len);
+    const int n0 = 8 * g;
+    const int c = cbase + n0;
+    const __nv_bfloat16 *xb = xbc + (size_t)b * len * ch + c;
+    __nv_bfloat16 *ob = act + ((size_t)(blockIdx.z * batch + b) * len) * kBC + n0;
+    auto raw = [&](int s, float (&v)[8]) {
+        if (s >= 0) {
+            const int tok = rev ? len - 1 - s : s;
+            unpack8(*reinterpret_cast<const uint4 *>(xb + (size_t)tok * ch), v);
+        } else if (!rev && tail) {
+            unpack8(*reinterpret_cast<const uint4 *>(tail + ((size_t)b * 4 + 4 + s) * ch + c), v);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = 0.0f;
+        }
+    };
+    if (!conv_w) {
+        for (int s = s_begin; s < s_end; ++s) {
+            float v[8];
+            raw(s, v);
+            *reinterpret_cast<uint4 *>(ob + (size_t)s * kBC) = pack8(v);
+        }
+        return;
+    }
+    float w0[8], w1[8], w2[8], w3[8], bb[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(conv_w + (size_t)(c + q) * 4);
+        w0[q] = t4.x; w1[q] = t4.y; w2[q] = t4.z; w3[q] = t4.w;
+        bb[q] = conv_b ? conv_b[c + q] : 0.0f;
+    }
+    float r0[8], r1[8], r2[8];
+    raw(s_begin - 3, r0);
+    raw(s_begin - 2, r1);
+    raw(s_begin - 1, r2);
+    for (int s = s_begin; s < s_end; ++s) {
+        float r3[8], o[8];
+        raw(s, r3);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            float acc = bb[q];
+            acc = fmaf(w0[q], r0[q], acc);
+            acc = fmaf(w1[q], r1[q], acc);
+            acc = fmaf(w2[q], r2[q], acc);
+            acc = fmaf(w3[q], r3[q], acc);
+            o[q] = tc::silu_tanh(acc);
+            r0[q] = r1[q]; r1[q] = r2[q]; r2[q] = r3[q];
+        }
+        *reinterpret_cast<uint4 *>(ob + (size_t)s * kBC) = pack8(o);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_bc,
+              const TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -133,30 +214,65 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_tc_kernel(const TcParams p)
     const uint32_t sbase = tc::smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x >> 1;
-    const bool rev = (blockIdx.x & 1) != 0;
+    const int dir = blockIdx.x & 1;
+    const bool rev = dir != 0;
     const int b = blockIdx.y;
     const int H = p.H, L = p.len, ch = p.ch;
 
     float *cum = reinterpret_cast<float *>(sm + kOffCum);
     float *dts = reinterpret_cast<float *>(sm + kOffDt);
-    float *wgt = reinterpret_cast<float *>(sm + kOffW);
     float4 *convw = reinterpret_cast<float4 *>(sm + kOffConvW);
     float *convb = reinterpret_cast<float *>(sm + kOffConvB);
-    float *wsum = reinterpret_cast<float *>(sm + kOffWsum);
     int *flag_slot = reinterpret_cast<int *>(sm + kOffFlag);
-    const uint32_t mbar = sbase + kOffMbar;
+    const uint32_t mbar_mma = sbase + kOffMbar;
+    const uint32_t mbar_x = sbase + kOffMbar + 8;
+    const uint32_t mbar_bc = sbase + kOffMbar + 16;
+    const __nv_bfloat16 *raw = reinterpret_cast<const __nv_bfloat16 *>(sm + kOffRaw);
 
-    // ---- setup: conv taps of this CTA's channels, TMEM, mbarrier
+    // geometry of walk chunk k: token chunk c, first token t0, valid slots cnt,
+    // walk step of slot 0
+    auto chunk_of = [&](int k, int &t0, int &cnt, int &s0) {
+        const int c = rev ? p.nchunks - 1 - k : k;
+        t0 = c * kQ;
+        cnt = min(kQ, L - t0);
+        s0 = rev ? L - t0 - cnt : t0;
+        return c;
+    };
+    // TMA producers (thread 0): raw x rows and the B/C operand tiles of chunk k
+    auto issue_x = [&](int k) {
+        int t0, cnt, s0;
+        chunk_of(k, t0, cnt, s0);
+        tc::mbar_expect_tx(mbar_x, kRawBytes);
+        tc::tma_load_3d(sbase + kOffRaw, &tm_x, h * kP, rev ? t0 : t0 - 3, b, mbar_x);
+    };
+    auto issue_bc = [&](int k) {
+        int t0, cnt, s0;
+        chunk_of(k, t0, cnt, s0);
+        const int zc = dir * p.batch + b;
+        tc::mbar_expect_tx(mbar_bc, kBCBytes);
+        tc::tma_load_3d(sbase + kOffB, &tm_bc, 0, s0, zc, mbar_bc);
+        tc::tma_load_3d(sbase + kOffB + 16384, &tm_bc, 64, s0, zc, mbar_bc);
+        tc::tma_load_3d(sbase + kOffC, &tm_bc, 128, s0, zc, mbar_bc);
+        tc::tma_load_3d(sbase + kOffC + 16384, &tm_bc, 192, s0, zc, mbar_bc);
+    };
+
+    // ---- setup: conv taps of this head's x channels, TMEM, barriers, first loads
     const bool has_conv = p.conv_w != nullptr;
-    for (int lc = tid; lc < kLocalCh; lc += kThreads) {
-        const int c = lc < kP ? h * kP + lc : H * kP + (lc - kP);
-        if (has_conv) {
-            convw[lc] = *reinterpret_cast<const float4 *>(p.conv_w + (size_t)c * 4);
-            convb[lc] = p.conv_b ? p.conv_b[c] : 0.0f;
-        }
+    if (tid < kP && has_conv) {
+        const int c = h * kP + tid;
+        convw[tid] = *reinterpret_cast<const float4 *>(p.conv_w + (size_t)c * 4);
+        convb[tid] = p.conv_b ? p.conv_b[c] : 0.0f;
     }
     if (warp == 0) tc::tmem_alloc(sbase + kOffTmem, kTmemCols);
-    if (tid == 0) tc::mbar_init(mbar, 1);
+    if (tid == 0) {
+        tc::prefetch_tmap(&tm_x);
+        tc::prefetch_tmap(&tm_bc);
+        tc::mbar_init(mbar_mma, 1);
+        tc::mbar_init(mbar_x, 1);
+        tc::mbar_init(mbar_bc, 1);
+        issue_x(0);
+        issue_bc(0);
+    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -181,140 +297,141 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_tc_kernel(const TcParams p)
     };
     store_state_bf16();
 
-    const __nv_bfloat16 *xb = p.xbc + (size_t)b * L * ch;
-    const __nv_bfloat16 *tailb = p.tail ? p.tail + (size_t)b * 4 * ch : nullptr;
     uint32_t phase = 0;
     bool ok = true;
 
-    for (int k = 0; k < p.nchunks; ++k) {
-        const int c = rev ? p.nchunks - 1 - k : k;  // token chunk
-        const int t0 = c * kQ;
-        const int cnt = min(kQ, L - t0);
-        const int s0 = rev ? L - t0 - cnt : t0;     // walk step of slot 0
-
-        // ---- A: dt, inclusive prefix sums of dt*A, state weights
-        if (tid < kQ) {
-            float d = 0.0f;
-            if (tid < cnt) {
-                const int s = s0 + tid;
+    // dt of walk chunk k for slots 4*lane .. 4*lane+3 (warp 0), zero past cnt
+    auto load_dt = [&](int k, float (&d)[4]) {
+        int t0, cnt, s0;
+        chunk_of(k, t0, cnt, s0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = 4 * lane + i;
+            d[i] = 0.0f;
+            if (j < cnt) {
+                const int s = s0 + j;
                 const int tok = rev ? L - 1 - s : s;
-                d = __bfloat162float(p.dt[((size_t)b * L + tok) * H + h]);
+                d[i] = __bfloat162float(p.dt[((size_t)b * L + tok) * H + h]);
             }
-            float a = d * Ah;
+        }
+    };
+    float dt_next[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (warp == 0) load_dt(0, dt_next);
+
+    for (int k = 0; k < p.nchunks; ++k) {
+        int t0, cnt, s0;
+        const int c = chunk_of(k, t0, cnt, s0);
+        const uint32_t tphase = k & 1;
+
+        // ---- A (warp 0): dt, inclusive prefix sums of dt*A over the chunk;
+        // the next chunk's dt is requested now and used one chunk later
+        // @phase A
+        if (warp == 0) {
+            float d[4], a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[i] = dt_next[i];
+            if (k + 1 < p.nchunks) load_dt(k + 1, dt_next);
+            a[0] = d[0] * Ah;
+#pragma unroll
+            for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Ah, a[i - 1]);
+            float run = a[3];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, a, o);
-                if (lane >= o) a += v;
+                const float v = __shfl_up_sync(0xffffffffu, run, o);
+                if (lane >= o) run += v;
             }
-            if (lane == 31) wsum[warp] = a;
-            dts[tid] = d;
-            cum[tid] = a;
+            const float excl = run - a[3];
+            *reinterpret_cast<float4 *>(dts + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
+            *reinterpret_cast<float4 *>(cum + 4 * lane) =
+                make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
         }
-        __syncthreads();
-        if (tid < kQ) {
-            float off = 0.0f;
-            for (int w = 0; w < (tid >> 5); ++w) off += wsum[w];
-            cum[tid] += off;
+        ok = tc::mbar_wait_bounded(mbar_x, tphase, kWaitCycles);
+        if (!__syncthreads_and(ok)) break;
+        // decode: the conv history before token 0 comes from the cached tail
+        if (!rev && c == 0 && p.tail) {
+            for (int e = tid; e < 3 * (kP / 8); e += kThreads) {
+                const int r = e / (kP / 8), g = e % (kP / 8);
+                *reinterpret_cast<uint4 *>(sm + kOffRaw + r * (kP * 2) + g * 16) =
+                    *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch + h * kP + 8 * g);
+            }
+            __syncthreads();
         }
-        __syncthreads();
         const float cum_last = cum[kQ - 1];
-        if (tid < kQ) wgt[tid] = __expf(cum_last - cum[tid]) * dts[tid];
-        __syncthreads();
 
-        // ---- B: conv+SiLU of x (this head), B, C into the swizzled tiles
-        for (int it = tid; it < (kLocalCh / 8) * (kQ / 8); it += kThreads) {
-            const int g = it % (kLocalCh / 8), r = it / (kLocalCh / 8);
-            const int j0 = r * 8;
-            const int lc0 = 8 * g;
-            const int cg = lc0 < kP ? h * kP + lc0 : H * kP + (lc0 - kP);
-            float o[8][8];
-            if (j0 >= cnt) {
+        // ---- B: conv+SiLU of this head's x (raw rows in shared memory) into
+        // X and wX.  Thread: 8 channels (group g) x 4 slots.  Raw row of token
+        // u: forward u - (t0 - 3), reverse u - t0.
+        {
+            const int g = tid & 7;
+            const int j0 = (tid >> 3) * 4;
+            float o[4][8];
+            if (has_conv) {
+                float w0[8], w1[8], w2[8], w3[8], bb[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int q = 0; q < 8; ++q) {
+                    const float4 t4 = convw[8 * g + q];
+                    w0[q] = t4.x; w1[q] = t4.y; w2[q] = t4.z; w3[q] = t4.w;
+                    bb[q] = convb[8 * g + q];
+                }
+                // the 7 raw rows slots j0..j0+3 read, oldest first in walk order
+                float rr[7][8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) o[i][q] = 0.0f;
-            } else {
-                auto raw = [&](int j, float (&v)[8]) {
-                    const int s = s0 + j;
-                    if (s >= 0) {
-                        const int tok = rev ? L - 1 - s : s;
-                        unpack8(*reinterpret_cast<const uint4 *>(xb + (size_t)tok * ch + cg), v);
-                    } else if (!rev && tailb) {
-                        unpack8(*reinterpret_cast<const uint4 *>(tailb + (size_t)(4 + s) * ch + cg), v);
+                for (int i = 0; i < 7; ++i) {
+                    // walk offset i-3 relative to slot j0
+                    const int jw = j0 + i - 3;
+                    const int rrow = rev ? cnt - 1 - jw : jw + 3;
+                    if (rrow >= 0 && rrow < kRawRows) {
+                        unpack8(*reinterpret_cast<const uint4 *>(raw + rrow * kP + 8 * g), rr[i]);
                     } else {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) v[q] = 0.0f;
+                        for (int q = 0; q < 8; ++q) rr[i][q] = 0.0f;
                     }
-                };
-                if (has_conv) {
-                    float w0[8], w1[8], w2[8], w3[8], bb[8];
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 t4 = convw[lc0 + q];
-                        w0[q] = t4.x; w1[q] = t4.y; w2[q] = t4.z; w3[q] = t4.w;
-                        bb[q] = convb[lc0 + q];
+                        float acc = bb[q];
+                        acc = fmaf(w0[q], rr[i][q], acc);
+                        acc = fmaf(w1[q], rr[i + 1][q], acc);
+                        acc = fmaf(w2[q], rr[i + 2][q], acc);
+                        acc = fmaf(w3[q], rr[i + 3][q], acc);
+                        o[i][q] = (j0 + i < cnt) ? tc::silu_tanh(acc) : 0.0f;
                     }
-                    float r0[8], r1[8], r2[8];
-                    raw(j0 - 3, r0);
-                    raw(j0 - 2, r1);
-                    raw(j0 - 1, r2);
+                }
+            } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        float r3[8];
-                        if (j0 + i < cnt) {
-                            raw(j0 + i, r3);
-                        } else {
+                for (int i = 0; i < 4; ++i) {
+                    const int jw = j0 + i;
+                    const int rrow = rev ? cnt - 1 - jw : jw + 3;
+                    if (jw < cnt) {
+                        unpack8(*reinterpret_cast<const uint4 *>(raw + rrow * kP + 8 * g), o[i]);
+                    } else {
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) r3[q] = 0.0f;
-                        }
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float acc = bb[q];
-                            acc = fmaf(w0[q], r0[q], acc);
-                            acc = fmaf(w1[q], r1[q], acc);
-                            acc = fmaf(w2[q], r2[q], acc);
-                            acc = fmaf(w3[q], r3[q], acc);
-                            o[i][q] = (j0 + i < cnt) ? silu_f(acc) : 0.0f;
-                            r0[q] = r1[q]; r1[q] = r2[q]; r2[q] = r3[q];
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (j0 + i < cnt) {
-                            raw(j0 + i, o[i]);
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) o[i][q] = 0.0f;
-                        }
+                        for (int q = 0; q < 8; ++q) o[i][q] = 0.0f;
                     }
                 }
             }
-            // store 8 rows (slots) x one 16-byte piece
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t rr = j0 + i;
-                if (g < kP / 8) {
-                    *reinterpret_cast<uint4 *>(sm + kOffX + tc::sw128(rr, g)) = pack8(o[i]);
-                    float xw[8];
-                    const float wj = wgt[rr];
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t rr_ = j0 + i;
+                *reinterpret_cast<uint4 *>(sm + kOffX + tc::sw128(rr_, g)) = pack8(o[i]);
+                float xw[8];
+                const float wj = __expf(cum_last - cum[rr_]) * dts[rr_];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) xw[q] = o[i][q] * wj;
-                    *reinterpret_cast<uint4 *>(sm + kOffXw + tc::sw128(rr, g)) = pack8(xw);
-                } else {
-                    const int n0 = lc0 - kP;                       // 0..255 over B then C
-                    const uint32_t base = n0 < kN ? kOffB : kOffC;
-                    const int nn = n0 < kN ? n0 : n0 - kN;         // 0..127
-                    *reinterpret_cast<uint4 *>(sm + base + (nn >> 6) * 16384 +
-                                               tc::sw128(rr, (nn & 63) >> 3)) = pack8(o[i]);
-                }
+                for (int q = 0; q < 8; ++q) xw[q] = o[i][q] * wj;
+                *reinterpret_cast<uint4 *>(sm + kOffXw + tc::sw128(rr_, g)) = pack8(xw);
             }
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        // raw x rows are consumed: prefetch the next chunk's
+        if (tid == 0 && k + 1 < p.nchunks) issue_x(k + 1);
 
-        // ---- C: G = C B^T
+        // ---- C: G = C B^T (after the B/C tiles of this chunk have landed)
+        ok = tc::mbar_wait_bounded(mbar_bc, tphase, kWaitCycles);
+        if (!__syncthreads_and(ok)) break;
         if (tid == 0) {
             tc::fence_after_sync();
             constexpr uint32_t idG = tc::idesc_bf16(128, 128, 0, 0);
@@ -324,16 +441,18 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_tc_kernel(const TcParams p)
                 tc::mma_bf16(tmem + kColG, tc::smem_desc(sbase + kOffC + koff, 16, 1024),
                              tc::smem_desc(sbase + kOffB + koff, 16, 1024), idG, ks > 0);
             }
-            tc::mma_commit(mbar);
+            tc::mma_commit(mbar_mma);
         }
-        ok = tc::mbar_wait_bounded(mbar, phase, kWaitCycles);
+        ok = tc::mbar_wait_bounded(mbar_mma, phase, kWaitCycles);
         phase ^= 1;
         if (!__syncthreads_and(ok)) break;
         tc::fence_after_sync();
 
         // ---- D: M = mask(G * exp(c_t - c_s) * dt_s) -> bf16 tile [t][s]
+        // (c_t is kept in a register: warp 0 may overwrite cum[] for the
+        // next chunk before every thread has finished this one)
+        const float ct = cum[row];
         {
-            const float ct = cum[row];
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int jb = 2 * half + jj;       // 32-column block of s
@@ -383,12 +502,44 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_tc_kernel(const TcParams p)
                 tc::mma_bf16(tmem + kColDS, tc::smem_desc(sbase + kOffB + ks * 2048, 16384, 1024),
                              tc::smem_desc(sbase + kOffXw + ks * 2048, 1024, 1024), idS, ks > 0);
             }
-            tc::mma_commit(mbar);
+            tc::mma_commit(mbar_mma);
+            // arrive at this chunk's forward/reverse meeting point while the
+            // MMAs run: the first of the two CTAs to arrive writes its output,
+            // the second adds its own to it
+            *flag_slot = atomicAdd(p.flags + (((size_t)b * H + h) * p.nchunks + c) * 2, 1);
         }
-        ok = tc::mbar_wait_bounded(mbar, phase, kWaitCycles);
+        ok = tc::mbar_wait_bounded(mbar_mma, phase, kWaitCycles);
         phase ^= 1;
         if (!__syncthreads_and(ok)) break;
         tc::fence_after_sync();
+        // the B/C tiles are consumed: prefetch the next chunk's
+        if (tid == 0 && k + 1 < p.nchunks) issue_bc(k + 1);
+        int *fl = p.flags + (((size_t)b * H + h) * p.nchunks + c) * 2;
+        const bool first = *flag_slot == 0;
+        const bool valid = row < cnt;
+        const int tok = rev ? t0 + cnt - 1 - row : t0 + row;
+        __nv_bfloat16 *yrow = p.y + ((size_t)b * L + tok) * ((size_t)H * kP) + h * kP + 32 * half;
+        uint4 prev_raw[4];
+        if (!first) {
+            // the partner CTA has arrived; wait (bounded) until its output is
+            // visible, then start loading it before the epilogue math
+            if (tid == 0) {
+                bool ready = ld_acquire(fl + 1) != 0;
+                if (!ready) {
+                    const long long w0 = clock64();
+                    while (!(ready = ld_acquire(fl + 1) != 0)) {
+                        if (clock64() - w0 > kWaitCycles) break;
+                    }
+                }
+                if (!ready) record_error(p.status, kStatusTimeout);
+            }
+            __syncthreads();
+            if (valid) {
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc)
+                    prev_raw[pc] = __ldcg(reinterpret_cast<const uint4 *>(yrow) + pc);
+            }
+        }
 
         // ---- F: state update and output
         {
@@ -403,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_tc_kernel(const TcParams p)
             float yd[32], yo[32];
             tc::tmem_ld32(tmem + lane_base + kColYd + 32 * half, yd);
             tc::tmem_ld32(tmem + lane_base + kColYo + 32 * half, yo);
-            const float et = __expf(cum[row]);
+            const float et = __expf(ct);
 #pragma unroll
             for (int pc = 0; pc < 4; ++pc) {
                 float xv[8];
@@ -418,47 +569,26 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_tc_kernel(const TcParams p)
         tc::fence_before_sync();
         store_state_bf16();   // the Y_off MMA that read the old copy has completed
 
-        // forward + reverse sum through the per-chunk handshake
-        int *fl = p.flags + (((size_t)b * H + h) * p.nchunks + c) * 2;
-        if (tid == 0) *flag_slot = atomicAdd(fl, 1);
-        __syncthreads();
-        const bool first = *flag_slot == 0;
-        const bool valid = row < cnt;
-        const int tok = rev ? t0 + cnt - 1 - row : t0 + row;
-        __nv_bfloat16 *yrow = p.y + ((size_t)b * L + tok) * ((size_t)H * kP) + h * kP + 32 * half;
+        // forward + reverse sum: store, or add the partner's output and store
         if (first) {
             if (valid) {
 #pragma unroll
                 for (int pc = 0; pc < 4; ++pc)
                     reinterpret_cast<uint4 *>(yrow)[pc] = pack8(yv + 8 * pc);
             }
-            __threadfence();
             __syncthreads();
-            if (tid == 0) atomicExch(fl + 1, 1);
+            if (tid == 0) st_release(fl + 1, 1);
         } else {
-            if (tid == 0) {
-                bool ready = ld_acquire(fl + 1) != 0;
-                if (!ready) {
-                    const long long w0 = clock64();
-                    while (!(ready = ld_acquire(fl + 1) != 0)) {
-                        if (clock64() - w0 > kWaitCycles) break;
-                    }
-                }
-                if (!ready) record_error(p.status, kStatusTimeout);
-            }
-            __syncthreads();
-            __threadfence();
             if (valid) {
 #pragma unroll
                 for (int pc = 0; pc < 4; ++pc) {
                     float prev[8];
-                    unpack8(__ldcg(reinterpret_cast<const uint4 *>(yrow) + pc), prev);
+                    unpack8(prev_raw[pc], prev);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) prev[q] += yv[8 * pc + q];
                     reinterpret_cast<uint4 *>(yrow)[pc] = pack8(prev);
                 }
             }
-            __syncthreads();
             if (tid == 0) {
                 fl[0] = 0;   // leave the workspace zeroed for the next call
                 fl[1] = 0;
@@ -470,7 +600,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_tc_kernel(const TcParams p)
 #pragma unroll
         for (int q = 0; q < 32; ++q) p.fin[sidx + (size_t)(32 * half + q) * kN + row] = S[q];
     }
-    if (!ok && tid == 0) record_error(p.status, kStatusTimeout);
+    if (!ok) {
+        if (tid == 0) record_error(p.status, kStatusTimeout);
+        // give loads still in flight a bounded chance to land before exit
+        tc::mbar_wait_bounded(mbar_x, 0, 1000000LL);
+        tc::mbar_wait_bounded(mbar_bc, 0, 1000000LL);
+    }
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
@@ -482,11 +617,49 @@ bool tc_path_supported(const bimamba_dims &d)
            d.d_conv == 4 && d.len > 0;
 }
 
-size_t tc_workspace_bytes(const bimamba_dims &d)
+// workspace: [flags: batch*H*nchunks*2 int32, 1 KB aligned][B/C activations:
+// 2 directions x batch x len x 256 bf16]
+static size_t flags_bytes(const bimamba_dims &d)
 {
     const size_t nchunks = ((size_t)d.len + kQ - 1) / kQ;
     const size_t bytes = (size_t)d.batch * d.heads * nchunks * 2 * sizeof(int);
-    return (bytes + 255) & ~(size_t)255;
+    return (bytes + 1023) & ~(size_t)1023;
+}
+
+size_t tc_workspace_bytes(const bimamba_dims &d)
+{
+    return flags_bytes(d) + (size_t)2 * d.batch * d.len * kBC * sizeof(__nv_bfloat16);
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+// 3-D bf16 tensor map: dims (inner, rows, planes), box (box0, box1, 1).
+static bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows,
+                     uint64_t planes, uint32_t box0, uint32_t box1, bool swizzle128)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {inner, rows, planes};
+    const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+    const cuuint32_t box[3] = {box0, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
@@ -509,12 +682,32 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
     p.H = d.heads;
     p.ch = d.heads * d.headdim + 2 * d.ngroups * d.d_state;
     p.nchunks = (d.len + kQ - 1) / kQ;
-    cudaError_t ea = cudaFuncSetAttribute(ssd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)kSmemBytes);
-    if (ea != cudaSuccess) return ea;
-    ssd_tc_kernel<<<dim3(2 * d.heads, d.batch), kThreads, kSmemBytes, stream>>>(p);
+    p.batch = d.batch;
+    __nv_bfloat16 *act = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(pr.workspace) +
+                                                           flags_bytes(d));
+
+    // prepass: B/C conv+SiLU in walk order for both directions
+    bc_prepass_kernel<<<dim3((d.len + 31) / 32, d.batch, 2), 128, 0, stream>>>(
+        p.xbc, p.tail, p.conv_w, p.conv_b, act, d.len, p.ch, d.heads * kP, d.batch);
     cudaError_t e = cudaGetLastError();
-    if (e == cudaSuccess) count_launch();
+    if (e != cudaSuccess) return e;
+    count_launch();
+
+    CUtensorMap tm_x, tm_bc;
+    if (!make_map(&tm_x, p.xbc, (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, kP, kRawRows,
+                  false) ||
+        !make_map(&tm_bc, act, (uint64_t)kBC, (uint64_t)d.len, (uint64_t)2 * d.batch, 64, kQ, true))
+        return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(ssd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const TimingEvents ev = timing_events();
+    if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
+    ssd_tc_kernel<<<dim3(2 * d.heads, d.batch), kThreads, kSmemBytes, stream>>>(tm_x, tm_bc, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch();
+    if (ev.stop) e = cudaEventRecord(ev.stop, stream);
     return e;
 }
 

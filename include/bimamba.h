@@ -80,6 +80,16 @@ int bimamba_version(void);
  * (host-side counter, all devices and streams).  For accounting only. */
 unsigned long long bimamba_launch_count(void);
 
+/*
+ * Timing hook for benchmarks.  When `start` and `stop` are non-NULL
+ * cudaEvent_t handles, every later bimamba_ssd_fwd_rev / bimamba_block_decode
+ * call on this host thread records `start` immediately before its main scan
+ * kernel and `stop` immediately after it, on the call's stream, so that
+ * cudaEventElapsedTime(start, stop) is that kernel's device time.  Pass NULL
+ * for both to switch it off.  Returns BIMAMBA_ERR_INVALID if only one is NULL.
+ */
+int bimamba_set_timing_events(void *start, void *stop);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *bimamba_strerror(int status);
 
