@@ -12,29 +12,35 @@
 // Chunked form used here (chunks of Q = 128 walk steps; c_j = inclusive
 // prefix sum of dt*A inside the chunk; S_in = state entering the chunk):
 //     G      = C B^T                                  (Q x Q,  K = N)
-//     M[t,s] = G[t,s] exp(c_t - c_s) dt_s  for s <= t, else 0
-//     Y      = M X + diag(exp(c)) C S_in^T + D X     (Q x P)
+//     M[t,s] = G[t,s] exp(c_t - c_s) dt_s  (s < t),  G[t,t] dt_t + D  (s = t)
+//     Y      = M X + diag(exp(c)) C S_in^T            (Q x P)
 //     S_out  = exp(c_last) S_in + sum_s exp(c_last - c_s) dt_s x_s B_s^T
 // The reverse stream is the same computation in walk order: chunk slots map
 // to tokens through t = len-1-s; no flipped copy of any tensor is made.
 //
-// Mapping: one CTA (256 threads) owns (batch b, head h, direction) and walks
-// the chunks of its sequence; the fp32 state lives in registers (thread
-// (n, half) holds S[32*half .. 32*half+31][n]); per chunk four MMAs run with
-// M = 128 (all products are 128 x 128 x {128, 64}):
-//     G        = C  . B^T      A = C  [t][n] K-major,  B = B  [s][n] K-major
-//     Y_diag   = M  . X        A = M  [t][s] K-major,  B = X  [s][p] MN-major
-//     Y_off    = C  . S_in^T   A = C  [t][n] K-major,  B = S^T[n][p] MN-major
-//     dS^T     = B^T. (wX)     A = B  [s][n] MN-major, B = wX [s][p] MN-major
-// TMEM: G in columns 0..127 (reused by Y_diag 0..63 and Y_off 64..127 once M
-// is built), dS^T in 128..191.
+// Mapping: one CTA (512 threads) owns (batch b, head pair, direction) and
+// walks the chunks of its sequence.  The two heads share B, C and G, so G is
+// computed once per chunk for both.  Per chunk (all M = 128):
+//     G        = C . B^T           A = C [t][n] K-major (smem), B = B [s][n] K-major
+//     Yd_h     = M_h . X_h         A = M_h in TMEM,            B = X_h [s][p] MN-major
+//     Yo       = C . [S_0;S_1]^T   A = C,                      B = S^T [n][p'] MN-major
+//     S^T     += B^T . [wX_0|wX_1] A = B [s][n] MN-major,      B = wX [s][p'] MN-major
+// The fp32 state S^T (n x p', both heads) lives in tensor memory: before the
+// chunk's MMAs the threads scale it by exp(c_last) in place (and keep a bf16
+// copy in shared memory as the Yo operand); the last MMA accumulates onto it.
+// TMEM columns: G 0..127 (then Yd_0 0..63, Yd_1 64..127), M_0 128..191,
+// M_1 192..255, Yo 256..383, S^T 384..511.
 // Descriptors: K-major operands use stride 1024 B between 8-row groups; an
 // MN-major operand uses leading offset = distance between its 64-element
-// blocks along M/N (16 KB for the 128-wide B tile; the 64-wide tiles have a
-// single block, where the field is unused and set equal to the 1024 B stride)
+// blocks along M/N (16 KB for the 128-wide tiles; for 64-wide tiles, which
+// have a single block, the unused field is set equal to the 1024 B stride)
 // and stride offset = 1024 B between groups of 8 rows along K.
+// Decay factors: for s in a 32-slot block below t's block,
+// exp(c_t - c_s) = exp(c_t - c_R) exp(c_R - c_s) with R the block's last
+// slot; both factors are <= 1, so nothing overflows, and only the diagonal
+// 32 x 32 blocks need one exponential per element.
 //
-// Forward+reverse sum: the two CTAs of a (b, h) pair meet per token chunk
+// Forward+reverse sum: the two CTAs of a (b, head pair) meet per token chunk
 // through a two-counter handshake in the caller's workspace: the first to
 // finish a chunk writes its output (bf16), the second adds its own to it.
 // The second one's wait is bounded; the first never waits.
@@ -49,38 +55,42 @@ namespace bimamba {
 
 namespace {
 
-constexpr int kQ = 128;  // chunk length
-constexpr int kP = 64;   // headdim of this kernel
-constexpr int kN = 128;  // d_state of this kernel
-constexpr int kThreads = 256;
-constexpr int kBC = 2 * kN;            // B and C channels
-constexpr int kRawRows = kQ + 3;       // raw x rows per chunk: 128 slots + 3-token conv halo
-constexpr uint32_t kTmemCols = 256;
+constexpr int kQ = 128;       // chunk length
+constexpr int kP = 64;        // headdim of this kernel
+constexpr int kN = 128;       // d_state of this kernel
+constexpr int kHeads = 2;     // heads per CTA
+constexpr int kPP = kHeads * kP;   // x channels per CTA (128)
+constexpr int kThreads = 512;
+constexpr int kBC = 2 * kN;   // B and C channels
+constexpr int kRawRows = kQ + 3;   // raw x rows per chunk: 128 slots + 3-token conv halo
+constexpr uint32_t kTmemCols = 512;
 
 // shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t kOffC = 0;        // C      [t][n]   2 x 16 KB blocks (TMA, swizzled)
-constexpr uint32_t kOffB = 32768;    // B      [s][n]   2 x 16 KB        (TMA, swizzled)
-constexpr uint32_t kOffM = 65536;    // M      [t][s]   2 x 16 KB
-constexpr uint32_t kOffX = 98304;    // X      [s][p]   16 KB
-constexpr uint32_t kOffXw = 114688;  // wX     [s][p]   16 KB
-constexpr uint32_t kOffS = 131072;   // S^T    [n][p]   16 KB (bf16 copy of the state)
-constexpr uint32_t kOffRaw = 147456; // raw x  [131][64] bf16, row-major (TMA)
-constexpr uint32_t kRawBytes = kRawRows * kP * 2;   // 16768
-constexpr uint32_t kOffCum = kOffRaw + 17408;   // f32[128] prefix sums of dt*A
-constexpr uint32_t kOffDt = kOffCum + 512;      // f32[128] dt
-constexpr uint32_t kOffConvW = kOffDt + 512;    // float4[64] conv taps of x
-constexpr uint32_t kOffConvB = kOffConvW + 16 * kP;   // f32[64]
-constexpr uint32_t kOffMbar = kOffConvB + 4 * kP;     // u64 x3: MMA, raw-x TMA, B/C TMA
-constexpr uint32_t kOffTmem = kOffMbar + 24;    // u32 TMEM base
-constexpr uint32_t kOffFlag = kOffTmem + 4;     // i32 handshake result
+constexpr uint32_t kOffC = 0;         // C      [t][n]   2 x 16 KB (TMA, swizzled)
+constexpr uint32_t kOffB = 32768;     // B      [s][n]   2 x 16 KB (TMA, swizzled)
+constexpr uint32_t kOffX = 65536;     // X      [s][p]   one 16 KB block per head
+constexpr uint32_t kOffXw = 98304;    // wX     [s][p']  2 x 16 KB
+constexpr uint32_t kOffS = 131072;    // S^T    [n][p']  2 x 16 KB (bf16 copy of the state)
+constexpr uint32_t kOffRaw = 163840;  // raw x  [131][128] bf16, row-major (TMA)
+constexpr uint32_t kRawBytes = kRawRows * kPP * 2;   // 33536
+constexpr uint32_t kOffCum = kOffRaw + 33792;    // f32[2][128] prefix sums of dt*A
+constexpr uint32_t kOffDt = kOffCum + 1024;      // f32[2][128] dt
+constexpr uint32_t kOffFB = kOffDt + 1024;       // f32[2][128] exp(c_R - c_s) dt_s, R = block end
+constexpr uint32_t kOffWgt = kOffFB + 1024;      // f32[2][128] exp(c_last - c_s) dt_s
+constexpr uint32_t kOffConvW = kOffWgt + 1024;   // float4[128] conv taps of x
+constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
+constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x3: MMA, raw-x TMA, B/C TMA
+constexpr uint32_t kOffTmem = kOffMbar + 24;     // u32 TMEM base
+constexpr uint32_t kOffFlag = kOffTmem + 4;      // i32 handshake result
 constexpr uint32_t kSmemUsed = kOffFlag + 4;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
-constexpr uint32_t kBCBytes = 4 * kQ * 64 * 2;     // four 128 x 64 bf16 boxes
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;   // + alignment slack
+constexpr uint32_t kBCBytes = 4 * kQ * 64 * 2;      // four 128 x 64 bf16 boxes
 
 constexpr uint32_t kColG = 0;
-constexpr uint32_t kColYd = 0;
-constexpr uint32_t kColYo = 64;
-constexpr uint32_t kColDS = 128;
+constexpr uint32_t kColYd = 0;     // + 64 * head
+constexpr uint32_t kColM = 128;    // + 64 * head (A operands, packed bf16 pairs)
+constexpr uint32_t kColYo = 256;   // + 64 * head
+constexpr uint32_t kColS = 384;    // + 64 * head
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 
@@ -95,7 +105,7 @@ struct TcParams {
     const float *init;
     float *fin;
     __nv_bfloat16 *y;
-    int *flags;   // [batch][H][nchunks][2]: arrivals, partial-ready
+    int *flags;   // [batch][H/2][nchunks][2]: arrivals, partial-ready
     int *status;
     int len, H, ch, nchunks, batch;
 };
@@ -213,14 +223,17 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                                               ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = tc::smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x >> 1;
+    const int hp = blockIdx.x >> 1;          // head pair: heads 2hp, 2hp+1
     const int dir = blockIdx.x & 1;
     const bool rev = dir != 0;
     const int b = blockIdx.y;
     const int H = p.H, L = p.len, ch = p.ch;
+    const int HP = H / kHeads;
 
-    float *cum = reinterpret_cast<float *>(sm + kOffCum);
+    float *cum = reinterpret_cast<float *>(sm + kOffCum);   // [head][slot]
     float *dts = reinterpret_cast<float *>(sm + kOffDt);
+    float *fB = reinterpret_cast<float *>(sm + kOffFB);
+    float *wgt = reinterpret_cast<float *>(sm + kOffWgt);
     float4 *convw = reinterpret_cast<float4 *>(sm + kOffConvW);
     float *convb = reinterpret_cast<float *>(sm + kOffConvB);
     int *flag_slot = reinterpret_cast<int *>(sm + kOffFlag);
@@ -229,8 +242,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     const uint32_t mbar_bc = sbase + kOffMbar + 16;
     const __nv_bfloat16 *raw = reinterpret_cast<const __nv_bfloat16 *>(sm + kOffRaw);
 
-    // geometry of walk chunk k: token chunk c, first token t0, valid slots cnt,
-    // walk step of slot 0
+    // thread roles: row = TMEM lane / tile row; rg = 32-column group of the
+    // head pair's 128 columns (head rg >> 1, half rg & 1)
+    const int row = tid & 127;
+    const int rg = tid >> 7;
+    const int hh = rg >> 1;
+    const int hsub = rg & 1;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const int quad = warp & 3;
+
     auto chunk_of = [&](int k, int &t0, int &cnt, int &s0) {
         const int c = rev ? p.nchunks - 1 - k : k;
         t0 = c * kQ;
@@ -238,12 +258,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         s0 = rev ? L - t0 - cnt : t0;
         return c;
     };
-    // TMA producers (thread 0): raw x rows and the B/C operand tiles of chunk k
     auto issue_x = [&](int k) {
         int t0, cnt, s0;
         chunk_of(k, t0, cnt, s0);
         tc::mbar_expect_tx(mbar_x, kRawBytes);
-        tc::tma_load_3d(sbase + kOffRaw, &tm_x, h * kP, rev ? t0 : t0 - 3, b, mbar_x);
+        tc::tma_load_3d(sbase + kOffRaw, &tm_x, hp * kPP, rev ? t0 : t0 - 3, b, mbar_x);
     };
     auto issue_bc = [&](int k) {
         int t0, cnt, s0;
@@ -255,14 +274,60 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         tc::tma_load_3d(sbase + kOffC, &tm_bc, 128, s0, zc, mbar_bc);
         tc::tma_load_3d(sbase + kOffC + 16384, &tm_bc, 192, s0, zc, mbar_bc);
     };
+    // dt of walk chunk k for head (warp index 0/1), slots 4*lane .. 4*lane+3
+    auto load_dt = [&](int k, int head, float (&d)[4]) {
+        int t0, cnt, s0;
+        chunk_of(k, t0, cnt, s0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = 4 * lane + i;
+            d[i] = 0.0f;
+            if (j < cnt) {
+                const int s = s0 + j;
+                const int tok = rev ? L - 1 - s : s;
+                d[i] = __bfloat162float(p.dt[((size_t)b * L + tok) * H + hp * kHeads + head]);
+            }
+        }
+    };
+    // warps 0 and 1: inclusive prefix sums of dt*A of one head for one chunk
+    auto scan_dt = [&](const float (&d)[4], float Aw, int head) {
+        float a[4];
+        a[0] = d[0] * Aw;
+#pragma unroll
+        for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Aw, a[i - 1]);
+        float run = a[3];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, run, o);
+            if (lane >= o) run += v;
+        }
+        const float excl = run - a[3];
+        *reinterpret_cast<float4 *>(dts + head * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
+        *reinterpret_cast<float4 *>(cum + head * kQ + 4 * lane) =
+            make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
+    };
+    // threads 0..255: per-slot decay factors of the chunk whose cum/dts are set
+    auto slot_factors = [&]() {
+        if (tid < kHeads * kQ) {
+            const int head = tid >> 7, s = tid & 127;
+            const float cs = cum[head * kQ + s];
+            const float d = dts[head * kQ + s];
+            fB[head * kQ + s] = __expf(cum[head * kQ + (s | 31)] - cs) * d;
+            wgt[head * kQ + s] = __expf(cum[head * kQ + kQ - 1] - cs) * d;
+        }
+    };
 
-    // ---- setup: conv taps of this head's x channels, TMEM, barriers, first loads
+    // ---- setup
     const bool has_conv = p.conv_w != nullptr;
-    if (tid < kP && has_conv) {
-        const int c = h * kP + tid;
-        convw[tid] = *reinterpret_cast<const float4 *>(p.conv_w + (size_t)c * 4);
-        convb[tid] = p.conv_b ? p.conv_b[c] : 0.0f;
+    if (tid < kPP && has_conv) {
+        // stored as [q][g] for local channel 8g + q, so that the 16 channel
+        // groups of a warp read 16 consecutive entries (no bank conflicts)
+        const int c = hp * kPP + tid;
+        const int slot = (tid & 7) * (kPP / 8) + (tid >> 3);
+        convw[slot] = *reinterpret_cast<const float4 *>(p.conv_w + (size_t)c * 4);
+        convb[slot] = p.conv_b ? p.conv_b[c] : 0.0f;
     }
+    const float Aw = warp < kHeads ? p.A[hp * kHeads + warp] : 0.0f;   // scan warps
     if (warp == 0) tc::tmem_alloc(sbase + kOffTmem, kTmemCols);
     if (tid == 0) {
         tc::prefetch_tmap(&tm_x);
@@ -273,163 +338,118 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         issue_x(0);
         issue_bc(0);
     }
+    float dt_next[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (warp < kHeads) {
+        float d[4];
+        load_dt(0, warp, d);
+        scan_dt(d, Aw, warp);
+        if (p.nchunks > 1) load_dt(1, warp, dt_next);
+    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kOffTmem);
+    slot_factors();
 
-    const int row = tid & 127;   // TMEM lane = tile row this thread serves
-    const int half = tid >> 7;   // which 32-column half of a 64-wide result
-    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const float Ah = p.A[h], Dh = p.D[h];
-    const size_t sidx = ((size_t)b * H + h) * kP * kN;
-
-    // ---- state: S^T[n = row][p = 32*half + k], fp32 in registers
-    float S[32];
+    // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg
+    const int head_g = hp * kHeads + hh;     // global head of this thread's columns
+    const size_t sidx = ((size_t)b * H + head_g) * kP * kN;
+    {
+        uint32_t r[16];
 #pragma unroll
-    for (int k = 0; k < 32; ++k)
-        S[k] = (!rev && p.init) ? p.init[sidx + (size_t)(32 * half + k) * kN + row] : 0.0f;
-    auto store_state_bf16 = [&]() {
-        uint8_t *Sb = sm + kOffS;
+        for (int half16 = 0; half16 < 2; ++half16) {
 #pragma unroll
-        for (int pc = 0; pc < 4; ++pc)
-            *reinterpret_cast<uint4 *>(Sb + tc::sw128(row, 4 * half + pc)) = pack8(S + 8 * pc);
-    };
-    store_state_bf16();
+            for (int i = 0; i < 16; ++i) {
+                const int pp = 32 * hsub + 16 * half16 + i;
+                const float v = (!rev && p.init) ? p.init[sidx + (size_t)pp * kN + row] : 0.0f;
+                r[i] = __float_as_uint(v);
+            }
+            tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
+        }
+    }
+    const float Dh = p.D[head_g];
 
     uint32_t phase = 0;
     bool ok = true;
-
-    // dt of walk chunk k for slots 4*lane .. 4*lane+3 (warp 0), zero past cnt
-    auto load_dt = [&](int k, float (&d)[4]) {
-        int t0, cnt, s0;
-        chunk_of(k, t0, cnt, s0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = 4 * lane + i;
-            d[i] = 0.0f;
-            if (j < cnt) {
-                const int s = s0 + j;
-                const int tok = rev ? L - 1 - s : s;
-                d[i] = __bfloat162float(p.dt[((size_t)b * L + tok) * H + h]);
-            }
-        }
-    };
-    float dt_next[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (warp == 0) load_dt(0, dt_next);
 
     for (int k = 0; k < p.nchunks; ++k) {
         int t0, cnt, s0;
         const int c = chunk_of(k, t0, cnt, s0);
         const uint32_t tphase = k & 1;
 
-        // ---- A (warp 0): dt, inclusive prefix sums of dt*A over the chunk;
-        // the next chunk's dt is requested now and used one chunk later
-        // @phase A
-        if (warp == 0) {
-            float d[4], a[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d[i] = dt_next[i];
-            if (k + 1 < p.nchunks) load_dt(k + 1, dt_next);
-            a[0] = d[0] * Ah;
-#pragma unroll
-            for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Ah, a[i - 1]);
-            float run = a[3];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, run, o);
-                if (lane >= o) run += v;
-            }
-            const float excl = run - a[3];
-            *reinterpret_cast<float4 *>(dts + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
-            *reinterpret_cast<float4 *>(cum + 4 * lane) =
-                make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
-        }
+        // ---- raw x rows of this chunk (+ decode conv history)
         ok = tc::mbar_wait_bounded(mbar_x, tphase, kWaitCycles);
         if (!__syncthreads_and(ok)) break;
-        // decode: the conv history before token 0 comes from the cached tail
         if (!rev && c == 0 && p.tail) {
-            for (int e = tid; e < 3 * (kP / 8); e += kThreads) {
-                const int r = e / (kP / 8), g = e % (kP / 8);
-                *reinterpret_cast<uint4 *>(sm + kOffRaw + r * (kP * 2) + g * 16) =
-                    *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch + h * kP + 8 * g);
+            for (int e = tid; e < 3 * (kPP / 8); e += kThreads) {
+                const int r = e / (kPP / 8), g = e % (kPP / 8);
+                *reinterpret_cast<uint4 *>(sm + kOffRaw + r * (kPP * 2) + g * 16) =
+                    *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
+                                                     hp * kPP + 8 * g);
             }
             __syncthreads();
         }
-        const float cum_last = cum[kQ - 1];
 
-        // ---- B: conv+SiLU of this head's x (raw rows in shared memory) into
-        // X and wX.  Thread: 8 channels (group g) x 4 slots.  Raw row of token
-        // u: forward u - (t0 - 3), reverse u - t0.
+        // ---- B: conv+SiLU of both heads' x into X and wX.  Thread: 8
+        // channels (group g: head g >> 3, piece g & 7) x 4 slots.  Raw row
+        // of token u: forward u - (t0 - 3), reverse u - t0.
         {
-            const int g = tid & 7;
-            const int j0 = (tid >> 3) * 4;
+            const int g = tid & 15;
+            const int gh = g >> 3, gp = g & 7;
+            const int j0 = (tid >> 4) * 4;
+            uint4 rr[7];
+#pragma unroll
+            for (int i = 0; i < 7; ++i) {
+                const int jw = j0 + i - 3;   // walk offset of the raw row
+                const int rrow = rev ? cnt - 1 - jw : jw + 3;
+                rr[i] = (rrow >= 0 && rrow < kRawRows)
+                            ? *reinterpret_cast<const uint4 *>(raw + rrow * kPP + 8 * g)
+                            : make_uint4(0, 0, 0, 0);
+            }
+            // o[i][q]: output slot j0 + i, channel 8g + q
             float o[4][8];
+            const __nv_bfloat16 *ru = reinterpret_cast<const __nv_bfloat16 *>(rr);
             if (has_conv) {
-                float w0[8], w1[8], w2[8], w3[8], bb[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const float4 t4 = convw[8 * g + q];
-                    w0[q] = t4.x; w1[q] = t4.y; w2[q] = t4.z; w3[q] = t4.w;
-                    bb[q] = convb[8 * g + q];
-                }
-                // the 7 raw rows slots j0..j0+3 read, oldest first in walk order
-                float rr[7][8];
+                    const float4 w4 = convw[q * (kPP / 8) + g];
+                    const float bq = convb[q * (kPP / 8) + g];
+                    float u[7];
 #pragma unroll
-                for (int i = 0; i < 7; ++i) {
-                    // walk offset i-3 relative to slot j0
-                    const int jw = j0 + i - 3;
-                    const int rrow = rev ? cnt - 1 - jw : jw + 3;
-                    if (rrow >= 0 && rrow < kRawRows) {
-                        unpack8(*reinterpret_cast<const uint4 *>(raw + rrow * kP + 8 * g), rr[i]);
-                    } else {
+                    for (int r = 0; r < 7; ++r) u[r] = __bfloat162float(ru[8 * r + q]);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) rr[i][q] = 0.0f;
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float acc = bb[q];
-                        acc = fmaf(w0[q], rr[i][q], acc);
-                        acc = fmaf(w1[q], rr[i + 1][q], acc);
-                        acc = fmaf(w2[q], rr[i + 2][q], acc);
-                        acc = fmaf(w3[q], rr[i + 3][q], acc);
+                    for (int i = 0; i < 4; ++i) {
+                        float acc = bq;
+                        acc = fmaf(w4.x, u[i], acc);
+                        acc = fmaf(w4.y, u[i + 1], acc);
+                        acc = fmaf(w4.z, u[i + 2], acc);
+                        acc = fmaf(w4.w, u[i + 3], acc);
                         o[i][q] = (j0 + i < cnt) ? tc::silu_tanh(acc) : 0.0f;
                     }
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int jw = j0 + i;
-                    const int rrow = rev ? cnt - 1 - jw : jw + 3;
-                    if (jw < cnt) {
-                        unpack8(*reinterpret_cast<const uint4 *>(raw + rrow * kP + 8 * g), o[i]);
-                    } else {
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) o[i][q] = 0.0f;
-                    }
-                }
+                    for (int q = 0; q < 8; ++q)
+                        o[i][q] = (j0 + i < cnt) ? __bfloat162float(ru[8 * (i + 3) + q]) : 0.0f;
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t rr_ = j0 + i;
-                *reinterpret_cast<uint4 *>(sm + kOffX + tc::sw128(rr_, g)) = pack8(o[i]);
-                float xw[8];
-                const float wj = __expf(cum_last - cum[rr_]) * dts[rr_];
+                const int j = j0 + i;
+                *reinterpret_cast<uint4 *>(sm + kOffX + gh * 16384 + tc::sw128(j, gp)) = pack8(o[i]);
+                const float wj = wgt[gh * kQ + j];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) xw[q] = o[i][q] * wj;
-                *reinterpret_cast<uint4 *>(sm + kOffXw + tc::sw128(rr_, g)) = pack8(xw);
+                for (int q = 0; q < 8; ++q) o[i][q] *= wj;
+                *reinterpret_cast<uint4 *>(sm + kOffXw + gh * 16384 + tc::sw128(j, gp)) = pack8(o[i]);
             }
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
-        // raw x rows are consumed: prefetch the next chunk's
-        if (tid == 0 && k + 1 < p.nchunks) issue_x(k + 1);
+        if (tid == 0 && k + 1 < p.nchunks) issue_x(k + 1);   // raw rows consumed
 
-        // ---- C: G = C B^T (after the B/C tiles of this chunk have landed)
+        // ---- C: G = C B^T
         ok = tc::mbar_wait_bounded(mbar_bc, tphase, kWaitCycles);
         if (!__syncthreads_and(ok)) break;
         if (tid == 0) {
@@ -448,81 +468,137 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         if (!__syncthreads_and(ok)) break;
         tc::fence_after_sync();
 
-        // ---- D: M = mask(G * exp(c_t - c_s) * dt_s) -> bf16 tile [t][s]
-        // (c_t is kept in a register: warp 0 may overwrite cum[] for the
-        // next chunk before every thread has finished this one)
-        const float ct = cum[row];
+        // ---- D: M_h (both heads, into TMEM) and the state's chunk-start
+        // scaling.  Thread (row t, rg): head hh, s-blocks 2*hsub, 2*hsub+1.
+        const float ct = cum[hh * kQ + row];            // kept for the epilogue
+        const float a_last = __expf(cum[hh * kQ + kQ - 1]);
         {
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
-                const int jb = 2 * half + jj;       // 32-column block of s
-                float m[32];
-                if (jb <= (warp & 3)) {             // warp-uniform: block has s <= t
+                const int jb = 2 * hsub + jj;           // 32-slot block of s
+                uint32_t packed[16];
+                if (jb > quad) {                        // warp-uniform: all s > t
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) packed[i] = 0u;
+                } else {
                     float gv[32];
                     tc::tmem_ld32(tmem + lane_base + kColG + 32 * jb, gv);
+                    const float *fbh = fB + hh * kQ + 32 * jb;
+                    if (jb < quad) {
+                        // whole block below the diagonal: factorised decay
+                        const float et = __expf(ct - cum[hh * kQ + 32 * jb + 31]);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int s = 32 * jb + i;
-                        const float e = __expf(fminf(ct - cum[s], 0.0f));
-                        m[i] = (s <= row) ? gv[i] * e * dts[s] : 0.0f;
+                        for (int i = 0; i < 16; ++i)
+                            packed[i] = tc::pack_bf16x2(gv[2 * i] * et * fbh[2 * i],
+                                                        gv[2 * i + 1] * et * fbh[2 * i + 1]);
+                    } else {
+                        // diagonal block: one exponential per element, D on the diagonal
+                        const float *ch_ = cum + hh * kQ + 32 * jb;
+                        const float *dh_ = dts + hh * kQ + 32 * jb;
+                        float m[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int s = 32 * jb + i;
+                            const float e = __expf(fminf(ct - ch_[i], 0.0f));
+                            float v = (s <= row) ? gv[i] * e * dh_[i] : 0.0f;
+                            if (s == row) v += Dh;
+                            m[i] = v;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) packed[i] = tc::pack_bf16x2(m[2 * i], m[2 * i + 1]);
                     }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) m[i] = 0.0f;
                 }
+                tc::tmem_st16(tmem + lane_base + kColM + 64 * hh + 16 * jb, packed);
+            }
+            // state: bf16 copy of S_in (the Yo operand), then S <- exp(c_last) S
+            float sv[32];
+            tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc)
-                    *reinterpret_cast<uint4 *>(sm + kOffM + (jb >> 1) * 16384 +
-                                               tc::sw128(row, 4 * (jb & 1) + pc)) = pack8(m + 8 * pc);
+            for (int pc = 0; pc < 4; ++pc)
+                *reinterpret_cast<uint4 *>(sm + kOffS + hh * 16384 + tc::sw128(row, 4 * hsub + pc)) =
+                    pack8(sv + 8 * pc);
+#pragma unroll
+            for (int half16 = 0; half16 < 2; ++half16) {
+                uint32_t r[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sv[16 * half16 + i] * a_last);
+                tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
             }
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
 
-        // ---- E: Y_diag = M X, Y_off = C S_in^T, dS^T = B^T (wX)
+        // ---- E: Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
         if (tid == 0) {
             tc::fence_after_sync();
-            constexpr uint32_t idY = tc::idesc_bf16(128, 64, 0, 1);
-            constexpr uint32_t idS = tc::idesc_bf16(128, 64, 1, 1);
+            constexpr uint32_t idYd = tc::idesc_bf16(128, 64, 0, 1);
+            constexpr uint32_t idYo = tc::idesc_bf16(128, 128, 0, 1);
+            constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
 #pragma unroll
-            for (int ks = 0; ks < kQ / 16; ++ks) {
-                const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                tc::mma_bf16(tmem + kColYd, tc::smem_desc(sbase + kOffM + koff, 16, 1024),
-                             tc::smem_desc(sbase + kOffX + ks * 2048, 1024, 1024), idY, ks > 0);
+            for (int hd = 0; hd < kHeads; ++hd) {
+#pragma unroll
+                for (int ks = 0; ks < kQ / 16; ++ks)
+                    tc::mma_bf16_tmemA(tmem + kColYd + 64 * hd, tmem + kColM + 64 * hd + 8 * ks,
+                                       tc::smem_desc(sbase + kOffX + hd * 16384 + ks * 2048, 1024, 1024),
+                                       idYd, ks > 0);
             }
 #pragma unroll
             for (int ks = 0; ks < kN / 16; ++ks) {
                 const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
                 tc::mma_bf16(tmem + kColYo, tc::smem_desc(sbase + kOffC + koff, 16, 1024),
-                             tc::smem_desc(sbase + kOffS + ks * 2048, 1024, 1024), idY, ks > 0);
+                             tc::smem_desc(sbase + kOffS + ks * 2048, 16384, 1024), idYo, ks > 0);
             }
 #pragma unroll
-            for (int ks = 0; ks < kQ / 16; ++ks) {
-                tc::mma_bf16(tmem + kColDS, tc::smem_desc(sbase + kOffB + ks * 2048, 16384, 1024),
-                             tc::smem_desc(sbase + kOffXw + ks * 2048, 1024, 1024), idS, ks > 0);
-            }
+            for (int ks = 0; ks < kQ / 16; ++ks)
+                tc::mma_bf16(tmem + kColS, tc::smem_desc(sbase + kOffB + ks * 2048, 16384, 1024),
+                             tc::smem_desc(sbase + kOffXw + ks * 2048, 16384, 1024), idS, 1);
             tc::mma_commit(mbar_mma);
-            // arrive at this chunk's forward/reverse meeting point while the
-            // MMAs run: the first of the two CTAs to arrive writes its output,
-            // the second adds its own to it
-            *flag_slot = atomicAdd(p.flags + (((size_t)b * H + h) * p.nchunks + c) * 2, 1);
+            *flag_slot = atomicAdd(p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2, 1);
+        }
+        // while the MMAs run: prefix sums of the next chunk's dt (cum/dts are
+        // no longer read for this chunk; the epilogue uses registers)
+        if (warp < kHeads && k + 1 < p.nchunks) {
+            float d[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[i] = dt_next[i];
+            if (k + 2 < p.nchunks) load_dt(k + 2, warp, dt_next);
+            scan_dt(d, Aw, warp);
         }
         ok = tc::mbar_wait_bounded(mbar_mma, phase, kWaitCycles);
         phase ^= 1;
         if (!__syncthreads_and(ok)) break;
         tc::fence_after_sync();
-        // the B/C tiles are consumed: prefetch the next chunk's
-        if (tid == 0 && k + 1 < p.nchunks) issue_bc(k + 1);
-        int *fl = p.flags + (((size_t)b * H + h) * p.nchunks + c) * 2;
+        if (tid == 0 && k + 1 < p.nchunks) issue_bc(k + 1);   // B/C tiles consumed
+        if (k + 1 < p.nchunks) slot_factors();                 // read next at B(k+1)
+
+        // ---- F: output rows, and the forward + reverse sum
+        int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
         const bool first = *flag_slot == 0;
         const bool valid = row < cnt;
         const int tok = rev ? t0 + cnt - 1 - row : t0 + row;
-        __nv_bfloat16 *yrow = p.y + ((size_t)b * L + tok) * ((size_t)H * kP) + h * kP + 32 * half;
-        uint4 prev_raw[4];
-        if (!first) {
-            // the partner CTA has arrived; wait (bounded) until its output is
-            // visible, then start loading it before the epilogue math
+        __nv_bfloat16 *yrow = p.y + ((size_t)b * L + tok) * ((size_t)H * kP) + head_g * kP + 32 * hsub;
+        float yv[32];
+        {
+            float yd[32], yo[32];
+            tc::tmem_ld32(tmem + lane_base + kColYd + 64 * hh + 32 * hsub, yd);
+            tc::tmem_ld32(tmem + lane_base + kColYo + 64 * hh + 32 * hsub, yo);
+            const float et = __expf(ct);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) yv[i] = fmaf(et, yo[i], yd[i]);
+        }
+        tc::fence_before_sync();
+        if (first) {
+            if (valid) {
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc)
+                    reinterpret_cast<uint4 *>(yrow)[pc] = pack8(yv + 8 * pc);
+            }
+            __syncthreads();
+            if (tid == 0) st_release(fl + 1, 1);
+        } else {
+            // the partner CTA arrived first; wait (bounded) until its output
+            // is visible, then add ours to it
             if (tid == 0) {
                 bool ready = ld_acquire(fl + 1) != 0;
                 if (!ready) {
@@ -535,51 +611,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             }
             __syncthreads();
             if (valid) {
+                uint4 prev_raw[4];
 #pragma unroll
                 for (int pc = 0; pc < 4; ++pc)
                     prev_raw[pc] = __ldcg(reinterpret_cast<const uint4 *>(yrow) + pc);
-            }
-        }
-
-        // ---- F: state update and output
-        {
-            float ds[32];
-            tc::tmem_ld32(tmem + lane_base + kColDS + 32 * half, ds);
-            const float a_last = __expf(cum_last);
-#pragma unroll
-            for (int q = 0; q < 32; ++q) S[q] = fmaf(a_last, S[q], ds[q]);
-        }
-        float yv[32];
-        {
-            float yd[32], yo[32];
-            tc::tmem_ld32(tmem + lane_base + kColYd + 32 * half, yd);
-            tc::tmem_ld32(tmem + lane_base + kColYo + 32 * half, yo);
-            const float et = __expf(ct);
-#pragma unroll
-            for (int pc = 0; pc < 4; ++pc) {
-                float xv[8];
-                unpack8(*reinterpret_cast<const uint4 *>(sm + kOffX + tc::sw128(row, 4 * half + pc)), xv);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int i = 8 * pc + q;
-                    yv[i] = fmaf(et, yo[i], yd[i]) + Dh * xv[q];
-                }
-            }
-        }
-        tc::fence_before_sync();
-        store_state_bf16();   // the Y_off MMA that read the old copy has completed
-
-        // forward + reverse sum: store, or add the partner's output and store
-        if (first) {
-            if (valid) {
-#pragma unroll
-                for (int pc = 0; pc < 4; ++pc)
-                    reinterpret_cast<uint4 *>(yrow)[pc] = pack8(yv + 8 * pc);
-            }
-            __syncthreads();
-            if (tid == 0) st_release(fl + 1, 1);
-        } else {
-            if (valid) {
 #pragma unroll
                 for (int pc = 0; pc < 4; ++pc) {
                     float prev[8];
@@ -597,12 +632,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     }
 
     if (ok && !rev && p.fin) {
+        tc::fence_after_sync();
+        float sv[32];
+        tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) p.fin[sidx + (size_t)(32 * half + q) * kN + row] = S[q];
+        for (int i = 0; i < 32; ++i) p.fin[sidx + (size_t)(32 * hsub + i) * kN + row] = sv[i];
     }
     if (!ok) {
         if (tid == 0) record_error(p.status, kStatusTimeout);
-        // give loads still in flight a bounded chance to land before exit
         tc::mbar_wait_bounded(mbar_x, 0, 1000000LL);
         tc::mbar_wait_bounded(mbar_bc, 0, 1000000LL);
     }
@@ -614,15 +651,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
 bool tc_path_supported(const bimamba_dims &d)
 {
     return d.dtype == BIMAMBA_BF16 && d.headdim == kP && d.d_state == kN && d.ngroups == 1 &&
-           d.d_conv == 4 && d.len > 0;
+           d.d_conv == 4 && d.len > 0 && d.heads % kHeads == 0;
 }
 
-// workspace: [flags: batch*H*nchunks*2 int32, 1 KB aligned][B/C activations:
+// workspace: [flags: batch*(H/2)*nchunks*2 int32, 1 KB aligned][B/C activations:
 // 2 directions x batch x len x 256 bf16]
 static size_t flags_bytes(const bimamba_dims &d)
 {
     const size_t nchunks = ((size_t)d.len + kQ - 1) / kQ;
-    const size_t bytes = (size_t)d.batch * d.heads * nchunks * 2 * sizeof(int);
+    const size_t bytes = (size_t)d.batch * (d.heads / kHeads) * nchunks * 2 * sizeof(int);
     return (bytes + 1023) & ~(size_t)1023;
 }
 
@@ -694,7 +731,7 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
     count_launch();
 
     CUtensorMap tm_x, tm_bc;
-    if (!make_map(&tm_x, p.xbc, (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, kP, kRawRows,
+    if (!make_map(&tm_x, p.xbc, (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, kPP, kRawRows,
                   false) ||
         !make_map(&tm_bc, act, (uint64_t)kBC, (uint64_t)d.len, (uint64_t)2 * d.batch, 64, kQ, true))
         return cudaErrorInvalidValue;
@@ -703,7 +740,7 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
     if (e != cudaSuccess) return e;
     const TimingEvents ev = timing_events();
     if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
-    ssd_tc_kernel<<<dim3(2 * d.heads, d.batch), kThreads, kSmemBytes, stream>>>(tm_x, tm_bc, p);
+    ssd_tc_kernel<<<dim3(d.heads, d.batch), kThreads, kSmemBytes, stream>>>(tm_x, tm_bc, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();
