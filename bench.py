@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--workload", choices=["layer1p3b", "long131k", "decode"], default="layer1p3b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences (decode: streams) per GPU; default: the workload's own")
     return ap.parse_args()
 
 
@@ -166,6 +168,7 @@ def run_ours(args):
 
     from bidirectional_mamba_ssm_b200 import _lib as lib
     from bidirectional_mamba_ssm_b200 import inputs as I
+    from bidirectional_mamba_ssm_b200 import replicas
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -178,6 +181,8 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     decode = args.workload == "decode"
     w, batch, seqlen = workload_spec(args.workload)
+    if args.batch is not None:
+        batch = args.batch
     H, P, N = w.heads, w.headdim, w.d_state
 
     # ---- inputs, generated on the device (seeded per rank)
@@ -250,15 +255,13 @@ def run_ours(args):
     assert lib.bimamba_get_error() == lib.BIMAMBA_OK
     ms_total = start.elapsed_time(end)
     per_call_ms = statistics.mean(a.elapsed_time(b_) for a, b_ in kev)
-    if world > 1:
-        t = torch.tensor([ms_total, per_call_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, per_call_ms = float(t[0]), float(t[1])
-        lt = torch.tensor([launches], device=dev, dtype=torch.float64)
-        dist.all_reduce(lt)
-        launches = int(lt.item())
-    ms_step = ms_total / args.steps
     tokens = batch * seqlen
+    # whole job: all ranks' tokens over the slowest rank's time
+    _, ms_total, _ = replicas.aggregate(tokens * args.steps, ms_total, device=dev)
+    _, per_call_ms, _ = replicas.aggregate(0, per_call_ms, device=dev)
+    launches, _, _ = replicas.aggregate(launches, 1.0, device=dev)
+    launches = int(launches)
+    ms_step = ms_total / args.steps
     value = tokens * world / (ms_step / 1e3)
 
     # ---- roofline of the dominant kernel (the main scan kernel of each step)
@@ -347,11 +350,8 @@ def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, 
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / args.e2e_steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
+    from bidirectional_mamba_ssm_b200 import replicas
+    _, ms, _ = replicas.aggregate(0, ms, device=dev)
     h2d = hx.numel() * hx.element_size() + hdt.numel() * hdt.element_size()
     d2h = hy.numel() * hy.element_size()
     return {"value": batch * seqlen * world / (ms / 1e3), "unit": "tokens/s",

@@ -66,25 +66,28 @@ constexpr int kRawRows = kQ + 3;   // raw x rows per chunk: 128 slots + 3-token 
 constexpr uint32_t kTmemCols = 512;
 
 // shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t kOffC = 0;         // C      [t][n]   2 x 16 KB (TMA, swizzled)
-constexpr uint32_t kOffB = 32768;     // B      [s][n]   2 x 16 KB (TMA, swizzled)
-constexpr uint32_t kOffX = 65536;     // X      [s][p]   one 16 KB block per head
-constexpr uint32_t kOffXw = 98304;    // wX     [s][p']  2 x 16 KB
-constexpr uint32_t kOffS = 131072;    // S^T    [n][p']  2 x 16 KB (bf16 copy of the state)
-constexpr uint32_t kOffRaw = 163840;  // raw x  [131][128] bf16, row-major (TMA)
-constexpr uint32_t kRawBytes = kRawRows * kPP * 2;   // 33536
-constexpr uint32_t kOffCum = kOffRaw + 33792;    // f32[2][128] prefix sums of dt*A
+constexpr uint32_t kOffC = 0;          // C      [t][n]   2 x 16 KB (TMA, swizzled)
+constexpr uint32_t kOffB = 32768;      // B      [s][n]   2 x 16 KB (TMA, swizzled)
+constexpr uint32_t kXbufBytes = 33792; // raw x [131][128] (TMA) -> X [s][p], 16 KB per head
+constexpr uint32_t kOffXbuf0 = 65536;  // x buffer of even walk chunks
+constexpr uint32_t kOffXbuf1 = kOffXbuf0 + kXbufBytes;   // odd walk chunks
+constexpr uint32_t kOffXw = kOffXbuf1 + kXbufBytes;      // wX [s][p'] 2 x 16 KB
+constexpr uint32_t kOffS = kOffXw + 32768;               // S^T bf16 [n][p'] 2 x 16 KB
+constexpr uint32_t kRawBytes = kRawRows * kPP * 2;       // 33536
+constexpr uint32_t kOffCum = kOffS + 32768;      // f32[2][128] prefix sums of dt*A
 constexpr uint32_t kOffDt = kOffCum + 1024;      // f32[2][128] dt
 constexpr uint32_t kOffFB = kOffDt + 1024;       // f32[2][128] exp(c_R - c_s) dt_s, R = block end
 constexpr uint32_t kOffWgt = kOffFB + 1024;      // f32[2][128] exp(c_last - c_s) dt_s
 constexpr uint32_t kOffConvW = kOffWgt + 1024;   // float4[128] conv taps of x
 constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
-constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x3: MMA, raw-x TMA, B/C TMA
-constexpr uint32_t kOffTmem = kOffMbar + 24;     // u32 TMEM base
+constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x4: MMA, B/C TMA, raw x 0/1
+constexpr uint32_t kOffTmem = kOffMbar + 32;     // u32 TMEM base
 constexpr uint32_t kOffFlag = kOffTmem + 4;      // i32 handshake result
 constexpr uint32_t kSmemUsed = kOffFlag + 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;   // + alignment slack
 constexpr uint32_t kBCBytes = 4 * kQ * 64 * 2;      // four 128 x 64 bf16 boxes
+static_assert(kOffXbuf1 % 1024 == 0 && kOffXw % 1024 == 0 && kOffS % 1024 == 0, "tile alignment");
+static_assert(kRawBytes <= kXbufBytes, "raw x tile must fit its buffer");
 
 constexpr uint32_t kColG = 0;
 constexpr uint32_t kColYd = 0;     // + 64 * head
@@ -238,9 +241,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     float *convb = reinterpret_cast<float *>(sm + kOffConvB);
     int *flag_slot = reinterpret_cast<int *>(sm + kOffFlag);
     const uint32_t mbar_mma = sbase + kOffMbar;
-    const uint32_t mbar_x = sbase + kOffMbar + 8;
-    const uint32_t mbar_bc = sbase + kOffMbar + 16;
-    const __nv_bfloat16 *raw = reinterpret_cast<const __nv_bfloat16 *>(sm + kOffRaw);
+    const uint32_t mbar_bc = sbase + kOffMbar + 8;
+    const uint32_t mbar_x0 = sbase + kOffMbar + 16;   // raw x into buffer 0 / 1
+    auto xbuf_off = [](int k) { return (k & 1) ? kOffXbuf1 : kOffXbuf0; };
 
     // thread roles: row = TMEM lane / tile row; rg = 32-column group of the
     // head pair's 128 columns (head rg >> 1, half rg & 1)
@@ -258,11 +261,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         s0 = rev ? L - t0 - cnt : t0;
         return c;
     };
+    // raw x rows of chunk k (+ conv halo) into x buffer k % 2
     auto issue_x = [&](int k) {
         int t0, cnt, s0;
         chunk_of(k, t0, cnt, s0);
-        tc::mbar_expect_tx(mbar_x, kRawBytes);
-        tc::tma_load_3d(sbase + kOffRaw, &tm_x, hp * kPP, rev ? t0 : t0 - 3, b, mbar_x);
+        const uint32_t mb = mbar_x0 + 8 * (k & 1);
+        tc::mbar_expect_tx(mb, kRawBytes);
+        tc::tma_load_3d(sbase + xbuf_off(k), &tm_x, hp * kPP, rev ? t0 : t0 - 3, b, mb);
     };
     auto issue_bc = [&](int k) {
         int t0, cnt, s0;
@@ -316,9 +321,79 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             wgt[head * kQ + s] = __expf(cum[head * kQ + kQ - 1] - cs) * d;
         }
     };
+    const bool has_conv = p.conv_w != nullptr;
+    // conv+SiLU of both heads' x for walk chunk k, in place: the raw rows in
+    // x buffer k % 2 become the swizzled X tile of the chunk.  Thread: 8
+    // channels (group g: head g >> 3, piece g & 7) x 4 slots.  Raw row of
+    // token u: forward u - (t0 - 3), reverse u - t0.  Every thread reads its
+    // raw rows before the barrier and writes after it.
+    auto conv_chunk = [&](int k) {
+        int t0, cnt, s0;
+        chunk_of(k, t0, cnt, s0);
+        uint8_t *buf = sm + xbuf_off(k);
+        const __nv_bfloat16 *rawp = reinterpret_cast<const __nv_bfloat16 *>(buf);
+        const int g = tid & 15;
+        const int gh = g >> 3, gp = g & 7;
+        const int j0 = (tid >> 4) * 4;
+        uint4 rr[7];
+#pragma unroll
+        for (int i = 0; i < 7; ++i) {
+            const int jw = j0 + i - 3;   // walk offset of the raw row
+            const int rrow = rev ? cnt - 1 - jw : jw + 3;
+            rr[i] = (rrow >= 0 && rrow < kRawRows)
+                        ? *reinterpret_cast<const uint4 *>(rawp + rrow * kPP + 8 * g)
+                        : make_uint4(0, 0, 0, 0);
+        }
+        __syncthreads();
+        float o[4][8];
+        const __nv_bfloat16 *ru = reinterpret_cast<const __nv_bfloat16 *>(rr);
+        if (has_conv) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 w4 = convw[q * (kPP / 8) + g];
+                const float bq = convb[q * (kPP / 8) + g];
+                float u[7];
+#pragma unroll
+                for (int r = 0; r < 7; ++r) u[r] = __bfloat162float(ru[8 * r + q]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float acc = bq;
+                    acc = fmaf(w4.x, u[i], acc);
+                    acc = fmaf(w4.y, u[i + 1], acc);
+                    acc = fmaf(w4.z, u[i + 2], acc);
+                    acc = fmaf(w4.w, u[i + 3], acc);
+                    o[i][q] = (j0 + i < cnt) ? tc::silu_tanh(acc) : 0.0f;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    o[i][q] = (j0 + i < cnt) ? __bfloat162float(ru[8 * (i + 3) + q]) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4 *>(buf + gh * 16384 + tc::sw128(j0 + i, gp)) = pack8(o[i]);
+    };
+    // wX = w_s * X for walk chunk k (X tile in x buffer k % 2)
+    auto weight_chunk = [&](int k) {
+        const uint8_t *xt = sm + xbuf_off(k);
+        const int j = tid & 127, q4 = tid >> 7;   // slot, quarter of the 128 columns
+        const int gh = q4 >> 1;
+        const float wj = wgt[gh * kQ + j];
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+            const uint32_t off = gh * 16384 + tc::sw128(j, 4 * (q4 & 1) + pc);
+            float v[8];
+            unpack8(*reinterpret_cast<const uint4 *>(xt + off), v);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] *= wj;
+            *reinterpret_cast<uint4 *>(sm + kOffXw + off) = pack8(v);
+        }
+    };
 
     // ---- setup
-    const bool has_conv = p.conv_w != nullptr;
     if (tid < kPP && has_conv) {
         // stored as [q][g] for local channel 8g + q, so that the 16 channel
         // groups of a warp read 16 consecutive entries (no bank conflicts)
@@ -333,9 +408,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         tc::prefetch_tmap(&tm_x);
         tc::prefetch_tmap(&tm_bc);
         tc::mbar_init(mbar_mma, 1);
-        tc::mbar_init(mbar_x, 1);
         tc::mbar_init(mbar_bc, 1);
+        tc::mbar_init(mbar_x0, 1);
+        tc::mbar_init(mbar_x0 + 8, 1);
         issue_x(0);
+        if (p.nchunks > 1) issue_x(1);
         issue_bc(0);
     }
     float dt_next[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -369,88 +446,42 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     }
     const float Dh = p.D[head_g];
 
+    // base shared-memory descriptors of every MMA operand (offsets are added per MMA)
+    const uint64_t dC = tc::smem_desc(sbase + kOffC, 16, 1024);       // K-major A (G, Yo)
+    const uint64_t dB = tc::smem_desc(sbase + kOffB, 16, 1024);       // K-major B (G)
+    const uint64_t dBmn = tc::smem_desc(sbase + kOffB, 16384, 1024);  // MN-major A (state)
+    const uint64_t dX0 = tc::smem_desc(sbase + kOffXbuf0, 1024, 1024);  // MN-major B (Yd)
+    const uint64_t dX1 = tc::smem_desc(sbase + kOffXbuf1, 1024, 1024);
+    const uint64_t dS = tc::smem_desc(sbase + kOffS, 16384, 1024);    // MN-major B (Yo)
+    const uint64_t dXw = tc::smem_desc(sbase + kOffXw, 16384, 1024);  // MN-major B (state)
+
     uint32_t phase = 0;
-    bool ok = true;
-
-    for (int k = 0; k < p.nchunks; ++k) {
-        int t0, cnt, s0;
-        const int c = chunk_of(k, t0, cnt, s0);
-        const uint32_t tphase = k & 1;
-
-        // ---- raw x rows of this chunk (+ decode conv history)
-        ok = tc::mbar_wait_bounded(mbar_x, tphase, kWaitCycles);
-        if (!__syncthreads_and(ok)) break;
-        if (!rev && c == 0 && p.tail) {
+    bool ok = tc::mbar_wait_bounded(mbar_x0, 0, kWaitCycles);
+    if (__syncthreads_and(ok)) {
+        // decode: the conv history before token 0 comes from the cached tail
+        if (!rev && p.tail) {
             for (int e = tid; e < 3 * (kPP / 8); e += kThreads) {
                 const int r = e / (kPP / 8), g = e % (kPP / 8);
-                *reinterpret_cast<uint4 *>(sm + kOffRaw + r * (kPP * 2) + g * 16) =
+                *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
                     *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
                                                      hp * kPP + 8 * g);
             }
             __syncthreads();
         }
-
-        // ---- B: conv+SiLU of both heads' x into X and wX.  Thread: 8
-        // channels (group g: head g >> 3, piece g & 7) x 4 slots.  Raw row
-        // of token u: forward u - (t0 - 3), reverse u - t0.
-        {
-            const int g = tid & 15;
-            const int gh = g >> 3, gp = g & 7;
-            const int j0 = (tid >> 4) * 4;
-            uint4 rr[7];
-#pragma unroll
-            for (int i = 0; i < 7; ++i) {
-                const int jw = j0 + i - 3;   // walk offset of the raw row
-                const int rrow = rev ? cnt - 1 - jw : jw + 3;
-                rr[i] = (rrow >= 0 && rrow < kRawRows)
-                            ? *reinterpret_cast<const uint4 *>(raw + rrow * kPP + 8 * g)
-                            : make_uint4(0, 0, 0, 0);
-            }
-            // o[i][q]: output slot j0 + i, channel 8g + q
-            float o[4][8];
-            const __nv_bfloat16 *ru = reinterpret_cast<const __nv_bfloat16 *>(rr);
-            if (has_conv) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 w4 = convw[q * (kPP / 8) + g];
-                    const float bq = convb[q * (kPP / 8) + g];
-                    float u[7];
-#pragma unroll
-                    for (int r = 0; r < 7; ++r) u[r] = __bfloat162float(ru[8 * r + q]);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float acc = bq;
-                        acc = fmaf(w4.x, u[i], acc);
-                        acc = fmaf(w4.y, u[i + 1], acc);
-                        acc = fmaf(w4.z, u[i + 2], acc);
-                        acc = fmaf(w4.w, u[i + 3], acc);
-                        o[i][q] = (j0 + i < cnt) ? tc::silu_tanh(acc) : 0.0f;
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        o[i][q] = (j0 + i < cnt) ? __bfloat162float(ru[8 * (i + 3) + q]) : 0.0f;
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int j = j0 + i;
-                *reinterpret_cast<uint4 *>(sm + kOffX + gh * 16384 + tc::sw128(j, gp)) = pack8(o[i]);
-                const float wj = wgt[gh * kQ + j];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) o[i][q] *= wj;
-                *reinterpret_cast<uint4 *>(sm + kOffXw + gh * 16384 + tc::sw128(j, gp)) = pack8(o[i]);
-            }
-        }
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
+        conv_chunk(0);
         __syncthreads();
-        if (tid == 0 && k + 1 < p.nchunks) issue_x(k + 1);   // raw rows consumed
+        weight_chunk(0);
+        tc::fence_proxy_async();
+    }
+
+    for (int k = 0; k < p.nchunks && ok; ++k) {
+        int t0, cnt, s0;
+        const int c = chunk_of(k, t0, cnt, s0);
+        const uint32_t xb_k = xbuf_off(k);
 
         // ---- C: G = C B^T
-        ok = tc::mbar_wait_bounded(mbar_bc, tphase, kWaitCycles);
+        ok = tc::mbar_wait_bounded(mbar_bc, k & 1, kWaitCycles);
+        tc::fence_before_sync();
         if (!__syncthreads_and(ok)) break;
         if (tid == 0) {
             tc::fence_after_sync();
@@ -458,8 +489,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
 #pragma unroll
             for (int ks = 0; ks < kN / 16; ++ks) {
                 const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                tc::mma_bf16(tmem + kColG, tc::smem_desc(sbase + kOffC + koff, 16, 1024),
-                             tc::smem_desc(sbase + kOffB + koff, 16, 1024), idG, ks > 0);
+                tc::mma_bf16(tmem + kColG, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
             }
             tc::mma_commit(mbar_mma);
         }
@@ -535,42 +565,49 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             constexpr uint32_t idYd = tc::idesc_bf16(128, 64, 0, 1);
             constexpr uint32_t idYo = tc::idesc_bf16(128, 128, 0, 1);
             constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
+            const uint64_t dX = (k & 1) ? dX1 : dX0;
 #pragma unroll
-            for (int hd = 0; hd < kHeads; ++hd) {
+            for (int ks = 0; ks < kQ / 16; ++ks) {
 #pragma unroll
-                for (int ks = 0; ks < kQ / 16; ++ks)
+                for (int hd = 0; hd < kHeads; ++hd)
                     tc::mma_bf16_tmemA(tmem + kColYd + 64 * hd, tmem + kColM + 64 * hd + 8 * ks,
-                                       tc::smem_desc(sbase + kOffX + hd * 16384 + ks * 2048, 1024, 1024),
-                                       idYd, ks > 0);
+                                       tc::desc_add(dX, hd * 16384 + ks * 2048), idYd, ks > 0);
             }
 #pragma unroll
             for (int ks = 0; ks < kN / 16; ++ks) {
                 const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                tc::mma_bf16(tmem + kColYo, tc::smem_desc(sbase + kOffC + koff, 16, 1024),
-                             tc::smem_desc(sbase + kOffS + ks * 2048, 16384, 1024), idYo, ks > 0);
+                tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048), idYo,
+                             ks > 0);
+                tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048), tc::desc_add(dXw, ks * 2048),
+                             idS, 1);
             }
-#pragma unroll
-            for (int ks = 0; ks < kQ / 16; ++ks)
-                tc::mma_bf16(tmem + kColS, tc::smem_desc(sbase + kOffB + ks * 2048, 16384, 1024),
-                             tc::smem_desc(sbase + kOffXw + ks * 2048, 16384, 1024), idS, 1);
             tc::mma_commit(mbar_mma);
             *flag_slot = atomicAdd(p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2, 1);
         }
-        // while the MMAs run: prefix sums of the next chunk's dt (cum/dts are
-        // no longer read for this chunk; the epilogue uses registers)
-        if (warp < kHeads && k + 1 < p.nchunks) {
+        // while the MMAs run: the next chunk's dt prefix sums (cum/dts are no
+        // longer read for this chunk) and its conv (into the other x buffer)
+        const bool more = k + 1 < p.nchunks;
+        if (warp < kHeads && more) {
             float d[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) d[i] = dt_next[i];
             if (k + 2 < p.nchunks) load_dt(k + 2, warp, dt_next);
             scan_dt(d, Aw, warp);
         }
+        if (more) {
+            ok = tc::mbar_wait_bounded(mbar_x0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1, kWaitCycles);
+            if (!__syncthreads_and(ok)) break;
+            conv_chunk(k + 1);
+        }
         ok = tc::mbar_wait_bounded(mbar_mma, phase, kWaitCycles);
         phase ^= 1;
         if (!__syncthreads_and(ok)) break;
         tc::fence_after_sync();
-        if (tid == 0 && k + 1 < p.nchunks) issue_bc(k + 1);   // B/C tiles consumed
-        if (k + 1 < p.nchunks) slot_factors();                 // read next at B(k+1)
+        if (tid == 0) {
+            if (more) issue_bc(k + 1);                     // B/C tiles consumed
+            if (k + 2 < p.nchunks) issue_x(k + 2);         // this chunk's X consumed
+        }
+        if (more) slot_factors();                          // next chunk's fB, w
 
         // ---- F: output rows, and the forward + reverse sum
         int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
@@ -578,6 +615,27 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         const bool valid = row < cnt;
         const int tok = rev ? t0 + cnt - 1 - row : t0 + row;
         __nv_bfloat16 *yrow = p.y + ((size_t)b * L + tok) * ((size_t)H * kP) + head_g * kP + 32 * hsub;
+        uint4 prev_raw[4];
+        if (!first) {
+            // the partner CTA arrived first; wait (bounded) until its output
+            // is visible, then start loading it before our epilogue math
+            if (tid == 0) {
+                bool ready = ld_acquire(fl + 1) != 0;
+                if (!ready) {
+                    const long long w0 = clock64();
+                    while (!(ready = ld_acquire(fl + 1) != 0)) {
+                        if (clock64() - w0 > kWaitCycles) break;
+                    }
+                }
+                if (!ready) record_error(p.status, kStatusTimeout);
+            }
+            __syncthreads();
+            if (valid) {
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc)
+                    prev_raw[pc] = __ldcg(reinterpret_cast<const uint4 *>(yrow) + pc);
+            }
+        }
         float yv[32];
         {
             float yd[32], yo[32];
@@ -597,24 +655,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             __syncthreads();
             if (tid == 0) st_release(fl + 1, 1);
         } else {
-            // the partner CTA arrived first; wait (bounded) until its output
-            // is visible, then add ours to it
-            if (tid == 0) {
-                bool ready = ld_acquire(fl + 1) != 0;
-                if (!ready) {
-                    const long long w0 = clock64();
-                    while (!(ready = ld_acquire(fl + 1) != 0)) {
-                        if (clock64() - w0 > kWaitCycles) break;
-                    }
-                }
-                if (!ready) record_error(p.status, kStatusTimeout);
-            }
-            __syncthreads();
             if (valid) {
-                uint4 prev_raw[4];
-#pragma unroll
-                for (int pc = 0; pc < 4; ++pc)
-                    prev_raw[pc] = __ldcg(reinterpret_cast<const uint4 *>(yrow) + pc);
 #pragma unroll
                 for (int pc = 0; pc < 4; ++pc) {
                     float prev[8];
@@ -628,6 +669,12 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 fl[0] = 0;   // leave the workspace zeroed for the next call
                 fl[1] = 0;
             }
+            __syncthreads();
+        }
+        // next chunk's wX (its factors were written before the barrier above)
+        if (more) {
+            weight_chunk(k + 1);
+            tc::fence_proxy_async();
         }
     }
 
@@ -640,7 +687,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     }
     if (!ok) {
         if (tid == 0) record_error(p.status, kStatusTimeout);
-        tc::mbar_wait_bounded(mbar_x, 0, 1000000LL);
         tc::mbar_wait_bounded(mbar_bc, 0, 1000000LL);
     }
     tc::fence_before_sync();

@@ -40,6 +40,15 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
     return d;
 }
 
+// Descriptor `d` with its start address advanced by `bytes` (a multiple of
+// 16; the address field does not overflow for shared-memory offsets).  Used
+// with compile-time offsets so that issuing an MMA costs one 64-bit add
+// instead of rebuilding the descriptor.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes)
+{
+    return d + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulate.
 // a_mn / b_mn: operand is MN-major (1) or K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn)
