@@ -8,7 +8,8 @@ the shared library.
 """
 __all__ = ["bimamba_version", "bimamba_launch_count", "bimamba_set_timing_events", "bimamba_strerror", "bimamba_get_error", "bimamba_conv_silu",
            "bimamba_workspace_bytes", "bimamba_ssd_fwd_rev", "bimamba_block_decode",
-           "make_dims", "new_workspace", "BimambaError"]
+           "make_dims", "new_workspace", "BimambaError",
+           "bimamba_noalloc_scratch_bytes", "bimamba_block_decode_noalloc"]
 
 
 def __getattr__(name):

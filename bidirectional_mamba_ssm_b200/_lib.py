@@ -36,6 +36,8 @@ EXPORTED = (
     "bimamba_workspace_bytes",
     "bimamba_ssd_fwd_rev",
     "bimamba_block_decode",
+    "bimamba_noalloc_scratch_bytes",
+    "bimamba_block_decode_noalloc",
 )
 
 
@@ -76,6 +78,10 @@ def _load() -> ctypes.CDLL:
     lib.bimamba_ssd_fwd_rev.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.bimamba_block_decode.restype = i
     lib.bimamba_block_decode.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.bimamba_noalloc_scratch_bytes.restype = sz
+    lib.bimamba_noalloc_scratch_bytes.argtypes = []
+    lib.bimamba_block_decode_noalloc.restype = i
+    lib.bimamba_block_decode_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     return lib
 
 
@@ -195,4 +201,26 @@ def bimamba_block_decode(xbc_block, dt_block, A, D, conv_w, conv_b, state, tail,
                                    _ptr(y), _ptr(state_out), _ptr(tail_out), _ptr(workspace), wsz,
                                    _stream(stream))
     _check(st, "bimamba_block_decode")
+    return y
+
+
+def bimamba_noalloc_scratch_bytes() -> int:
+    """Size of the fixed scratch array bimamba_block_decode_noalloc uses."""
+    return int(_lib.bimamba_noalloc_scratch_bytes())
+
+
+def bimamba_block_decode_noalloc(xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, y,
+                                 state_out, tail_out, *, heads, headdim, d_state, ngroups=1,
+                                 stream=None):
+    """Cached block decode for callers that cannot allocate device memory:
+    same as bimamba_block_decode, but the scratch is the library's own fixed
+    array (no workspace argument).  Calls sharing that array must not
+    overlap on the GPU."""
+    S, L, _ = xbc_block.shape
+    dims = make_dims(S, L, heads, headdim, d_state, _dtype_code(xbc_block), ngroups)
+    st = _lib.bimamba_block_decode_noalloc(ctypes.byref(dims), _ptr(xbc_block), _ptr(dt_block),
+                                           _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b),
+                                           _ptr(state), _ptr(tail), _ptr(y), _ptr(state_out),
+                                           _ptr(tail_out), _stream(stream))
+    _check(st, "bimamba_block_decode_noalloc")
     return y

@@ -178,6 +178,38 @@ int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block,
                          float *state_out, void *tail_out, void *workspace,
                          size_t workspace_bytes, bimamba_stream_t stream);
 
+/*
+ * Cached block decode without a caller workspace.  The paper has no
+ * counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory: a serving process whose memory pool already holds
+ * the whole device (an allocation by the library would fail or fight that
+ * pool), or a decode loop whose rules forbid allocating once it serves.
+ * Arguments, layouts and result are those of bimamba_block_decode, minus the
+ * workspace.  The scratch comes from one fixed array of
+ * bimamba_noalloc_scratch_bytes() bytes (16 MiB) inside this library, which
+ * every GPU that loads the library holds until the process exits.
+ *  - Returns BIMAMBA_ERR_WORKSPACE when the call needs more scratch than the
+ *    array holds (bimamba_workspace_bytes(d) > bimamba_noalloc_scratch_bytes();
+ *    for bf16, headdim 64, d_state 128 that is about 16 000 tokens, i.e.
+ *    streams x block length, per call).  Nothing is launched then.
+ *  - The first call on a device looks up the array's device address, so make
+ *    that first call before any stream capture.
+ *  - Each call clears the part of the array it uses (asynchronous memset on
+ *    `stream`), then runs the same kernels as bimamba_block_decode.
+ *  - All calls share the one array: calls that overlap on the GPU (on
+ *    different streams, or from several host threads without ordering) race
+ *    and corrupt each other's results.  Serialise them.
+ *  - It allocates and frees nothing.
+ */
+size_t bimamba_noalloc_scratch_bytes(void);
+
+int bimamba_block_decode_noalloc(const bimamba_dims *d, const void *xbc_block,
+                                 const void *dt_block, const float *A, const float *D,
+                                 const float *conv_w, const float *conv_b,
+                                 const float *state, const void *tail, void *y,
+                                 float *state_out, void *tail_out,
+                                 bimamba_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
