@@ -60,7 +60,10 @@ constexpr int kP = 64;        // headdim of this kernel
 constexpr int kN = 128;       // d_state of this kernel
 constexpr int kHeads = 2;     // heads per CTA
 constexpr int kPP = kHeads * kP;   // x channels per CTA (128)
-constexpr int kThreads = 512;
+constexpr int kAluThreads = 512;          // compute group (16 warps)
+constexpr int kProducerWarp = 16;         // issues every MMA and TMA load
+constexpr int kProducerTid = 32 * kProducerWarp;
+constexpr int kThreads = kAluThreads + 32;
 constexpr int kBC = 2 * kN;   // B and C channels
 constexpr int kRawRows = kQ + 3;   // raw x rows per chunk: 128 slots + 3-token conv halo
 constexpr uint32_t kTmemCols = 512;
@@ -80,8 +83,8 @@ constexpr uint32_t kOffFB = kOffDt + 1024;       // f32[2][128] exp(c_R - c_s) d
 constexpr uint32_t kOffWgt = kOffFB + 1024;      // f32[2][128] exp(c_last - c_s) dt_s
 constexpr uint32_t kOffConvW = kOffWgt + 1024;   // float4[128] conv taps of x
 constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
-constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x4: MMA, B/C TMA, raw x 0/1
-constexpr uint32_t kOffTmem = kOffMbar + 32;     // u32 TMEM base
+constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x6 (see the kernel)
+constexpr uint32_t kOffTmem = kOffMbar + 48;     // u32 TMEM base
 constexpr uint32_t kOffFlag = kOffTmem + 4;      // i32 handshake result
 constexpr uint32_t kSmemUsed = kOffFlag + 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;   // + alignment slack
@@ -89,13 +92,13 @@ constexpr uint32_t kBCBytes = 4 * kQ * 64 * 2;      // four 128 x 64 bf16 boxes
 static_assert(kOffXbuf1 % 1024 == 0 && kOffXw % 1024 == 0 && kOffS % 1024 == 0, "tile alignment");
 static_assert(kRawBytes <= kXbufBytes, "raw x tile must fit its buffer");
 
-constexpr uint32_t kColG = 0;
-constexpr uint32_t kColYd = 0;     // + 64 * head
-constexpr uint32_t kColM = 128;    // + 64 * head (A operands, packed bf16 pairs)
+// TMEM columns: 0..255 hold G/Yd of one chunk and M of the other (the two
+// 128-column regions alternate per chunk); Yo and the state are fixed.
 constexpr uint32_t kColYo = 256;   // + 64 * head
 constexpr uint32_t kColS = 384;    // + 64 * head
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+constexpr int kArriveTid = 480;   // a thread outside warp 0 (which issues the MMAs)
 
 struct TcParams {
     const __nv_bfloat16 *xbc;
@@ -125,6 +128,25 @@ __device__ __forceinline__ int ld_acquire(const int *p)
 __device__ __forceinline__ void st_release(int *p, int v)
 {
     asm volatile("st.release.gpu.global.b32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+// Barrier over the compute group only (named barrier 1, 512 threads); the
+// producer warp never joins it.
+__device__ __forceinline__ void alu_sync()
+{
+    asm volatile("bar.sync 1, 512;" ::: "memory");
+}
+
+__device__ __forceinline__ bool alu_sync_and(bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 512, p;\n\t"
+        "selp.b32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"((uint32_t)pred) : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ void unpack8(uint4 r, float (&v)[8])
@@ -240,19 +262,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     float4 *convw = reinterpret_cast<float4 *>(sm + kOffConvW);
     float *convb = reinterpret_cast<float *>(sm + kOffConvB);
     int *flag_slot = reinterpret_cast<int *>(sm + kOffFlag);
-    const uint32_t mbar_mma = sbase + kOffMbar;
-    const uint32_t mbar_bc = sbase + kOffMbar + 8;
-    const uint32_t mbar_x0 = sbase + kOffMbar + 16;   // raw x into buffer 0 / 1
+    // mbarriers: B/C tiles landed, raw x landed (buffer 0 / 1), G done,
+    // M/state ready for the chunk's MMAs, chunk MMAs done
+    const uint32_t mb_bc = sbase + kOffMbar;
+    const uint32_t mb_x0 = sbase + kOffMbar + 8;
+    const uint32_t mb_g = sbase + kOffMbar + 24;
+    const uint32_t mb_m = sbase + kOffMbar + 32;
+    const uint32_t mb_e = sbase + kOffMbar + 40;
     auto xbuf_off = [](int k) { return (k & 1) ? kOffXbuf1 : kOffXbuf0; };
-
-    // thread roles: row = TMEM lane / tile row; rg = 32-column group of the
-    // head pair's 128 columns (head rg >> 1, half rg & 1)
-    const int row = tid & 127;
-    const int rg = tid >> 7;
-    const int hh = rg >> 1;
-    const int hsub = rg & 1;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const int quad = warp & 3;
+    // TMEM regions that alternate between chunks: G(k) and Yd(k) use
+    // columns gcol(k) .. +127, M(k) uses mcol(k) .. +127 (the other region)
+    auto gcol = [](int k) -> uint32_t { return (k & 1) ? 128u : 0u; };
+    auto mcol = [](int k) -> uint32_t { return (k & 1) ? 0u : 128u; };
 
     auto chunk_of = [&](int k, int &t0, int &cnt, int &s0) {
         const int c = rev ? p.nchunks - 1 - k : k;
@@ -265,7 +286,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     auto issue_x = [&](int k) {
         int t0, cnt, s0;
         chunk_of(k, t0, cnt, s0);
-        const uint32_t mb = mbar_x0 + 8 * (k & 1);
+        const uint32_t mb = mb_x0 + 8 * (k & 1);
         tc::mbar_expect_tx(mb, kRawBytes);
         tc::tma_load_3d(sbase + xbuf_off(k), &tm_x, hp * kPP, rev ? t0 : t0 - 3, b, mb);
     };
@@ -273,127 +294,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         int t0, cnt, s0;
         chunk_of(k, t0, cnt, s0);
         const int zc = dir * p.batch + b;
-        tc::mbar_expect_tx(mbar_bc, kBCBytes);
-        tc::tma_load_3d(sbase + kOffB, &tm_bc, 0, s0, zc, mbar_bc);
-        tc::tma_load_3d(sbase + kOffB + 16384, &tm_bc, 64, s0, zc, mbar_bc);
-        tc::tma_load_3d(sbase + kOffC, &tm_bc, 128, s0, zc, mbar_bc);
-        tc::tma_load_3d(sbase + kOffC + 16384, &tm_bc, 192, s0, zc, mbar_bc);
-    };
-    // dt of walk chunk k for head (warp index 0/1), slots 4*lane .. 4*lane+3
-    auto load_dt = [&](int k, int head, float (&d)[4]) {
-        int t0, cnt, s0;
-        chunk_of(k, t0, cnt, s0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = 4 * lane + i;
-            d[i] = 0.0f;
-            if (j < cnt) {
-                const int s = s0 + j;
-                const int tok = rev ? L - 1 - s : s;
-                d[i] = __bfloat162float(p.dt[((size_t)b * L + tok) * H + hp * kHeads + head]);
-            }
-        }
-    };
-    // warps 0 and 1: inclusive prefix sums of dt*A of one head for one chunk
-    auto scan_dt = [&](const float (&d)[4], float Aw, int head) {
-        float a[4];
-        a[0] = d[0] * Aw;
-#pragma unroll
-        for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Aw, a[i - 1]);
-        float run = a[3];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, run, o);
-            if (lane >= o) run += v;
-        }
-        const float excl = run - a[3];
-        *reinterpret_cast<float4 *>(dts + head * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
-        *reinterpret_cast<float4 *>(cum + head * kQ + 4 * lane) =
-            make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
-    };
-    // threads 0..255: per-slot decay factors of the chunk whose cum/dts are set
-    auto slot_factors = [&]() {
-        if (tid < kHeads * kQ) {
-            const int head = tid >> 7, s = tid & 127;
-            const float cs = cum[head * kQ + s];
-            const float d = dts[head * kQ + s];
-            fB[head * kQ + s] = __expf(cum[head * kQ + (s | 31)] - cs) * d;
-            wgt[head * kQ + s] = __expf(cum[head * kQ + kQ - 1] - cs) * d;
-        }
-    };
-    const bool has_conv = p.conv_w != nullptr;
-    // conv+SiLU of both heads' x for walk chunk k, in place: the raw rows in
-    // x buffer k % 2 become the swizzled X tile of the chunk.  Thread: 8
-    // channels (group g: head g >> 3, piece g & 7) x 4 slots.  Raw row of
-    // token u: forward u - (t0 - 3), reverse u - t0.  Every thread reads its
-    // raw rows before the barrier and writes after it.
-    auto conv_chunk = [&](int k) {
-        int t0, cnt, s0;
-        chunk_of(k, t0, cnt, s0);
-        uint8_t *buf = sm + xbuf_off(k);
-        const __nv_bfloat16 *rawp = reinterpret_cast<const __nv_bfloat16 *>(buf);
-        const int g = tid & 15;
-        const int gh = g >> 3, gp = g & 7;
-        const int j0 = (tid >> 4) * 4;
-        uint4 rr[7];
-#pragma unroll
-        for (int i = 0; i < 7; ++i) {
-            const int jw = j0 + i - 3;   // walk offset of the raw row
-            const int rrow = rev ? cnt - 1 - jw : jw + 3;
-            rr[i] = (rrow >= 0 && rrow < kRawRows)
-                        ? *reinterpret_cast<const uint4 *>(rawp + rrow * kPP + 8 * g)
-                        : make_uint4(0, 0, 0, 0);
-        }
-        __syncthreads();
-        float o[4][8];
-        const __nv_bfloat16 *ru = reinterpret_cast<const __nv_bfloat16 *>(rr);
-        if (has_conv) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 w4 = convw[q * (kPP / 8) + g];
-                const float bq = convb[q * (kPP / 8) + g];
-                float u[7];
-#pragma unroll
-                for (int r = 0; r < 7; ++r) u[r] = __bfloat162float(ru[8 * r + q]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float acc = bq;
-                    acc = fmaf(w4.x, u[i], acc);
-                    acc = fmaf(w4.y, u[i + 1], acc);
-                    acc = fmaf(w4.z, u[i + 2], acc);
-                    acc = fmaf(w4.w, u[i + 3], acc);
-                    o[i][q] = (j0 + i < cnt) ? tc::silu_tanh(acc) : 0.0f;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    o[i][q] = (j0 + i < cnt) ? __bfloat162float(ru[8 * (i + 3) + q]) : 0.0f;
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<uint4 *>(buf + gh * 16384 + tc::sw128(j0 + i, gp)) = pack8(o[i]);
-    };
-    // wX = w_s * X for walk chunk k (X tile in x buffer k % 2)
-    auto weight_chunk = [&](int k) {
-        const uint8_t *xt = sm + xbuf_off(k);
-        const int j = tid & 127, q4 = tid >> 7;   // slot, quarter of the 128 columns
-        const int gh = q4 >> 1;
-        const float wj = wgt[gh * kQ + j];
-#pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
-            const uint32_t off = gh * 16384 + tc::sw128(j, 4 * (q4 & 1) + pc);
-            float v[8];
-            unpack8(*reinterpret_cast<const uint4 *>(xt + off), v);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) v[q] *= wj;
-            *reinterpret_cast<uint4 *>(sm + kOffXw + off) = pack8(v);
-        }
+        tc::mbar_expect_tx(mb_bc, kBCBytes);
+        tc::tma_load_3d(sbase + kOffB, &tm_bc, 0, s0, zc, mb_bc);
+        tc::tma_load_3d(sbase + kOffB + 16384, &tm_bc, 64, s0, zc, mb_bc);
+        tc::tma_load_3d(sbase + kOffC, &tm_bc, 128, s0, zc, mb_bc);
+        tc::tma_load_3d(sbase + kOffC + 16384, &tm_bc, 192, s0, zc, mb_bc);
     };
 
-    // ---- setup
+    // ---- setup (all threads)
+    const bool has_conv = p.conv_w != nullptr;
     if (tid < kPP && has_conv) {
         // stored as [q][g] for local channel 8g + q, so that the 16 channel
         // groups of a warp read 16 consecutive entries (no bank conflicts)
@@ -402,224 +311,374 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         convw[slot] = *reinterpret_cast<const float4 *>(p.conv_w + (size_t)c * 4);
         convb[slot] = p.conv_b ? p.conv_b[c] : 0.0f;
     }
-    const float Aw = warp < kHeads ? p.A[hp * kHeads + warp] : 0.0f;   // scan warps
     if (warp == 0) tc::tmem_alloc(sbase + kOffTmem, kTmemCols);
-    if (tid == 0) {
+    if (tid == kProducerTid) {
         tc::prefetch_tmap(&tm_x);
         tc::prefetch_tmap(&tm_bc);
-        tc::mbar_init(mbar_mma, 1);
-        tc::mbar_init(mbar_bc, 1);
-        tc::mbar_init(mbar_x0, 1);
-        tc::mbar_init(mbar_x0 + 8, 1);
+        tc::mbar_init(mb_bc, 1);
+        tc::mbar_init(mb_x0, 1);
+        tc::mbar_init(mb_x0 + 8, 1);
+        tc::mbar_init(mb_g, 1);
+        tc::mbar_init(mb_m, 1);
+        tc::mbar_init(mb_e, 1);
         issue_x(0);
         if (p.nchunks > 1) issue_x(1);
         issue_bc(0);
-    }
-    float dt_next[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (warp < kHeads) {
-        float d[4];
-        load_dt(0, warp, d);
-        scan_dt(d, Aw, warp);
-        if (p.nchunks > 1) load_dt(1, warp, dt_next);
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kOffTmem);
-    slot_factors();
 
-    // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg
-    const int head_g = hp * kHeads + hh;     // global head of this thread's columns
-    const size_t sidx = ((size_t)b * H + head_g) * kP * kN;
-    {
-        uint32_t r[16];
-#pragma unroll
-        for (int half16 = 0; half16 < 2; ++half16) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int pp = 32 * hsub + 16 * half16 + i;
-                const float v = (!rev && p.init) ? p.init[sidx + (size_t)pp * kN + row] : 0.0f;
-                r[i] = __float_as_uint(v);
-            }
-            tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
-        }
-    }
-    const float Dh = p.D[head_g];
-
-    // base shared-memory descriptors of every MMA operand (offsets are added per MMA)
-    const uint64_t dC = tc::smem_desc(sbase + kOffC, 16, 1024);       // K-major A (G, Yo)
-    const uint64_t dB = tc::smem_desc(sbase + kOffB, 16, 1024);       // K-major B (G)
-    const uint64_t dBmn = tc::smem_desc(sbase + kOffB, 16384, 1024);  // MN-major A (state)
-    const uint64_t dX0 = tc::smem_desc(sbase + kOffXbuf0, 1024, 1024);  // MN-major B (Yd)
-    const uint64_t dX1 = tc::smem_desc(sbase + kOffXbuf1, 1024, 1024);
-    const uint64_t dS = tc::smem_desc(sbase + kOffS, 16384, 1024);    // MN-major B (Yo)
-    const uint64_t dXw = tc::smem_desc(sbase + kOffXw, 16384, 1024);  // MN-major B (state)
-
-    uint32_t phase = 0;
-    bool ok = tc::mbar_wait_bounded(mbar_x0, 0, kWaitCycles);
-    if (__syncthreads_and(ok)) {
-        // decode: the conv history before token 0 comes from the cached tail
-        if (!rev && p.tail) {
-            for (int e = tid; e < 3 * (kPP / 8); e += kThreads) {
-                const int r = e / (kPP / 8), g = e % (kPP / 8);
-                *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
-                    *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
-                                                     hp * kPP + 8 * g);
-            }
-            __syncthreads();
-        }
-        conv_chunk(0);
-        __syncthreads();
-        weight_chunk(0);
-        tc::fence_proxy_async();
-    }
-
-    for (int k = 0; k < p.nchunks && ok; ++k) {
-        int t0, cnt, s0;
-        const int c = chunk_of(k, t0, cnt, s0);
-        const uint32_t xb_k = xbuf_off(k);
-
-        // ---- C: G = C B^T
-        ok = tc::mbar_wait_bounded(mbar_bc, k & 1, kWaitCycles);
-        tc::fence_before_sync();
-        if (!__syncthreads_and(ok)) break;
-        if (tid == 0) {
-            tc::fence_after_sync();
+    if (warp == kProducerWarp) {
+        // ================= producer: every MMA and every TMA load ==========
+        if (lane == 0) {
+            const uint64_t dC = tc::smem_desc(sbase + kOffC, 16, 1024);       // K-major A (G, Yo)
+            const uint64_t dB = tc::smem_desc(sbase + kOffB, 16, 1024);       // K-major B (G)
+            const uint64_t dBmn = tc::smem_desc(sbase + kOffB, 16384, 1024);  // MN-major A (state)
+            const uint64_t dX0 = tc::smem_desc(sbase + kOffXbuf0, 1024, 1024);  // MN-major B (Yd)
+            const uint64_t dX1 = tc::smem_desc(sbase + kOffXbuf1, 1024, 1024);
+            const uint64_t dS = tc::smem_desc(sbase + kOffS, 16384, 1024);    // MN-major B (Yo)
+            const uint64_t dXw = tc::smem_desc(sbase + kOffXw, 16384, 1024);  // MN-major B (state)
             constexpr uint32_t idG = tc::idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-            for (int ks = 0; ks < kN / 16; ++ks) {
-                const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                tc::mma_bf16(tmem + kColG, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
-            }
-            tc::mma_commit(mbar_mma);
-        }
-        ok = tc::mbar_wait_bounded(mbar_mma, phase, kWaitCycles);
-        phase ^= 1;
-        if (!__syncthreads_and(ok)) break;
-        tc::fence_after_sync();
-
-        // ---- D: M_h (both heads, into TMEM) and the state's chunk-start
-        // scaling.  Thread (row t, rg): head hh, s-blocks 2*hsub, 2*hsub+1.
-        const float ct = cum[hh * kQ + row];            // kept for the epilogue
-        const float a_last = __expf(cum[hh * kQ + kQ - 1]);
-        {
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int jb = 2 * hsub + jj;           // 32-slot block of s
-                uint32_t packed[16];
-                if (jb > quad) {                        // warp-uniform: all s > t
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) packed[i] = 0u;
-                } else {
-                    float gv[32];
-                    tc::tmem_ld32(tmem + lane_base + kColG + 32 * jb, gv);
-                    const float *fbh = fB + hh * kQ + 32 * jb;
-                    if (jb < quad) {
-                        // whole block below the diagonal: factorised decay
-                        const float et = __expf(ct - cum[hh * kQ + 32 * jb + 31]);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            packed[i] = tc::pack_bf16x2(gv[2 * i] * et * fbh[2 * i],
-                                                        gv[2 * i + 1] * et * fbh[2 * i + 1]);
-                    } else {
-                        // diagonal block: one exponential per element, D on the diagonal
-                        const float *ch_ = cum + hh * kQ + 32 * jb;
-                        const float *dh_ = dts + hh * kQ + 32 * jb;
-                        float m[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int s = 32 * jb + i;
-                            const float e = __expf(fminf(ct - ch_[i], 0.0f));
-                            float v = (s <= row) ? gv[i] * e * dh_[i] : 0.0f;
-                            if (s == row) v += Dh;
-                            m[i] = v;
-                        }
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) packed[i] = tc::pack_bf16x2(m[2 * i], m[2 * i + 1]);
-                    }
-                }
-                tc::tmem_st16(tmem + lane_base + kColM + 64 * hh + 16 * jb, packed);
-            }
-            // state: bf16 copy of S_in (the Yo operand), then S <- exp(c_last) S
-            float sv[32];
-            tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
-#pragma unroll
-            for (int pc = 0; pc < 4; ++pc)
-                *reinterpret_cast<uint4 *>(sm + kOffS + hh * 16384 + tc::sw128(row, 4 * hsub + pc)) =
-                    pack8(sv + 8 * pc);
-#pragma unroll
-            for (int half16 = 0; half16 < 2; ++half16) {
-                uint32_t r[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sv[16 * half16 + i] * a_last);
-                tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
-            }
-        }
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
-        __syncthreads();
-
-        // ---- E: Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
-        if (tid == 0) {
-            tc::fence_after_sync();
             constexpr uint32_t idYd = tc::idesc_bf16(128, 64, 0, 1);
             constexpr uint32_t idYo = tc::idesc_bf16(128, 128, 0, 1);
             constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
-            const uint64_t dX = (k & 1) ? dX1 : dX0;
+            bool pok = true;
+            for (int k = 0; k < p.nchunks && pok; ++k) {
+                // G(k) overwrites region gcol(k), last used by M(k-1): wait
+                // for the MMAs of chunk k-1, and for this chunk's B/C tiles
+                if (k > 0) pok = tc::mbar_wait_bounded(mb_e, (k - 1) & 1, kWaitCycles);
+                if (pok) pok = tc::mbar_wait_bounded(mb_bc, k & 1, kWaitCycles);
+                if (!pok) break;
+                tc::fence_after_sync();
+                const uint32_t g = tmem + gcol(k);
 #pragma unroll
-            for (int ks = 0; ks < kQ / 16; ++ks) {
+                for (int ks = 0; ks < kN / 16; ++ks) {
+                    const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    tc::mma_bf16(g, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
+                }
+                tc::mma_commit(mb_g);
+                // Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
+                pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
+                if (!pok) break;
+                tc::fence_after_sync();
+                const uint64_t dX = (k & 1) ? dX1 : dX0;
+                const uint32_t mc = tmem + mcol(k);
 #pragma unroll
-                for (int hd = 0; hd < kHeads; ++hd)
-                    tc::mma_bf16_tmemA(tmem + kColYd + 64 * hd, tmem + kColM + 64 * hd + 8 * ks,
-                                       tc::desc_add(dX, hd * 16384 + ks * 2048), idYd, ks > 0);
+                for (int ks = 0; ks < kQ / 16; ++ks) {
+#pragma unroll
+                    for (int hd = 0; hd < kHeads; ++hd)
+                        tc::mma_bf16_tmemA(g + 64 * hd, mc + 64 * hd + 8 * ks,
+                                           tc::desc_add(dX, hd * 16384 + ks * 2048), idYd, ks > 0);
+                }
+#pragma unroll
+                for (int ks = 0; ks < kN / 16; ++ks) {
+                    const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048),
+                                 idYo, ks > 0);
+                    tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048),
+                                 tc::desc_add(dXw, ks * 2048), idS, 1);
+                }
+                tc::mma_commit(mb_e);
+                // once they complete, the B/C tiles and this chunk's x buffer
+                // are free: load the next chunk's tiles and the chunk after
+                // next's raw x rows
+                if (k + 1 < p.nchunks) {
+                    pok = tc::mbar_wait_bounded(mb_e, k & 1, kWaitCycles);
+                    if (!pok) break;
+                    issue_bc(k + 1);
+                    if (k + 2 < p.nchunks) issue_x(k + 2);
+                }
             }
-#pragma unroll
-            for (int ks = 0; ks < kN / 16; ++ks) {
-                const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048), idYo,
-                             ks > 0);
-                tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048), tc::desc_add(dXw, ks * 2048),
-                             idS, 1);
-            }
-            tc::mma_commit(mbar_mma);
-            *flag_slot = atomicAdd(p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2, 1);
+            if (!pok) record_error(p.status, kStatusTimeout);
         }
-        // while the MMAs run: the next chunk's dt prefix sums (cum/dts are no
-        // longer read for this chunk) and its conv (into the other x buffer)
-        const bool more = k + 1 < p.nchunks;
-        if (warp < kHeads && more) {
-            float d[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d[i] = dt_next[i];
-            if (k + 2 < p.nchunks) load_dt(k + 2, warp, dt_next);
-            scan_dt(d, Aw, warp);
-        }
-        if (more) {
-            ok = tc::mbar_wait_bounded(mbar_x0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1, kWaitCycles);
-            if (!__syncthreads_and(ok)) break;
-            conv_chunk(k + 1);
-        }
-        ok = tc::mbar_wait_bounded(mbar_mma, phase, kWaitCycles);
-        phase ^= 1;
-        if (!__syncthreads_and(ok)) break;
-        tc::fence_after_sync();
-        if (tid == 0) {
-            if (more) issue_bc(k + 1);                     // B/C tiles consumed
-            if (k + 2 < p.nchunks) issue_x(k + 2);         // this chunk's X consumed
-        }
-        if (more) slot_factors();                          // next chunk's fB, w
+    } else {
+        // ================= compute group: 512 threads ======================
+        // thread roles: row = TMEM lane / tile row; rg = 32-column group of
+        // the head pair's 128 columns (head rg >> 1, half rg & 1)
+        const int row = tid & 127;
+        const int rg = tid >> 7;
+        const int hh = rg >> 1;
+        const int hsub = rg & 1;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        const int quad = warp & 3;
+        constexpr float kLog2e = 1.4426950408889634f;
 
-        // ---- F: output rows, and the forward + reverse sum
-        int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
-        const bool first = *flag_slot == 0;
-        const bool valid = row < cnt;
-        const int tok = rev ? t0 + cnt - 1 - row : t0 + row;
-        __nv_bfloat16 *yrow = p.y + ((size_t)b * L + tok) * ((size_t)H * kP) + head_g * kP + 32 * hsub;
-        uint4 prev_raw[4];
-        if (!first) {
-            // the partner CTA arrived first; wait (bounded) until its output
-            // is visible, then start loading it before our epilogue math
-            if (tid == 0) {
+        // dt of walk chunk k for head (warp index 0/1), slots 4*lane .. +3
+        auto load_dt = [&](int k, int head, float (&d)[4]) {
+            int t0, cnt, s0;
+            chunk_of(k, t0, cnt, s0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int j = 4 * lane + i;
+                d[i] = 0.0f;
+                if (j < cnt) {
+                    const int s = s0 + j;
+                    const int tok = rev ? L - 1 - s : s;
+                    d[i] = __bfloat162float(p.dt[((size_t)b * L + tok) * H + hp * kHeads + head]);
+                }
+            }
+        };
+        // warps 0 and 1: inclusive prefix sums of dt*A of one head for one
+        // chunk, in log2 units (Aw carries the factor log2(e)) so that every
+        // decay factor is one 2^x on the special-function unit
+        auto scan_dt = [&](const float (&d)[4], float Aw, int head) {
+            float a[4];
+            a[0] = d[0] * Aw;
+#pragma unroll
+            for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Aw, a[i - 1]);
+            float run = a[3];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, run, o);
+                if (lane >= o) run += v;
+            }
+            const float excl = run - a[3];
+            *reinterpret_cast<float4 *>(dts + head * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
+            *reinterpret_cast<float4 *>(cum + head * kQ + 4 * lane) =
+                make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
+        };
+        // threads 0..255: per-slot decay factors of the chunk whose cum/dts are set
+        auto slot_factors = [&]() {
+            if (tid < kHeads * kQ) {
+                const int head = tid >> 7, s = tid & 127;
+                const float cs = cum[head * kQ + s];
+                const float d = dts[head * kQ + s];
+                fB[head * kQ + s] = tc::exp2_approx(cum[head * kQ + (s | 31)] - cs) * d;
+                wgt[head * kQ + s] = tc::exp2_approx(cum[head * kQ + kQ - 1] - cs) * d;
+            }
+        };
+        // conv+SiLU of both heads' x for walk chunk k, in place: the raw
+        // rows in x buffer k % 2 become the swizzled X tile of the chunk.
+        // Thread: 8 channels (group g: head g >> 3, piece g & 7) x 4 slots.
+        // Raw row of token u: forward u - (t0 - 3), reverse u - t0.  Every
+        // thread reads its raw rows before the barrier and writes after it.
+        auto conv_chunk = [&](int k) {
+            int t0, cnt, s0;
+            chunk_of(k, t0, cnt, s0);
+            uint8_t *buf = sm + xbuf_off(k);
+            const __nv_bfloat16 *rawp = reinterpret_cast<const __nv_bfloat16 *>(buf);
+            const int g = tid & 15;
+            const int gh = g >> 3, gp = g & 7;
+            const int j0 = (tid >> 4) * 4;
+            uint4 rr[7];
+#pragma unroll
+            for (int i = 0; i < 7; ++i) {
+                const int jw = j0 + i - 3;   // walk offset of the raw row
+                const int rrow = rev ? cnt - 1 - jw : jw + 3;
+                rr[i] = (rrow >= 0 && rrow < kRawRows)
+                            ? *reinterpret_cast<const uint4 *>(rawp + rrow * kPP + 8 * g)
+                            : make_uint4(0, 0, 0, 0);
+            }
+            alu_sync();
+            float o[4][8];
+            const __nv_bfloat16 *ru = reinterpret_cast<const __nv_bfloat16 *>(rr);
+            if (has_conv) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 w4 = convw[q * (kPP / 8) + g];
+                    const float bq = convb[q * (kPP / 8) + g];
+                    float u[7];
+#pragma unroll
+                    for (int r = 0; r < 7; ++r) u[r] = __bfloat162float(ru[8 * r + q]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float acc = bq;
+                        acc = fmaf(w4.x, u[i], acc);
+                        acc = fmaf(w4.y, u[i + 1], acc);
+                        acc = fmaf(w4.z, u[i + 2], acc);
+                        acc = fmaf(w4.w, u[i + 3], acc);
+                        o[i][q] = (j0 + i < cnt) ? tc::silu_tanh(acc) : 0.0f;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        o[i][q] = (j0 + i < cnt) ? __bfloat162float(ru[8 * (i + 3) + q]) : 0.0f;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4 *>(buf + gh * 16384 + tc::sw128(j0 + i, gp)) = pack8(o[i]);
+        };
+        // wX = w_s * X for walk chunk k (X tile in x buffer k % 2)
+        auto weight_chunk = [&](int k) {
+            const uint8_t *xt = sm + xbuf_off(k);
+            const int j = tid & 127, q4 = tid >> 7;   // slot, quarter of the 128 columns
+            const int gh = q4 >> 1;
+            const float wj = wgt[gh * kQ + j];
+#pragma unroll
+            for (int pc = 0; pc < 4; ++pc) {
+                const uint32_t off = gh * 16384 + tc::sw128(j, 4 * (q4 & 1) + pc);
+                float v[8];
+                unpack8(*reinterpret_cast<const uint4 *>(xt + off), v);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] *= wj;
+                *reinterpret_cast<uint4 *>(sm + kOffXw + off) = pack8(v);
+            }
+        };
+        // one thread polls an mbarrier; the group barrier releases the rest
+        auto wait_all = [&](uint32_t mb, uint32_t parity) -> bool {
+            bool w = true;
+            if (tid == 0) w = tc::mbar_wait_bounded(mb, parity, kWaitCycles);
+            return alu_sync_and(w);
+        };
+
+        const float Aw = warp < kHeads ? p.A[hp * kHeads + warp] * kLog2e : 0.0f;   // scan warps
+        float dt_next[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (warp < kHeads) {
+            float d[4];
+            load_dt(0, warp, d);
+            scan_dt(d, Aw, warp);
+            if (p.nchunks > 1) load_dt(1, warp, dt_next);
+        }
+        alu_sync();
+        slot_factors();
+
+        // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg
+        const int head_g = hp * kHeads + hh;     // global head of this thread's columns
+        const size_t sidx = ((size_t)b * H + head_g) * kP * kN;
+        {
+            uint32_t r[16];
+#pragma unroll
+            for (int half16 = 0; half16 < 2; ++half16) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int pp = 32 * hsub + 16 * half16 + i;
+                    const float v = (!rev && p.init) ? p.init[sidx + (size_t)pp * kN + row] : 0.0f;
+                    r[i] = __float_as_uint(v);
+                }
+                tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
+            }
+        }
+        const float Dh = p.D[head_g];
+
+        int arrival = 0;   // result of this chunk's arrival atomic (thread kArriveTid)
+        bool ok = wait_all(mb_x0, 0);
+        if (ok) {
+            // decode: the conv history before token 0 comes from the cached tail
+            if (!rev && p.tail) {
+                for (int e = tid; e < 3 * (kPP / 8); e += kAluThreads) {
+                    const int r = e / (kPP / 8), g = e % (kPP / 8);
+                    *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
+                        *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
+                                                         hp * kPP + 8 * g);
+                }
+                alu_sync();
+            }
+            conv_chunk(0);
+            alu_sync();
+            weight_chunk(0);
+        }
+
+        for (int k = 0; k < p.nchunks && ok; ++k) {
+            int t0, cnt, s0;
+            const int c = chunk_of(k, t0, cnt, s0);
+            const bool more = k + 1 < p.nchunks;
+
+            // arrive at this chunk's forward/reverse meeting point; the
+            // result is read only after the chunk's MMAs
+            if (tid == kArriveTid)
+                arrival = atomicAdd(p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2, 1);
+
+            // ---- D: M_h (both heads, into TMEM) and the state's chunk-start
+            // scaling, once G(k) is done.  Thread (row t, rg): head hh,
+            // s-blocks 2*hsub, 2*hsub+1.
+            tc::fence_proxy_async();          // wX of this chunk (written last iteration)
+            ok = wait_all(mb_g, k & 1);
+            if (!ok) break;
+            tc::fence_after_sync();
+            const float ct = cum[hh * kQ + row];            // kept for the epilogue
+            const float a_last = tc::exp2_approx(cum[hh * kQ + kQ - 1]);
+            {
+                const uint32_t gc = gcol(k), mc = mcol(k);
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int jb = 2 * hsub + jj;           // 32-slot block of s
+                    uint32_t packed[16];
+                    if (jb > quad) {                        // warp-uniform: all s > t
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) packed[i] = 0u;
+                    } else {
+                        float gv[32];
+                        tc::tmem_ld32(tmem + lane_base + gc + 32 * jb, gv);
+                        const float *fbh = fB + hh * kQ + 32 * jb;
+                        if (jb < quad) {
+                            // whole block below the diagonal: factorised decay
+                            const float et = tc::exp2_approx(ct - cum[hh * kQ + 32 * jb + 31]);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                packed[i] = tc::pack_bf16x2(gv[2 * i] * et * fbh[2 * i],
+                                                            gv[2 * i + 1] * et * fbh[2 * i + 1]);
+                        } else {
+                            // diagonal block: one exponential per element, D on the diagonal
+                            const float *ch_ = cum + hh * kQ + 32 * jb;
+                            const float *dh_ = dts + hh * kQ + 32 * jb;
+                            const int r31 = row & 31;
+                            float m[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const float e = tc::exp2_approx(fminf(ct - ch_[i], 0.0f));
+                                const float add = (i == r31) ? Dh : 0.0f;
+                                const float v = fmaf(gv[i] * e, dh_[i], add);
+                                m[i] = (i <= r31) ? v : 0.0f;
+                            }
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) packed[i] = tc::pack_bf16x2(m[2 * i], m[2 * i + 1]);
+                        }
+                    }
+                    tc::tmem_st16(tmem + lane_base + mc + 64 * hh + 16 * jb, packed);
+                }
+                // state: bf16 copy of S_in (the Yo operand), then S <- exp(c_last) S
+                float sv[32];
+                tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc)
+                    *reinterpret_cast<uint4 *>(sm + kOffS + hh * 16384 + tc::sw128(row, 4 * hsub + pc)) =
+                        pack8(sv + 8 * pc);
+#pragma unroll
+                for (int half16 = 0; half16 < 2; ++half16) {
+                    uint32_t r[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sv[16 * half16 + i] * a_last);
+                    tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
+                }
+            }
+            tc::fence_proxy_async();
+            tc::fence_before_sync();
+            alu_sync();
+            if (tid == 0) tc::mbar_arrive(mb_m);    // the producer issues the MMAs
+
+            // ---- while the MMAs run: next chunk's dt prefix sums and conv
+            if (warp < kHeads && more) {
+                float d[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d[i] = dt_next[i];
+                if (k + 2 < p.nchunks) load_dt(k + 2, warp, dt_next);
+                scan_dt(d, Aw, warp);
+            }
+            if (more) {
+                ok = wait_all(mb_x0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
+                if (!ok) break;
+                conv_chunk(k + 1);
+            }
+            if (tid == kArriveTid) *flag_slot = arrival;
+            ok = wait_all(mb_e, k & 1);
+            if (!ok) break;
+            tc::fence_after_sync();
+            if (more) slot_factors();                          // next chunk's fB, w
+
+            // ---- F: output rows, and the forward + reverse sum
+            int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
+            const bool first = *flag_slot == 0;
+            const bool valid = row < cnt;
+            const int tok = rev ? t0 + cnt - 1 - row : t0 + row;
+            __nv_bfloat16 *yrow = p.y + ((size_t)b * L + tok) * ((size_t)H * kP) + head_g * kP + 32 * hsub;
+            if (!first && tid == 0) {
+                // the partner CTA arrived first; wait (bounded) until its
+                // output is visible
                 bool ready = ld_acquire(fl + 1) != 0;
                 if (!ready) {
                     const long long w0 = clock64();
@@ -629,65 +688,57 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 }
                 if (!ready) record_error(p.status, kStatusTimeout);
             }
-            __syncthreads();
-            if (valid) {
+            alu_sync();   // also publishes the next chunk's factors
+            // the next chunk's wX first, while the partner's rows can be fetched
+            if (more) weight_chunk(k + 1);
+            float yv[32];
+            {
+                float yd[32], yo[32];
+                tc::tmem_ld32(tmem + lane_base + gcol(k) + 64 * hh + 32 * hsub, yd);
+                tc::tmem_ld32(tmem + lane_base + kColYo + 64 * hh + 32 * hsub, yo);
+                const float et = tc::exp2_approx(ct);
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc)
-                    prev_raw[pc] = __ldcg(reinterpret_cast<const uint4 *>(yrow) + pc);
+                for (int i = 0; i < 32; ++i) yv[i] = fmaf(et, yo[i], yd[i]);
             }
-        }
-        float yv[32];
-        {
-            float yd[32], yo[32];
-            tc::tmem_ld32(tmem + lane_base + kColYd + 64 * hh + 32 * hsub, yd);
-            tc::tmem_ld32(tmem + lane_base + kColYo + 64 * hh + 32 * hsub, yo);
-            const float et = __expf(ct);
+            tc::fence_before_sync();
+            if (first) {
+                if (valid) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) yv[i] = fmaf(et, yo[i], yd[i]);
-        }
-        tc::fence_before_sync();
-        if (first) {
-            if (valid) {
+                    for (int pc = 0; pc < 4; ++pc)
+                        reinterpret_cast<uint4 *>(yrow)[pc] = pack8(yv + 8 * pc);
+                }
+                alu_sync();
+                if (tid == 0) st_release(fl + 1, 1);
+            } else {
+                if (valid) {
+                    uint4 prev_raw[4];
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc)
-                    reinterpret_cast<uint4 *>(yrow)[pc] = pack8(yv + 8 * pc);
-            }
-            __syncthreads();
-            if (tid == 0) st_release(fl + 1, 1);
-        } else {
-            if (valid) {
+                    for (int pc = 0; pc < 4; ++pc)
+                        prev_raw[pc] = __ldcg(reinterpret_cast<const uint4 *>(yrow) + pc);
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc) {
-                    float prev[8];
-                    unpack8(prev_raw[pc], prev);
+                    for (int pc = 0; pc < 4; ++pc) {
+                        float prev[8];
+                        unpack8(prev_raw[pc], prev);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) prev[q] += yv[8 * pc + q];
-                    reinterpret_cast<uint4 *>(yrow)[pc] = pack8(prev);
+                        for (int q = 0; q < 8; ++q) prev[q] += yv[8 * pc + q];
+                        reinterpret_cast<uint4 *>(yrow)[pc] = pack8(prev);
+                    }
+                }
+                if (tid == 0) {
+                    fl[0] = 0;   // leave the workspace zeroed for the next call
+                    fl[1] = 0;
                 }
             }
-            if (tid == 0) {
-                fl[0] = 0;   // leave the workspace zeroed for the next call
-                fl[1] = 0;
-            }
-            __syncthreads();
         }
-        // next chunk's wX (its factors were written before the barrier above)
-        if (more) {
-            weight_chunk(k + 1);
-            tc::fence_proxy_async();
-        }
-    }
 
-    if (ok && !rev && p.fin) {
-        tc::fence_after_sync();
-        float sv[32];
-        tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
+        if (ok && !rev && p.fin) {
+            tc::fence_after_sync();
+            float sv[32];
+            tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) p.fin[sidx + (size_t)(32 * hsub + i) * kN + row] = sv[i];
-    }
-    if (!ok) {
-        if (tid == 0) record_error(p.status, kStatusTimeout);
-        tc::mbar_wait_bounded(mbar_bc, 0, 1000000LL);
+            for (int i = 0; i < 32; ++i) p.fin[sidx + (size_t)(32 * hsub + i) * kN + row] = sv[i];
+        }
+        if (!ok && tid == 0) record_error(p.status, kStatusTimeout);
     }
     tc::fence_before_sync();
     __syncthreads();

@@ -203,6 +203,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity
     return true;
 }
 
+// Arrive once on `mbar` (release semantics at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(mbar) : "memory");
+}
+
 // Expect `bytes` more transaction bytes on `mbar` and arrive once.
 __device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes)
 {
@@ -228,12 +234,21 @@ __device__ __forceinline__ void prefetch_tmap(const void *tmap)
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
-// SiLU through the hardware tanh: x * sigmoid(x), sigmoid(x) = (1 + tanh(x/2)) / 2.
+// SiLU through the hardware tanh: x sigmoid(x) = h + h tanh(h) with h = x/2.
 __device__ __forceinline__ float silu_tanh(float x)
 {
+    const float h = 0.5f * x;
     float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-    return x * fmaf(0.5f, t, 0.5f);
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
+}
+
+// 2^x on the special-function unit (inputs are <= 0 here; underflow gives 0).
+__device__ __forceinline__ float exp2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
