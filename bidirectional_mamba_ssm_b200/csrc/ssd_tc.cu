@@ -673,9 +673,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             // ---- F: output rows, and the forward + reverse sum
             int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
             const bool first = *flag_slot == 0;
-            const bool valid = row < cnt;
-            const int tok = rev ? t0 + cnt - 1 - row : t0 + row;
-            __nv_bfloat16 *yrow = p.y + ((size_t)b * L + tok) * ((size_t)H * kP) + head_g * kP + 32 * hsub;
             if (!first && tid == 0) {
                 // the partner CTA arrived first; wait (bounded) until its
                 // output is visible
@@ -691,39 +688,61 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             alu_sync();   // also publishes the next chunk's factors
             // the next chunk's wX first, while the partner's rows can be fetched
             if (more) weight_chunk(k + 1);
-            float yv[32];
+            // Coalesced output: each thread stages its 32 outputs in shared
+            // memory (the bf16 state copy's buffer, free until the next
+            // chunk's phase D), then 16 threads per token row move whole
+            // 256-byte rows.  Staging layout: [t][16 pieces of 16 B], piece
+            // q of row t stored at q ^ (t & 15) (conflict-free both ways).
+            const int cp = tid & 15;          // 16-byte piece of a row (8 channels)
+            const int cr = tid >> 4;          // rows cr, cr+32, cr+64, cr+96
+            auto ypiece = [&](int r) -> uint4 * {
+                const int tk = rev ? t0 + cnt - 1 - r : t0 + r;
+                return reinterpret_cast<uint4 *>(p.y + ((size_t)b * L + tk) * ((size_t)H * kP) +
+                                                 hp * kPP) + cp;
+            };
+            uint4 prev[4];
+            if (!first) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int r = cr + 32 * j;
+                    prev[j] = r < cnt ? __ldcg(ypiece(r)) : make_uint4(0, 0, 0, 0);
+                }
+            }
             {
                 float yd[32], yo[32];
                 tc::tmem_ld32(tmem + lane_base + gcol(k) + 64 * hh + 32 * hsub, yd);
                 tc::tmem_ld32(tmem + lane_base + kColYo + 64 * hh + 32 * hsub, yo);
                 const float et = tc::exp2_approx(ct);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) yv[i] = fmaf(et, yo[i], yd[i]);
+                for (int i = 0; i < 32; ++i) yd[i] = fmaf(et, yo[i], yd[i]);
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc)
+                    *reinterpret_cast<uint4 *>(sm + kOffS + row * 256 +
+                                               (((4 * rg + pc) ^ (row & 15)) << 4)) = pack8(yd + 8 * pc);
             }
             tc::fence_before_sync();
-            if (first) {
-                if (valid) {
+            alu_sync();
 #pragma unroll
-                    for (int pc = 0; pc < 4; ++pc)
-                        reinterpret_cast<uint4 *>(yrow)[pc] = pack8(yv + 8 * pc);
+            for (int j = 0; j < 4; ++j) {
+                const int r = cr + 32 * j;
+                if (r < cnt) {
+                    uint4 v = *reinterpret_cast<const uint4 *>(sm + kOffS + r * 256 + ((cp ^ (r & 15)) << 4));
+                    if (!first) {
+                        float a[8], c8[8];
+                        unpack8(v, a);
+                        unpack8(prev[j], c8);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) a[q] += c8[q];
+                        v = pack8(a);
+                    }
+                    *ypiece(r) = v;
                 }
+            }
+            if (first) {
                 alu_sync();
                 if (tid == 0) st_release(fl + 1, 1);
             } else {
-                if (valid) {
-                    uint4 prev_raw[4];
-#pragma unroll
-                    for (int pc = 0; pc < 4; ++pc)
-                        prev_raw[pc] = __ldcg(reinterpret_cast<const uint4 *>(yrow) + pc);
-#pragma unroll
-                    for (int pc = 0; pc < 4; ++pc) {
-                        float prev[8];
-                        unpack8(prev_raw[pc], prev);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) prev[q] += yv[8 * pc + q];
-                        reinterpret_cast<uint4 *>(yrow)[pc] = pack8(prev);
-                    }
-                }
+                alu_sync();   // the staging buffer is rewritten by the next chunk's phase D
                 if (tid == 0) {
                     fl[0] = 0;   // leave the workspace zeroed for the next call
                     fl[1] = 0;
