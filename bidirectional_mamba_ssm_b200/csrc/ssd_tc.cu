@@ -86,7 +86,8 @@ constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
 constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x6 (see the kernel)
 constexpr uint32_t kOffTmem = kOffMbar + 48;     // u32 TMEM base
 constexpr uint32_t kOffFlag = kOffTmem + 4;      // i32 handshake result
-constexpr uint32_t kSmemUsed = kOffFlag + 4;
+constexpr uint32_t kOffDtBuf = kOffFlag + 12;    // [2][128] bf16x2: dt of both heads, by cp.async
+constexpr uint32_t kSmemUsed = kOffDtBuf + 2 * kQ * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;   // + alignment slack
 constexpr uint32_t kBCBytes = 4 * kQ * 64 * 2;      // four 128 x 64 bf16 boxes
 static_assert(kOffXbuf1 % 1024 == 0 && kOffXw % 1024 == 0 && kOffS % 1024 == 0, "tile alignment");
@@ -404,40 +405,61 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         const int quad = warp & 3;
         constexpr float kLog2e = 1.4426950408889634f;
+        const float A0 = p.A[hp * kHeads] * kLog2e, A1 = p.A[hp * kHeads + 1] * kLog2e;
 
-        // dt of walk chunk k for head (warp index 0/1), slots 4*lane .. +3
-        auto load_dt = [&](int k, int head, float (&d)[4]) {
+        // warp 0: asynchronous copy of walk chunk k's dt (both heads of the
+        // pair are adjacent: one 4-byte copy per token) into dt buffer k % 2;
+        // slots past the chunk end are zero.  Nothing is held in registers.
+        auto load_dt_async = [&](int k) {
             int t0, cnt, s0;
             chunk_of(k, t0, cnt, s0);
+            uint32_t *dst = reinterpret_cast<uint32_t *>(sm + kOffDtBuf) + (k & 1) * kQ;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int j = 4 * lane + i;
-                d[i] = 0.0f;
                 if (j < cnt) {
                     const int s = s0 + j;
                     const int tok = rev ? L - 1 - s : s;
-                    d[i] = __bfloat162float(p.dt[((size_t)b * L + tok) * H + hp * kHeads + head]);
+                    const __nv_bfloat16 *src = p.dt + ((size_t)b * L + tok) * H + hp * kHeads;
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
+                                 :: "r"(tc::smem_u32(dst + j)), "l"(src) : "memory");
+                } else {
+                    dst[j] = 0u;
                 }
             }
+            asm volatile("cp.async.commit_group;" ::: "memory");
         };
-        // warps 0 and 1: inclusive prefix sums of dt*A of one head for one
-        // chunk, in log2 units (Aw carries the factor log2(e)) so that every
-        // decay factor is one 2^x on the special-function unit
-        auto scan_dt = [&](const float (&d)[4], float Aw, int head) {
-            float a[4];
-            a[0] = d[0] * Aw;
+        // warp 0: inclusive prefix sums of dt*A of both heads for walk chunk
+        // k (its dt copies must have landed), in log2 units (A carries the
+        // factor log2(e)) so that every decay factor is one 2^x on the
+        // special-function unit
+        auto scan_dt = [&](int k) {
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            const __nv_bfloat162 *src =
+                reinterpret_cast<const __nv_bfloat162 *>(sm + kOffDtBuf) + (k & 1) * kQ + 4 * lane;
 #pragma unroll
-            for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Aw, a[i - 1]);
-            float run = a[3];
+            for (int head = 0; head < kHeads; ++head) {
+                float d[4], a[4];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, run, o);
-                if (lane >= o) run += v;
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(src[i]);
+                    d[i] = head ? f.y : f.x;
+                }
+                const float Aw = head ? A1 : A0;
+                a[0] = d[0] * Aw;
+#pragma unroll
+                for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Aw, a[i - 1]);
+                float run = a[3];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, run, o);
+                    if (lane >= o) run += v;
+                }
+                const float excl = run - a[3];
+                *reinterpret_cast<float4 *>(dts + head * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
+                *reinterpret_cast<float4 *>(cum + head * kQ + 4 * lane) =
+                    make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
             }
-            const float excl = run - a[3];
-            *reinterpret_cast<float4 *>(dts + head * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
-            *reinterpret_cast<float4 *>(cum + head * kQ + 4 * lane) =
-                make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
         };
         // threads 0..255: per-slot decay factors of the chunk whose cum/dts are set
         auto slot_factors = [&]() {
@@ -526,13 +548,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             return alu_sync_and(w);
         };
 
-        const float Aw = warp < kHeads ? p.A[hp * kHeads + warp] * kLog2e : 0.0f;   // scan warps
-        float dt_next[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if (warp < kHeads) {
-            float d[4];
-            load_dt(0, warp, d);
-            scan_dt(d, Aw, warp);
-            if (p.nchunks > 1) load_dt(1, warp, dt_next);
+        if (warp == 0) {
+            load_dt_async(0);
+            scan_dt(0);
+            if (p.nchunks > 1) load_dt_async(1);
         }
         alu_sync();
         slot_factors();
@@ -652,12 +671,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             if (tid == 0) tc::mbar_arrive(mb_m);    // the producer issues the MMAs
 
             // ---- while the MMAs run: next chunk's dt prefix sums and conv
-            if (warp < kHeads && more) {
-                float d[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) d[i] = dt_next[i];
-                if (k + 2 < p.nchunks) load_dt(k + 2, warp, dt_next);
-                scan_dt(d, Aw, warp);
+            if (warp == 0 && more) {
+                scan_dt(k + 1);                       // its copies were issued a chunk ago
+                if (k + 2 < p.nchunks) load_dt_async(k + 2);
             }
             if (more) {
                 ok = wait_all(mb_x0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);

@@ -179,14 +179,17 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// One bounded try of a phase wait.  The suspend-time hint (ns) lets the
+// hardware park the thread until the phase completes instead of having it
+// spin and take issue slots from the other warps of its scheduler.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
+        : "=r"(ok) : "r"(mbar), "r"(parity), "r"(1000000u) : "memory");
     return ok != 0;
 }
 
