@@ -284,3 +284,63 @@ def test_block_decode_32_streams_65k_prefix_sampled(lib):
         assert rel_err(to_np(y[s:s + 1])[..., ycols], ry) <= TOL["bf16"]
         assert rel_err(to_np(so[s:s + 1, heads]), rso) <= TOL["bf16"]
     np.testing.assert_array_equal(to_np(to), to_np(blk_in["xbc"][:, -4:]))
+
+
+# ------------------------------------------------- tensor-core path edges
+TC_EDGES = [1, 3, 64, 128, 129, 255, 256, 257]
+
+
+@pytest.mark.parametrize("L", TC_EDGES)
+@pytest.mark.parametrize("variant", ["plain", "init+bias"])
+def test_tensor_core_path_chunk_boundaries(lib, L, variant):
+    """bf16, headdim 64, d_state 128 (the chunked tensor-core kernel) at
+    lengths around the 128-token chunk size, long-memory decays so that
+    state carried across chunk boundaries dominates."""
+    bsz, H, P, N = 2, 4, 64, 128
+    w = inp_mod.Workload("edge", bsz, L, H, P, N, dtype="bf16", bc_scale=1.0 / math.sqrt(N))
+    cpu = inp_mod.make_inputs(w, seed=1000 + L, a_range=(1e-3, 1e-2), conv_bias="bias" in variant)
+    init = inp_mod.make_state(bsz, H, P, N, seed=L, scale=0.3) if "init" in variant else None
+    y, fin = _run_scan(lib, w, _dev(cpu), None if init is None else init.cuda(), want_final=True)
+    n = _np_inputs(cpu)
+    ry, rfin = oracle.bimamba(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], n["conv_b"],
+                              heads=H, headdim=P, d_state=N, init=to_np(init), want_final=True)
+    for b in range(bsz):
+        assert rel_err(to_np(y)[b], ry[b]) <= TOL["bf16"], (L, b)
+        assert rel_err(to_np(fin)[b], rfin[b]) <= TOL["bf16"], (L, b)
+
+
+def test_odd_head_count_uses_a_valid_path(lib):
+    """Three heads cannot be paired: the library must still compute it."""
+    w = inp_mod.Workload("odd", 1, 150, 3, 64, 128, dtype="bf16", bc_scale=1.0 / math.sqrt(128))
+    cpu = inp_mod.make_inputs(w, seed=3)
+    y, _ = _run_scan(lib, w, _dev(cpu))
+    n = _np_inputs(cpu)
+    ry = oracle.bimamba(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], None, heads=3,
+                        headdim=64, d_state=128)
+    assert rel_err(to_np(y), ry) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("blk,prefix", [(1, 5), (128, 300), (200, 64)])
+def test_block_decode_multi_chunk_blocks(lib, blk, prefix):
+    """Decode blocks of 1, 128 and 200 tokens (one, one full and two chunks)."""
+    _decode_case(lib, "bf16", 2, blk, prefix, 4, 64, 128, (1e-3, 1e-2))
+
+
+def test_repeated_calls_reuse_the_workspace(lib):
+    """The handshake counters must come back to zero: three calls on one
+    workspace give the same result."""
+    w = inp_mod.Workload("rep", 2, 300, 4, 64, 128, dtype="bf16", bc_scale=1.0 / math.sqrt(128))
+    g = _dev(inp_mod.make_inputs(w, seed=5))
+    dims = lib.make_dims(2, 300, 4, 64, 128, torch.bfloat16)
+    ws = lib.new_workspace(dims)
+    outs = []
+    for _ in range(3):
+        y = torch.empty((2, 300, 256), dtype=torch.bfloat16, device="cuda")
+        lib.bimamba_ssd_fwd_rev(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], None, None, None, y,
+                                ws, heads=4, headdim=64, d_state=128)
+        outs.append(y)
+    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+    nflags = 2 * 2 * 3    # batch x head pairs x chunks, two counters each
+    assert torch.count_nonzero(ws[: 4 * 2 * nflags]).item() == 0
+    for o in outs[1:]:
+        assert rel_err(to_np(o), to_np(outs[0])) <= 1e-2
