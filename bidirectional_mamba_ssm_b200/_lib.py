@@ -34,6 +34,7 @@ EXPORTED = (
     "bimamba_get_error",
     "bimamba_conv_silu",
     "bimamba_workspace_bytes",
+    "bimamba_launch_plan",
     "bimamba_ssd_fwd_rev",
     "bimamba_block_decode",
     "bimamba_noalloc_scratch_bytes",
@@ -74,6 +75,8 @@ def _load() -> ctypes.CDLL:
     lib.bimamba_conv_silu.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
     lib.bimamba_workspace_bytes.restype = sz
     lib.bimamba_workspace_bytes.argtypes = [dp]
+    lib.bimamba_launch_plan.restype = i
+    lib.bimamba_launch_plan.argtypes = [dp, ctypes.POINTER(ctypes.c_int)]
     lib.bimamba_ssd_fwd_rev.restype = i
     lib.bimamba_ssd_fwd_rev.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.bimamba_block_decode.restype = i
@@ -158,6 +161,15 @@ def make_dims(batch, seqlen, heads, headdim, d_state, dtype, ngroups=1, d_conv=4
 
 def bimamba_workspace_bytes(dims: Dims) -> int:
     return int(_lib.bimamba_workspace_bytes(ctypes.byref(dims)))
+
+
+def bimamba_launch_plan(dims: Dims) -> dict:
+    """How a call with these dims is launched (host only): tensor-core path
+    or not, segments per direction, chunks per segment, state-only items."""
+    out = (ctypes.c_int * 4)()
+    _check(_lib.bimamba_launch_plan(ctypes.byref(dims), out), "bimamba_launch_plan")
+    return {"tensor_core": bool(out[0]), "segments": out[1], "seg_chunks": out[2],
+            "items": out[3]}
 
 
 def new_workspace(dims: Dims, device=None) -> torch.Tensor:

@@ -145,6 +145,22 @@ size_t bimamba_workspace_bytes(const bimamba_dims *d)
     return workspace_bytes_for(*d);
 }
 
+int bimamba_launch_plan(const bimamba_dims *d, int *out)
+{
+    if (!out) return BIMAMBA_ERR_INVALID;
+    const int st = check_dims(d);
+    if (st != BIMAMBA_OK) return st;
+    out[0] = tc_path_supported(*d) ? 1 : 0;
+    if (out[0]) {
+        tc_launch_plan(*d, out + 1);
+    } else {
+        out[1] = 1;
+        out[2] = (d->len + 127) / 128;
+        out[3] = 0;
+    }
+    return BIMAMBA_OK;
+}
+
 // Shared by the full scan and the cached block decode.
 static int run_bimamba(const bimamba_dims *d, const void *xbc, const void *dt, const float *A,
                        const float *D, const float *conv_w, const float *conv_b,

@@ -33,6 +33,8 @@ cudaError_t launch_bimamba(const Problem &p, cudaStream_t stream);
 // chunked tensor-core path (bf16, headdim 64, d_state 128)
 bool tc_path_supported(const bimamba_dims &d);
 size_t tc_workspace_bytes(const bimamba_dims &d);
+// out[0..2]: segments per direction, chunks per segment, state-only items
+void tc_launch_plan(const bimamba_dims &d, int *out);
 cudaError_t launch_ssd_tc(const Problem &p, cudaStream_t stream);
 
 template <typename T>

@@ -48,6 +48,7 @@
 #include "dispatch.h"
 #include "tc_ptx.cuh"
 
+#include <algorithm>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -114,6 +115,12 @@ struct TcParams {
     __nv_bfloat16 *y;
     int *flags;   // [batch][H/2][nchunks][2]: arrivals, partial-ready
     int *status;
+    // segments (blockIdx.z): walk chunks [z * seg_chunks, +seg_chunks)
+    float *seg_state;   // [dir][batch][H/2][nitems][2][kP][kN] item end states from zero
+    float *seg_dec;     // [dir][batch][H/2][nitems][2] item decays, log2 units
+    int seg_chunks;     // walk chunks per CTA
+    int item_chunks;    // walk chunks per state-only item (0: no items)
+    int nitems;
     int len, H, ch, nchunks, batch;
 };
 
@@ -240,6 +247,11 @@ bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc, const __nv_bfloat16 *__
     }
 }
 
+// kStateOnly = false: outputs of walk chunks [k0, k0 + nk) of one segment,
+// entering it with the state chained from the items before it.
+// kStateOnly = true: only the state recurrence over one item's chunks, from a
+// zero state; writes the item's end state and its total decay.
+template <bool kStateOnly>
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_bc,
               const TcParams p)
@@ -255,6 +267,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     const int b = blockIdx.y;
     const int H = p.H, L = p.len, ch = p.ch;
     const int HP = H / kHeads;
+    const int k0 = blockIdx.z * p.seg_chunks;           // first walk chunk of this CTA
+    const int nk = min(p.seg_chunks, p.nchunks - k0);   // walk chunks it covers
+    const size_t item_row = ((size_t)(dir * p.batch + b) * HP + hp) * p.nitems;
 
     float *cum = reinterpret_cast<float *>(sm + kOffCum);   // [head][slot]
     float *dts = reinterpret_cast<float *>(sm + kOffDt);
@@ -277,7 +292,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     auto mcol = [](int k) -> uint32_t { return (k & 1) ? 0u : 128u; };
 
     auto chunk_of = [&](int k, int &t0, int &cnt, int &s0) {
-        const int c = rev ? p.nchunks - 1 - k : k;
+        const int kg = k0 + k;
+        const int c = rev ? p.nchunks - 1 - kg : kg;
         t0 = c * kQ;
         cnt = min(kQ, L - t0);
         s0 = rev ? L - t0 - cnt : t0;
@@ -295,11 +311,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         int t0, cnt, s0;
         chunk_of(k, t0, cnt, s0);
         const int zc = dir * p.batch + b;
-        tc::mbar_expect_tx(mb_bc, kBCBytes);
+        tc::mbar_expect_tx(mb_bc, kStateOnly ? kBCBytes / 2 : kBCBytes);
         tc::tma_load_3d(sbase + kOffB, &tm_bc, 0, s0, zc, mb_bc);
         tc::tma_load_3d(sbase + kOffB + 16384, &tm_bc, 64, s0, zc, mb_bc);
-        tc::tma_load_3d(sbase + kOffC, &tm_bc, 128, s0, zc, mb_bc);
-        tc::tma_load_3d(sbase + kOffC + 16384, &tm_bc, 192, s0, zc, mb_bc);
+        if constexpr (!kStateOnly) {
+            tc::tma_load_3d(sbase + kOffC, &tm_bc, 128, s0, zc, mb_bc);
+            tc::tma_load_3d(sbase + kOffC + 16384, &tm_bc, 192, s0, zc, mb_bc);
+        }
     };
 
     // ---- setup (all threads)
@@ -323,7 +341,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         tc::mbar_init(mb_m, 1);
         tc::mbar_init(mb_e, 1);
         issue_x(0);
-        if (p.nchunks > 1) issue_x(1);
+        if (nk > 1) issue_x(1);
         issue_bc(0);
     }
     tc::fence_before_sync();
@@ -346,38 +364,43 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             constexpr uint32_t idYo = tc::idesc_bf16(128, 128, 0, 1);
             constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
             bool pok = true;
-            for (int k = 0; k < p.nchunks && pok; ++k) {
+            for (int k = 0; k < nk && pok; ++k) {
                 // G(k) overwrites region gcol(k), last used by M(k-1): wait
                 // for the MMAs of chunk k-1, and for this chunk's B/C tiles
-                if (k > 0) pok = tc::mbar_wait_bounded(mb_e, (k - 1) & 1, kWaitCycles);
+                if (!kStateOnly && k > 0) pok = tc::mbar_wait_bounded(mb_e, (k - 1) & 1, kWaitCycles);
                 if (pok) pok = tc::mbar_wait_bounded(mb_bc, k & 1, kWaitCycles);
                 if (!pok) break;
                 tc::fence_after_sync();
                 const uint32_t g = tmem + gcol(k);
+                if constexpr (!kStateOnly) {
 #pragma unroll
-                for (int ks = 0; ks < kN / 16; ++ks) {
-                    const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    tc::mma_bf16(g, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
+                    for (int ks = 0; ks < kN / 16; ++ks) {
+                        const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        tc::mma_bf16(g, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
+                    }
+                    tc::mma_commit(mb_g);
                 }
-                tc::mma_commit(mb_g);
                 // Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
                 pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
                 if (!pok) break;
                 tc::fence_after_sync();
-                const uint64_t dX = (k & 1) ? dX1 : dX0;
-                const uint32_t mc = tmem + mcol(k);
+                if constexpr (!kStateOnly) {
+                    const uint64_t dX = (k & 1) ? dX1 : dX0;
+                    const uint32_t mc = tmem + mcol(k);
 #pragma unroll
-                for (int ks = 0; ks < kQ / 16; ++ks) {
+                    for (int ks = 0; ks < kQ / 16; ++ks) {
 #pragma unroll
-                    for (int hd = 0; hd < kHeads; ++hd)
-                        tc::mma_bf16_tmemA(g + 64 * hd, mc + 64 * hd + 8 * ks,
-                                           tc::desc_add(dX, hd * 16384 + ks * 2048), idYd, ks > 0);
+                        for (int hd = 0; hd < kHeads; ++hd)
+                            tc::mma_bf16_tmemA(g + 64 * hd, mc + 64 * hd + 8 * ks,
+                                               tc::desc_add(dX, hd * 16384 + ks * 2048), idYd, ks > 0);
+                    }
                 }
 #pragma unroll
                 for (int ks = 0; ks < kN / 16; ++ks) {
                     const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048),
-                                 idYo, ks > 0);
+                    if constexpr (!kStateOnly)
+                        tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048),
+                                     idYo, ks > 0);
                     tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048),
                                  tc::desc_add(dXw, ks * 2048), idS, 1);
                 }
@@ -385,11 +408,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 // once they complete, the B/C tiles and this chunk's x buffer
                 // are free: load the next chunk's tiles and the chunk after
                 // next's raw x rows
-                if (k + 1 < p.nchunks) {
+                if (k + 1 < nk) {
                     pok = tc::mbar_wait_bounded(mb_e, k & 1, kWaitCycles);
                     if (!pok) break;
                     issue_bc(k + 1);
-                    if (k + 2 < p.nchunks) issue_x(k + 2);
+                    if (k + 2 < nk) issue_x(k + 2);
                 }
             }
             if (!pok) record_error(p.status, kStatusTimeout);
@@ -551,34 +574,46 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         if (warp == 0) {
             load_dt_async(0);
             scan_dt(0);
-            if (p.nchunks > 1) load_dt_async(1);
+            if (nk > 1) load_dt_async(1);
         }
         alu_sync();
         slot_factors();
 
-        // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg
+        // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg.
+        // A segment's entering state: the caller's initial state (forward
+        // stream) or zero, carried through the items before the segment:
+        // S <- 2^dec_i S + S_i, with S_i item i's end state from zero.
         const int head_g = hp * kHeads + hh;     // global head of this thread's columns
         const size_t sidx = ((size_t)b * H + head_g) * kP * kN;
         {
-            uint32_t r[16];
+            float sv[32];
+            const bool use_init = !kStateOnly && !rev && p.init;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                sv[i] = use_init ? p.init[sidx + (size_t)(32 * hsub + i) * kN + row] : 0.0f;
+            const int n_in = (kStateOnly || p.item_chunks == 0) ? 0 : k0 / p.item_chunks;
+            for (int it = 0; it < n_in; ++it) {
+                const float *si = p.seg_state + ((item_row + it) * kHeads + hh) * kP * kN;
+                const float a = tc::exp2_approx(p.seg_dec[(item_row + it) * kHeads + hh]);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[i] = fmaf(sv[i], a, si[(size_t)(32 * hsub + i) * kN + row]);
+            }
 #pragma unroll
             for (int half16 = 0; half16 < 2; ++half16) {
+                uint32_t r[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int pp = 32 * hsub + 16 * half16 + i;
-                    const float v = (!rev && p.init) ? p.init[sidx + (size_t)pp * kN + row] : 0.0f;
-                    r[i] = __float_as_uint(v);
-                }
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sv[16 * half16 + i]);
                 tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
             }
         }
+        float dec = 0.0f;   // state-only: total decay of the item (log2 units)
         const float Dh = p.D[head_g];
 
         int arrival = 0;   // result of this chunk's arrival atomic (thread kArriveTid)
         bool ok = wait_all(mb_x0, 0);
         if (ok) {
             // decode: the conv history before token 0 comes from the cached tail
-            if (!rev && p.tail) {
+            if (!rev && p.tail && k0 == 0) {
                 for (int e = tid; e < 3 * (kPP / 8); e += kAluThreads) {
                     const int r = e / (kPP / 8), g = e % (kPP / 8);
                     *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
@@ -592,71 +627,78 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             weight_chunk(0);
         }
 
-        for (int k = 0; k < p.nchunks && ok; ++k) {
+        for (int k = 0; k < nk && ok; ++k) {
             int t0, cnt, s0;
             const int c = chunk_of(k, t0, cnt, s0);
-            const bool more = k + 1 < p.nchunks;
+            const bool more = k + 1 < nk;
 
             // arrive at this chunk's forward/reverse meeting point; the
             // result is read only after the chunk's MMAs
-            if (tid == kArriveTid)
+            if (!kStateOnly && tid == kArriveTid)
                 arrival = atomicAdd(p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2, 1);
 
             // ---- D: M_h (both heads, into TMEM) and the state's chunk-start
             // scaling, once G(k) is done.  Thread (row t, rg): head hh,
             // s-blocks 2*hsub, 2*hsub+1.
             tc::fence_proxy_async();          // wX of this chunk (written last iteration)
-            ok = wait_all(mb_g, k & 1);
-            if (!ok) break;
+            if constexpr (!kStateOnly) {
+                ok = wait_all(mb_g, k & 1);
+                if (!ok) break;
+            }
             tc::fence_after_sync();
             const float ct = cum[hh * kQ + row];            // kept for the epilogue
             const float a_last = tc::exp2_approx(cum[hh * kQ + kQ - 1]);
+            if constexpr (kStateOnly) dec += cum[hh * kQ + kQ - 1];
             {
                 const uint32_t gc = gcol(k), mc = mcol(k);
+                if constexpr (!kStateOnly) {
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    const int jb = 2 * hsub + jj;           // 32-slot block of s
-                    uint32_t packed[16];
-                    if (jb > quad) {                        // warp-uniform: all s > t
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int jb = 2 * hsub + jj;           // 32-slot block of s
+                        uint32_t packed[16];
+                        if (jb > quad) {                        // warp-uniform: all s > t
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) packed[i] = 0u;
-                    } else {
-                        float gv[32];
-                        tc::tmem_ld32(tmem + lane_base + gc + 32 * jb, gv);
-                        const float *fbh = fB + hh * kQ + 32 * jb;
-                        if (jb < quad) {
-                            // whole block below the diagonal: factorised decay
-                            const float et = tc::exp2_approx(ct - cum[hh * kQ + 32 * jb + 31]);
-#pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                packed[i] = tc::pack_bf16x2(gv[2 * i] * et * fbh[2 * i],
-                                                            gv[2 * i + 1] * et * fbh[2 * i + 1]);
+                            for (int i = 0; i < 16; ++i) packed[i] = 0u;
                         } else {
-                            // diagonal block: one exponential per element, D on the diagonal
-                            const float *ch_ = cum + hh * kQ + 32 * jb;
-                            const float *dh_ = dts + hh * kQ + 32 * jb;
-                            const int r31 = row & 31;
-                            float m[32];
+                            float gv[32];
+                            tc::tmem_ld32(tmem + lane_base + gc + 32 * jb, gv);
+                            const float *fbh = fB + hh * kQ + 32 * jb;
+                            if (jb < quad) {
+                                // whole block below the diagonal: factorised decay
+                                const float et = tc::exp2_approx(ct - cum[hh * kQ + 32 * jb + 31]);
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const float e = tc::exp2_approx(fminf(ct - ch_[i], 0.0f));
-                                const float add = (i == r31) ? Dh : 0.0f;
-                                const float v = fmaf(gv[i] * e, dh_[i], add);
-                                m[i] = (i <= r31) ? v : 0.0f;
+                                for (int i = 0; i < 16; ++i)
+                                    packed[i] = tc::pack_bf16x2(gv[2 * i] * et * fbh[2 * i],
+                                                                gv[2 * i + 1] * et * fbh[2 * i + 1]);
+                            } else {
+                                // diagonal block: one exponential per element, D on the diagonal
+                                const float *ch_ = cum + hh * kQ + 32 * jb;
+                                const float *dh_ = dts + hh * kQ + 32 * jb;
+                                const int r31 = row & 31;
+                                float m[32];
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) {
+                                    const float e = tc::exp2_approx(fminf(ct - ch_[i], 0.0f));
+                                    const float add = (i == r31) ? Dh : 0.0f;
+                                    const float v = fmaf(gv[i] * e, dh_[i], add);
+                                    m[i] = (i <= r31) ? v : 0.0f;
+                                }
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) packed[i] = tc::pack_bf16x2(m[2 * i], m[2 * i + 1]);
                             }
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) packed[i] = tc::pack_bf16x2(m[2 * i], m[2 * i + 1]);
                         }
+                        tc::tmem_st16(tmem + lane_base + mc + 64 * hh + 16 * jb, packed);
                     }
-                    tc::tmem_st16(tmem + lane_base + mc + 64 * hh + 16 * jb, packed);
                 }
                 // state: bf16 copy of S_in (the Yo operand), then S <- exp(c_last) S
                 float sv[32];
                 tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
+                if constexpr (!kStateOnly) {
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc)
-                    *reinterpret_cast<uint4 *>(sm + kOffS + hh * 16384 + tc::sw128(row, 4 * hsub + pc)) =
-                        pack8(sv + 8 * pc);
+                    for (int pc = 0; pc < 4; ++pc)
+                        *reinterpret_cast<uint4 *>(sm + kOffS + hh * 16384 +
+                                                   tc::sw128(row, 4 * hsub + pc)) = pack8(sv + 8 * pc);
+                }
 #pragma unroll
                 for (int half16 = 0; half16 < 2; ++half16) {
                     uint32_t r[16];
@@ -673,18 +715,23 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             // ---- while the MMAs run: next chunk's dt prefix sums and conv
             if (warp == 0 && more) {
                 scan_dt(k + 1);                       // its copies were issued a chunk ago
-                if (k + 2 < p.nchunks) load_dt_async(k + 2);
+                if (k + 2 < nk) load_dt_async(k + 2);
             }
             if (more) {
                 ok = wait_all(mb_x0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
                 if (!ok) break;
                 conv_chunk(k + 1);
             }
-            if (tid == kArriveTid) *flag_slot = arrival;
+            if (!kStateOnly && tid == kArriveTid) *flag_slot = arrival;
             ok = wait_all(mb_e, k & 1);
             if (!ok) break;
             tc::fence_after_sync();
             if (more) slot_factors();                          // next chunk's fB, w
+            if constexpr (kStateOnly) {
+                alu_sync();   // publishes the next chunk's factors
+                if (more) weight_chunk(k + 1);
+                continue;
+            }
 
             // ---- F: output rows, and the forward + reverse sum
             int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
@@ -766,7 +813,19 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             }
         }
 
-        if (ok && !rev && p.fin) {
+        if constexpr (kStateOnly) {
+            if (ok) {
+                // the item's end state and total decay
+                tc::fence_after_sync();
+                float sv[32];
+                tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
+                const size_t item = item_row + blockIdx.z;
+                float *so = p.seg_state + (item * kHeads + hh) * kP * kN;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) so[(size_t)(32 * hsub + i) * kN + row] = sv[i];
+                if (row == 0 && hsub == 0) p.seg_dec[item * kHeads + hh] = dec;
+            }
+        } else if (ok && !rev && p.fin && k0 + nk == p.nchunks) {
             tc::fence_after_sync();
             float sv[32];
             tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
@@ -786,8 +845,40 @@ bool tc_path_supported(const bimamba_dims &d)
            d.d_conv == 4 && d.len > 0 && d.heads % kHeads == 0;
 }
 
+// Segments.  One CTA per (batch, head pair, direction) fills the 148 SMs
+// only when batch * heads >= 148.  Otherwise each direction's walk is cut
+// into nseg segments of seg_chunks chunks, run side by side.  A segment must
+// start from the state the walk carries into it, so a state-only pass first
+// reduces each of the nitems = (nseg - 1) * r items (seg_chunks / r chunks
+// each) before the last segment to its end state from zero and its total
+// decay; a segment's CTA then chains the items before it (the recurrence is
+// linear in the state, so S_in = 2^dec_i S_in + S_i over the items in order).
+// r > 1 splits the state-only pass finer than the segments, so that it too
+// fills the SMs.
+struct SegPlan {
+    int nseg, seg_chunks, item_chunks, nitems;
+};
+
+constexpr int kPlanSMs = 148;   // SMs of a B200
+
+static SegPlan seg_plan(const bimamba_dims &d)
+{
+    const int nchunks = (int)(((long long)d.len + kQ - 1) / kQ);
+    const SegPlan whole{1, nchunks, 0, 0};
+    const long long ctas = (long long)d.heads * d.batch;   // head pairs x 2 directions
+    if (ctas <= 0 || ctas * 2 > kPlanSMs || nchunks < 4) return whole;
+    const int nseg_target = (int)(kPlanSMs / ctas);
+    const int r = (int)std::max<long long>(1, kPlanSMs / (ctas * (nseg_target - 1)));
+    const int item_chunks = (nchunks + nseg_target * r - 1) / (nseg_target * r);
+    const int seg_chunks = r * item_chunks;
+    const int nseg = (nchunks + seg_chunks - 1) / seg_chunks;
+    if (nseg < 2) return whole;
+    return SegPlan{nseg, seg_chunks, item_chunks, (nseg - 1) * r};
+}
+
 // workspace: [flags: batch*(H/2)*nchunks*2 int32, 1 KB aligned][B/C activations:
-// 2 directions x batch x len x 256 bf16]
+// 2 directions x batch x len x 256 bf16][item states: 2 x batch x H/2 x nitems
+// x 2 x kP x kN f32][item decays: 2 x batch x H/2 x nitems x 2 f32]
 static size_t flags_bytes(const bimamba_dims &d)
 {
     const size_t nchunks = ((size_t)d.len + kQ - 1) / kQ;
@@ -795,9 +886,30 @@ static size_t flags_bytes(const bimamba_dims &d)
     return (bytes + 1023) & ~(size_t)1023;
 }
 
+static size_t act_bytes(const bimamba_dims &d)
+{
+    return (size_t)2 * d.batch * d.len * kBC * sizeof(__nv_bfloat16);
+}
+
+static size_t items(const bimamba_dims &d, const SegPlan &sp)
+{
+    return (size_t)2 * d.batch * (d.heads / kHeads) * sp.nitems;
+}
+
+void tc_launch_plan(const bimamba_dims &d, int *out)
+{
+    const SegPlan sp = seg_plan(d);
+    out[0] = sp.nseg;
+    out[1] = sp.seg_chunks;
+    out[2] = sp.nitems;
+}
+
 size_t tc_workspace_bytes(const bimamba_dims &d)
 {
-    return flags_bytes(d) + (size_t)2 * d.batch * d.len * kBC * sizeof(__nv_bfloat16);
+    const SegPlan sp = seg_plan(d);
+    const size_t n = items(d, sp);
+    return flags_bytes(d) + act_bytes(d) + n * kHeads * kP * kN * sizeof(float) +
+           n * kHeads * sizeof(float);
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -852,8 +964,15 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
     p.ch = d.heads * d.headdim + 2 * d.ngroups * d.d_state;
     p.nchunks = (d.len + kQ - 1) / kQ;
     p.batch = d.batch;
-    __nv_bfloat16 *act = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(pr.workspace) +
-                                                           flags_bytes(d));
+    char *ws = static_cast<char *>(pr.workspace);
+    __nv_bfloat16 *act = reinterpret_cast<__nv_bfloat16 *>(ws + flags_bytes(d));
+    const SegPlan sp = seg_plan(d);
+    const size_t n_items = items(d, sp);
+    p.seg_state = reinterpret_cast<float *>(ws + flags_bytes(d) + act_bytes(d));
+    p.seg_dec = p.seg_state + n_items * kHeads * kP * kN;
+    p.seg_chunks = sp.seg_chunks;
+    p.item_chunks = sp.item_chunks;
+    p.nitems = sp.nitems;
 
     // prepass: B/C conv+SiLU in walk order for both directions
     bc_prepass_kernel<<<dim3((d.len + 31) / 32, d.batch, 2), 128, 0, stream>>>(
@@ -867,12 +986,25 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
                   false) ||
         !make_map(&tm_bc, act, (uint64_t)kBC, (uint64_t)d.len, (uint64_t)2 * d.batch, 64, kQ, true))
         return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(ssd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(ssd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ssd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const TimingEvents ev = timing_events();
     if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
-    ssd_tc_kernel<<<dim3(d.heads, d.batch), kThreads, kSmemBytes, stream>>>(tm_x, tm_bc, p);
+    if (sp.nitems > 0) {
+        TcParams q = p;
+        q.seg_chunks = sp.item_chunks;   // one CTA per item
+        ssd_tc_kernel<true><<<dim3(d.heads, d.batch, sp.nitems), kThreads, kSmemBytes, stream>>>(
+            tm_x, tm_bc, q);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        count_launch();
+    }
+    ssd_tc_kernel<false><<<dim3(d.heads, d.batch, sp.nseg), kThreads, kSmemBytes, stream>>>(
+        tm_x, tm_bc, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();

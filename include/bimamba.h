@@ -124,11 +124,32 @@ int bimamba_conv_silu(const void *u, void *out, const float *w, const float *bia
  * Bytes of scratch workspace bimamba_ssd_fwd_rev / bimamba_block_decode need
  * for dims `d`.  The caller allocates it once (device memory, 256-byte
  * aligned), zero-fills it before first use, and may reuse it for any later
- * call whose workspace size is not larger.  The kernels leave it zeroed.
+ * call whose workspace size is not larger.  The kernels return its
+ * forward/reverse meeting counters to zero, so it needs no clearing between
+ * calls (the rest holds per-call intermediates that every call rewrites).
  * Calls that share one workspace must not run concurrently.
  * Returns 0 for invalid dims.
  */
 size_t bimamba_workspace_bytes(const bimamba_dims *d);
+
+/*
+ * How a bimamba_ssd_fwd_rev / bimamba_block_decode call with dims `d` is
+ * launched; host only, no device work.  The chunked scan ("Mamba-2" state
+ * space duality, chunkwise form: intra-chunk contraction, chunk states,
+ * state passing) parallelises over (sequence, head pair, direction); when
+ * that gives fewer than two CTAs per 148 SMs each direction's walk is cut
+ * into segments, and a state-only pass first reduces the walk before each
+ * segment to end states that the segment chains from.
+ *   out[0] : 1 chunked tensor-core path, 0 sequential fp32 path
+ *   out[1] : segments per direction (1: no segmentation)
+ *   out[2] : 128-token chunks per segment
+ *   out[3] : state-only items per (sequence, head pair, direction)
+ *            (0: no state-only pass)
+ * out must point to 4 writable ints.  Returns BIMAMBA_ERR_INVALID for
+ * invalid dims or a NULL out, else BIMAMBA_OK (the same shape checks as the
+ * compute calls, so UNSUPPORTED dims are reported too).
+ */
+int bimamba_launch_plan(const bimamba_dims *d, int *out);
 
 /*
  * Full bidirectional mixer core (steps: load, conv+SiLU both ways, decay,

@@ -92,3 +92,54 @@ def test_workspace_size_is_monotone(lib):
     a = lib.bimamba_workspace_bytes(lib.make_dims(8, 4096, 64, 64, 128, 1))
     b = lib.bimamba_workspace_bytes(lib.make_dims(8, 8192, 64, 64, 128, 1))
     assert 0 <= a <= b
+
+
+def test_launch_plan_covers_the_walk(lib):
+    """Segment plans (host only): segments tile the chunk walk, state-only
+    items tile the walk before the last segment and nest in the segments, and
+    a segmented launch stays within one wave of the 148 SMs."""
+    import torch
+    assert lib.bimamba_launch_plan(lib.make_dims(1, 256, 4, 32, 16, torch.float32)) == {
+        "tensor_core": False, "segments": 1, "seg_chunks": 2, "items": 0}
+    # the benchmarked layer (512 CTAs) is not segmented
+    assert lib.bimamba_launch_plan(lib.make_dims(8, 4096, 64, 64, 128, torch.bfloat16)) == {
+        "tensor_core": True, "segments": 1, "seg_chunks": 32, "items": 0}
+    seen_split_items = False
+    for bsz in (1, 2, 3, 8):
+        for H in (2, 4, 16, 32, 64):
+            for L in (1, 127, 128, 513, 1100, 1300, 4096, 131072):
+                p = lib.bimamba_launch_plan(lib.make_dims(bsz, L, H, 64, 128, torch.bfloat16))
+                nchunks = (L + 127) // 128
+                S, sc, items = p["segments"], p["seg_chunks"], p["items"]
+                assert p["tensor_core"]
+                assert S >= 1 and sc >= 1
+                assert (S - 1) * sc < nchunks <= S * sc, (bsz, H, L, p)
+                ctas = bsz * H
+                if S == 1:
+                    assert items == 0
+                    continue
+                assert ctas * S <= 148 and ctas * items <= 148, (bsz, H, L, p)
+                assert items % (S - 1) == 0
+                r = items // (S - 1)
+                assert sc % r == 0
+                seen_split_items |= r > 1
+    assert seen_split_items
+
+
+def test_launch_plan_rejects_bad_arguments(lib):
+    import torch
+    L = lib.library()
+    d = lib.make_dims(1, 8, 0, 64, 128, torch.bfloat16)
+    out = (ctypes.c_int * 4)()
+    assert L.bimamba_launch_plan(ctypes.byref(d), out) == lib.BIMAMBA_ERR_INVALID
+    d = lib.make_dims(1, 8, 2, 64, 128, torch.bfloat16)
+    assert L.bimamba_launch_plan(ctypes.byref(d), None) == lib.BIMAMBA_ERR_INVALID
+
+
+def test_workspace_grows_with_the_state_only_items(lib):
+    import torch
+    d1 = lib.make_dims(1, 1300, 2, 64, 128, torch.bfloat16)    # 10 items
+    flags = 1024                                                 # 11 chunks x 2 counters, 1 KB
+    act = 2 * 1 * 1300 * 256 * 2
+    items = 2 * 1 * 1 * 10
+    assert lib.bimamba_workspace_bytes(d1) == flags + act + items * 2 * 64 * 128 * 4 + items * 2 * 4

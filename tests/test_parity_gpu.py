@@ -320,10 +320,49 @@ def test_odd_head_count_uses_a_valid_path(lib):
     assert rel_err(to_np(y), ry) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("blk,prefix", [(1, 5), (128, 300), (200, 64)])
+@pytest.mark.parametrize("blk,prefix", [(1, 5), (128, 300), (200, 64), (900, 100)])
 def test_block_decode_multi_chunk_blocks(lib, blk, prefix):
-    """Decode blocks of 1, 128 and 200 tokens (one, one full and two chunks)."""
+    """Decode blocks of 1, 128, 200 and 900 tokens (one, one full, two and
+    eight chunks; the 900-token block is walked as segments, so the cached
+    state, the conv tail and the commit meet segment boundaries)."""
     _decode_case(lib, "bf16", 2, blk, prefix, 4, 64, 128, (1e-3, 1e-2))
+
+
+# ------------------------------------------------------- segmented walks
+SEGMENTED = [
+    # batch, L, H, variant, heads the oracle checks (None: all)
+    (1, 1300, 2, "plain", None),          # 11 one-chunk segments, 10 state-only items
+    (2, 700, 4, "init+bias", None),       # 6 one-chunk segments, initial state chained
+    (1, 1100, 64, "init+bias", [0, 17, 62, 63]),   # 2 segments of 6 chunks, items of 3
+]
+
+
+@pytest.mark.parametrize("case", SEGMENTED, ids=lambda c: f"b{c[0]}-L{c[1]}-H{c[2]}-{c[3]}")
+@pytest.mark.parametrize("memory", ["short", "long"])
+def test_segmented_walks(lib, case, memory):
+    """Few (sequence, head pair) tasks: each direction's walk is split into
+    segments that start from states chained out of a state-only pass.  With
+    long-memory decays the chained state dominates every segment's output."""
+    bsz, L, H, variant, heads = case
+    P, N = 64, 128
+    plan = lib.bimamba_launch_plan(lib.make_dims(bsz, L, H, P, N, torch.bfloat16))
+    assert plan["tensor_core"] and plan["segments"] > 1 and plan["items"] > 0, plan
+    w = inp_mod.Workload("seg", bsz, L, H, P, N, dtype="bf16", bc_scale=1.0 / math.sqrt(N))
+    a = (1.0, 16.0) if memory == "short" else (1e-3, 1e-2)
+    cpu = inp_mod.make_inputs(w, seed=L + H, a_range=a, conv_bias="bias" in variant)
+    init = inp_mod.make_state(bsz, H, P, N, seed=11, scale=0.3) if "init" in variant else None
+    y, fin = _run_scan(lib, w, _dev(cpu), None if init is None else init.cuda(), want_final=True)
+    n = _np_inputs(cpu)
+    heads = list(range(H)) if heads is None else heads
+    sub, _ = head_subset(n, heads, H, P, N)
+    ry, rfin = oracle.bimamba(sub["xbc"], sub["dt"], sub["A"], sub["D"], sub["conv_w"],
+                              sub["conv_b"], heads=len(heads), headdim=P, d_state=N,
+                              init=None if init is None else to_np(init[:, heads]),
+                              want_final=True)
+    cols = y_cols(heads, P)
+    for b in range(bsz):
+        assert rel_err(to_np(y)[b][..., cols], ry[b]) <= TOL["bf16"], b
+        assert rel_err(to_np(fin)[b][heads], rfin[b]) <= TOL["bf16"], b
 
 
 def test_repeated_calls_reuse_the_workspace(lib):
