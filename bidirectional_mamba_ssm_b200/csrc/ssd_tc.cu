@@ -78,14 +78,14 @@ constexpr uint32_t kOffXbuf1 = kOffXbuf0 + kXbufBytes;   // odd walk chunks
 constexpr uint32_t kOffXw = kOffXbuf1 + kXbufBytes;      // wX [s][p'] 2 x 16 KB
 constexpr uint32_t kOffS = kOffXw + 32768;               // S^T bf16 [n][p'] 2 x 16 KB
 constexpr uint32_t kRawBytes = kRawRows * kPP * 2;       // 33536
-constexpr uint32_t kOffCum = kOffS + 32768;      // f32[2][128] prefix sums of dt*A
-constexpr uint32_t kOffDt = kOffCum + 1024;      // f32[2][128] dt
-constexpr uint32_t kOffFB = kOffDt + 1024;       // f32[2][128] exp(c_R - c_s) dt_s, R = block end
+constexpr uint32_t kOffCum = kOffS + 32768;      // f32[2][2][128] prefix sums of dt*A (chunk parity, head)
+constexpr uint32_t kOffDt = kOffCum + 2048;      // f32[2][2][128] dt
+constexpr uint32_t kOffFB = kOffDt + 2048;       // f32[2][128] exp(c_R - c_s) dt_s, R = block end
 constexpr uint32_t kOffWgt = kOffFB + 1024;      // f32[2][128] exp(c_last - c_s) dt_s
 constexpr uint32_t kOffConvW = kOffWgt + 1024;   // float4[128] conv taps of x
 constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
-constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x6 (see the kernel)
-constexpr uint32_t kOffTmem = kOffMbar + 48;     // u32 TMEM base
+constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x8 (see the kernel)
+constexpr uint32_t kOffTmem = kOffMbar + 64;     // u32 TMEM base
 constexpr uint32_t kOffFlag = kOffTmem + 4;      // i32 handshake result
 constexpr uint32_t kOffDtBuf = kOffFlag + 12;    // [2][128] bf16x2: dt of both heads, by cp.async
 constexpr uint32_t kSmemUsed = kOffDtBuf + 2 * kQ * 4;
@@ -271,7 +271,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     const int nk = min(p.seg_chunks, p.nchunks - k0);   // walk chunks it covers
     const size_t item_row = ((size_t)(dir * p.batch + b) * HP + hp) * p.nitems;
 
-    float *cum = reinterpret_cast<float *>(sm + kOffCum);   // [head][slot]
+    float *cum = reinterpret_cast<float *>(sm + kOffCum);   // [chunk parity][head][slot]
     float *dts = reinterpret_cast<float *>(sm + kOffDt);
     float *fB = reinterpret_cast<float *>(sm + kOffFB);
     float *wgt = reinterpret_cast<float *>(sm + kOffWgt);
@@ -279,12 +279,19 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     float *convb = reinterpret_cast<float *>(sm + kOffConvB);
     int *flag_slot = reinterpret_cast<int *>(sm + kOffFlag);
     // mbarriers: B/C tiles landed, raw x landed (buffer 0 / 1), G done,
-    // M/state ready for the chunk's MMAs, chunk MMAs done
+    // M/state ready for the chunk's MMAs, chunk MMAs done, the dt prefix
+    // sums of an even / odd walk chunk written (one barrier per buffer, so
+    // that the producer may run a chunk ahead without phase aliasing)
     const uint32_t mb_bc = sbase + kOffMbar;
     const uint32_t mb_x0 = sbase + kOffMbar + 8;
     const uint32_t mb_g = sbase + kOffMbar + 24;
     const uint32_t mb_m = sbase + kOffMbar + 32;
     const uint32_t mb_e = sbase + kOffMbar + 40;
+    const uint32_t mb_dt0 = sbase + kOffMbar + 48;   // + 8 * (chunk & 1)
+    auto dt_ready = [&](int k, uint32_t &mb, uint32_t &parity) {
+        mb = mb_dt0 + 8 * (k & 1);
+        parity = (k >> 1) & 1;
+    };
     auto xbuf_off = [](int k) { return (k & 1) ? kOffXbuf1 : kOffXbuf0; };
     // TMEM regions that alternate between chunks: G(k) and Yd(k) use
     // columns gcol(k) .. +127, M(k) uses mcol(k) .. +127 (the other region)
@@ -320,6 +327,67 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         }
     };
 
+    constexpr float kLog2e = 1.4426950408889634f;
+    const float A0 = p.A[hp * kHeads] * kLog2e, A1 = p.A[hp * kHeads + 1] * kLog2e;
+
+    // producer warp: asynchronous copy of walk chunk k's dt (both heads of
+    // the pair are adjacent: one 4-byte copy per token) into dt buffer
+    // k % 2; slots past the chunk end are zero.
+    auto load_dt_async = [&](int k) {
+        int t0, cnt, s0;
+        chunk_of(k, t0, cnt, s0);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(sm + kOffDtBuf) + (k & 1) * kQ;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = 4 * lane + i;
+            if (j < cnt) {
+                const int s = s0 + j;
+                const int tok = rev ? L - 1 - s : s;
+                const __nv_bfloat16 *src = p.dt + ((size_t)b * L + tok) * H + hp * kHeads;
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
+                             :: "r"(tc::smem_u32(dst + j)), "l"(src) : "memory");
+            } else {
+                dst[j] = 0u;
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // producer warp: inclusive prefix sums of dt*A of both heads for walk
+    // chunk k into cum/dts buffer k % 2, in log2 units (A carries the factor
+    // log2(e)) so that every decay factor is one 2^x on the special-function
+    // unit.  Waits for this thread's outstanding dt copies, which are chunk
+    // k's (and, before the first chunk, chunk 1's).
+    auto scan_dt = [&](int k) {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        const __nv_bfloat162 *src =
+            reinterpret_cast<const __nv_bfloat162 *>(sm + kOffDtBuf) + (k & 1) * kQ + 4 * lane;
+#pragma unroll
+        for (int head = 0; head < kHeads; ++head) {
+            float d[4], a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(src[i]);
+                d[i] = head ? f.y : f.x;
+            }
+            const float Aw = head ? A1 : A0;
+            a[0] = d[0] * Aw;
+#pragma unroll
+            for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Aw, a[i - 1]);
+            float run = a[3];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, run, o);
+                if (lane >= o) run += v;
+            }
+            const float excl = run - a[3];
+            float *db = dts + ((k & 1) * kHeads + head) * kQ + 4 * lane;
+            float *cb = cum + ((k & 1) * kHeads + head) * kQ + 4 * lane;
+            *reinterpret_cast<float4 *>(db) = make_float4(d[0], d[1], d[2], d[3]);
+            *reinterpret_cast<float4 *>(cb) =
+                make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
+        }
+    };
+
     // ---- setup (all threads)
     const bool has_conv = p.conv_w != nullptr;
     if (tid < kPP && has_conv) {
@@ -340,6 +408,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         tc::mbar_init(mb_g, 1);
         tc::mbar_init(mb_m, 1);
         tc::mbar_init(mb_e, 1);
+        tc::mbar_init(mb_dt0, 32);       // every producer lane arrives after its part of a scan
+        tc::mbar_init(mb_dt0 + 8, 32);
         issue_x(0);
         if (nk > 1) issue_x(1);
         issue_bc(0);
@@ -350,73 +420,96 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kOffTmem);
 
     if (warp == kProducerWarp) {
-        // ================= producer: every MMA and every TMA load ==========
-        if (lane == 0) {
-            const uint64_t dC = tc::smem_desc(sbase + kOffC, 16, 1024);       // K-major A (G, Yo)
-            const uint64_t dB = tc::smem_desc(sbase + kOffB, 16, 1024);       // K-major B (G)
-            const uint64_t dBmn = tc::smem_desc(sbase + kOffB, 16384, 1024);  // MN-major A (state)
-            const uint64_t dX0 = tc::smem_desc(sbase + kOffXbuf0, 1024, 1024);  // MN-major B (Yd)
-            const uint64_t dX1 = tc::smem_desc(sbase + kOffXbuf1, 1024, 1024);
-            const uint64_t dS = tc::smem_desc(sbase + kOffS, 16384, 1024);    // MN-major B (Yo)
-            const uint64_t dXw = tc::smem_desc(sbase + kOffXw, 16384, 1024);  // MN-major B (state)
-            constexpr uint32_t idG = tc::idesc_bf16(128, 128, 0, 0);
-            constexpr uint32_t idYd = tc::idesc_bf16(128, 64, 0, 1);
-            constexpr uint32_t idYo = tc::idesc_bf16(128, 128, 0, 1);
-            constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
-            bool pok = true;
-            for (int k = 0; k < nk && pok; ++k) {
+        // ================= producer: every MMA and every TMA load (lane 0),
+        // and each chunk's dt prefix sums (whole warp), computed while the
+        // compute group builds the previous chunk's M
+        load_dt_async(0);
+        if (nk > 1) load_dt_async(1);
+        scan_dt(0);
+        tc::mbar_arrive(mb_dt0);
+        const uint64_t dC = tc::smem_desc(sbase + kOffC, 16, 1024);       // K-major A (G, Yo)
+        const uint64_t dB = tc::smem_desc(sbase + kOffB, 16, 1024);       // K-major B (G)
+        const uint64_t dBmn = tc::smem_desc(sbase + kOffB, 16384, 1024);  // MN-major A (state)
+        const uint64_t dX0 = tc::smem_desc(sbase + kOffXbuf0, 1024, 1024);  // MN-major B (Yd)
+        const uint64_t dX1 = tc::smem_desc(sbase + kOffXbuf1, 1024, 1024);
+        const uint64_t dS = tc::smem_desc(sbase + kOffS, 16384, 1024);    // MN-major B (Yo)
+        const uint64_t dXw = tc::smem_desc(sbase + kOffXw, 16384, 1024);  // MN-major B (state)
+        constexpr uint32_t idG = tc::idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t idYd = tc::idesc_bf16(128, 64, 0, 1);
+        constexpr uint32_t idYo = tc::idesc_bf16(128, 128, 0, 1);
+        constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
+        bool pok = true;
+        for (int k = 0; k < nk && pok; ++k) {
+            const uint32_t g = tmem + gcol(k);
+            if (lane == 0) {
                 // G(k) overwrites region gcol(k), last used by M(k-1): wait
                 // for the MMAs of chunk k-1, and for this chunk's B/C tiles
                 if (!kStateOnly && k > 0) pok = tc::mbar_wait_bounded(mb_e, (k - 1) & 1, kWaitCycles);
                 if (pok) pok = tc::mbar_wait_bounded(mb_bc, k & 1, kWaitCycles);
-                if (!pok) break;
-                tc::fence_after_sync();
-                const uint32_t g = tmem + gcol(k);
-                if constexpr (!kStateOnly) {
+                if (pok) {
+                    tc::fence_after_sync();
+                    if constexpr (!kStateOnly) {
+#pragma unroll
+                        for (int ks = 0; ks < kN / 16; ++ks) {
+                            const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            tc::mma_bf16(g, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
+                        }
+                        tc::mma_commit(mb_g);
+                    }
+                }
+            }
+            pok = __shfl_sync(0xffffffffu, pok, 0);
+            if (!pok) break;
+            // while the compute group builds M(k): the next chunk's dt prefix
+            // sums (buffer (k+1) % 2, last read for chunk k-1)
+            if (k + 1 < nk) {
+                scan_dt(k + 1);
+                if (k + 2 < nk) load_dt_async(k + 2);
+                tc::mbar_arrive(mb_dt0 + 8 * ((k + 1) & 1));
+            }
+            if (lane == 0) {
+                // Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
+                pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
+                if (pok) {
+                    tc::fence_after_sync();
+                    if constexpr (!kStateOnly) {
+                        const uint64_t dX = (k & 1) ? dX1 : dX0;
+                        const uint32_t mc = tmem + mcol(k);
+#pragma unroll
+                        for (int ks = 0; ks < kQ / 16; ++ks) {
+#pragma unroll
+                            for (int hd = 0; hd < kHeads; ++hd)
+                                tc::mma_bf16_tmemA(g + 64 * hd, mc + 64 * hd + 8 * ks,
+                                                   tc::desc_add(dX, hd * 16384 + ks * 2048), idYd, ks > 0);
+                        }
+                    }
 #pragma unroll
                     for (int ks = 0; ks < kN / 16; ++ks) {
                         const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        tc::mma_bf16(g, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
+                        if constexpr (!kStateOnly)
+                            tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048),
+                                         idYo, ks > 0);
+                        tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048),
+                                     tc::desc_add(dXw, ks * 2048), idS, 1);
                     }
-                    tc::mma_commit(mb_g);
+                    tc::mma_commit(mb_e);
                 }
-                // Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
-                pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
-                if (!pok) break;
-                tc::fence_after_sync();
-                if constexpr (!kStateOnly) {
-                    const uint64_t dX = (k & 1) ? dX1 : dX0;
-                    const uint32_t mc = tmem + mcol(k);
-#pragma unroll
-                    for (int ks = 0; ks < kQ / 16; ++ks) {
-#pragma unroll
-                        for (int hd = 0; hd < kHeads; ++hd)
-                            tc::mma_bf16_tmemA(g + 64 * hd, mc + 64 * hd + 8 * ks,
-                                               tc::desc_add(dX, hd * 16384 + ks * 2048), idYd, ks > 0);
-                    }
-                }
-#pragma unroll
-                for (int ks = 0; ks < kN / 16; ++ks) {
-                    const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    if constexpr (!kStateOnly)
-                        tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048),
-                                     idYo, ks > 0);
-                    tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048),
-                                 tc::desc_add(dXw, ks * 2048), idS, 1);
-                }
-                tc::mma_commit(mb_e);
-                // once they complete, the B/C tiles and this chunk's x buffer
-                // are free: load the next chunk's tiles and the chunk after
-                // next's raw x rows
-                if (k + 1 < nk) {
-                    pok = tc::mbar_wait_bounded(mb_e, k & 1, kWaitCycles);
-                    if (!pok) break;
+            }
+            pok = __shfl_sync(0xffffffffu, pok, 0);
+            if (!pok || k + 1 >= nk) break;
+            // once they complete, the B/C tiles and this chunk's x buffer
+            // are free: load the next chunk's tiles and the chunk after
+            // next's raw x rows
+            if (lane == 0) {
+                pok = tc::mbar_wait_bounded(mb_e, k & 1, kWaitCycles);
+                if (pok) {
                     issue_bc(k + 1);
                     if (k + 2 < nk) issue_x(k + 2);
                 }
             }
-            if (!pok) record_error(p.status, kStatusTimeout);
+            pok = __shfl_sync(0xffffffffu, pok, 0);
         }
+        if (lane == 0 && !pok) record_error(p.status, kStatusTimeout);
     } else {
         // ================= compute group: 512 threads ======================
         // thread roles: row = TMEM lane / tile row; rg = 32-column group of
@@ -427,71 +520,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         const int hsub = rg & 1;
         const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         const int quad = warp & 3;
-        constexpr float kLog2e = 1.4426950408889634f;
-        const float A0 = p.A[hp * kHeads] * kLog2e, A1 = p.A[hp * kHeads + 1] * kLog2e;
-
-        // warp 0: asynchronous copy of walk chunk k's dt (both heads of the
-        // pair are adjacent: one 4-byte copy per token) into dt buffer k % 2;
-        // slots past the chunk end are zero.  Nothing is held in registers.
-        auto load_dt_async = [&](int k) {
-            int t0, cnt, s0;
-            chunk_of(k, t0, cnt, s0);
-            uint32_t *dst = reinterpret_cast<uint32_t *>(sm + kOffDtBuf) + (k & 1) * kQ;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int j = 4 * lane + i;
-                if (j < cnt) {
-                    const int s = s0 + j;
-                    const int tok = rev ? L - 1 - s : s;
-                    const __nv_bfloat16 *src = p.dt + ((size_t)b * L + tok) * H + hp * kHeads;
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
-                                 :: "r"(tc::smem_u32(dst + j)), "l"(src) : "memory");
-                } else {
-                    dst[j] = 0u;
-                }
-            }
-            asm volatile("cp.async.commit_group;" ::: "memory");
-        };
-        // warp 0: inclusive prefix sums of dt*A of both heads for walk chunk
-        // k (its dt copies must have landed), in log2 units (A carries the
-        // factor log2(e)) so that every decay factor is one 2^x on the
-        // special-function unit
-        auto scan_dt = [&](int k) {
-            asm volatile("cp.async.wait_all;" ::: "memory");
-            const __nv_bfloat162 *src =
-                reinterpret_cast<const __nv_bfloat162 *>(sm + kOffDtBuf) + (k & 1) * kQ + 4 * lane;
-#pragma unroll
-            for (int head = 0; head < kHeads; ++head) {
-                float d[4], a[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __bfloat1622float2(src[i]);
-                    d[i] = head ? f.y : f.x;
-                }
-                const float Aw = head ? A1 : A0;
-                a[0] = d[0] * Aw;
-#pragma unroll
-                for (int i = 1; i < 4; ++i) a[i] = fmaf(d[i], Aw, a[i - 1]);
-                float run = a[3];
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, run, o);
-                    if (lane >= o) run += v;
-                }
-                const float excl = run - a[3];
-                *reinterpret_cast<float4 *>(dts + head * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
-                *reinterpret_cast<float4 *>(cum + head * kQ + 4 * lane) =
-                    make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
-            }
-        };
-        // threads 0..255: per-slot decay factors of the chunk whose cum/dts are set
-        auto slot_factors = [&]() {
+        // threads 0..255: per-slot decay factors of walk chunk k
+        auto slot_factors = [&](int k) {
             if (tid < kHeads * kQ) {
                 const int head = tid >> 7, s = tid & 127;
-                const float cs = cum[head * kQ + s];
-                const float d = dts[head * kQ + s];
-                fB[head * kQ + s] = tc::exp2_approx(cum[head * kQ + (s | 31)] - cs) * d;
-                wgt[head * kQ + s] = tc::exp2_approx(cum[head * kQ + kQ - 1] - cs) * d;
+                const float *ck = cum + ((k & 1) * kHeads + head) * kQ;
+                const float cs = ck[s];
+                const float d = dts[((k & 1) * kHeads + head) * kQ + s];
+                fB[head * kQ + s] = tc::exp2_approx(ck[s | 31] - cs) * d;
+                wgt[head * kQ + s] = tc::exp2_approx(ck[kQ - 1] - cs) * d;
             }
         };
         // conv+SiLU of both heads' x for walk chunk k, in place: the raw
@@ -564,20 +601,21 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 *reinterpret_cast<uint4 *>(sm + kOffXw + off) = pack8(v);
             }
         };
-        // one thread polls an mbarrier; the group barrier releases the rest
-        auto wait_all = [&](uint32_t mb, uint32_t parity) -> bool {
+        // one thread polls an mbarrier (two if mb2 != 0); the group barrier
+        // releases the rest
+        auto wait_all = [&](uint32_t mb, uint32_t parity, uint32_t mb2 = 0, uint32_t parity2 = 0) -> bool {
             bool w = true;
-            if (tid == 0) w = tc::mbar_wait_bounded(mb, parity, kWaitCycles);
+            if (tid == 0) {
+                w = tc::mbar_wait_bounded(mb, parity, kWaitCycles);
+                if (w && mb2) w = tc::mbar_wait_bounded(mb2, parity2, kWaitCycles);
+            }
             return alu_sync_and(w);
         };
 
-        if (warp == 0) {
-            load_dt_async(0);
-            scan_dt(0);
-            if (nk > 1) load_dt_async(1);
-        }
-        alu_sync();
-        slot_factors();
+        uint32_t mbd, pard;
+        dt_ready(0, mbd, pard);
+        bool ok = wait_all(mbd, pard);   // chunk 0's prefix sums
+        slot_factors(0);
 
         // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg.
         // A segment's entering state: the caller's initial state (forward
@@ -610,7 +648,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         const float Dh = p.D[head_g];
 
         int arrival = 0;   // result of this chunk's arrival atomic (thread kArriveTid)
-        bool ok = wait_all(mb_x0, 0);
+        ok = ok && wait_all(mb_x0, 0);
         if (ok) {
             // decode: the conv history before token 0 comes from the cached tail
             if (!rev && p.tail && k0 == 0) {
@@ -646,9 +684,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 if (!ok) break;
             }
             tc::fence_after_sync();
-            const float ct = cum[hh * kQ + row];            // kept for the epilogue
-            const float a_last = tc::exp2_approx(cum[hh * kQ + kQ - 1]);
-            if constexpr (kStateOnly) dec += cum[hh * kQ + kQ - 1];
+            const float *cumk = cum + ((k & 1) * kHeads + hh) * kQ;   // this chunk, this head
+            const float *dtsk = dts + ((k & 1) * kHeads + hh) * kQ;
+            const float ct = cumk[row];                     // kept for the epilogue
+            const float a_last = tc::exp2_approx(cumk[kQ - 1]);
+            if constexpr (kStateOnly) dec += cumk[kQ - 1];
             {
                 const uint32_t gc = gcol(k), mc = mcol(k);
                 if constexpr (!kStateOnly) {
@@ -665,15 +705,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                             const float *fbh = fB + hh * kQ + 32 * jb;
                             if (jb < quad) {
                                 // whole block below the diagonal: factorised decay
-                                const float et = tc::exp2_approx(ct - cum[hh * kQ + 32 * jb + 31]);
+                                const float et = tc::exp2_approx(ct - cumk[32 * jb + 31]);
 #pragma unroll
                                 for (int i = 0; i < 16; ++i)
                                     packed[i] = tc::pack_bf16x2(gv[2 * i] * et * fbh[2 * i],
                                                                 gv[2 * i + 1] * et * fbh[2 * i + 1]);
                             } else {
                                 // diagonal block: one exponential per element, D on the diagonal
-                                const float *ch_ = cum + hh * kQ + 32 * jb;
-                                const float *dh_ = dts + hh * kQ + 32 * jb;
+                                const float *ch_ = cumk + 32 * jb;
+                                const float *dh_ = dtsk + 32 * jb;
                                 const int r31 = row & 31;
                                 float m[32];
 #pragma unroll
@@ -712,21 +752,19 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             alu_sync();
             if (tid == 0) tc::mbar_arrive(mb_m);    // the producer issues the MMAs
 
-            // ---- while the MMAs run: next chunk's dt prefix sums and conv
-            if (warp == 0 && more) {
-                scan_dt(k + 1);                       // its copies were issued a chunk ago
-                if (k + 2 < nk) load_dt_async(k + 2);
-            }
+            // ---- while the MMAs run: the next chunk's conv
             if (more) {
                 ok = wait_all(mb_x0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
                 if (!ok) break;
                 conv_chunk(k + 1);
             }
             if (!kStateOnly && tid == kArriveTid) *flag_slot = arrival;
-            ok = wait_all(mb_e, k & 1);
+            // the chunk's MMAs done, and (producer) the next chunk's prefix sums
+            dt_ready(k + 1, mbd, pard);
+            ok = more ? wait_all(mb_e, k & 1, mbd, pard) : wait_all(mb_e, k & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            if (more) slot_factors();                          // next chunk's fB, w
+            if (more) slot_factors(k + 1);                     // next chunk's fB, w
             if constexpr (kStateOnly) {
                 alu_sync();   // publishes the next chunk's factors
                 if (more) weight_chunk(k + 1);
