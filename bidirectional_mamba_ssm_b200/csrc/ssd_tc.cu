@@ -84,8 +84,8 @@ constexpr uint32_t kOffFB = kOffDt + 2048;       // f32[2][128] exp(c_R - c_s) d
 constexpr uint32_t kOffWgt = kOffFB + 1024;      // f32[2][128] exp(c_last - c_s) dt_s
 constexpr uint32_t kOffConvW = kOffWgt + 1024;   // float4[128] conv taps of x
 constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
-constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x8 (see the kernel)
-constexpr uint32_t kOffTmem = kOffMbar + 64;     // u32 TMEM base
+constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x10 + 2 flag pointers (see the kernel)
+constexpr uint32_t kOffTmem = kOffMbar + 96;     // u32 TMEM base
 constexpr uint32_t kOffFlag = kOffTmem + 4;      // i32 handshake result
 constexpr uint32_t kOffDtBuf = kOffFlag + 12;    // [2][128] bf16x2: dt of both heads, by cp.async
 constexpr uint32_t kSmemUsed = kOffDtBuf + 2 * kQ * 4;
@@ -288,6 +288,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     const uint32_t mb_m = sbase + kOffMbar + 32;
     const uint32_t mb_e = sbase + kOffMbar + 40;
     const uint32_t mb_dt0 = sbase + kOffMbar + 48;   // + 8 * (chunk & 1)
+    // a chunk's output rows stored (even / odd walk chunk), and the handshake
+    // flag the producer then raises for it (null: nothing to publish)
+    const uint32_t mb_rows0 = sbase + kOffMbar + 64;
+    int **rel_flag = reinterpret_cast<int **>(sm + kOffMbar + 80);
     auto dt_ready = [&](int k, uint32_t &mb, uint32_t &parity) {
         mb = mb_dt0 + 8 * (k & 1);
         parity = (k >> 1) & 1;
@@ -410,6 +414,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         tc::mbar_init(mb_e, 1);
         tc::mbar_init(mb_dt0, 32);       // every producer lane arrives after its part of a scan
         tc::mbar_init(mb_dt0 + 8, 32);
+        tc::mbar_init(mb_rows0, 1);
+        tc::mbar_init(mb_rows0 + 8, 1);
         issue_x(0);
         if (nk > 1) issue_x(1);
         issue_bc(0);
@@ -438,6 +444,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         constexpr uint32_t idYd = tc::idesc_bf16(128, 64, 0, 1);
         constexpr uint32_t idYo = tc::idesc_bf16(128, 128, 0, 1);
         constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
+        // lane 0: once chunk j's rows are stored, publish them to the partner
+        // CTA if this CTA arrived first (GPU-scope release; the rows were
+        // made visible to this thread through the group barrier and the
+        // mbarrier).  Done here so that the compute group never waits on it.
+        auto release_rows = [&](int j) -> bool {
+            const bool w = tc::mbar_wait_bounded(mb_rows0 + 8 * (j & 1), (j >> 1) & 1, kWaitCycles);
+            if (w) {
+                int *f = rel_flag[j & 1];
+                if (f) st_release(f, 1);
+            }
+            return w;
+        };
         bool pok = true;
         for (int k = 0; k < nk && pok; ++k) {
             const uint32_t g = tmem + gcol(k);
@@ -468,8 +486,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 tc::mbar_arrive(mb_dt0 + 8 * ((k + 1) & 1));
             }
             if (lane == 0) {
+                if (!kStateOnly && k > 0) pok = release_rows(k - 1);
                 // Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
-                pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
+                if (pok) pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
                 if (pok) {
                     tc::fence_after_sync();
                     if constexpr (!kStateOnly) {
@@ -509,6 +528,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             }
             pok = __shfl_sync(0xffffffffu, pok, 0);
         }
+        if (!kStateOnly && lane == 0 && pok && nk > 0) pok = release_rows(nk - 1);
         if (lane == 0 && !pok) record_error(p.status, kStatusTimeout);
     } else {
         // ================= compute group: 512 threads ======================
@@ -839,15 +859,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                     *ypiece(r) = v;
                 }
             }
-            if (first) {
-                alu_sync();
-                if (tid == 0) st_release(fl + 1, 1);
-            } else {
-                alu_sync();   // the staging buffer is rewritten by the next chunk's phase D
-                if (tid == 0) {
+            alu_sync();   // rows stored; the staging buffer is rewritten by the next chunk's phase D
+            if (tid == 0) {
+                if (!first) {
                     fl[0] = 0;   // leave the workspace zeroed for the next call
                     fl[1] = 0;
                 }
+                rel_flag[k & 1] = first ? fl + 1 : nullptr;
+                tc::mbar_arrive(mb_rows0 + 8 * (k & 1));   // the producer publishes them
             }
         }
 
