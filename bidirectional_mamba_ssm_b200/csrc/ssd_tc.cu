@@ -64,7 +64,8 @@ constexpr int kPP = kHeads * kP;   // x channels per CTA (128)
 constexpr int kAluThreads = 512;          // compute group (16 warps)
 constexpr int kProducerWarp = 16;         // issues every MMA and TMA load
 constexpr int kProducerTid = 32 * kProducerWarp;
-constexpr int kThreads = kAluThreads + 32;
+constexpr int kHelperWarp = 17;           // dt copies, prefix sums, slot factors
+constexpr int kThreads = kAluThreads + 64;
 constexpr int kBC = 2 * kN;   // B and C channels
 constexpr int kRawRows = kQ + 3;   // raw x rows per chunk: 128 slots + 3-token conv halo
 constexpr uint32_t kTmemCols = 512;
@@ -80,12 +81,12 @@ constexpr uint32_t kOffS = kOffXw + 32768;               // S^T bf16 [n][p'] 2 x
 constexpr uint32_t kRawBytes = kRawRows * kPP * 2;       // 33536
 constexpr uint32_t kOffCum = kOffS + 32768;      // f32[2][2][128] prefix sums of dt*A (chunk parity, head)
 constexpr uint32_t kOffDt = kOffCum + 2048;      // f32[2][2][128] dt
-constexpr uint32_t kOffFB = kOffDt + 2048;       // f32[2][128] exp(c_R - c_s) dt_s, R = block end
-constexpr uint32_t kOffWgt = kOffFB + 1024;      // f32[2][128] exp(c_last - c_s) dt_s
-constexpr uint32_t kOffConvW = kOffWgt + 1024;   // float4[128] conv taps of x
+constexpr uint32_t kOffFB = kOffDt + 2048;       // f32[2][2][128] exp(c_R - c_s) dt_s, R = block end
+constexpr uint32_t kOffWgt = kOffFB + 2048;      // f32[2][2][128] exp(c_last - c_s) dt_s
+constexpr uint32_t kOffConvW = kOffWgt + 2048;   // float4[128] conv taps of x
 constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
-constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x10 + 2 flag pointers (see the kernel)
-constexpr uint32_t kOffTmem = kOffMbar + 96;     // u32 TMEM base
+constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x12 + 2 flag pointers (see the kernel)
+constexpr uint32_t kOffTmem = kOffMbar + 112;    // u32 TMEM base
 constexpr uint32_t kOffFlag = kOffTmem + 4;      // i32 handshake result
 constexpr uint32_t kOffDtBuf = kOffFlag + 12;    // [2][128] bf16x2: dt of both heads, by cp.async
 constexpr uint32_t kSmemUsed = kOffDtBuf + 2 * kQ * 4;
@@ -292,6 +293,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     // flag the producer then raises for it (null: nothing to publish)
     const uint32_t mb_rows0 = sbase + kOffMbar + 64;
     int **rel_flag = reinterpret_cast<int **>(sm + kOffMbar + 80);
+    // phase D of an even / odd walk chunk done: its cum/dts/fB buffer is free
+    const uint32_t mb_free0 = sbase + kOffMbar + 96;
     auto dt_ready = [&](int k, uint32_t &mb, uint32_t &parity) {
         mb = mb_dt0 + 8 * (k & 1);
         parity = (k >> 1) & 1;
@@ -334,7 +337,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     constexpr float kLog2e = 1.4426950408889634f;
     const float A0 = p.A[hp * kHeads] * kLog2e, A1 = p.A[hp * kHeads + 1] * kLog2e;
 
-    // producer warp: asynchronous copy of walk chunk k's dt (both heads of
+    // helper warp: asynchronous copy of walk chunk k's dt (both heads of
     // the pair are adjacent: one 4-byte copy per token) into dt buffer
     // k % 2; slots past the chunk end are zero.
     auto load_dt_async = [&](int k) {
@@ -356,11 +359,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    // producer warp: inclusive prefix sums of dt*A of both heads for walk
+    // helper warp: inclusive prefix sums of dt*A of both heads for walk
     // chunk k into cum/dts buffer k % 2, in log2 units (A carries the factor
     // log2(e)) so that every decay factor is one 2^x on the special-function
-    // unit.  Waits for this thread's outstanding dt copies, which are chunk
-    // k's (and, before the first chunk, chunk 1's).
+    // unit, then the chunk's per-slot factors.  Waits for this thread's
+    // outstanding dt copies (chunk k's and, if issued, chunk k+1's).
     auto scan_dt = [&](int k) {
         asm volatile("cp.async.wait_all;" ::: "memory");
         const __nv_bfloat162 *src =
@@ -390,6 +393,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             *reinterpret_cast<float4 *>(cb) =
                 make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
         }
+        // per-slot decay factors, from the sums the other lanes just wrote:
+        // fB = exp(c_R - c_s) dt_s (R = end of s's 32-slot block) and
+        // w = exp(c_last - c_s) dt_s
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kHeads * kQ / 32; ++i) {
+            const int e = (k & 1) * kHeads * kQ + 32 * i + lane;   // [parity][head][slot]
+            const float cs = cum[e];
+            const float d = dts[e];
+            fB[e] = tc::exp2_approx(cum[e | 31] - cs) * d;
+            wgt[e] = tc::exp2_approx(cum[e | (kQ - 1)] - cs) * d;
+        }
     };
 
     // ---- setup (all threads)
@@ -412,8 +427,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         tc::mbar_init(mb_g, 1);
         tc::mbar_init(mb_m, 1);
         tc::mbar_init(mb_e, 1);
-        tc::mbar_init(mb_dt0, 32);       // every producer lane arrives after its part of a scan
+        tc::mbar_init(mb_dt0, 32);       // every helper lane arrives after its part of a scan
         tc::mbar_init(mb_dt0 + 8, 32);
+        tc::mbar_init(mb_free0, 1);
+        tc::mbar_init(mb_free0 + 8, 1);
         tc::mbar_init(mb_rows0, 1);
         tc::mbar_init(mb_rows0 + 8, 1);
         issue_x(0);
@@ -426,13 +443,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kOffTmem);
 
     if (warp == kProducerWarp) {
-        // ================= producer: every MMA and every TMA load (lane 0),
-        // and each chunk's dt prefix sums (whole warp), computed while the
-        // compute group builds the previous chunk's M
-        load_dt_async(0);
-        if (nk > 1) load_dt_async(1);
-        scan_dt(0);
-        tc::mbar_arrive(mb_dt0);
+        // ================= producer: every MMA and every TMA load, and the
+        // release of each chunk's rows (lane 0)
         const uint64_t dC = tc::smem_desc(sbase + kOffC, 16, 1024);       // K-major A (G, Yo)
         const uint64_t dB = tc::smem_desc(sbase + kOffB, 16, 1024);       // K-major B (G)
         const uint64_t dBmn = tc::smem_desc(sbase + kOffB, 16384, 1024);  // MN-major A (state)
@@ -476,17 +488,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                     }
                 }
             }
-            pok = __shfl_sync(0xffffffffu, pok, 0);
-            if (!pok) break;
-            // while the compute group builds M(k): the next chunk's dt prefix
-            // sums (buffer (k+1) % 2, last read for chunk k-1)
-            if (k + 1 < nk) {
-                scan_dt(k + 1);
-                if (k + 2 < nk) load_dt_async(k + 2);
-                tc::mbar_arrive(mb_dt0 + 8 * ((k + 1) & 1));
-            }
             if (lane == 0) {
-                if (!kStateOnly && k > 0) pok = release_rows(k - 1);
+                if (!kStateOnly && k > 0 && pok) pok = release_rows(k - 1);
                 // Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
                 if (pok) pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
                 if (pok) {
@@ -530,6 +533,26 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         }
         if (!kStateOnly && lane == 0 && pok && nk > 0) pok = release_rows(nk - 1);
         if (lane == 0 && !pok) record_error(p.status, kStatusTimeout);
+    } else if (warp == kHelperWarp) {
+        // ================= helper: dt copies, prefix sums and slot factors
+        // of each chunk, up to two chunks ahead of phase D
+        load_dt_async(0);
+        if (nk > 1) load_dt_async(1);
+        bool hok = true;
+        for (int j = 0; j < nk; ++j) {
+            if (j >= 2) {
+                // buffer j % 2 last held chunk j-2, read up to its phase D
+                if (lane == 0)
+                    hok = tc::mbar_wait_bounded(mb_free0 + 8 * (j & 1), ((j >> 1) - 1) & 1, kWaitCycles);
+                hok = __shfl_sync(0xffffffffu, hok, 0);
+                if (!hok) break;
+            }
+            scan_dt(j);
+            if (j + 2 < nk) load_dt_async(j + 2);
+            tc::mbar_arrive(mb_dt0 + 8 * (j & 1));
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (lane == 0 && !hok) record_error(p.status, kStatusTimeout);
     } else {
         // ================= compute group: 512 threads ======================
         // thread roles: row = TMEM lane / tile row; rg = 32-column group of
@@ -540,17 +563,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         const int hsub = rg & 1;
         const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         const int quad = warp & 3;
-        // threads 0..255: per-slot decay factors of walk chunk k
-        auto slot_factors = [&](int k) {
-            if (tid < kHeads * kQ) {
-                const int head = tid >> 7, s = tid & 127;
-                const float *ck = cum + ((k & 1) * kHeads + head) * kQ;
-                const float cs = ck[s];
-                const float d = dts[((k & 1) * kHeads + head) * kQ + s];
-                fB[head * kQ + s] = tc::exp2_approx(ck[s | 31] - cs) * d;
-                wgt[head * kQ + s] = tc::exp2_approx(ck[kQ - 1] - cs) * d;
-            }
-        };
         // conv+SiLU of both heads' x for walk chunk k, in place: the raw
         // rows in x buffer k % 2 become the swizzled X tile of the chunk.
         // Thread: 8 channels (group g: head g >> 3, piece g & 7) x 4 slots.
@@ -610,7 +622,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             const uint8_t *xt = sm + xbuf_off(k);
             const int j = tid & 127, q4 = tid >> 7;   // slot, quarter of the 128 columns
             const int gh = q4 >> 1;
-            const float wj = wgt[gh * kQ + j];
+            const float wj = wgt[((k & 1) * kHeads + gh) * kQ + j];
 #pragma unroll
             for (int pc = 0; pc < 4; ++pc) {
                 const uint32_t off = gh * 16384 + tc::sw128(j, 4 * (q4 & 1) + pc);
@@ -634,8 +646,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
 
         uint32_t mbd, pard;
         dt_ready(0, mbd, pard);
-        bool ok = wait_all(mbd, pard);   // chunk 0's prefix sums
-        slot_factors(0);
+        bool ok = wait_all(mbd, pard);   // chunk 0's prefix sums and slot factors
 
         // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg.
         // A segment's entering state: the caller's initial state (forward
@@ -722,7 +733,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                         } else {
                             float gv[32];
                             tc::tmem_ld32(tmem + lane_base + gc + 32 * jb, gv);
-                            const float *fbh = fB + hh * kQ + 32 * jb;
+                            const float *fbh = fB + ((k & 1) * kHeads + hh) * kQ + 32 * jb;
                             if (jb < quad) {
                                 // whole block below the diagonal: factorised decay
                                 const float et = tc::exp2_approx(ct - cumk[32 * jb + 31]);
@@ -770,7 +781,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             tc::fence_proxy_async();
             tc::fence_before_sync();
             alu_sync();
-            if (tid == 0) tc::mbar_arrive(mb_m);    // the producer issues the MMAs
+            if (tid == 0) {
+                tc::mbar_arrive(mb_m);                  // the producer issues the MMAs
+                tc::mbar_arrive(mb_free0 + 8 * (k & 1));   // the helper may reuse this chunk's buffers
+            }
 
             // ---- while the MMAs run: the next chunk's conv
             if (more) {
@@ -779,14 +793,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 conv_chunk(k + 1);
             }
             if (!kStateOnly && tid == kArriveTid) *flag_slot = arrival;
-            // the chunk's MMAs done, and (producer) the next chunk's prefix sums
+            // the chunk's MMAs done, and (helper) the next chunk's prefix sums
+            // and slot factors
             dt_ready(k + 1, mbd, pard);
             ok = more ? wait_all(mb_e, k & 1, mbd, pard) : wait_all(mb_e, k & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            if (more) slot_factors(k + 1);                     // next chunk's fB, w
             if constexpr (kStateOnly) {
-                alu_sync();   // publishes the next chunk's factors
                 if (more) weight_chunk(k + 1);
                 continue;
             }
@@ -806,7 +819,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 }
                 if (!ready) record_error(p.status, kStatusTimeout);
             }
-            alu_sync();   // also publishes the next chunk's factors
+            alu_sync();   // releases the group after thread 0's wait for the partner
             // the next chunk's wX first, while the partner's rows can be fetched
             if (more) weight_chunk(k + 1);
             // Coalesced output: each thread stages its 32 outputs in shared
