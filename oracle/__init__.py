@@ -56,6 +56,7 @@ def _load():
                                            i, i, i, i, i, i, i, dp, dp, dp, dp]
             lib.oracle_block_decode.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp,
                                                 i, i, i, i, i, i, i, dp, dp, dp]
+            lib.oracle_bimamba_untied.argtypes = [dp] * 13 + [i] * 8 + [dp, dp]
             _lib = lib
     return _lib
 
@@ -147,6 +148,32 @@ def bimamba(xbc, dt, A, D, conv_w=None, conv_b=None, *, heads, headdim, d_state,
     if want_dirs:
         out.append((yf, yr))
     return out[0] if len(out) == 1 else tuple(out)
+
+
+def bimamba_untied(xbc_f, xbc_r, dt_f, dt_r, A_f, A_r, D_f, D_r, conv_w_f=None, conv_w_r=None,
+                   conv_b_f=None, conv_b_r=None, *, heads, headdim, d_state, ngroups=1,
+                   init=None, concat=False, want_final=False):
+    """Untied directions: each stream with its own parameters, outputs summed
+    (y: (batch, len, H*P)) or concatenated per token as [forward | reverse]
+    (y: (batch, len, 2*H*P)).  Returns y [, forward final state]."""
+    lib = _load()
+    (xbc_f, xbc_r, dt_f, dt_r, A_f, A_r, D_f, D_r, conv_w_f, conv_w_r, conv_b_f, conv_b_r,
+     init) = map(_f64, (xbc_f, xbc_r, dt_f, dt_r, A_f, A_r, D_f, D_r, conv_w_f, conv_w_r,
+                        conv_b_f, conv_b_r, init))
+    bsz, L, ch = xbc_f.shape
+    H, P, N, G = heads, headdim, d_state, ngroups
+    assert ch == H * P + 2 * G * N and xbc_r.shape == xbc_f.shape
+    K = 4
+    for w in (conv_w_f, conv_w_r):
+        if w is not None:
+            K = w.shape[1]
+    y = np.empty((bsz, L, (2 if concat else 1) * H * P))
+    fin = np.empty((bsz, H, P, N)) if want_final else None
+    lib.oracle_bimamba_untied(_ptr(xbc_f), _ptr(xbc_r), _ptr(dt_f), _ptr(dt_r), _ptr(A_f),
+                              _ptr(A_r), _ptr(D_f), _ptr(D_r), _ptr(conv_w_f), _ptr(conv_w_r),
+                              _ptr(conv_b_f), _ptr(conv_b_r), _ptr(init), bsz, L, H, P, N, G, K,
+                              int(bool(concat)), _ptr(y), _ptr(fin))
+    return (y, fin) if want_final else y
 
 
 def block_decode(block, dt, A, D, conv_w, conv_b, state, tail, *, heads, headdim,

@@ -261,3 +261,68 @@ void oracle_block_decode(const double *block, const double *dt, const double *A,
         }
     }
 }
+
+/*
+ * Untied directions.  The blog post "DiffuMamba" (metaphor-xennon),
+ * network-architecture listing, builds the bidirectional mixer from two
+ * separate Mamba modules: one reads the sequence as it is, the other reads
+ * it reversed and its output is reversed back; the two outputs are
+ * concatenated and a Linear layer maps 2d back to d.  The technical
+ * summaries (section 2) combine the two streams by addition instead.  This
+ * function gives each stream its own parameters and offers both fusions:
+ *   *_f, *_r : forward / reverse stream inputs and parameters (xbc, dt, A,
+ *              D, conv taps, conv bias), shaped as in oracle_bimamba
+ *   init     : (batch, H, P, N) or NULL -- forward initial state
+ *   concat   : 0 -> y (batch, len, H*P) = forward + reverse
+ *              1 -> y (batch, len, 2*H*P), per token [forward | reverse]
+ *              (the Linear after the concatenation is not part of the scan)
+ *   fin      : (batch, H, P, N) or NULL -- forward final state
+ * Each stream is exactly the corresponding stream of oracle_bimamba run
+ * with that stream's parameters.
+ */
+void oracle_bimamba_untied(const double *xbc_f, const double *xbc_r,
+                           const double *dt_f, const double *dt_r,
+                           const double *A_f, const double *A_r,
+                           const double *D_f, const double *D_r,
+                           const double *conv_w_f, const double *conv_w_r,
+                           const double *conv_b_f, const double *conv_b_r,
+                           const double *init, int batch, int len, int H,
+                           int P, int N, int G, int K, int concat, double *y,
+                           double *fin)
+{
+    int ch = H * P + 2 * G * N;
+    size_t nt = (size_t)batch * len;
+    size_t hp = (size_t)H * P;
+    double *act = (double *)malloc(sizeof(double) * nt * ch);
+    double *x = (double *)malloc(sizeof(double) * nt * hp);
+    double *Bm = (double *)malloc(sizeof(double) * nt * G * N);
+    double *Cm = (double *)malloc(sizeof(double) * nt * G * N);
+    double *of = (double *)malloc(sizeof(double) * nt * hp);
+    double *orv = (double *)malloc(sizeof(double) * nt * hp);
+
+    /* forward stream, forward parameters */
+    if (conv_w_f)
+        oracle_conv(xbc_f, conv_w_f, conv_b_f, NULL, batch, len, ch, K, 0, 1, act);
+    else
+        memcpy(act, xbc_f, sizeof(double) * nt * ch);
+    split_xbc(act, batch, len, H, P, N, G, x, Bm, Cm);
+    oracle_scan(x, Bm, Cm, dt_f, A_f, D_f, init, batch, len, H, P, N, G, 0, of, fin);
+
+    /* reverse stream, reverse parameters: mirrored conv, zero state */
+    if (conv_w_r)
+        oracle_conv(xbc_r, conv_w_r, conv_b_r, NULL, batch, len, ch, K, 1, 1, act);
+    else
+        memcpy(act, xbc_r, sizeof(double) * nt * ch);
+    split_xbc(act, batch, len, H, P, N, G, x, Bm, Cm);
+    oracle_scan(x, Bm, Cm, dt_r, A_r, D_r, NULL, batch, len, H, P, N, G, 1, orv, NULL);
+
+    for (size_t r = 0; r < nt; ++r) {
+        if (concat) {
+            memcpy(y + r * 2 * hp, of + r * hp, sizeof(double) * hp);
+            memcpy(y + r * 2 * hp + hp, orv + r * hp, sizeof(double) * hp);
+        } else {
+            for (size_t i = 0; i < hp; ++i) y[r * hp + i] = of[r * hp + i] + orv[r * hp + i];
+        }
+    }
+    free(act); free(x); free(Bm); free(Cm); free(of); free(orv);
+}

@@ -302,3 +302,92 @@ def test_decode_golden_scalar():
     y = oracle.bimamba(u, one, np.array([-math.log(2.0)]), np.array([0.0]),
                        heads=1, headdim=1, d_state=1, init=np.full((1, 1, 1, 1), 2.5))
     assert abs(y.ravel()[0] - 7.25) < 1e-14
+
+
+# ------------------------------------------------------- untied directions
+def _brute_force_dir(x, B, C, dt, A, D, reverse):
+    """One direction of the materialised quadratic form (no conv):
+    forward  M[t,s] = (C_t . B_s) exp(A sum_{r=s+1..t} dt_r) dt_s   (s <= t)
+    reverse  M[t,s] = (C_t . B_s) exp(A sum_{r=t..s-1} dt_r) dt_s   (s >= t)
+    y = M x + D x.  Explicit double loops, independent of the recurrence."""
+    bsz, L, H, P = x.shape
+    G = B.shape[2]
+    hpg = H // G
+    y = np.zeros_like(x)
+    for b in range(bsz):
+        for h in range(H):
+            g = h // hpg
+            CB = C[b, :, g, :] @ B[b, :, g, :].T
+            M = np.zeros((L, L))
+            for t in range(L):
+                for s in range(L):
+                    if not reverse and s <= t:
+                        M[t, s] = CB[t, s] * math.exp(A[h] * dt[b, s + 1:t + 1, h].sum()) * dt[b, s, h]
+                    if reverse and s >= t:
+                        M[t, s] = CB[t, s] * math.exp(A[h] * dt[b, t:s, h].sum()) * dt[b, s, h]
+            y[b, :, h, :] = M @ x[b, :, h, :] + D[h] * x[b, :, h, :]
+    return y
+
+
+@pytest.mark.parametrize("L,H,P,N,G", [(1, 1, 1, 1, 1), (9, 2, 3, 4, 1), (40, 4, 2, 5, 2)])
+@pytest.mark.parametrize("memory", ["short", "long"])
+@pytest.mark.parametrize("concat", [False, True])
+def test_untied_equals_quadratic_forms(L, H, P, N, G, memory, concat):
+    """Untied directions (separate x, B, C, dt, A, D per stream, as in the
+    blog's two-module listing): the sum, or the per-token concatenation
+    [forward | reverse], of two independently parameterised quadratic forms."""
+    rng = np.random.default_rng(L * 7 + H + 100 * concat)
+    a = (1.0, 16.0) if memory == "short" else (1e-3, 1e-2)
+    xf, Bf, Cf, dtf, Af, Df = _rand(rng, 2, L, H, P, N, G, *a)
+    xr, Br, Cr, dtr, Ar, Dr = _rand(rng, 2, L, H, P, N, G, *a)
+    y = oracle.bimamba_untied(_xbc(xf, Bf, Cf), _xbc(xr, Br, Cr), dtf, dtr, Af, Ar, Df, Dr,
+                              heads=H, headdim=P, d_state=N, ngroups=G, concat=concat)
+    yf = _brute_force_dir(xf, Bf, Cf, dtf, Af, Df, False).reshape(2, L, H * P)
+    yr = _brute_force_dir(xr, Br, Cr, dtr, Ar, Dr, True).reshape(2, L, H * P)
+    ref = np.concatenate([yf, yr], axis=-1) if concat else yf + yr
+    assert y.shape == ref.shape
+    assert np.max(np.abs(y - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_untied_with_equal_parameters_is_the_tied_mixer():
+    rng = np.random.default_rng(5)
+    L, H, P, N = 30, 2, 4, 8
+    x, B, C, dt, A, D = _rand(rng, 2, L, H, P, N)
+    u = _xbc(x, B, C)
+    ch = u.shape[-1]
+    w = rng.normal(0, 0.5, (ch, 4))
+    bias = rng.normal(0, 0.1, ch)
+    init = rng.normal(0, 0.3, (2, H, P, N))
+    ref, rfin = oracle.bimamba(u, dt, A, D, w, bias, heads=H, headdim=P, d_state=N, init=init,
+                               want_final=True, want_dirs=False)
+    y, fin = oracle.bimamba_untied(u, u, dt, dt, A, A, D, D, w, w, bias, bias, heads=H, headdim=P,
+                                   d_state=N, init=init, want_final=True)
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(fin, rfin, rtol=0, atol=1e-13)
+
+
+def test_untied_streams_read_only_their_own_parameters():
+    """Changing every reverse-stream input leaves the forward half of the
+    concatenation (and the forward final state) bit-identical, and the other
+    way round."""
+    rng = np.random.default_rng(8)
+    L, H, P, N = 25, 2, 3, 4
+    f = _rand(rng, 1, L, H, P, N)
+    r1 = _rand(rng, 1, L, H, P, N)
+    r2 = _rand(rng, 1, L, H, P, N)
+    ch = H * P + 2 * N
+    wf, w1, w2 = (rng.normal(0, 0.5, (ch, 4)) for _ in range(3))
+
+    def run(fp, rp, wr):
+        xf, Bf, Cf, dtf, Af, Df = fp
+        xr, Br, Cr, dtr, Ar, Dr = rp
+        return oracle.bimamba_untied(_xbc(xf, Bf, Cf), _xbc(xr, Br, Cr), dtf, dtr, Af, Ar, Df, Dr,
+                                     wf, wr, heads=H, headdim=P, d_state=N, concat=True,
+                                     want_final=True)
+    y1, fin1 = run(f, r1, w1)
+    y2, fin2 = run(f, r2, w2)
+    np.testing.assert_array_equal(y1[..., :H * P], y2[..., :H * P])
+    np.testing.assert_array_equal(fin1, fin2)
+    assert np.max(np.abs(y1[..., H * P:] - y2[..., H * P:])) > 1e-3
+    y3, _ = run(r1, r1, w1)
+    np.testing.assert_array_equal(y3[..., H * P:], y1[..., H * P:])
