@@ -43,7 +43,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer1p3b", "long131k", "decode"], default="layer1p3b")
+    ap.add_argument("--workload", choices=["layer1p3b", "long131k", "decode", "untied1p3b"],
+                    default="layer1p3b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--batch", type=int, default=None,
@@ -60,20 +61,23 @@ def workload_spec(name):
         return I.LONG_131K, 1, I.LONG_131K.seqlen
     if name == "decode":
         return I.LAYER_1P3B, I.DECODE_STREAMS, I.DECODE_BLOCK
+    if name == "untied1p3b":   # the same layer with untied directions, outputs concatenated
+        return I.LAYER_1P3B, I.LAYER_1P3B.batch, I.LAYER_1P3B.seqlen
     raise ValueError(name)
 
 
-def algorithmic(w, batch, seqlen, decode=False):
+def algorithmic(w, batch, seqlen, decode=False, untied=False):
     """Algorithmic bytes and flops of one step (definitions in the design doc).
 
     bytes/token = raw xBC in (H*P + 2N) + dt (H) + y out (H*P), in the
     activation dtype; decode adds the fp32 state read (H*P*N*4 per stream)
-    and the conv tail (4 tokens of xBC) per stream.
+    and the conv tail (4 tokens of xBC) per stream.  Untied directions read
+    both streams' xBC and dt and write both halves of the concatenated y.
     flops/token = 2*(2*Q*N + H*(Q*P + 4*P*N)) with Q = 64 fixed.
     """
     esz = 2 if w.dtype == "bf16" else 4
     H, P, N = w.heads, w.headdim, w.d_state
-    per_tok = esz * ((H * P + 2 * N) + H + H * P)
+    per_tok = esz * ((H * P + 2 * N) + H + H * P) * (2 if untied else 1)
     tokens = batch * seqlen
     nbytes = per_tok * tokens
     if decode:
@@ -180,15 +184,18 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     decode = args.workload == "decode"
+    untied = args.workload == "untied1p3b"
     w, batch, seqlen = workload_spec(args.workload)
     if args.batch is not None:
         batch = args.batch
     H, P, N = w.heads, w.headdim, w.d_state
 
-    # ---- inputs, generated on the device (seeded per rank)
+    # ---- inputs, generated on the device (seeded per rank); untied
+    # directions draw the reverse stream's inputs and parameters separately
     g = I.make_inputs(w, seed=rank, device=dev, seqlen=seqlen, batch=batch,
                       conv_bias=decode)
-    y = torch.empty((batch, seqlen, H * P), dtype=torch.bfloat16, device=dev)
+    gr = I.make_inputs(w, seed=10000 + rank, device=dev, seqlen=seqlen, batch=batch) if untied else None
+    y = torch.empty((batch, seqlen, (2 if untied else 1) * H * P), dtype=torch.bfloat16, device=dev)
     dims = lib.make_dims(batch, seqlen, H, P, N, torch.bfloat16)
     ws = lib.new_workspace(dims, device=dev)
     if decode:
@@ -209,6 +216,10 @@ def run_ours(args):
         def step():
             lib.bimamba_block_decode(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], g["conv_b"],
                                      state, tail, y, None, None, ws, heads=H, headdim=P, d_state=N)
+    elif untied:
+        def step():
+            lib.bimamba_ssd_fwd_rev_untied(g, gr, None, None, y, ws, heads=H, headdim=P,
+                                           d_state=N, concat=True)
     else:
         def step():
             lib.bimamba_ssd_fwd_rev(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], None, None,
@@ -266,7 +277,7 @@ def run_ours(args):
 
     # ---- roofline of the dominant kernel (the main scan kernel of each step)
     peaks, peak_kind = load_peaks()
-    nbytes, flops = algorithmic(w, batch, seqlen, decode)
+    nbytes, flops = algorithmic(w, batch, seqlen, decode, untied)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
     kernel_s = per_call_ms / 1e3
@@ -288,16 +299,16 @@ def run_ours(args):
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, locals().get("state"),
-                  locals().get("tail"), dev, world)
+                  locals().get("tail"), dev, world, gr)
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name if not decode else
-                   f"cached block decode: {batch} streams x {seqlen}-token block, "
-                   f"H64x64 N128 bf16, 65536-token prefix state",
+        "config": {"workload": (f"cached block decode: {batch} streams x {seqlen}-token block, "
+                                f"H64x64 N128 bf16, 65536-token prefix state") if decode else
+                   (w.name + ", untied directions, outputs concatenated") if untied else w.name,
                    "batch_per_gpu": batch, "seqlen": seqlen, "heads": H, "headdim": P,
                    "d_state": N, "state_dtype": "f32",
                    "l2": "inputs larger than L2 (xbc + y per step > 126 MB)" if not decode
@@ -315,7 +326,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, world):
+def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, world, gr=None):
     """Same metric through the public API from pinned HOST buffers.  Every step
     copies its inputs (xbc, dt) host->device, runs the call, and copies y back
     to the host.  Steps are pipelined the way a serving loop would run them:
@@ -323,12 +334,14 @@ def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, 
     streams with two device buffer sets, ordered by events."""
     import torch
     H, P, N = w.heads, w.headdim, w.d_state
-    hx = g["xbc"].cpu().pin_memory()
-    hdt = g["dt"].cpu().pin_memory()
-    hy = torch.empty((batch, seqlen, H * P), dtype=torch.bfloat16).pin_memory()
-    dx = [torch.empty_like(g["xbc"]) for _ in range(2)]
-    ddt = [torch.empty_like(g["dt"]) for _ in range(2)]
-    dy = [torch.empty((batch, seqlen, H * P), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    untied = gr is not None
+    # per-step inputs: xbc and dt of each stream (one stream when tied)
+    srcs = [g] + ([gr] if untied else [])
+    hin = [t.cpu().pin_memory() for d in srcs for t in (d["xbc"], d["dt"])]
+    ywidth = (2 if untied else 1) * H * P
+    hy = torch.empty((batch, seqlen, ywidth), dtype=torch.bfloat16).pin_memory()
+    din = [[torch.empty_like(t, device=dev) for t in hin] for _ in range(2)]
+    dy = [torch.empty((batch, seqlen, ywidth), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     wss = [ws, lib.new_workspace(dims, device=dev)]
     s_up, s_run, s_down = (torch.cuda.Stream(device=dev) for _ in range(3))
     up_done = [torch.cuda.Event() for _ in range(2)]
@@ -341,17 +354,23 @@ def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, 
         j = i & 1
         s_up.wait_event(run_done[j])            # buffers j free once step i-2 has run
         with torch.cuda.stream(s_up):
-            dx[j].copy_(hx, non_blocking=True)
-            ddt[j].copy_(hdt, non_blocking=True)
+            for dst, src in zip(din[j], hin):
+                dst.copy_(src, non_blocking=True)
         up_done[j].record(s_up)
         s_run.wait_event(up_done[j])
         s_run.wait_event(down_done[j])          # y buffer j read back by step i-2
+        dx, ddt = din[j][0], din[j][1]
         if decode:
-            lib.bimamba_block_decode(dx[j], ddt[j], g["A"], g["D"], g["conv_w"], g["conv_b"], state,
+            lib.bimamba_block_decode(dx, ddt, g["A"], g["D"], g["conv_w"], g["conv_b"], state,
                                      tail, dy[j], None, None, wss[j], heads=H, headdim=P, d_state=N,
                                      stream=s_run)
+        elif untied:
+            fwd = dict(g, xbc=dx, dt=ddt)
+            rev = dict(gr, xbc=din[j][2], dt=din[j][3])
+            lib.bimamba_ssd_fwd_rev_untied(fwd, rev, None, None, dy[j], wss[j], heads=H, headdim=P,
+                                           d_state=N, concat=True, stream=s_run)
         else:
-            lib.bimamba_ssd_fwd_rev(dx[j], ddt[j], g["A"], g["D"], g["conv_w"], None, None, None,
+            lib.bimamba_ssd_fwd_rev(dx, ddt, g["A"], g["D"], g["conv_w"], None, None, None,
                                     dy[j], wss[j], heads=H, headdim=P, d_state=N, stream=s_run)
         run_done[j].record(s_run)
         s_down.wait_event(run_done[j])
@@ -373,7 +392,7 @@ def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, 
     ms = a.elapsed_time(b) / args.e2e_steps
     from bidirectional_mamba_ssm_b200 import replicas
     _, ms, _ = replicas.aggregate(0, ms, device=dev)
-    h2d = hx.numel() * hx.element_size() + hdt.numel() * hdt.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in hin)
     d2h = hy.numel() * hy.element_size()
     return {"value": batch * seqlen * world / (ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
@@ -391,8 +410,14 @@ def oracle_sample_step(w, workload, seq_tokens, seed=0):
     cpu = I.make_inputs(w, seed=seed, seqlen=seq_tokens, batch=1, conv_bias=decode)
     n = {k: (None if v is None else v.float().double().numpy()) for k, v in cpu.items()}
     kw = dict(heads=w.heads, headdim=w.headdim, d_state=w.d_state)
+    if workload == "untied1p3b":
+        cr = I.make_inputs(w, seed=seed + 10000, seqlen=seq_tokens, batch=1)
+        r = {k: (None if v is None else v.float().double().numpy()) for k, v in cr.items()}
     t0 = time.perf_counter()
-    if decode:
+    if workload == "untied1p3b":
+        oracle.bimamba_untied(n["xbc"], r["xbc"], n["dt"], r["dt"], n["A"], r["A"], n["D"], r["D"],
+                              n["conv_w"], r["conv_w"], None, None, concat=True, **kw)
+    elif decode:
         state = np.zeros((1, w.heads, w.headdim, w.d_state))
         tail = np.zeros((1, 4, w.channels))
         oracle.block_decode(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], n["conv_b"], state,
@@ -440,7 +465,9 @@ def run_reference(args):
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name if args.workload != "decode" else "cached block decode",
+        "config": {"workload": {"decode": "cached block decode",
+                                "untied1p3b": w.name + ", untied directions, outputs concatenated"}
+                   .get(args.workload, w.name),
                    "batch_per_gpu": batch, "seqlen": seqlen, "heads": w.heads,
                    "headdim": w.headdim, "d_state": w.d_state},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",

@@ -24,6 +24,8 @@ BIMAMBA_ERR_TIMEOUT = 4
 BIMAMBA_ERR_WORKSPACE = 5
 BIMAMBA_F32 = 0
 BIMAMBA_BF16 = 1
+BIMAMBA_FUSE_SUM = 0
+BIMAMBA_FUSE_CONCAT = 1
 
 # every symbol include/bimamba.h declares
 EXPORTED = (
@@ -36,6 +38,7 @@ EXPORTED = (
     "bimamba_workspace_bytes",
     "bimamba_launch_plan",
     "bimamba_ssd_fwd_rev",
+    "bimamba_ssd_fwd_rev_untied",
     "bimamba_block_decode",
     "bimamba_noalloc_scratch_bytes",
     "bimamba_block_decode_noalloc",
@@ -79,6 +82,8 @@ def _load() -> ctypes.CDLL:
     lib.bimamba_launch_plan.argtypes = [dp, ctypes.POINTER(ctypes.c_int)]
     lib.bimamba_ssd_fwd_rev.restype = i
     lib.bimamba_ssd_fwd_rev.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.bimamba_ssd_fwd_rev_untied.restype = i
+    lib.bimamba_ssd_fwd_rev_untied.argtypes = [dp] + [vp] * 15 + [i, vp, sz, vp]
     lib.bimamba_block_decode.restype = i
     lib.bimamba_block_decode.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.bimamba_noalloc_scratch_bytes.restype = sz
@@ -199,6 +204,25 @@ def bimamba_ssd_fwd_rev(xbc, dt, A, D, conv_w, conv_b, init_state, final_state, 
                                   _ptr(conv_w), _ptr(conv_b), _ptr(init_state), _ptr(final_state),
                                   _ptr(y), _ptr(workspace), wsz, _stream(stream))
     _check(st, "bimamba_ssd_fwd_rev")
+    return y
+
+
+def bimamba_ssd_fwd_rev_untied(fwd, rev, init_state, final_state, y, workspace, *, heads,
+                               headdim, d_state, concat=False, ngroups=1, stream=None):
+    """Untied directions: `fwd` and `rev` are dicts with keys xbc, dt, A, D,
+    conv_w, conv_b (conv_w/conv_b may be None) holding each stream's own
+    inputs.  y = forward + reverse (concat=False, (batch, len, H*P)) or
+    per token [forward | reverse] (concat=True, (batch, len, 2*H*P))."""
+    bsz, L, _ = fwd["xbc"].shape
+    dims = make_dims(bsz, L, heads, headdim, d_state, _dtype_code(fwd["xbc"]), ngroups)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    g = lambda d, k: _ptr(d.get(k))
+    st = _lib.bimamba_ssd_fwd_rev_untied(
+        ctypes.byref(dims), g(fwd, "xbc"), g(rev, "xbc"), g(fwd, "dt"), g(rev, "dt"), g(fwd, "A"),
+        g(rev, "A"), g(fwd, "D"), g(rev, "D"), g(fwd, "conv_w"), g(rev, "conv_w"), g(fwd, "conv_b"),
+        g(rev, "conv_b"), _ptr(init_state), _ptr(final_state), _ptr(y),
+        BIMAMBA_FUSE_CONCAT if concat else BIMAMBA_FUSE_SUM, _ptr(workspace), wsz, _stream(stream))
+    _check(st, "bimamba_ssd_fwd_rev_untied")
     return y
 
 

@@ -161,9 +161,11 @@ int bimamba_launch_plan(const bimamba_dims *d, int *out)
     return BIMAMBA_OK;
 }
 
-// Shared by the full scan and the cached block decode.
-static int run_bimamba(const bimamba_dims *d, const void *xbc, const void *dt, const float *A,
-                       const float *D, const float *conv_w, const float *conv_b,
+// Shared by the full scan (tied or untied) and the cached block decode.
+// Index 0 of each pair is the forward stream's input, index 1 the reverse's.
+static int run_bimamba(const bimamba_dims *d, const void *const xbc[2], const void *const dt[2],
+                       const float *const A[2], const float *const D[2],
+                       const float *const conv_w[2], const float *const conv_b[2], int concat,
                        const void *tail, const float *init, float *fin, void *y,
                        void *workspace, size_t workspace_bytes, cudaStream_t s)
 {
@@ -172,12 +174,39 @@ static int run_bimamba(const bimamba_dims *d, const void *xbc, const void *dt, c
         return BIMAMBA_ERR_WORKSPACE;
     Problem pr{};
     pr.dims = *d;
-    pr.xbc = xbc; pr.dt = dt; pr.A = A; pr.D = D;
-    pr.conv_w = conv_w; pr.conv_b = conv_b; pr.tail = tail;
+    for (int i = 0; i < 2; ++i) {
+        pr.xbc[i] = xbc[i]; pr.dt[i] = dt[i]; pr.A[i] = A[i]; pr.D[i] = D[i];
+        pr.conv_w[i] = conv_w[i]; pr.conv_b[i] = conv_b[i];
+    }
+    pr.concat = concat;
+    pr.tail = tail;
     pr.init = init; pr.fin = fin; pr.y = y;
     pr.workspace = workspace; pr.workspace_bytes = workspace_bytes;
     pr.status = device_status_word();
     return cuda_status(launch_bimamba(pr, s));
+}
+
+static int run_tied(const bimamba_dims *d, const void *xbc, const void *dt, const float *A,
+                    const float *D, const float *conv_w, const float *conv_b, const void *tail,
+                    const float *init, float *fin, void *y, void *workspace,
+                    size_t workspace_bytes, cudaStream_t s)
+{
+    const void *x2[2] = {xbc, xbc}, *dt2[2] = {dt, dt};
+    const float *A2[2] = {A, A}, *D2[2] = {D, D}, *w2[2] = {conv_w, conv_w}, *b2[2] = {conv_b, conv_b};
+    return run_bimamba(d, x2, dt2, A2, D2, w2, b2, 0, tail, init, fin, y, workspace,
+                       workspace_bytes, s);
+}
+
+// Empty sequence: y is empty; the forward state passes through.
+static int pass_state_through(const bimamba_dims *d, const float *init_state, float *final_state,
+                              cudaStream_t s)
+{
+    const size_t state_bytes = sizeof(float) * (size_t)d->batch * d->heads * d->headdim * d->d_state;
+    if (!final_state || init_state == final_state) return BIMAMBA_OK;
+    cudaError_t e = init_state ? cudaMemcpyAsync(final_state, init_state, state_bytes,
+                                                 cudaMemcpyDeviceToDevice, s)
+                               : cudaMemsetAsync(final_state, 0, state_bytes, s);
+    return cuda_status(e);
 }
 
 int bimamba_ssd_fwd_rev(const bimamba_dims *d, const void *xbc, const void *dt, const float *A,
@@ -188,25 +217,43 @@ int bimamba_ssd_fwd_rev(const bimamba_dims *d, const void *xbc, const void *dt, 
     int st = check_dims(d);
     if (st != BIMAMBA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const size_t state_bytes = sizeof(float) * (size_t)d->batch * d->heads * d->headdim * d->d_state;
     if (d->batch == 0) return BIMAMBA_OK;
-    if (d->len == 0) {
-        // empty sequence: y is empty; the forward state passes through
-        if (!final_state) return BIMAMBA_OK;
-        if (init_state == final_state) return BIMAMBA_OK;
-        cudaError_t e = init_state
-                            ? cudaMemcpyAsync(final_state, init_state, state_bytes,
-                                              cudaMemcpyDeviceToDevice, s)
-                            : cudaMemsetAsync(final_state, 0, state_bytes, s);
-        return cuda_status(e);
-    }
+    if (d->len == 0) return pass_state_through(d, init_state, final_state, s);
     if (!xbc || !dt || !A || !D || !y) return BIMAMBA_ERR_INVALID;
     if (conv_b && !conv_w) return BIMAMBA_ERR_INVALID;
     const void *ptrs[] = {xbc, dt, A, D, y, conv_w, conv_b, init_state, final_state};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
-    return run_bimamba(d, xbc, dt, A, D, conv_w, conv_b, nullptr, init_state, final_state, y,
-                       workspace, workspace_bytes, s);
+    return run_tied(d, xbc, dt, A, D, conv_w, conv_b, nullptr, init_state, final_state, y,
+                    workspace, workspace_bytes, s);
+}
+
+int bimamba_ssd_fwd_rev_untied(const bimamba_dims *d, const void *xbc_f, const void *xbc_r,
+                               const void *dt_f, const void *dt_r, const float *A_f,
+                               const float *A_r, const float *D_f, const float *D_r,
+                               const float *conv_w_f, const float *conv_w_r,
+                               const float *conv_b_f, const float *conv_b_r,
+                               const float *init_state, float *final_state, void *y, int fusion,
+                               void *workspace, size_t workspace_bytes, bimamba_stream_t stream)
+{
+    int st = check_dims(d);
+    if (st != BIMAMBA_OK) return st;
+    if (fusion != BIMAMBA_FUSE_SUM && fusion != BIMAMBA_FUSE_CONCAT) return BIMAMBA_ERR_INVALID;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d->batch == 0) return BIMAMBA_OK;
+    if (d->len == 0) return pass_state_through(d, init_state, final_state, s);
+    if (!xbc_f || !xbc_r || !dt_f || !dt_r || !A_f || !A_r || !D_f || !D_r || !y)
+        return BIMAMBA_ERR_INVALID;
+    if ((conv_b_f && !conv_w_f) || (conv_b_r && !conv_w_r)) return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {xbc_f, xbc_r, dt_f, dt_r, A_f, A_r, D_f, D_r, y, conv_w_f, conv_w_r,
+                          conv_b_f, conv_b_r, init_state, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
+    const void *x2[2] = {xbc_f, xbc_r}, *dt2[2] = {dt_f, dt_r};
+    const float *A2[2] = {A_f, A_r}, *D2[2] = {D_f, D_r};
+    const float *w2[2] = {conv_w_f, conv_w_r}, *b2[2] = {conv_b_f, conv_b_r};
+    return run_bimamba(d, x2, dt2, A2, D2, w2, b2, fusion == BIMAMBA_FUSE_CONCAT, nullptr,
+                       init_state, final_state, y, workspace, workspace_bytes, s);
 }
 
 int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block, const void *dt_block,
@@ -231,8 +278,8 @@ int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block, const voi
         if (a < b + tail_bytes && b < a + tail_bytes) return BIMAMBA_ERR_INVALID;
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    st = run_bimamba(d, xbc_block, dt_block, A, D, conv_w, conv_b, tail, state, state_out, y,
-                     workspace, workspace_bytes, s);
+    st = run_tied(d, xbc_block, dt_block, A, D, conv_w, conv_b, tail, state, state_out, y,
+                  workspace, workspace_bytes, s);
     if (st != BIMAMBA_OK || !tail_out) return st;
     cudaError_t e = d->dtype == BIMAMBA_F32
                         ? launch_tail_commit<float>(xbc_block, tail, tail_out, d->batch, d->len, ch, s)

@@ -16,13 +16,8 @@ cudaError_t launch_bimamba(const Problem &p, cudaStream_t stream)
     // needs a 1e-4 bound that bf16 operands cannot hold) and other head
     // shapes run on the sequential fp32 kernel.
     if (tc_path_supported(d)) return launch_ssd_tc(p, stream);
-    if (d.dtype == BIMAMBA_F32)
-        return launch_scan_seq<float>(p.xbc, p.dt, p.A, p.D, p.conv_w, p.conv_b, p.tail, p.init,
-                                      p.fin, p.y, d.batch, d.len, d.heads, d.headdim, d.d_state,
-                                      stream);
-    return launch_scan_seq<__nv_bfloat16>(p.xbc, p.dt, p.A, p.D, p.conv_w, p.conv_b, p.tail,
-                                          p.init, p.fin, p.y, d.batch, d.len, d.heads, d.headdim,
-                                          d.d_state, stream);
+    if (d.dtype == BIMAMBA_F32) return launch_scan_seq<float>(p, stream);
+    return launch_scan_seq<__nv_bfloat16>(p, stream);
 }
 
 }  // namespace bimamba

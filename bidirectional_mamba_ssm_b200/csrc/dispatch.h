@@ -10,14 +10,17 @@
 namespace bimamba {
 
 // One validated call of the bidirectional mixer core (full scan or decode).
+// Per-direction inputs: [0] the forward stream, [1] the reverse stream (the
+// same pointers when the directions share their parameters).
 struct Problem {
     bimamba_dims dims;
-    const void *xbc;
-    const void *dt;
-    const float *A;
-    const float *D;
-    const float *conv_w;   // null: xbc already activated
-    const float *conv_b;
+    const void *xbc[2];
+    const void *dt[2];
+    const float *A[2];
+    const float *D[2];
+    const float *conv_w[2];   // null: xbc already activated
+    const float *conv_b[2];
+    int concat;            // 0: y = forward + reverse; 1: y = [forward | reverse] per token
     const void *tail;      // forward conv history (decode) or null
     const float *init;     // forward initial state or null
     float *fin;            // forward final state or null
@@ -43,10 +46,7 @@ cudaError_t launch_conv_silu(const void *u, void *out, const float *w, const flo
                              cudaStream_t stream);
 
 template <typename T>
-cudaError_t launch_scan_seq(const void *xbc, const void *dt, const float *A, const float *D,
-                            const float *conv_w, const float *conv_b, const void *tail,
-                            const float *init, float *fin, void *y, int batch, int len, int H,
-                            int P, int N, cudaStream_t stream);
+cudaError_t launch_scan_seq(const Problem &p, cudaStream_t stream);
 
 template <typename T>
 cudaError_t launch_tail_commit(const void *block, const void *tail, void *tail_out, int streams,

@@ -14,7 +14,9 @@
 // outputs are added.
 //
 // One CTA owns (batch b, head h) and runs both directions one after the
-// other: the forward pass writes y, the reverse pass adds to it.  Thread
+// other: the forward pass writes y, the reverse pass adds to it (or, with
+// the concatenating fusion of untied directions, writes its own half of
+// each output row).  Each direction reads its own inputs and parameters.  Thread
 // (p, q) owns state row p, columns n = q + NS*k (k < NPT), so each thread
 // carries NPT fp32 state values in registers; the y dot product is reduced
 // over the NS threads of a row with warp shuffles.  Activated x, B, C and dt
@@ -27,12 +29,13 @@ namespace bimamba {
 constexpr int kSeqChunk = 32;
 
 struct SeqParams {
-    const void *xbc;
-    const void *dt;
-    const float *A;
-    const float *D;
-    const float *conv_w;
-    const float *conv_b;
+    const void *xbc[2];     // [0] forward stream, [1] reverse stream
+    const void *dt[2];
+    const float *A[2];
+    const float *D[2];
+    const float *conv_w[2];
+    const float *conv_b[2];
+    int concat;        // y rows are [forward | reverse] (2*H*P wide)
     const void *tail;  // forward conv history (batch, 4, ch) or null
     const float *init;
     float *fin;
@@ -56,11 +59,8 @@ scan_seq_kernel(SeqParams p)
     float *ys = cs + kSeqChunk * N;      // [kSeqChunk][P]
     float *dts = ys + kSeqChunk * P;     // [kSeqChunk]
 
-    const T *xbc = static_cast<const T *>(p.xbc) + (size_t)b * len * ch;
-    const T *dtp = static_cast<const T *>(p.dt) + (size_t)b * len * H;
     const T *tail = p.tail ? static_cast<const T *>(p.tail) + (size_t)b * 4 * ch : nullptr;
-    T *y = static_cast<T *>(p.y) + (size_t)b * len * H * P;
-    const float Ah = p.A[h], Dh = p.D[h];
+    const size_t ystride = (size_t)(p.concat ? 2 : 1) * H * P;   // y row length
     const int nch = P + 2 * N;
     // lanes present in this warp (the block need not be a multiple of 32)
     const int wbase = tid & ~31;
@@ -70,6 +70,13 @@ scan_seq_kernel(SeqParams p)
 
     for (int dir = 0; dir < 2; ++dir) {
         const bool rev = dir == 1;
+        // selects, not a run-time index into the parameter arrays
+        const T *xbc = static_cast<const T *>(rev ? p.xbc[1] : p.xbc[0]) + (size_t)b * len * ch;
+        const T *dtp = static_cast<const T *>(rev ? p.dt[1] : p.dt[0]) + (size_t)b * len * H;
+        const float *conv_w = rev ? p.conv_w[1] : p.conv_w[0];
+        const float *conv_b = rev ? p.conv_b[1] : p.conv_b[0];
+        T *y = static_cast<T *>(p.y) + (size_t)b * len * ystride + (p.concat ? dir * H * P : 0);
+        const float Ah = (rev ? p.A[1] : p.A[0])[h], Dh = (rev ? p.D[1] : p.D[0])[h];
         float st[NPT];
 #pragma unroll
         for (int k = 0; k < NPT; ++k)
@@ -91,10 +98,10 @@ scan_seq_kernel(SeqParams p)
                     if (!rev && tail) return Elem<T>::load(tail + (size_t)(4 + s) * ch + c);
                     return 0.0f;
                 };
-                if (p.conv_w) {
-                    const float w0 = p.conv_w[c * 4 + 0], w1 = p.conv_w[c * 4 + 1];
-                    const float w2 = p.conv_w[c * 4 + 2], w3 = p.conv_w[c * 4 + 3];
-                    const float bias = p.conv_b ? p.conv_b[c] : 0.0f;
+                if (conv_w) {
+                    const float w0 = conv_w[c * 4 + 0], w1 = conv_w[c * 4 + 1];
+                    const float w2 = conv_w[c * 4 + 2], w3 = conv_w[c * 4 + 3];
+                    const float bias = conv_b ? conv_b[c] : 0.0f;
                     float r0 = raw(s0 - 3), r1 = raw(s0 - 2), r2 = raw(s0 - 1);
                     for (int i = 0; i < cnt; ++i) {
                         float r3 = raw(s0 + i);
@@ -134,14 +141,14 @@ scan_seq_kernel(SeqParams p)
             }
             __syncthreads();
 
-            // ---- write back; the reverse pass adds to the forward result.
-            // Visibility of the forward writes to other threads of this CTA
-            // is ordered by the __syncthreads() calls in between.
+            // ---- write back; the reverse pass adds to the forward result
+            // (sum fusion).  Visibility of the forward writes to other threads
+            // of this CTA is ordered by the __syncthreads() calls in between.
             for (int e = tid; e < cnt * P; e += blockDim.x) {
                 const int i = e / P, pc = e % P;
-                T *yp = y + (size_t)walk_token(s0 + i, len, rev) * H * P + h * P + pc;
+                T *yp = y + (size_t)walk_token(s0 + i, len, rev) * ystride + h * P + pc;
                 float v = ys[e];
-                if (rev) v += Elem<T>::load(yp);
+                if (rev && !p.concat) v += Elem<T>::load(yp);
                 Elem<T>::store(yp, v);
             }
         }
@@ -171,12 +178,21 @@ static cudaError_t launch_seq_t(const SeqParams &p, int batch, cudaStream_t stre
 }
 
 template <typename T>
-cudaError_t launch_scan_seq(const void *xbc, const void *dt, const float *A, const float *D,
-                            const float *conv_w, const float *conv_b, const void *tail,
-                            const float *init, float *fin, void *y, int batch, int len, int H,
-                            int P, int N, cudaStream_t stream)
+cudaError_t launch_scan_seq(const Problem &pr, cudaStream_t stream)
 {
-    SeqParams p{xbc, dt, A, D, conv_w, conv_b, tail, init, fin, y, len, H, P, N, H * P + 2 * N};
+    const bimamba_dims &d = pr.dims;
+    const int batch = d.batch, len = d.len, H = d.heads, P = d.headdim, N = d.d_state;
+    SeqParams p{};
+    for (int i = 0; i < 2; ++i) {
+        p.xbc[i] = pr.xbc[i]; p.dt[i] = pr.dt[i]; p.A[i] = pr.A[i]; p.D[i] = pr.D[i];
+        p.conv_w[i] = pr.conv_w[i]; p.conv_b[i] = pr.conv_b[i];
+    }
+    p.concat = pr.concat;
+    p.tail = pr.tail;
+    p.init = pr.init;
+    p.fin = pr.fin;
+    p.y = pr.y;
+    p.len = len; p.H = H; p.P = P; p.N = N; p.ch = H * P + 2 * N;
     // at most 512 threads per CTA: P * (N / NPT) <= 512 for P <= 128, N <= 256
     if (N >= 64 && P * (N / 32) > 512) return launch_seq_t<T, 64>(p, batch, stream);
     if (N >= 32) return launch_seq_t<T, 32>(p, batch, stream);
@@ -184,14 +200,8 @@ cudaError_t launch_scan_seq(const void *xbc, const void *dt, const float *A, con
     return launch_seq_t<T, 8>(p, batch, stream);
 }
 
-template cudaError_t launch_scan_seq<float>(const void *, const void *, const float *,
-                                            const float *, const float *, const float *,
-                                            const void *, const float *, float *, void *, int,
-                                            int, int, int, int, cudaStream_t);
-template cudaError_t launch_scan_seq<__nv_bfloat16>(const void *, const void *, const float *,
-                                                    const float *, const float *, const float *,
-                                                    const void *, const float *, float *, void *,
-                                                    int, int, int, int, int, cudaStream_t);
+template cudaError_t launch_scan_seq<float>(const Problem &, cudaStream_t);
+template cudaError_t launch_scan_seq<__nv_bfloat16>(const Problem &, cudaStream_t);
 
 // tail_out[s][k] = (prefix | block)[len - 4 + k], oldest first.
 template <typename T>

@@ -103,13 +103,15 @@ constexpr uint32_t kColS = 384;    // + 64 * head
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 constexpr int kArriveTid = 480;   // a thread outside warp 0 (which issues the MMAs)
 
+// Per-direction inputs are indexed [0] forward stream, [1] reverse stream
+// (the same pointers when the directions share their parameters); a CTA
+// picks its direction's with a select, never a run-time array index.
 struct TcParams {
-    const __nv_bfloat16 *xbc;
-    const __nv_bfloat16 *dt;
-    const float *A;
-    const float *D;
-    const float *conv_w;
-    const float *conv_b;
+    const __nv_bfloat16 *dt[2];
+    const float *A[2];
+    const float *D[2];
+    const float *conv_w[2];
+    const float *conv_b[2];
     const __nv_bfloat16 *tail;
     const float *init;
     float *fin;
@@ -187,13 +189,19 @@ __device__ __forceinline__ uint4 pack8(const float *v)
 // values are copied.  One thread: 8 channels x 8 walk steps, 3-step window in
 // registers; a warp covers one token's 256 channels (512 contiguous bytes).
 __global__ void __launch_bounds__(128)
-bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc, const __nv_bfloat16 *__restrict__ tail,
-                  const float *__restrict__ conv_w, const float *__restrict__ conv_b,
-                  __nv_bfloat16 *__restrict__ act, int len, int ch, int cbase, int batch)
+bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc_f, const __nv_bfloat16 *__restrict__ xbc_r,
+                  const __nv_bfloat16 *__restrict__ tail, const float *__restrict__ conv_w_f,
+                  const float *__restrict__ conv_w_r, const float *__restrict__ conv_b_f,
+                  const float *__restrict__ conv_b_r, __nv_bfloat16 *__restrict__ act, int len,
+                  int ch, int cbase, int batch)
 {
     const int g = threadIdx.x & 31, sub = threadIdx.x >> 5;
     const int b = blockIdx.y;
     const bool rev = blockIdx.z != 0;
+    // each direction's own raw input and conv parameters
+    const __nv_bfloat16 *xbc = rev ? xbc_r : xbc_f;
+    const float *conv_w = rev ? conv_w_r : conv_w_f;
+    const float *conv_b = rev ? conv_b_r : conv_b_f;
     const int s_begin = blockIdx.x * 32 + sub * 8;
     if (s_begin >= len) return;
     const int s_end = min(s_begin + 8, len);
@@ -252,10 +260,12 @@ bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc, const __nv_bfloat16 *__
 // entering it with the state chained from the items before it.
 // kStateOnly = true: only the state recurrence over one item's chunks, from a
 // zero state; writes the item's end state and its total decay.
-template <bool kStateOnly>
+// kConcat: untied directions with concatenated outputs; each direction
+// stores its own half of every output row and the CTAs never meet.
+template <bool kStateOnly, bool kConcat>
 __global__ void __launch_bounds__(kThreads, 1)
-ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_bc,
-              const TcParams p)
+ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant__ CUtensorMap tm_x_r,
+              const __grid_constant__ CUtensorMap tm_bc, const TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -319,7 +329,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         chunk_of(k, t0, cnt, s0);
         const uint32_t mb = mb_x0 + 8 * (k & 1);
         tc::mbar_expect_tx(mb, kRawBytes);
-        tc::tma_load_3d(sbase + xbuf_off(k), &tm_x, hp * kPP, rev ? t0 : t0 - 3, b, mb);
+        tc::tma_load_3d(sbase + xbuf_off(k), rev ? &tm_x_r : &tm_x_f, hp * kPP, rev ? t0 : t0 - 3, b,
+                        mb);
     };
     auto issue_bc = [&](int k) {
         int t0, cnt, s0;
@@ -335,7 +346,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     };
 
     constexpr float kLog2e = 1.4426950408889634f;
-    const float A0 = p.A[hp * kHeads] * kLog2e, A1 = p.A[hp * kHeads + 1] * kLog2e;
+    const float *Adir = rev ? p.A[1] : p.A[0];
+    const float A0 = Adir[hp * kHeads] * kLog2e, A1 = Adir[hp * kHeads + 1] * kLog2e;
 
     // helper warp: asynchronous copy of walk chunk k's dt (both heads of
     // the pair are adjacent: one 4-byte copy per token) into dt buffer
@@ -350,7 +362,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             if (j < cnt) {
                 const int s = s0 + j;
                 const int tok = rev ? L - 1 - s : s;
-                const __nv_bfloat16 *src = p.dt + ((size_t)b * L + tok) * H + hp * kHeads;
+                const __nv_bfloat16 *src = (rev ? p.dt[1] : p.dt[0]) + ((size_t)b * L + tok) * H + hp * kHeads;
                 asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
                              :: "r"(tc::smem_u32(dst + j)), "l"(src) : "memory");
             } else {
@@ -408,18 +420,20 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     };
 
     // ---- setup (all threads)
-    const bool has_conv = p.conv_w != nullptr;
+    const float *conv_w = rev ? p.conv_w[1] : p.conv_w[0];
+    const float *conv_b = rev ? p.conv_b[1] : p.conv_b[0];
+    const bool has_conv = conv_w != nullptr;
     if (tid < kPP && has_conv) {
         // stored as [q][g] for local channel 8g + q, so that the 16 channel
         // groups of a warp read 16 consecutive entries (no bank conflicts)
         const int c = hp * kPP + tid;
         const int slot = (tid & 7) * (kPP / 8) + (tid >> 3);
-        convw[slot] = *reinterpret_cast<const float4 *>(p.conv_w + (size_t)c * 4);
-        convb[slot] = p.conv_b ? p.conv_b[c] : 0.0f;
+        convw[slot] = *reinterpret_cast<const float4 *>(conv_w + (size_t)c * 4);
+        convb[slot] = conv_b ? conv_b[c] : 0.0f;
     }
     if (warp == 0) tc::tmem_alloc(sbase + kOffTmem, kTmemCols);
     if (tid == kProducerTid) {
-        tc::prefetch_tmap(&tm_x);
+        tc::prefetch_tmap(rev ? &tm_x_r : &tm_x_f);
         tc::prefetch_tmap(&tm_bc);
         tc::mbar_init(mb_bc, 1);
         tc::mbar_init(mb_x0, 1);
@@ -676,7 +690,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             }
         }
         float dec = 0.0f;   // state-only: total decay of the item (log2 units)
-        const float Dh = p.D[head_g];
+        const float Dh = (rev ? p.D[1] : p.D[0])[head_g];
 
         int arrival = 0;   // result of this chunk's arrival atomic (thread kArriveTid)
         ok = ok && wait_all(mb_x0, 0);
@@ -703,7 +717,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
 
             // arrive at this chunk's forward/reverse meeting point; the
             // result is read only after the chunk's MMAs
-            if (!kStateOnly && tid == kArriveTid)
+            if (!kStateOnly && !kConcat && tid == kArriveTid)
                 arrival = atomicAdd(p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2, 1);
 
             // ---- D: M_h (both heads, into TMEM) and the state's chunk-start
@@ -831,8 +845,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             const int cr = tid >> 4;          // rows cr, cr+32, cr+64, cr+96
             auto ypiece = [&](int r) -> uint4 * {
                 const int tk = rev ? t0 + cnt - 1 - r : t0 + r;
-                return reinterpret_cast<uint4 *>(p.y + ((size_t)b * L + tk) * ((size_t)H * kP) +
-                                                 hp * kPP) + cp;
+                const size_t row0 = kConcat ? ((size_t)b * L + tk) * 2 * H * kP + dir * H * kP
+                                            : ((size_t)b * L + tk) * H * kP;
+                return reinterpret_cast<uint4 *>(p.y + row0 + hp * kPP) + cp;
             };
             uint4 prev[4];
             if (!first) {
@@ -878,7 +893,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                     fl[0] = 0;   // leave the workspace zeroed for the next call
                     fl[1] = 0;
                 }
-                rel_flag[k & 1] = first ? fl + 1 : nullptr;
+                rel_flag[k & 1] = (first && !kConcat) ? fl + 1 : nullptr;
                 tc::mbar_arrive(mb_rows0 + 8 * (k & 1));   // the producer publishes them
             }
         }
@@ -1017,16 +1032,20 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
 {
     const bimamba_dims &d = pr.dims;
     TcParams p;
-    p.xbc = static_cast<const __nv_bfloat16 *>(pr.xbc);
-    p.dt = static_cast<const __nv_bfloat16 *>(pr.dt);
-    p.A = pr.A;
-    p.D = pr.D;
-    p.conv_w = pr.conv_w;
-    p.conv_b = pr.conv_b;
+    const __nv_bfloat16 *xbc[2];
+    for (int i = 0; i < 2; ++i) {
+        xbc[i] = static_cast<const __nv_bfloat16 *>(pr.xbc[i]);
+        p.dt[i] = static_cast<const __nv_bfloat16 *>(pr.dt[i]);
+        p.A[i] = pr.A[i];
+        p.D[i] = pr.D[i];
+        p.conv_w[i] = pr.conv_w[i];
+        p.conv_b[i] = pr.conv_b[i];
+    }
     p.tail = static_cast<const __nv_bfloat16 *>(pr.tail);
     p.init = pr.init;
     p.fin = pr.fin;
     p.y = static_cast<__nv_bfloat16 *>(pr.y);
+
     p.flags = static_cast<int *>(pr.workspace);
     p.status = pr.status;
     p.len = d.len;
@@ -1046,20 +1065,23 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
 
     // prepass: B/C conv+SiLU in walk order for both directions
     bc_prepass_kernel<<<dim3((d.len + 31) / 32, d.batch, 2), 128, 0, stream>>>(
-        p.xbc, p.tail, p.conv_w, p.conv_b, act, d.len, p.ch, d.heads * kP, d.batch);
+        xbc[0], xbc[1], p.tail, p.conv_w[0], p.conv_w[1], p.conv_b[0], p.conv_b[1], act, d.len, p.ch,
+        d.heads * kP, d.batch);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();
 
-    CUtensorMap tm_x, tm_bc;
-    if (!make_map(&tm_x, p.xbc, (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, kPP, kRawRows,
+    CUtensorMap tm_x_f, tm_x_r, tm_bc;
+    if (!make_map(&tm_x_f, xbc[0], (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, kPP, kRawRows,
+                  false) ||
+        !make_map(&tm_x_r, xbc[1], (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, kPP, kRawRows,
                   false) ||
         !make_map(&tm_bc, act, (uint64_t)kBC, (uint64_t)d.len, (uint64_t)2 * d.batch, 64, kQ, true))
         return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(ssd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
+    auto main_kernel = pr.concat ? ssd_tc_kernel<false, true> : ssd_tc_kernel<false, false>;
+    e = cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(ssd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(ssd_tc_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const TimingEvents ev = timing_events();
@@ -1067,14 +1089,14 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
     if (sp.nitems > 0) {
         TcParams q = p;
         q.seg_chunks = sp.item_chunks;   // one CTA per item
-        ssd_tc_kernel<true><<<dim3(d.heads, d.batch, sp.nitems), kThreads, kSmemBytes, stream>>>(
-            tm_x, tm_bc, q);
+        ssd_tc_kernel<true, false><<<dim3(d.heads, d.batch, sp.nitems), kThreads, kSmemBytes, stream>>>(
+            tm_x_f, tm_x_r, tm_bc, q);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         count_launch();
     }
-    ssd_tc_kernel<false><<<dim3(d.heads, d.batch, sp.nseg), kThreads, kSmemBytes, stream>>>(
-        tm_x, tm_bc, p);
+    main_kernel<<<dim3(d.heads, d.batch, sp.nseg), kThreads, kSmemBytes, stream>>>(tm_x_f, tm_x_r, tm_bc,
+                                                                                 p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();

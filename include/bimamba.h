@@ -62,6 +62,9 @@ typedef enum {
 
 typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype;
 
+/* How bimamba_ssd_fwd_rev_untied combines its two streams. */
+typedef enum { BIMAMBA_FUSE_SUM = 0, BIMAMBA_FUSE_CONCAT = 1 } bimamba_fusion;
+
 typedef struct {
     int batch;    /* independent sequences (decode: streams)                */
     int len;      /* tokens per sequence (decode: active block length)      */
@@ -171,6 +174,41 @@ int bimamba_ssd_fwd_rev(const bimamba_dims *d, const void *xbc, const void *dt,
                         const float *conv_b, const float *init_state,
                         float *final_state, void *y, void *workspace,
                         size_t workspace_bytes, bimamba_stream_t stream);
+
+/*
+ * Bidirectional mixer core with UNTIED directions: the forward stream and
+ * the reverse stream each have their own inputs and parameters.  The blog
+ * post "DiffuMamba", network-architecture listing, builds the mixer from two
+ * separate Mamba modules (one on the sequence, one on the reversed
+ * sequence, output reversed back), concatenates their outputs and maps 2d
+ * back to d with a Linear layer; the technical summaries add the two
+ * streams.  Both fusions are offered; the Linear after a concatenation is a
+ * plain GEMM outside this call.
+ *   xbc_f, xbc_r : (batch, len, ch) raw xBC of the forward / reverse stream
+ *   dt_f, dt_r   : (batch, len, H) dtype, already positive
+ *   A_f, A_r, D_f, D_r : (H) fp32
+ *   conv_w_f, conv_w_r : (ch, 4) fp32 or NULL (that stream's xbc is taken as
+ *                        activated); conv_b_f, conv_b_r : (ch) fp32 or NULL
+ *                        (a bias needs its taps)
+ *   init_state, final_state : the forward stream's, as in bimamba_ssd_fwd_rev
+ *   fusion : BIMAMBA_FUSE_SUM    -> y (batch, len, H*P) = forward + reverse
+ *            BIMAMBA_FUSE_CONCAT -> y (batch, len, 2*H*P), per token
+ *                                   [forward (H*P) | reverse (H*P)]
+ *   workspace : bimamba_workspace_bytes(d) bytes, as above
+ * With every *_f pointer equal to its *_r pointer and BIMAMBA_FUSE_SUM this
+ * is bimamba_ssd_fwd_rev.  Returns BIMAMBA_ERR_INVALID for an unknown
+ * fusion, a missing input, a bias without taps or a misaligned pointer.
+ */
+int bimamba_ssd_fwd_rev_untied(const bimamba_dims *d, const void *xbc_f,
+                               const void *xbc_r, const void *dt_f,
+                               const void *dt_r, const float *A_f,
+                               const float *A_r, const float *D_f,
+                               const float *D_r, const float *conv_w_f,
+                               const float *conv_w_r, const float *conv_b_f,
+                               const float *conv_b_r, const float *init_state,
+                               float *final_state, void *y, int fusion,
+                               void *workspace, size_t workspace_bytes,
+                               bimamba_stream_t stream);
 
 /*
  * Cached block decode for block diffusion: d->batch independent streams,

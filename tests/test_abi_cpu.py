@@ -143,3 +143,37 @@ def test_workspace_grows_with_the_state_only_items(lib):
     act = 2 * 1 * 1300 * 256 * 2
     items = 2 * 1 * 1 * 10
     assert lib.bimamba_workspace_bytes(d1) == flags + act + items * 2 * 64 * 128 * 4 + items * 2 * 4
+
+
+def test_untied_host_validation(lib):
+    """bimamba_ssd_fwd_rev_untied rejects bad arguments on the host, before
+    anything touches a device."""
+    import torch
+    L = lib.library()
+    d = lib.make_dims(1, 8, 2, 64, 128, torch.bfloat16)
+
+    def call(fusion=0, **over):
+        a = dict(xf=16, xr=16, dtf=16, dtr=16, Af=16, Ar=16, Df=16, Dr=16, wf=None, wr=None,
+                 bf=None, br=None, init=None, fin=None, y=16)
+        a.update(over)
+        return L.bimamba_ssd_fwd_rev_untied(
+            ctypes.byref(d), a["xf"], a["xr"], a["dtf"], a["dtr"], a["Af"], a["Ar"], a["Df"],
+            a["Dr"], a["wf"], a["wr"], a["bf"], a["br"], a["init"], a["fin"], a["y"], fusion,
+            None, 0, None)
+
+    assert call(fusion=2) == lib.BIMAMBA_ERR_INVALID
+    assert call(fusion=-1) == lib.BIMAMBA_ERR_INVALID
+    for k in ("xf", "xr", "dtf", "dtr", "Af", "Ar", "Df", "Dr", "y"):
+        assert call(**{k: None}) == lib.BIMAMBA_ERR_INVALID, k
+    assert call(br=16) == lib.BIMAMBA_ERR_INVALID          # a bias without its taps
+    assert call(bf=16, wf=None) == lib.BIMAMBA_ERR_INVALID
+    assert call(xr=24) == lib.BIMAMBA_ERR_INVALID          # misaligned
+    assert call(fusion=1, dtr=8) == lib.BIMAMBA_ERR_INVALID
+    # unsupported / invalid dims are reported the same way as for the tied call
+    bad = lib.make_dims(1, 8, 0, 64, 128, torch.bfloat16)
+    assert L.bimamba_ssd_fwd_rev_untied(ctypes.byref(bad), *([16] * 8), *([None] * 6), 16, 0,
+                                        None, 0, None) == lib.BIMAMBA_ERR_INVALID
+    # an empty batch is a valid no-op
+    empty = lib.make_dims(0, 8, 2, 64, 128, torch.bfloat16)
+    assert L.bimamba_ssd_fwd_rev_untied(ctypes.byref(empty), *([16] * 8), *([None] * 6), 16, 1,
+                                        None, 0, None) == lib.BIMAMBA_OK

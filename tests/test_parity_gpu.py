@@ -383,3 +383,88 @@ def test_repeated_calls_reuse_the_workspace(lib):
     assert torch.count_nonzero(ws[: 4 * 2 * nflags]).item() == 0
     for o in outs[1:]:
         assert rel_err(to_np(o), to_np(outs[0])) <= 1e-2
+
+
+# ------------------------------------------------------- untied directions
+UNTIED = [
+    # dtype, batch, L, H, P, N
+    ("f32", 2, 129, 3, 16, 32),      # sequential fp32 path
+    ("bf16", 2, 300, 4, 64, 128),    # tensor-core path, several chunks and a ragged tail
+    ("bf16", 1, 1300, 2, 64, 128),   # tensor-core path, segmented walk (state-only items)
+    ("bf16", 1, 200, 3, 32, 64),     # sequential path for bf16 shapes the tensor cores do not take
+]
+
+
+def _untied_inputs(w, a, seed):
+    f = inp_mod.make_inputs(w, seed=seed, a_range=a, conv_bias=True)
+    r = inp_mod.make_inputs(w, seed=seed + 1, a_range=a, conv_bias=True)
+    return f, r
+
+
+@pytest.mark.parametrize("case", UNTIED, ids=lambda c: "-".join(map(str, c)))
+@pytest.mark.parametrize("fusion", ["sum", "concat"])
+@pytest.mark.parametrize("memory", ["short", "long"])
+@pytest.mark.parametrize("convs", ["both", "forward-only"])
+def test_untied_directions(lib, case, fusion, memory, convs):
+    """Each stream with its own x/B/C, dt, A, D and conv parameters; outputs
+    summed or concatenated [forward | reverse] per token."""
+    dtype, bsz, L, H, P, N = case
+    w = inp_mod.Workload("u", bsz, L, H, P, N, dtype=dtype,
+                         bc_scale=1.0 if dtype == "f32" else 1.0 / math.sqrt(N))
+    a = (1.0, 16.0) if memory == "short" else (1e-3, 1e-2)
+    f, r = _untied_inputs(w, a, seed=L + 31 * H)
+    if convs == "forward-only":
+        r["conv_w"] = None
+        r["conv_b"] = None
+    init = inp_mod.make_state(bsz, H, P, N, seed=17, scale=0.3)
+    concat = fusion == "concat"
+    td = inp_mod.torch_dtype(dtype)
+    y = torch.full((bsz, L, (2 if concat else 1) * H * P), float("nan"), dtype=td, device="cuda")
+    fin = torch.full((bsz, H, P, N), float("nan"), device="cuda")
+    ws = lib.new_workspace(lib.make_dims(bsz, L, H, P, N, td))
+    lib.bimamba_ssd_fwd_rev_untied(_dev(f), _dev(r), init.cuda(), fin, y, ws, heads=H, headdim=P,
+                                   d_state=N, concat=concat)
+    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+    nf, nr = _np_inputs(f), _np_inputs(r)
+    ry, rfin = oracle.bimamba_untied(nf["xbc"], nr["xbc"], nf["dt"], nr["dt"], nf["A"], nr["A"],
+                                     nf["D"], nr["D"], nf["conv_w"], nr["conv_w"], nf["conv_b"],
+                                     nr["conv_b"], heads=H, headdim=P, d_state=N, init=to_np(init),
+                                     concat=concat, want_final=True)
+    tol = TOL[dtype]
+    for b in range(bsz):
+        if concat:
+            # each half against its own stream's scale
+            assert rel_err(to_np(y)[b][..., :H * P], ry[b][..., :H * P]) <= tol, b
+            assert rel_err(to_np(y)[b][..., H * P:], ry[b][..., H * P:]) <= tol, b
+        else:
+            assert rel_err(to_np(y)[b], ry[b]) <= tol, b
+        assert rel_err(to_np(fin)[b], rfin[b]) <= tol, b
+
+
+def test_untied_1p3b_concat_sampled_heads(lib):
+    """b8 L4096 H64x64 N128 bf16 untied, concatenated, as benchmarked; 2 heads x
+    2 sequences checked."""
+    w = inp_mod.LAYER_1P3B
+    f = inp_mod.make_inputs(w, seed=0)
+    r = inp_mod.make_inputs(w, seed=1)
+    H, P, N = w.heads, w.headdim, w.d_state
+    y = torch.full((w.batch, w.seqlen, 2 * H * P), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = lib.new_workspace(lib.make_dims(w.batch, w.seqlen, H, P, N, torch.bfloat16))
+    lib.bimamba_ssd_fwd_rev_untied(_dev(f), _dev(r), None, None, y, ws, heads=H, headdim=P,
+                                   d_state=N, concat=True)
+    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+    y = y.cpu()
+    heads = [3, 60]
+    nf, nr = _np_inputs(f), _np_inputs(r)
+    sf, _ = head_subset(nf, heads, H, P, N)
+    sr, _ = head_subset(nr, heads, H, P, N)
+    cols = y_cols(heads, P)
+    for b in (0, 7):
+        sl = slice(b, b + 1)
+        ry = oracle.bimamba_untied(sf["xbc"][sl], sr["xbc"][sl], sf["dt"][sl], sr["dt"][sl], sf["A"],
+                                   sr["A"], sf["D"], sr["D"], sf["conv_w"], sr["conv_w"], None, None,
+                                   heads=len(heads), headdim=P, d_state=N, concat=True)
+        got = to_np(y[sl])
+        hp = len(heads) * P
+        assert rel_err(got[..., cols], ry[..., :hp]) <= TOL["bf16"], b
+        assert rel_err(got[..., H * P + cols], ry[..., hp:]) <= TOL["bf16"], b
