@@ -451,6 +451,23 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         if (nk > 1) issue_x(1);
         issue_bc(0);
     }
+    // Global loads that need nothing from the set-up start before its
+    // barrier, so that their latencies overlap (they dominate a CTA that
+    // covers a single chunk, as in block decode): the helper's first dt
+    // copies, and each compute thread's share of the caller's initial state.
+    if (warp == kHelperWarp) {
+        load_dt_async(0);
+        if (nk > 1) load_dt_async(1);
+    }
+    float sv_init[32];
+    {
+        const int row = tid & 127, rg = tid >> 7;
+        const size_t sidx0 = ((size_t)b * H + hp * kHeads + (rg >> 1)) * kP * kN;
+        const bool use_init = !kStateOnly && !rev && p.init && tid < kAluThreads;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            sv_init[i] = use_init ? __ldg(p.init + sidx0 + (size_t)(32 * (rg & 1) + i) * kN + row) : 0.0f;
+    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -549,9 +566,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         if (lane == 0 && !pok) record_error(p.status, kStatusTimeout);
     } else if (warp == kHelperWarp) {
         // ================= helper: dt copies, prefix sums and slot factors
-        // of each chunk, up to two chunks ahead of phase D
-        load_dt_async(0);
-        if (nk > 1) load_dt_async(1);
+        // of each chunk, up to two chunks ahead of phase D (the copies of
+        // chunks 0 and 1 were issued before the set-up barrier)
         bool hok = true;
         for (int j = 0; j < nk; ++j) {
             if (j >= 2) {
@@ -658,22 +674,17 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             return alu_sync_and(w);
         };
 
-        uint32_t mbd, pard;
-        dt_ready(0, mbd, pard);
-        bool ok = wait_all(mbd, pard);   // chunk 0's prefix sums and slot factors
-
         // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg.
         // A segment's entering state: the caller's initial state (forward
-        // stream) or zero, carried through the items before the segment:
-        // S <- 2^dec_i S + S_i, with S_i item i's end state from zero.
+        // stream; loaded before the set-up barrier) or zero, carried through
+        // the items before the segment: S <- 2^dec_i S + S_i, with S_i item
+        // i's end state from zero.
         const int head_g = hp * kHeads + hh;     // global head of this thread's columns
         const size_t sidx = ((size_t)b * H + head_g) * kP * kN;
         {
             float sv[32];
-            const bool use_init = !kStateOnly && !rev && p.init;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                sv[i] = use_init ? p.init[sidx + (size_t)(32 * hsub + i) * kN + row] : 0.0f;
+            for (int i = 0; i < 32; ++i) sv[i] = sv_init[i];
             const int n_in = (kStateOnly || p.item_chunks == 0) ? 0 : k0 / p.item_chunks;
             for (int it = 0; it < n_in; ++it) {
                 const float *si = p.seg_state + ((item_row + it) * kHeads + hh) * kP * kN;
@@ -689,6 +700,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
             }
         }
+        uint32_t mbd, pard;
+        dt_ready(0, mbd, pard);
+        bool ok = wait_all(mbd, pard);   // chunk 0's prefix sums and slot factors
         float dec = 0.0f;   // state-only: total decay of the item (log2 units)
         const float Dh = (rev ? p.D[1] : p.D[0])[head_g];
 
