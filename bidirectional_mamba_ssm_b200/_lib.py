@@ -39,6 +39,8 @@ EXPORTED = (
     "bimamba_launch_plan",
     "bimamba_ssd_fwd_rev",
     "bimamba_ssd_fwd_rev_untied",
+    "bimamba_shard_states",
+    "bimamba_ssd_fwd_rev_shard",
     "bimamba_block_decode",
     "bimamba_noalloc_scratch_bytes",
     "bimamba_block_decode_noalloc",
@@ -84,6 +86,10 @@ def _load() -> ctypes.CDLL:
     lib.bimamba_ssd_fwd_rev.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.bimamba_ssd_fwd_rev_untied.restype = i
     lib.bimamba_ssd_fwd_rev_untied.argtypes = [dp] + [vp] * 15 + [i, vp, sz, vp]
+    lib.bimamba_shard_states.restype = i
+    lib.bimamba_shard_states.argtypes = [dp] + [vp] * 10 + [sz, vp]
+    lib.bimamba_ssd_fwd_rev_shard.restype = i
+    lib.bimamba_ssd_fwd_rev_shard.argtypes = [dp] + [vp] * 11 + [i, i, vp, vp, vp, sz, vp]
     lib.bimamba_block_decode.restype = i
     lib.bimamba_block_decode.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.bimamba_noalloc_scratch_bytes.restype = sz
@@ -223,6 +229,37 @@ def bimamba_ssd_fwd_rev_untied(fwd, rev, init_state, final_state, y, workspace, 
         g(rev, "conv_b"), _ptr(init_state), _ptr(final_state), _ptr(y),
         BIMAMBA_FUSE_CONCAT if concat else BIMAMBA_FUSE_SUM, _ptr(workspace), wsz, _stream(stream))
     _check(st, "bimamba_ssd_fwd_rev_untied")
+    return y
+
+
+def bimamba_shard_states(xbc, dt, A, conv_w, conv_b, tail, head, states, decays, workspace, *,
+                         heads, headdim, d_state, ngroups=1, stream=None):
+    """One sequence shard's end states from zero, (2, batch, H, P, N) [forward,
+    reverse], and log2 decays (2, batch, H).  tail/head: (batch, 4, ch) raw
+    tokens before/after the shard, or None (zeros)."""
+    bsz, L, _ = xbc.shape
+    dims = make_dims(bsz, L, heads, headdim, d_state, _dtype_code(xbc), ngroups)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.bimamba_shard_states(ctypes.byref(dims), _ptr(xbc), _ptr(dt), _ptr(A), _ptr(conv_w),
+                                   _ptr(conv_b), _ptr(tail), _ptr(head), _ptr(states),
+                                   _ptr(decays), _ptr(workspace), wsz, _stream(stream))
+    _check(st, "bimamba_shard_states")
+    return states, decays
+
+
+def bimamba_ssd_fwd_rev_shard(xbc, dt, A, D, conv_w, conv_b, tail, head, init_state, all_states,
+                              all_decays, rank, nranks, final_state, y, workspace, *, heads,
+                              headdim, d_state, ngroups=1, stream=None):
+    """One sequence shard's outputs, entering with the states the other
+    shards hand on (all_states / all_decays: every rank's shard states)."""
+    bsz, L, _ = xbc.shape
+    dims = make_dims(bsz, L, heads, headdim, d_state, _dtype_code(xbc), ngroups)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.bimamba_ssd_fwd_rev_shard(
+        ctypes.byref(dims), _ptr(xbc), _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b),
+        _ptr(tail), _ptr(head), _ptr(init_state), _ptr(all_states), _ptr(all_decays), int(rank),
+        int(nranks), _ptr(final_state), _ptr(y), _ptr(workspace), wsz, _stream(stream))
+    _check(st, "bimamba_ssd_fwd_rev_shard")
     return y
 
 

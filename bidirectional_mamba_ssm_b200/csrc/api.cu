@@ -256,6 +256,93 @@ int bimamba_ssd_fwd_rev_untied(const bimamba_dims *d, const void *xbc_f, const v
                        init_state, final_state, y, workspace, workspace_bytes, s);
 }
 
+// Sequence shards: a shard's inputs, halos and tied parameters into a Problem.
+static int shard_problem(const bimamba_dims *d, const void *xbc, const void *dt, const float *A,
+                         const float *D, const float *conv_w, const float *conv_b,
+                         const void *tail, const void *head, void *workspace,
+                         size_t workspace_bytes, Problem &pr)
+{
+    int st = check_dims(d);
+    if (st != BIMAMBA_OK) return st;
+    if (!tc_path_supported(*d)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!xbc || !dt || !A) return BIMAMBA_ERR_INVALID;
+    if (conv_b && !conv_w) return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {xbc, dt, A, D, conv_w, conv_b, tail, head};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return BIMAMBA_ERR_INVALID;
+    const size_t need = workspace_bytes_for(*d);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+        return BIMAMBA_ERR_WORKSPACE;
+    pr = Problem{};
+    pr.dims = *d;
+    for (int i = 0; i < 2; ++i) {
+        pr.xbc[i] = xbc; pr.dt[i] = dt; pr.A[i] = A; pr.D[i] = D;
+        pr.conv_w[i] = conv_w; pr.conv_b[i] = conv_b;
+    }
+    pr.tail = tail;
+    pr.head = head;
+    pr.workspace = workspace;
+    pr.workspace_bytes = workspace_bytes;
+    pr.status = device_status_word();
+    return BIMAMBA_OK;
+}
+
+int bimamba_shard_states(const bimamba_dims *d, const void *xbc, const void *dt, const float *A,
+                         const float *conv_w, const float *conv_b, const void *tail,
+                         const void *head, float *states, float *decays, void *workspace,
+                         size_t workspace_bytes, bimamba_stream_t stream)
+{
+    Problem pr;
+    int st = shard_problem(d, xbc, dt, A, nullptr, conv_w, conv_b, tail, head, workspace,
+                           workspace_bytes, pr);
+    if (st != BIMAMBA_OK) return st;
+    if (!states || !decays || !aligned16(states) || !aligned16(decays)) return BIMAMBA_ERR_INVALID;
+    if (d->batch == 0) return BIMAMBA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d->len == 0) {
+        // an empty shard leaves every state unchanged: zero states, zero log-decay
+        const size_t ns = (size_t)2 * d->batch * d->heads * d->headdim * d->d_state;
+        cudaError_t e = cudaMemsetAsync(states, 0, ns * sizeof(float), s);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(decays, 0, (size_t)2 * d->batch * d->heads * sizeof(float), s);
+        return cuda_status(e);
+    }
+    pr.states_out = states;
+    pr.dec_out = decays;
+    return cuda_status(launch_shard_states(pr, s));
+}
+
+int bimamba_ssd_fwd_rev_shard(const bimamba_dims *d, const void *xbc, const void *dt,
+                              const float *A, const float *D, const float *conv_w,
+                              const float *conv_b, const void *tail, const void *head,
+                              const float *init_state, const float *all_states,
+                              const float *all_decays, int rank, int nranks, float *final_state,
+                              void *y, void *workspace, size_t workspace_bytes,
+                              bimamba_stream_t stream)
+{
+    Problem pr;
+    int st = shard_problem(d, xbc, dt, A, D, conv_w, conv_b, tail, head, workspace,
+                           workspace_bytes, pr);
+    if (st != BIMAMBA_OK) return st;
+    if (!D || !y || nranks < 1 || rank < 0 || rank >= nranks) return BIMAMBA_ERR_INVALID;
+    if (nranks > 1 && (!all_states || !all_decays)) return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {init_state, all_states, all_decays, final_state, y};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return BIMAMBA_ERR_INVALID;
+    if (d->batch == 0 || d->len == 0) return d->len == 0 && d->batch > 0 ? BIMAMBA_ERR_INVALID
+                                                                       : BIMAMBA_OK;
+    pr.init = init_state;
+    pr.fin = final_state;
+    pr.y = y;
+    if (nranks > 1) {
+        pr.shard_states = all_states;
+        pr.shard_dec = all_decays;
+    }
+    pr.rank = rank;
+    pr.nranks = nranks;
+    return cuda_status(launch_bimamba(pr, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block, const void *dt_block,
                          const float *A, const float *D, const float *conv_w,
                          const float *conv_b, const float *state, const void *tail, void *y,

@@ -21,7 +21,15 @@ struct Problem {
     const float *conv_w[2];   // null: xbc already activated
     const float *conv_b[2];
     int concat;            // 0: y = forward + reverse; 1: y = [forward | reverse] per token
-    const void *tail;      // forward conv history (decode) or null
+    const void *tail;      // forward conv history (decode, sequence shards) or null
+    const void *head;      // raw tokens after a sequence shard (reverse conv) or null
+    // sequence shards: all ranks' shard end states and log2 decays, this rank
+    const float *shard_states;
+    const float *shard_dec;
+    int rank, nranks;
+    // states-only call: write this shard's end states / decays, no outputs
+    float *states_out;
+    float *dec_out;
     const float *init;     // forward initial state or null
     float *fin;            // forward final state or null
     void *y;
@@ -39,6 +47,9 @@ size_t tc_workspace_bytes(const bimamba_dims &d);
 // out[0..2]: segments per direction, chunks per segment, state-only items
 void tc_launch_plan(const bimamba_dims &d, int *out);
 cudaError_t launch_ssd_tc(const Problem &p, cudaStream_t stream);
+// end states from zero and log2 decays of a whole sequence (shard), both
+// directions; tensor-core path only
+cudaError_t launch_shard_states(const Problem &p, cudaStream_t stream);
 
 template <typename T>
 cudaError_t launch_conv_silu(const void *u, void *out, const float *w, const float *bias,

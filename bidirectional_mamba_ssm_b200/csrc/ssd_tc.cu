@@ -112,10 +112,16 @@ struct TcParams {
     const float *D[2];
     const float *conv_w[2];
     const float *conv_b[2];
-    const __nv_bfloat16 *tail;
+    const __nv_bfloat16 *tail;   // (batch, 4, ch) raw tokens before the sequence, or null
+    const __nv_bfloat16 *head;   // (batch, 4, ch) raw tokens after it (sequence shards), or null
     const float *init;
     float *fin;
     __nv_bfloat16 *y;
+    // sequence shards: every rank's shard end states from zero
+    // [nranks][2 dir][batch][H][kP][kN] and log2 decays [nranks][2][batch][H]
+    const float *shard_states;
+    const float *shard_dec;
+    int rank, nranks;
     int *flags;   // [batch][H/2][nchunks][2]: arrivals, partial-ready
     int *status;
     // segments (blockIdx.z): walk chunks [z * seg_chunks, +seg_chunks)
@@ -190,7 +196,8 @@ __device__ __forceinline__ uint4 pack8(const float *v)
 // registers; a warp covers one token's 256 channels (512 contiguous bytes).
 __global__ void __launch_bounds__(128)
 bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc_f, const __nv_bfloat16 *__restrict__ xbc_r,
-                  const __nv_bfloat16 *__restrict__ tail, const float *__restrict__ conv_w_f,
+                  const __nv_bfloat16 *__restrict__ tail, const __nv_bfloat16 *__restrict__ head,
+                  const float *__restrict__ conv_w_f,
                   const float *__restrict__ conv_w_r, const float *__restrict__ conv_b_f,
                   const float *__restrict__ conv_b_r, __nv_bfloat16 *__restrict__ act, int len,
                   int ch, int cbase, int batch)
@@ -215,6 +222,8 @@ bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc_f, const __nv_bfloat16 *
             unpack8(*reinterpret_cast<const uint4 *>(xb + (size_t)tok * ch), v);
         } else if (!rev && tail) {
             unpack8(*reinterpret_cast<const uint4 *>(tail + ((size_t)b * 4 + 4 + s) * ch + c), v);
+        } else if (rev && head) {   // walk step s < 0 of the reverse stream: token len - 1 - s
+            unpack8(*reinterpret_cast<const uint4 *>(head + ((size_t)b * 4 - 1 - s) * ch + c), v);
         } else {
 #pragma unroll
             for (int q = 0; q < 8; ++q) v[q] = 0.0f;
@@ -685,6 +694,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             float sv[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) sv[i] = sv_init[i];
+            // sequence shards: the walk enters this shard with the state the
+            // shards before it in walk order leave (forward: ranks 0..rank-1
+            // from the initial state; reverse: ranks nranks-1..rank+1 from zero)
+            const int n_sh = (kStateOnly || !p.shard_states) ? 0 : (rev ? p.nranks - 1 - p.rank : p.rank);
+            for (int it = 0; it < n_sh; ++it) {
+                const int q = rev ? p.nranks - 1 - it : it;
+                const size_t e = (((size_t)q * 2 + dir) * p.batch + b) * H + head_g;
+                const float *si = p.shard_states + e * kP * kN;
+                const float a = tc::exp2_approx(p.shard_dec[e]);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[i] = fmaf(sv[i], a, si[(size_t)(32 * hsub + i) * kN + row]);
+            }
             const int n_in = (kStateOnly || p.item_chunks == 0) ? 0 : k0 / p.item_chunks;
             for (int it = 0; it < n_in; ++it) {
                 const float *si = p.seg_state + ((item_row + it) * kHeads + hh) * kP * kN;
@@ -704,17 +725,31 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         dt_ready(0, mbd, pard);
         bool ok = wait_all(mbd, pard);   // chunk 0's prefix sums and slot factors
         float dec = 0.0f;   // state-only: total decay of the item (log2 units)
-        const float Dh = (rev ? p.D[1] : p.D[0])[head_g];
+        const float Dh = kStateOnly ? 0.0f : (rev ? p.D[1] : p.D[0])[head_g];   // no D for states
 
         int arrival = 0;   // result of this chunk's arrival atomic (thread kArriveTid)
         ok = ok && wait_all(mb_x0, 0);
         if (ok) {
-            // decode: the conv history before token 0 comes from the cached tail
+            // decode and sequence shards: the conv history before token 0
+            // comes from the tail; for sequence shards the reverse stream's
+            // conv reads the tokens after the shard from the head (raw rows
+            // cnt .. cnt+2 of the walk's first chunk, past the shard end)
             if (!rev && p.tail && k0 == 0) {
                 for (int e = tid; e < 3 * (kPP / 8); e += kAluThreads) {
                     const int r = e / (kPP / 8), g = e % (kPP / 8);
                     *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
                         *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
+                                                         hp * kPP + 8 * g);
+                }
+                alu_sync();
+            }
+            if (rev && p.head && k0 == 0) {
+                int t0, cnt, s0;
+                chunk_of(0, t0, cnt, s0);
+                for (int e = tid; e < 3 * (kPP / 8); e += kAluThreads) {
+                    const int r = e / (kPP / 8), g = e % (kPP / 8);
+                    *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + (cnt + r) * (kPP * 2) + g * 16) =
+                        *reinterpret_cast<const uint4 *>(p.head + ((size_t)b * 4 + r) * ch +
                                                          hp * kPP + 8 * g);
                 }
                 alu_sync();
@@ -1042,6 +1077,11 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
+cudaError_t launch_shard_states(const Problem &pr, cudaStream_t stream)
+{
+    return launch_ssd_tc(pr, stream);   // pr.states_out selects the states-only launch
+}
+
 cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
 {
     const bimamba_dims &d = pr.dims;
@@ -1056,6 +1096,11 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
         p.conv_b[i] = pr.conv_b[i];
     }
     p.tail = static_cast<const __nv_bfloat16 *>(pr.tail);
+    p.head = static_cast<const __nv_bfloat16 *>(pr.head);
+    p.shard_states = pr.shard_states;
+    p.shard_dec = pr.shard_dec;
+    p.rank = pr.rank;
+    p.nranks = pr.nranks;
     p.init = pr.init;
     p.fin = pr.fin;
     p.y = static_cast<__nv_bfloat16 *>(pr.y);
@@ -1079,8 +1124,8 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
 
     // prepass: B/C conv+SiLU in walk order for both directions
     bc_prepass_kernel<<<dim3((d.len + 31) / 32, d.batch, 2), 128, 0, stream>>>(
-        xbc[0], xbc[1], p.tail, p.conv_w[0], p.conv_w[1], p.conv_b[0], p.conv_b[1], act, d.len, p.ch,
-        d.heads * kP, d.batch);
+        xbc[0], xbc[1], p.tail, p.head, p.conv_w[0], p.conv_w[1], p.conv_b[0], p.conv_b[1], act, d.len,
+        p.ch, d.heads * kP, d.batch);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();
@@ -1100,6 +1145,22 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
     if (e != cudaSuccess) return e;
     const TimingEvents ev = timing_events();
     if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
+    if (pr.states_out) {
+        // states only: one item per walk, the whole sequence, written to the
+        // caller's [2][batch][H][kP][kN] states and [2][batch][H] decays
+        TcParams q = p;
+        q.seg_state = pr.states_out;
+        q.seg_dec = pr.dec_out;
+        q.nitems = 1;
+        q.item_chunks = q.seg_chunks = p.nchunks;
+        ssd_tc_kernel<true, false><<<dim3(d.heads, d.batch, 1), kThreads, kSmemBytes, stream>>>(
+            tm_x_f, tm_x_r, tm_bc, q);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        count_launch();
+        if (ev.stop) e = cudaEventRecord(ev.stop, stream);
+        return e;
+    }
     if (sp.nitems > 0) {
         TcParams q = p;
         q.seg_chunks = sp.item_chunks;   // one CTA per item

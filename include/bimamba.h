@@ -211,6 +211,65 @@ int bimamba_ssd_fwd_rev_untied(const bimamba_dims *d, const void *xbc_f,
                                bimamba_stream_t stream);
 
 /*
+ * Sequence shards (one sequence split across ranks, e.g. one GPU each).
+ * The recurrence is linear in the state, so a shard's effect on the state
+ * that crosses it is h -> 2^dec h + S, where S is the state the shard leaves
+ * when entered with zero and dec the log2 of the product of its per-token
+ * decay factors exp(dt A).  Each rank computes (S, dec) of its shard for both
+ * directions, the ranks exchange them (an all-gather: 2 x H x P x N fp32 plus
+ * 2 x H per sequence and rank), and each rank then computes its outputs
+ * entering its shard with the states the other shards hand on.  This is the
+ * exchange step of the scan on a sharded sequence dimension.  The tokens next
+ * to a shard that its conv reads (3 before for the forward stream, 3 after
+ * for the reverse stream) come from the neighbouring shards as halos.
+ * Tensor-core path only (bf16, headdim 64, d_state 128, even H); other
+ * shapes return BIMAMBA_ERR_UNSUPPORTED.
+ *
+ * bimamba_shard_states: this rank's (S, dec), no outputs.
+ *   d      : the shard's dims (len = shard length)
+ *   xbc, dt, A, conv_w, conv_b : as in bimamba_ssd_fwd_rev, for the shard
+ *   tail   : (batch, 4, ch) dtype or NULL -- the 4 raw tokens before the shard
+ *            (oldest first; NULL or zeros for the first shard)
+ *   head   : (batch, 4, ch) dtype or NULL -- the 4 raw tokens after the shard
+ *            (in order; NULL or zeros for the last shard)
+ *   states : (2, batch, H, P, N) fp32, written: [0] the forward stream's state
+ *            after the shard, [1] the reverse stream's state after walking the
+ *            shard from its last token to its first, both from zero
+ *   decays : (2, batch, H) fp32, written: dec per direction (equal up to the
+ *            rounding of the two summation orders)
+ *   workspace : bimamba_workspace_bytes(d) bytes
+ */
+int bimamba_shard_states(const bimamba_dims *d, const void *xbc, const void *dt,
+                         const float *A, const float *conv_w, const float *conv_b,
+                         const void *tail, const void *head, float *states,
+                         float *decays, void *workspace, size_t workspace_bytes,
+                         bimamba_stream_t stream);
+
+/*
+ * bimamba_ssd_fwd_rev_shard: this rank's outputs.  The forward stream enters
+ * the shard with init_state carried through shards 0 .. rank-1; the reverse
+ * stream enters with zero carried through shards nranks-1 .. rank+1.
+ *   xbc, dt, A, D, conv_w, conv_b, tail, head : as above
+ *   init_state : (batch, H, P, N) fp32 or NULL -- forward state before shard 0
+ *   all_states : (nranks, 2, batch, H, P, N) fp32 -- every rank's `states`,
+ *                in rank order (may be NULL when nranks == 1)
+ *   all_decays : (nranks, 2, batch, H) fp32 -- every rank's `decays`
+ *   rank, nranks : this shard's position, 0 <= rank < nranks
+ *   final_state : (batch, H, P, N) fp32 or NULL -- the forward state after
+ *                this shard (the sequence's final state on the last rank)
+ *   y          : (batch, len, H*P) dtype -- the shard's outputs
+ * Concatenating every rank's y gives bimamba_ssd_fwd_rev on the whole sequence.
+ */
+int bimamba_ssd_fwd_rev_shard(const bimamba_dims *d, const void *xbc,
+                              const void *dt, const float *A, const float *D,
+                              const float *conv_w, const float *conv_b,
+                              const void *tail, const void *head,
+                              const float *init_state, const float *all_states,
+                              const float *all_decays, int rank, int nranks,
+                              float *final_state, void *y, void *workspace,
+                              size_t workspace_bytes, bimamba_stream_t stream);
+
+/*
  * Cached block decode for block diffusion: d->batch independent streams,
  * each with an active block of d->len tokens.  The forward stream resumes
  * from `state` with the conv history `tail`; the reverse stream covers the

@@ -177,3 +177,25 @@ def test_untied_host_validation(lib):
     empty = lib.make_dims(0, 8, 2, 64, 128, torch.bfloat16)
     assert L.bimamba_ssd_fwd_rev_untied(ctypes.byref(empty), *([16] * 8), *([None] * 6), 16, 1,
                                         None, 0, None) == lib.BIMAMBA_OK
+
+
+def _declared_arity():
+    """Parameter count of every entry point, from include/bimamba.h."""
+    src = open(os.path.join(ROOT, "include", "bimamba.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(bimamba_\w+)\s*\(([^)]*)\)\s*;", src):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header(lib):
+    """Every ctypes prototype has exactly as many arguments as the C
+    declaration (a short prototype passes later arguments with the wrong
+    types, which crashes the host process)."""
+    so = lib.library()
+    arity = _declared_arity()
+    assert set(arity) == set(lib.EXPORTED)
+    for name, n in arity.items():
+        assert len(getattr(so, name).argtypes) == n, (name, len(getattr(so, name).argtypes), n)

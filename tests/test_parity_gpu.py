@@ -468,3 +468,82 @@ def test_untied_1p3b_concat_sampled_heads(lib):
         hp = len(heads) * P
         assert rel_err(got[..., cols], ry[..., :hp]) <= TOL["bf16"], b
         assert rel_err(got[..., H * P + cols], ry[..., hp:]) <= TOL["bf16"], b
+
+
+# ------------------------------------------------------- sequence shards
+SHARDED = [
+    # batch, shard lengths, H, variant, heads the oracle checks (None: all)
+    (2, (334, 333, 333), 4, "init+bias", None),        # 3 ranks, ragged shards
+    (1, (700, 5, 600, 130), 2, "plain", None),         # 4 ranks; a 5-token shard; segmented shards
+    (1, (1500, 1700), 64, "init+bias", [0, 41, 63]),   # 64 heads: items inside each shard too
+]
+
+
+def _run_shards(lib, g, lens, H, P, N, init):
+    """Every rank's two calls, one rank after the other on this GPU (no rank
+    waits on another inside a kernel); the all-gather becomes a stack."""
+    full_x, full_dt = g["xbc"], g["dt"]
+    bsz, total, ch = full_x.shape
+    starts = [sum(lens[:r]) for r in range(len(lens))]
+    zeros = torch.zeros((bsz, 4, ch), dtype=full_x.dtype, device="cuda")
+    parts = []
+    for r, (s0, n) in enumerate(zip(starts, lens)):
+        # fresh allocations (a rank holds its own shard); slices of one tensor
+        # can start off the 16-byte alignment the library requires
+        x = full_x[:, s0:s0 + n].clone()
+        dt = full_dt[:, s0:s0 + n].clone()
+        tail = full_x[:, s0 - 4:s0].clone() if r > 0 else zeros
+        head = full_x[:, s0 + n:s0 + n + 4].clone() if r + 1 < len(lens) else zeros
+        ws = lib.new_workspace(lib.make_dims(bsz, n, H, P, N, torch.bfloat16))
+        st = torch.full((2, bsz, H, P, N), float("nan"), device="cuda")
+        dc = torch.full((2, bsz, H), float("nan"), device="cuda")
+        lib.bimamba_shard_states(x, dt, g["A"], g["conv_w"], g["conv_b"], tail, head, st, dc, ws,
+                                 heads=H, headdim=P, d_state=N)
+        parts.append((x, dt, tail, head, ws, st, dc))
+    all_states = torch.stack([p_[5] for p_ in parts])
+    all_decays = torch.stack([p_[6] for p_ in parts])
+    ys, fin = [], None
+    for r, (x, dt, tail, head, ws, _, _) in enumerate(parts):
+        y = torch.full((bsz, lens[r], H * P), float("nan"), dtype=torch.bfloat16, device="cuda")
+        f = torch.full((bsz, H, P, N), float("nan"), device="cuda")
+        lib.bimamba_ssd_fwd_rev_shard(x, dt, g["A"], g["D"], g["conv_w"], g["conv_b"], tail, head,
+                                      init, all_states, all_decays, r, len(lens), f, y, ws,
+                                      heads=H, headdim=P, d_state=N)
+        ys.append(y)
+        fin = f
+    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+    return torch.cat(ys, dim=1), fin, all_decays
+
+
+@pytest.mark.parametrize("case", SHARDED, ids=lambda c: f"b{c[0]}-{len(c[1])}ranks-H{c[2]}-{c[3]}")
+@pytest.mark.parametrize("memory", ["short", "long"])
+def test_sequence_shards_equal_the_whole_sequence(lib, case, memory):
+    """One sequence cut into shards: each rank's state-only pass, the exchange
+    (here a stack) and each rank's shard call together give the oracle's
+    output over the whole sequence and its final forward state."""
+    bsz, lens, H, variant, heads = case
+    P, N = 64, 128
+    L = sum(lens)
+    w = inp_mod.Workload("shard", bsz, L, H, P, N, dtype="bf16", bc_scale=1.0 / math.sqrt(N))
+    a = (1.0, 16.0) if memory == "short" else (1e-3, 1e-2)
+    cpu = inp_mod.make_inputs(w, seed=L + 7 * H, a_range=a, conv_bias="bias" in variant)
+    init = inp_mod.make_state(bsz, H, P, N, seed=23, scale=0.3) if "init" in variant else None
+    g = _dev(cpu)
+    y, fin, decays = _run_shards(lib, g, lens, H, P, N, None if init is None else init.cuda())
+    # the decays are log2 of the shards' decay products
+    starts = [sum(lens[:r]) for r in range(len(lens))]
+    want = torch.stack([(cpu["dt"][:, s:s + n].float() * cpu["A"]).sum(1) for s, n in zip(starts, lens)])
+    got = decays.cpu()
+    torch.testing.assert_close(got[:, 0], want / math.log(2.0), rtol=2e-4, atol=1e-3)
+    # both directions sum the same terms, in opposite orders
+    torch.testing.assert_close(got[:, 1], got[:, 0], rtol=1e-5, atol=1e-5)
+    n = _np_inputs(cpu)
+    heads = list(range(H)) if heads is None else heads
+    sub, _ = head_subset(n, heads, H, P, N)
+    ry, rfin = oracle.bimamba(sub["xbc"], sub["dt"], sub["A"], sub["D"], sub["conv_w"],
+                              sub["conv_b"], heads=len(heads), headdim=P, d_state=N,
+                              init=None if init is None else to_np(init[:, heads]), want_final=True)
+    cols = y_cols(heads, P)
+    for b in range(bsz):
+        assert rel_err(to_np(y)[b][..., cols], ry[b]) <= TOL["bf16"], b
+        assert rel_err(to_np(fin)[b][heads], rfin[b]) <= TOL["bf16"], b
