@@ -898,14 +898,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                                             : ((size_t)b * L + tk) * H * kP;
                 return reinterpret_cast<uint4 *>(p.y + row0 + hp * kPP) + cp;
             };
-            uint4 prev[4];
-            if (!first) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = cr + 32 * j;
-                    prev[j] = r < cnt ? __ldcg(ypiece(r)) : make_uint4(0, 0, 0, 0);
-                }
-            }
             {
                 float yd[32], yo[32];
                 tc::tmem_ld32(tmem + lane_base + gcol(k) + 64 * hh + 32 * hsub, yd);
@@ -924,16 +916,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             for (int j = 0; j < 4; ++j) {
                 const int r = cr + 32 * j;
                 if (r < cnt) {
-                    uint4 v = *reinterpret_cast<const uint4 *>(sm + kOffS + r * 256 + ((cp ^ (r & 15)) << 4));
-                    if (!first) {
-                        float a[8], c8[8];
-                        unpack8(v, a);
-                        unpack8(prev[j], c8);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) a[q] += c8[q];
-                        v = pack8(a);
+                    const uint4 v = *reinterpret_cast<const uint4 *>(sm + kOffS + r * 256 +
+                                                                     ((cp ^ (r & 15)) << 4));
+                    if (first) {
+                        *ypiece(r) = v;
+                    } else {
+                        // second to reach the chunk: add to the partner's rows
+                        // at L2 (bf16 reductions, ordered after the partner's
+                        // release through thread 0's acquire and the barrier)
+                        asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};"
+                                     :: "l"(ypiece(r)), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                                     : "memory");
                     }
-                    *ypiece(r) = v;
                 }
             }
             alu_sync();   // rows stored; the staging buffer is rewritten by the next chunk's phase D
