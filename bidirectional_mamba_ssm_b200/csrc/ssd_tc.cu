@@ -83,7 +83,8 @@ constexpr uint32_t kOffCum = kOffS + 32768;      // f32[2][2][128] prefix sums o
 constexpr uint32_t kOffDt = kOffCum + 2048;      // f32[2][2][128] dt
 constexpr uint32_t kOffFB = kOffDt + 2048;       // f32[2][2][128] exp(c_R - c_s) dt_s, R = block end
 constexpr uint32_t kOffWgt = kOffFB + 2048;      // f32[2][2][128] exp(c_last - c_s) dt_s
-constexpr uint32_t kOffConvW = kOffWgt + 2048;   // float4[128] conv taps of x
+constexpr uint32_t kOffF4 = kOffWgt + 2048;      // f32[2][2][128] exp(c_R4 - c_s) dt_s, R4 = s | 3
+constexpr uint32_t kOffConvW = kOffF4 + 2048;    // float4[128] conv taps of x
 constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
 constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x12 + 2 flag pointers (see the kernel)
 constexpr uint32_t kOffTmem = kOffMbar + 112;    // u32 TMEM base
@@ -295,6 +296,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     float *dts = reinterpret_cast<float *>(sm + kOffDt);
     float *fB = reinterpret_cast<float *>(sm + kOffFB);
     float *wgt = reinterpret_cast<float *>(sm + kOffWgt);
+    float *f4 = reinterpret_cast<float *>(sm + kOffF4);
     float4 *convw = reinterpret_cast<float4 *>(sm + kOffConvW);
     float *convb = reinterpret_cast<float *>(sm + kOffConvB);
     int *flag_slot = reinterpret_cast<int *>(sm + kOffFlag);
@@ -415,16 +417,19 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
         }
         // per-slot decay factors, from the sums the other lanes just wrote:
-        // fB = exp(c_R - c_s) dt_s (R = end of s's 32-slot block) and
-        // w = exp(c_last - c_s) dt_s
+        // w = exp(c_last - c_s) dt_s, fB = exp(c_R - c_s) dt_s (R = end of
+        // s's 32-slot block) and f4 = exp(c_R4 - c_s) dt_s (R4 = s | 3)
         __syncwarp();
 #pragma unroll
         for (int i = 0; i < kHeads * kQ / 32; ++i) {
             const int e = (k & 1) * kHeads * kQ + 32 * i + lane;   // [parity][head][slot]
             const float cs = cum[e];
             const float d = dts[e];
-            fB[e] = tc::exp2_approx(cum[e | 31] - cs) * d;
             wgt[e] = tc::exp2_approx(cum[e | (kQ - 1)] - cs) * d;
+            if constexpr (!kStateOnly) {   // M's factors; the state-only pass needs w only
+                fB[e] = tc::exp2_approx(cum[e | 31] - cs) * d;
+                f4[e] = tc::exp2_approx(cum[e | 3] - cs) * d;
+            }
         }
     };
 
@@ -805,20 +810,35 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                                     packed[i] = tc::pack_bf16x2(gv[2 * i] * et * fbh[2 * i],
                                                                 gv[2 * i + 1] * et * fbh[2 * i + 1]);
                             } else {
-                                // diagonal block: one exponential per element, D on the diagonal
+                                // diagonal block, D on the diagonal
                                 const float *ch_ = cumk + 32 * jb;
-                                const float *dh_ = dtsk + 32 * jb;
                                 const int r31 = row & 31;
-                                float m[32];
+                                if (ch_[0] - ch_[31] <= 60.0f) {   // warp-uniform (head, block)
+                                    // 4-slot sub-blocks: exp(c_t - c_s) = exp(c_t - c_R4)
+                                    // exp(c_R4 - c_s), R4 = s | 3.  With the block's whole
+                                    // decay at most 2^60 neither factor overflows; for s <= t
+                                    // the product is the decay itself
+                                    const float *f4h = f4 + ((k & 1) * kHeads + hh) * kQ + 32 * jb;
+                                    float rf[8];
 #pragma unroll
-                                for (int i = 0; i < 32; ++i) {
-                                    const float e = tc::exp2_approx(fminf(ct - ch_[i], 0.0f));
-                                    const float add = (i == r31) ? Dh : 0.0f;
-                                    const float v = fmaf(gv[i] * e, dh_[i], add);
-                                    m[i] = (i <= r31) ? v : 0.0f;
+                                    for (int j = 0; j < 8; ++j) rf[j] = tc::exp2_approx(ct - ch_[4 * j + 3]);
+#pragma unroll
+                                    for (int i = 0; i < 32; ++i) {
+                                        const float v = fmaf(gv[i] * rf[i >> 2], f4h[i], (i == r31) ? Dh : 0.0f);
+                                        gv[i] = (i <= r31) ? v : 0.0f;
+                                    }
+                                } else {
+                                    // steep decays: one exponential per element, each <= 1
+                                    const float *dh_ = dtsk + 32 * jb;
+#pragma unroll
+                                    for (int i = 0; i < 32; ++i) {
+                                        const float e = tc::exp2_approx(fminf(ct - ch_[i], 0.0f));
+                                        const float v = fmaf(gv[i] * e, dh_[i], (i == r31) ? Dh : 0.0f);
+                                        gv[i] = (i <= r31) ? v : 0.0f;
+                                    }
                                 }
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) packed[i] = tc::pack_bf16x2(m[2 * i], m[2 * i + 1]);
+                                for (int i = 0; i < 16; ++i) packed[i] = tc::pack_bf16x2(gv[2 * i], gv[2 * i + 1]);
                             }
                         }
                         tc::tmem_st16(tmem + lane_base + mc + 64 * hh + 16 * jb, packed);
