@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -97,16 +98,25 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_sha(text):
+    """sha256[:16] of a C/CUDA source with its comments and whitespace
+    removed: the same for two versions that differ only in comments."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = re.sub(r"\s+", " ", text).strip()
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
+
+
 def kernel_traffic(kernel_file):
     """dram bytes per launch from the committed ncu summary, if it was taken
-    on the current source of the kernel (sha256 recorded there); else None."""
+    on the current code of the kernel (code_sha recorded there); else None."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     src = os.path.join(ROOT, "bidirectional_mamba_ssm_b200", "csrc", kernel_file)
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        sha = code_sha(open(src).read())
         for line in open(path):
             parts = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
-            if parts.get("file") == kernel_file and parts.get("sha") == sha:
+            if parts.get("file") == kernel_file and parts.get("code_sha") == sha:
                 return float(parts["dram_bytes_per_launch"])
     except OSError:
         pass

@@ -18,9 +18,13 @@
 // The reverse stream is the same computation in walk order: chunk slots map
 // to tokens through t = len-1-s; no flipped copy of any tensor is made.
 //
-// Mapping: one CTA (512 threads) owns (batch b, head pair, direction) and
-// walks the chunks of its sequence.  The two heads share B, C and G, so G is
-// computed once per chunk for both.  Per chunk (all M = 128):
+// Mapping: one CTA owns (batch b, head pair, direction) and walks the chunks
+// of its sequence (or of one segment of it).  Warps: 16 compute warps (512
+// threads: conv, M, state scaling, epilogue), one producer warp (every MMA
+// and TMA load, and the handshake releases) and one helper warp (dt copies,
+// prefix sums and per-slot decay factors, up to two chunks ahead).  The two
+// heads share B, C and G, so G is computed once per chunk for both.  Per
+// chunk (all M = 128):
 //     G        = C . B^T           A = C [t][n] K-major (smem), B = B [s][n] K-major
 //     Yd_h     = M_h . X_h         A = M_h in TMEM,            B = X_h [s][p] MN-major
 //     Yo       = C . [S_0;S_1]^T   A = C,                      B = S^T [n][p'] MN-major
@@ -37,13 +41,17 @@
 // and stride offset = 1024 B between groups of 8 rows along K.
 // Decay factors: for s in a 32-slot block below t's block,
 // exp(c_t - c_s) = exp(c_t - c_R) exp(c_R - c_s) with R the block's last
-// slot; both factors are <= 1, so nothing overflows, and only the diagonal
-// 32 x 32 blocks need one exponential per element.
+// slot; both factors are <= 1, so nothing overflows.  The diagonal 32 x 32
+// blocks factorise the same way through 4-slot sub-blocks when the block's
+// whole decay is at most 2^60 (so the row factor, >= 1 inside t's own
+// sub-block, stays finite), else take one exponential per element.
 //
 // Forward+reverse sum: the two CTAs of a (b, head pair) meet per token chunk
 // through a two-counter handshake in the caller's workspace: the first to
-// finish a chunk writes its output (bf16), the second adds its own to it.
-// The second one's wait is bounded; the first never waits.
+// finish a chunk writes its output (bf16), the second adds its own to it
+// with bf16 reductions at L2.  The second one's wait is bounded; the first
+// never waits.  (Untied directions with concatenated outputs, kConcat, do
+// not meet: each direction stores its own half of every output row.)
 #include "common.cuh"
 #include "dispatch.h"
 #include "tc_ptx.cuh"
