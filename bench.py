@@ -68,7 +68,9 @@ def workload_spec(name):
 
 
 def algorithmic(w, batch, seqlen, decode=False, untied=False):
-    """Algorithmic bytes and flops of one step (definitions in the design doc).
+    """Algorithmic bytes and flops of one step: the bytes the operation must
+    move through HBM once and the flops of its chunked form, counted with a
+    fixed chunk length so that the kernel's own chunking cannot change them.
 
     bytes/token = raw xBC in (H*P + 2N) + dt (H) + y out (H*P), in the
     activation dtype; decode adds the fp32 state read (H*P*N*4 per stream)
