@@ -199,3 +199,22 @@ def test_binding_argument_counts_match_the_header(lib):
     assert set(arity) == set(lib.EXPORTED)
     for name, n in arity.items():
         assert len(getattr(so, name).argtypes) == n, (name, len(getattr(so, name).argtypes), n)
+
+
+def test_plain_c_program_uses_the_abi(lib, tmp_path):
+    """The boundary is a C ABI: a C99 program that includes only
+    include/bimamba.h and links libbimamba.so builds with gcc and gets the
+    documented answers from the entry points that need no device."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_host"
+    libdir = os.path.dirname(lib.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_host.c"), "-L", libdir, "-lbimamba",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "abi ok"
