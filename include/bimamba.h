@@ -259,6 +259,9 @@ int bimamba_shard_states(const bimamba_dims *d, const void *xbc, const void *dt,
  *                this shard (the sequence's final state on the last rank)
  *   y          : (batch, len, H*P) dtype -- the shard's outputs
  * Concatenating every rank's y gives bimamba_ssd_fwd_rev on the whole sequence.
+ * A shard must hold at least one token (an empty shard returns
+ * BIMAMBA_ERR_INVALID here; bimamba_shard_states reports it as zero states
+ * and zero decay, which leave the crossing state unchanged).
  */
 int bimamba_ssd_fwd_rev_shard(const bimamba_dims *d, const void *xbc,
                               const void *dt, const float *A, const float *D,
