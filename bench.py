@@ -44,7 +44,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer1p3b", "long131k", "decode", "untied1p3b"],
+    ap.add_argument("--workload", choices=["layer1p3b", "long131k", "decode", "untied1p3b", "sweep"],
                     default="layer1p3b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
@@ -54,6 +54,9 @@ def parse_args():
 
 
 # --------------------------------------------------------------------------- workloads
+SWEEP_LENGTHS = (1024, 4096, 16384, 65536, 262144)
+
+
 def workload_spec(name):
     from bidirectional_mamba_ssm_b200 import inputs as I
     if name == "layer1p3b":
@@ -64,6 +67,8 @@ def workload_spec(name):
         return I.LAYER_1P3B, I.DECODE_STREAMS, I.DECODE_BLOCK
     if name == "untied1p3b":   # the same layer with untied directions, outputs concatenated
         return I.LAYER_1P3B, I.LAYER_1P3B.batch, I.LAYER_1P3B.seqlen
+    if name == "sweep":   # one sequence, prefill at 1k..256k tokens; the line's value at 256k
+        return I.LONG_131K, 1, SWEEP_LENGTHS[-1]
     raise ValueError(name)
 
 
@@ -329,6 +334,12 @@ def run_ours(args):
         "roofline": roof, "roofline_hbm_context": hbm_ctx,
         "e2e": e2e, "clocks": clocks, "gpu_launches": launches,
     }
+    if args.workload == "sweep":
+        del g, y, ws
+        torch.cuda.empty_cache()
+        result["config"]["workload"] = (f"sweep: one sequence, prefill at {SWEEP_LENGTHS[0]}.."
+                                        f"{SWEEP_LENGTHS[-1]} tokens, H64x64 N128 bf16")
+        result["sweep"] = run_sweep(args, lib, w, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.workload)
     if rank == 0:
@@ -336,6 +347,51 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_sweep(args, lib, w, dev, peaks):
+    """Prefill time per token of one sequence at each length: the scan's
+    cost should be linear in the length (flat per token).  Every timed call
+    starts with L2 flushed (a 256 MB write between calls, outside the timed
+    region), so the short lengths, whose inputs would fit in L2, are timed
+    cold like the long ones."""
+    import torch
+    from bidirectional_mamba_ssm_b200 import inputs as I
+    H, P, N = w.heads, w.headdim, w.d_state
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    out = []
+    for L in SWEEP_LENGTHS:
+        g = I.make_inputs(w, seed=7, device=dev, seqlen=L, batch=1)
+        y = torch.empty((1, L, H * P), dtype=torch.bfloat16, device=dev)
+        ws = lib.new_workspace(lib.make_dims(1, L, H, P, N, torch.bfloat16), device=dev)
+
+        def call():
+            lib.bimamba_ssd_fwd_rev(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], None, None,
+                                    None, y, ws, heads=H, headdim=P, d_state=N)
+        for _ in range(max(3, args.warmup)):
+            call()
+        times = []
+        for _ in range(max(5, min(args.steps, 20))):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+        ms = statistics.median(times)
+        _, flops = algorithmic(w, 1, L)
+        plan = lib.bimamba_launch_plan(lib.make_dims(1, L, H, P, N, torch.bfloat16))
+        out.append({"seqlen": L, "ms_per_step": ms, "ns_per_token": ms * 1e6 / L,
+                    "tokens_per_s": L / (ms / 1e3),
+                    "tensor_frac": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                    "segments": plan["segments"], "state_only_items": plan["items"]})
+        del g, y, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, world, gr=None):
