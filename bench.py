@@ -2,12 +2,17 @@
 """Throughput of the bidirectional Mamba-2 mixer core on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload layer1p3b|long131k|decode] [--no-cpu-baseline]
+                    [--workload layer1p3b|long131k|decode|untied1p3b|sweep]
+                    [--no-cpu-baseline]
 
 One step = one bimamba_ssd_fwd_rev call over one batch of the workload
 (conv+SiLU both ways, forward and reverse SSD scans, summed output), inputs
 resident in HBM.  Default workload: b8 x L4096, 64 heads x headdim 64,
 d_state 128, bf16 activations, fp32 state (one 1.3B-model mixer layer).
+Other workloads: one 131072-token sequence; cached block decode (32 streams x
+64-token block); the layer with untied directions and concatenated outputs;
+and a prefill sweep of one sequence at 1k..256k tokens (the line's value at
+256k, a "sweep" field with every length).
 Every rank runs its own copy of the workload (independent sequences, no
 data-path collective): scaling is weak, value = all ranks' tokens / the
 slowest rank's time.  Rank 0 prints one JSON line.
