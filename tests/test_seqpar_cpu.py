@@ -108,3 +108,39 @@ def test_shards_shorter_than_the_halo_are_refused():
             seqpar.exchange_halos(torch.zeros(1, 3, 8))
     finally:
         dist.destroy_process_group()
+
+
+def test_orchestration_calls_match_the_binding_signatures():
+    """The recorders above accept anything; this binds the orchestration's
+    actual calls against the real binding functions' signatures, so that an
+    argument added, dropped or reordered in either place fails on CPU."""
+    import inspect
+    import torch.distributed as dist
+    from bidirectional_mamba_ssm_b200 import build
+    build.build()
+    from bidirectional_mamba_ssm_b200 import _lib, seqpar
+
+    class Binder:
+        def __init__(self):
+            self.bound = []
+
+        def __getattr__(self, name):
+            real = getattr(_lib, name)
+
+            def call(*a, **kw):
+                inspect.signature(real).bind(*a, **kw)   # raises TypeError on a mismatch
+                self.bound.append(name)
+            return call
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(_free_port())
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        b = Binder()
+        x = torch.zeros(1, 8, 24)
+        seqpar.bimamba_sequence_parallel(x, torch.zeros(1, 8, 2), torch.zeros(2), torch.zeros(2),
+                                         None, None, None, torch.zeros(1, 8, 8), None, heads=2,
+                                         headdim=4, d_state=8, kernels=b)
+        assert b.bound == ["bimamba_shard_states", "bimamba_ssd_fwd_rev_shard"]
+    finally:
+        dist.destroy_process_group()
