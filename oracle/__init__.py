@@ -57,6 +57,7 @@ def _load():
             lib.oracle_block_decode.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp,
                                                 i, i, i, i, i, i, i, dp, dp, dp]
             lib.oracle_bimamba_untied.argtypes = [dp] * 13 + [i] * 8 + [dp, dp]
+            lib.oracle_scan_backward.argtypes = [dp] * 8 + [i] * 7 + [dp] * 7
             _lib = lib
     return _lib
 
@@ -148,6 +149,36 @@ def bimamba(xbc, dt, A, D, conv_w=None, conv_b=None, *, heads, headdim, d_state,
     if want_dirs:
         out.append((yf, yr))
     return out[0] if len(out) == 1 else tuple(out)
+
+
+def scan_backward(x, B, C, dt, A, D, dy, init=None, reverse=False, grads=None):
+    """Gradients of L = sum(dy * y) for one direction of the scan (no conv),
+    y = scan(x, B, C, dt, A, D, init, reverse).  Returns a dict of float64
+    arrays (x, B, C, dt, A, D, init); pass `grads` to accumulate into it."""
+    lib = _load()
+    x, B, C, dt, A, D, dy, init = map(_f64, (x, B, C, dt, A, D, dy, init))
+    bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if grads is None:
+        grads = {"x": np.zeros_like(x), "B": np.zeros_like(B), "C": np.zeros_like(C),
+                 "dt": np.zeros_like(dt), "A": np.zeros_like(A), "D": np.zeros_like(D),
+                 "init": np.zeros((bsz, H, P, N))}
+    lib.oracle_scan_backward(_ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(D), _ptr(init),
+                             _ptr(dy), bsz, L, H, P, N, G, int(bool(reverse)), _ptr(grads["x"]),
+                             _ptr(grads["B"]), _ptr(grads["C"]), _ptr(grads["dt"]),
+                             _ptr(grads["A"]), _ptr(grads["D"]), _ptr(grads["init"]))
+    return grads
+
+
+def bimamba_backward(x, B, C, dt, A, D, dy, init=None):
+    """Gradients of L = sum(dy * y) for the bidirectional scan without conv,
+    y = scan(forward, from init) + scan(reverse, from zero): the two
+    directions' adjoints summed (the initial state only enters forward)."""
+    g = scan_backward(x, B, C, dt, A, D, dy, init=init, reverse=False)
+    init_grad = g["init"].copy()
+    g = scan_backward(x, B, C, dt, A, D, dy, init=None, reverse=True, grads=g)
+    g["init"] = init_grad
+    return g
 
 
 def bimamba_untied(xbc_f, xbc_r, dt_f, dt_r, A_f, A_r, D_f, D_r, conv_w_f=None, conv_w_r=None,

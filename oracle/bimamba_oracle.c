@@ -326,3 +326,93 @@ void oracle_bimamba_untied(const double *xbc_f, const double *xbc_r,
     }
     free(act); free(x); free(Bm); free(Cm); free(of); free(orv);
 }
+
+/*
+ * Backward of one direction of the selective scan (no conv): the adjoint of
+ * the recurrence above, for the training objective the cached-decode page's
+ * block-causal training implies.  Given dy = dL/dy (same shape as y), it ADDS
+ * dL/d(input) into the gradient buffers (any of which may be NULL), so that
+ * calling it once per direction accumulates the bidirectional gradient.
+ * With g_s = dL/dh_s carried backward along the walk:
+ *   g_s      = dy_s C_s^T + a_{s+1} g_{s+1}
+ *   dC_s    += h_s^T dy_s            dD   += dy_s . x_s
+ *   dx_s    += D dy_s + dt_s g_s B_s dB_s += dt_s g_s^T x_s
+ *   ddt_s   += <g_s, x_s B_s^T> + A a_s <g_s, h_{s-1}>
+ *   dA      += dt_s a_s <g_s, h_{s-1}>
+ *   dinit   += a_0 g_0    (the state entering the walk)
+ * Shapes as in oracle_scan; dA, dD : (H); dinit : (batch, H, P, N).
+ * Sequential (the group-shared B, C and the per-head A, D gradients are sums
+ * over heads, batch and time).
+ */
+void oracle_scan_backward(const double *x, const double *Bm, const double *Cm,
+                          const double *dt, const double *A, const double *D,
+                          const double *init, const double *dy, int batch,
+                          int len, int H, int P, int N, int G, int reverse,
+                          double *dx, double *dB, double *dC, double *ddt,
+                          double *dA, double *dD, double *dinit)
+{
+    int hpg = H / G;
+    size_t pn = (size_t)P * N;
+    double *hs = (double *)malloc(sizeof(double) * pn * (size_t)(len + 1));
+    double *g = (double *)malloc(sizeof(double) * pn);
+    for (int b = 0; b < batch; ++b) {
+        for (int h = 0; h < H; ++h) {
+            int grp = h / hpg;
+            /* forward pass, keeping every state: hs[0] = entering state,
+               hs[s + 1] = state after walk step s */
+            if (init)
+                memcpy(hs, init + ((size_t)b * H + h) * pn, sizeof(double) * pn);
+            else
+                memset(hs, 0, sizeof(double) * pn);
+            for (int s = 0; s < len; ++s) {
+                int t = reverse ? len - 1 - s : s;
+                double d = dt[((size_t)b * len + t) * H + h];
+                double a = exp(d * A[h]);
+                const double *xt = x + (((size_t)b * len + t) * H + h) * P;
+                const double *bt = Bm + (((size_t)b * len + t) * G + grp) * N;
+                const double *prev = hs + (size_t)s * pn;
+                double *cur = hs + (size_t)(s + 1) * pn;
+                for (int p = 0; p < P; ++p)
+                    for (int n = 0; n < N; ++n)
+                        cur[(size_t)p * N + n] = a * prev[(size_t)p * N + n] + d * xt[p] * bt[n];
+            }
+            /* backward along the walk */
+            memset(g, 0, sizeof(double) * pn);
+            for (int s = len - 1; s >= 0; --s) {
+                int t = reverse ? len - 1 - s : s;
+                size_t ti = (size_t)b * len + t;
+                double d = dt[ti * H + h];
+                double a = exp(d * A[h]);
+                const double *xt = x + (ti * H + h) * P;
+                const double *bt = Bm + (ti * G + grp) * N;
+                const double *ct = Cm + (ti * G + grp) * N;
+                const double *dyt = dy + (ti * H + h) * P;
+                const double *cur = hs + (size_t)(s + 1) * pn;
+                const double *prev = hs + (size_t)s * pn;
+                double da = 0.0, dd_in = 0.0, dDh = 0.0;
+                for (int p = 0; p < P; ++p) {
+                    double gx = 0.0;
+                    for (int n = 0; n < N; ++n) {
+                        double *gp = g + (size_t)p * N + n;
+                        *gp += dyt[p] * ct[n];
+                        if (dC) dC[(ti * G + grp) * N + n] += cur[(size_t)p * N + n] * dyt[p];
+                        if (dB) dB[(ti * G + grp) * N + n] += d * (*gp) * xt[p];
+                        gx += (*gp) * bt[n];
+                        da += (*gp) * prev[(size_t)p * N + n];
+                        dd_in += (*gp) * xt[p] * bt[n];
+                    }
+                    if (dx) dx[(ti * H + h) * P + p] += D[h] * dyt[p] + d * gx;
+                    dDh += dyt[p] * xt[p];
+                }
+                if (dD) dD[h] += dDh;
+                if (ddt) ddt[ti * H + h] += dd_in + A[h] * a * da;
+                if (dA) dA[h] += d * a * da;
+                for (size_t i = 0; i < pn; ++i) g[i] *= a;
+            }
+            if (dinit)
+                for (size_t i = 0; i < pn; ++i) dinit[((size_t)b * H + h) * pn + i] += g[i];
+        }
+    }
+    free(hs);
+    free(g);
+}

@@ -391,3 +391,70 @@ def test_untied_streams_read_only_their_own_parameters():
     assert np.max(np.abs(y1[..., H * P:] - y2[..., H * P:])) > 1e-3
     y3, _ = run(r1, r1, w1)
     np.testing.assert_array_equal(y3[..., H * P:], y1[..., H * P:])
+
+
+# ------------------------------------------------------- backward (adjoint)
+def _loss(x, B, C, dt, A, D, dy, init, reverse):
+    y = oracle.scan(x, B, C, dt, A, D, init=init, reverse=reverse)
+    return float(np.sum(y * dy))
+
+
+def _fd_grad(f, arr, eps=1e-6):
+    """Central finite differences of the scalar f() w.r.t. every element of
+    arr (perturbed in place)."""
+    out = np.zeros_like(arr)
+    it = np.nditer(arr, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        v = arr[i]
+        arr[i] = v + eps
+        hi = f()
+        arr[i] = v - eps
+        lo = f()
+        arr[i] = v
+        out[i] = (hi - lo) / (2 * eps)
+    return out
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("memory", ["short", "long"])
+def test_scan_backward_matches_finite_differences(reverse, memory):
+    """The adjoint recurrence against central differences of the forward
+    recurrence, for every element of every input (x, B, C, dt, A, D and the
+    initial state), one direction at a time, with two heads sharing a group."""
+    rng = np.random.default_rng(11 + reverse)
+    L, H, P, N, G = 6, 2, 2, 3, 1
+    a = (1.0, 4.0) if memory == "short" else (1e-3, 1e-2)
+    x, B, C, dt, A, D = _rand(rng, 1, L, H, P, N, G, *a)
+    dy = rng.normal(size=x.shape)
+    init = rng.normal(0, 0.5, (1, H, P, N)) if not reverse else None
+    g = oracle.scan_backward(x, B, C, dt, A, D, dy, init=init, reverse=reverse)
+    inputs = {"x": x, "B": B, "C": C, "dt": dt, "A": A, "D": D}
+    if init is not None:
+        inputs["init"] = init
+    for name, arr in inputs.items():
+        fd = _fd_grad(lambda: _loss(x, B, C, dt, A, D, dy, init, reverse), arr)
+        scale = max(1.0, np.max(np.abs(fd)))
+        assert np.max(np.abs(g[name] - fd)) <= 1e-6 * scale, name
+
+
+def test_bidirectional_backward_matches_finite_differences():
+    """Both directions' adjoints summed, against central differences of
+    y = forward(init) + reverse(0)."""
+    rng = np.random.default_rng(21)
+    L, H, P, N, G = 5, 2, 2, 2, 1
+    x, B, C, dt, A, D = _rand(rng, 2, L, H, P, N, G, 1.0, 8.0)
+    dy = rng.normal(size=x.shape)
+    init = rng.normal(0, 0.5, (2, H, P, N))
+
+    def loss():
+        yf = oracle.scan(x, B, C, dt, A, D, init=init)
+        yr = oracle.scan(x, B, C, dt, A, D, reverse=True)
+        return float(np.sum((yf + yr) * dy))
+    g = oracle.bimamba_backward(x, B, C, dt, A, D, dy, init=init)
+    for name, arr in {"x": x, "B": B, "C": C, "dt": dt, "A": A, "D": D, "init": init}.items():
+        fd = _fd_grad(loss, arr)
+        scale = max(1.0, np.max(np.abs(fd)))
+        assert np.max(np.abs(g[name] - fd)) <= 1e-6 * scale, name
+    # D enters each direction once per token: dL/dD_h = 2 sum_t dy_t . x_t
+    np.testing.assert_allclose(g["D"], 2 * np.einsum("blhp,blhp->h", dy, x), rtol=1e-12)
