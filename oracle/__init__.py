@@ -58,6 +58,7 @@ def _load():
                                                 i, i, i, i, i, i, i, dp, dp, dp]
             lib.oracle_bimamba_untied.argtypes = [dp] * 13 + [i] * 8 + [dp, dp]
             lib.oracle_scan_backward.argtypes = [dp] * 8 + [i] * 7 + [dp] * 7
+            lib.oracle_conv_backward.argtypes = [dp] * 4 + [i] * 5 + [dp] * 3
             _lib = lib
     return _lib
 
@@ -179,6 +180,51 @@ def bimamba_backward(x, B, C, dt, A, D, dy, init=None):
     g = scan_backward(x, B, C, dt, A, D, dy, init=None, reverse=True, grads=g)
     g["init"] = init_grad
     return g
+
+
+def conv_backward(u, w, bias, dout, reverse=False):
+    """Gradients of L = sum(dout * conv_silu(u)) w.r.t. u, w and bias (no
+    tail): returns (du, dw, dbias)."""
+    lib = _load()
+    u, w, bias, dout = map(_f64, (u, w, bias, dout))
+    bsz, L, ch = u.shape
+    du, dw, db = np.zeros_like(u), np.zeros_like(w), np.zeros(ch)
+    lib.oracle_conv_backward(_ptr(u), _ptr(w), _ptr(bias), _ptr(dout), bsz, L, ch, w.shape[1],
+                             int(bool(reverse)), _ptr(du), _ptr(dw), _ptr(db))
+    return du, dw, db
+
+
+def bimamba_mixer_backward(xbc, dt, A, D, conv_w, conv_b, dy, *, heads, headdim, d_state,
+                           init=None):
+    """Gradients of L = sum(dy * y) for the whole bidirectional mixer core
+    (conv+SiLU per direction, both scans, summed; one group): each
+    direction's scan adjoint gives the gradient of its activated x, B and C,
+    which its conv's backward carries to the raw xBC and the conv taps.
+    Returns a dict: xbc, dt, A, D, conv_w, conv_b, init."""
+    xbc, dt, A, D, conv_w, conv_b, dy, init = map(_f64, (xbc, dt, A, D, conv_w, conv_b, dy, init))
+    bsz, L, ch = xbc.shape
+    H, P, N = heads, headdim, d_state
+    out = {"xbc": np.zeros_like(xbc), "dt": np.zeros_like(dt), "A": np.zeros_like(A),
+           "D": np.zeros_like(D), "conv_w": np.zeros_like(conv_w), "conv_b": np.zeros(ch),
+           "init": np.zeros((bsz, H, P, N))}
+    for reverse in (False, True):
+        act = conv(xbc, conv_w, conv_b, reverse=reverse)
+        x = act[..., :H * P].reshape(bsz, L, H, P)
+        Bm = act[..., H * P:H * P + N].reshape(bsz, L, 1, N)
+        Cm = act[..., H * P + N:].reshape(bsz, L, 1, N)
+        g = scan_backward(x, Bm, Cm, dt, A, D, dy.reshape(bsz, L, H, P),
+                          init=None if reverse else init, reverse=reverse)
+        dact = np.concatenate([g["x"].reshape(bsz, L, H * P), g["B"].reshape(bsz, L, N),
+                               g["C"].reshape(bsz, L, N)], axis=-1)
+        du, dw, db = conv_backward(xbc, conv_w, conv_b, dact, reverse=reverse)
+        out["xbc"] += du
+        out["conv_w"] += dw
+        out["conv_b"] += db
+        for k in ("dt", "A", "D"):
+            out[k] += g[k]
+        if not reverse:
+            out["init"] += g["init"]
+    return out
 
 
 def bimamba_untied(xbc_f, xbc_r, dt_f, dt_r, A_f, A_r, D_f, D_r, conv_w_f=None, conv_w_r=None,

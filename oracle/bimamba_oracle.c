@@ -416,3 +416,39 @@ void oracle_scan_backward(const double *x, const double *Bm, const double *Cm,
     free(hs);
     free(g);
 }
+
+/*
+ * Backward of oracle_conv (with SiLU) without a tail: given dout = dL/dout,
+ * ADDS dL/du, dL/dw and dL/dbias (any may be NULL).  With pre the conv's
+ * pre-activation, silu'(v) = s(v) (1 + v (1 - s(v))), s the logistic sigmoid:
+ *   dpre[t,c]    = dout[t,c] silu'(pre[t,c])
+ *   du[src,c]   += w[c,j] dpre[t,c]   for each tap j (src as in the forward)
+ *   dw[c,j]     += dpre[t,c] u[src,c]
+ *   dbias[c]    += dpre[t,c]
+ */
+void oracle_conv_backward(const double *u, const double *w, const double *bias,
+                          const double *dout, int batch, int len, int ch, int K,
+                          int reverse, double *du, double *dw, double *dbias)
+{
+    for (int b = 0; b < batch; ++b) {
+        for (int t = 0; t < len; ++t) {
+            for (int c = 0; c < ch; ++c) {
+                double pre = bias ? bias[c] : 0.0;
+                for (int j = 0; j < K; ++j) {
+                    long src = reverse ? (long)t + (K - 1) - j : (long)t - (K - 1) + j;
+                    if (src >= 0 && src < len)
+                        pre += w[(size_t)c * K + j] * u[((size_t)b * len + src) * ch + c];
+                }
+                double sg = 1.0 / (1.0 + exp(-pre));
+                double dpre = dout[((size_t)b * len + t) * ch + c] * sg * (1.0 + pre * (1.0 - sg));
+                if (dbias) dbias[c] += dpre;
+                for (int j = 0; j < K; ++j) {
+                    long src = reverse ? (long)t + (K - 1) - j : (long)t - (K - 1) + j;
+                    if (src < 0 || src >= len) continue;
+                    if (du) du[((size_t)b * len + src) * ch + c] += w[(size_t)c * K + j] * dpre;
+                    if (dw) dw[(size_t)c * K + j] += dpre * u[((size_t)b * len + src) * ch + c];
+                }
+            }
+        }
+    }
+}
