@@ -7,15 +7,20 @@
 
 One step = one bimamba_ssd_fwd_rev call over one batch of the workload
 (conv+SiLU both ways, forward and reverse SSD scans, summed output), inputs
-resident in HBM.  Default workload: b8 x L4096, 64 heads x headdim 64,
-d_state 128, bf16 activations, fp32 state (one 1.3B-model mixer layer).
-Other workloads: one 131072-token sequence; cached block decode (32 streams x
-64-token block); the layer with untied directions and concatenated outputs;
-and a prefill sweep of one sequence at 1k..256k tokens (the line's value at
-256k, a "sweep" field with every length).
+resident in HBM.  Default workload: the largest single-GPU configuration,
+one 131072-token sequence, 64 heads x headdim 64, d_state 128, bf16
+activations, fp32 state; the same line carries the 1.3B-layer workload
+(b8 x L4096) as its "layer1p3b" field.  Other workloads: the 1.3B layer
+alone; cached block decode (32 streams x 64-token block, HBM-cold: the
+timed steps rotate over state/input sets larger than L2); the layer with
+untied directions and concatenated outputs; and a sweep of one sequence at
+1k..256k tokens, prefill and cached decode at each length (the line's value
+at 256k, a "sweep" field with every length).
 Every rank runs its own copy of the workload (independent sequences, no
 data-path collective): scaling is weak, value = all ranks' tokens / the
-slowest rank's time.  Rank 0 prints one JSON line.
+slowest rank's time.  Rank 0 prints one JSON line.  `--gpus N` without a
+torchrun environment launches N local ranks itself (torch.distributed.run);
+under torchrun, N must equal WORLD_SIZE.
 
 --impl reference times the CPU oracle (the double-precision sequential
 recurrence under oracle/) on the host cores, a bounded sample per step, and
@@ -49,8 +54,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer1p3b", "long131k", "decode", "untied1p3b", "sweep"],
-                    default="layer1p3b")
+    ap.add_argument("--workload", choices=["long131k", "layer1p3b", "decode", "untied1p3b", "sweep"],
+                    default="long131k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--batch", type=int, default=None,
@@ -186,58 +191,114 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-# --------------------------------------------------------------------------- our arm
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
-    from datetime import timedelta
+# --------------------------------------------------------------------------- peaks
+def tensor_peak(peaks, clocks):
+    """The bf16 tensor peak a kernel timed inside this run is held against.
 
-    from bidirectional_mamba_ssm_b200 import _lib as lib
-    from bidirectional_mamba_ssm_b200 import inputs as I
+    The burst figure (a cuBLAS GEMM timed alone, at full clock) applies when
+    the clocks sampled during the timed region show no power capping; when
+    sw_power_cap was active the burst figure is scaled by the sampled median
+    SM clock over the maximum clock.  Returns (TFLOP/s, rule)."""
+    burst = peaks["bf16_tflops"]
+    if not clocks:
+        return burst, "burst (no clock samples)"
+    if "sw_power_cap" in clocks.get("reasons", []):
+        f = clocks["sm_mhz"] / max(clocks["sm_max_mhz"], 1.0)
+        return burst * f, f"burst x median/max SM clock ({f:.3f}): sw_power_cap active"
+    return burst, "burst: no sw_power_cap in the clock samples"
+
+
+def roofline(peaks, peak_kind, clocks, nbytes, flops, kernel_s, decode, kernel_file):
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    tpeak, rule = tensor_peak(peaks, clocks)
+    t_tc = flops / (tpeak * 1e12)
+    if decode or t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": nbytes / kernel_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "peak_source": f"{peak_kind} (copy)"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / kernel_s / 1e12, "peak": tpeak,
+                "unit": "TFLOP/s", "peak_source": f"{peak_kind} ({rule})"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = kernel_traffic(kernel_file)
+    roof["kernel"] = kernel_file
+    ctx = {"achieved_gbs": nbytes / kernel_s / 1e9, "peak_gbs": peaks["hbm_gbs"],
+           "frac": nbytes / kernel_s / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
+           "algorithmic_flops": flops, "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6,
+           "tensor_peak_tflops": tpeak}
+    return roof, ctx
+
+
+# --------------------------------------------------------------------------- ranks
+def resolve_world(gpus, env):
+    """How this process runs `--gpus gpus` given its environment `env`:
+    ("run", world) inside a torchrun rank or for one GPU, ("spawn", gpus) to
+    launch gpus local ranks, ("refuse", why) when they disagree."""
+    if gpus < 1:
+        return "refuse", f"--gpus {gpus}: need at least one GPU"
+    ws = env.get("WORLD_SIZE")
+    if ws is None:
+        return ("spawn", gpus) if gpus > 1 else ("run", 1)
+    if int(ws) != gpus:
+        return "refuse", f"--gpus {gpus} but WORLD_SIZE={ws}: launch one rank per GPU"
+    return "run", int(ws)
+
+
+def spawn_ranks(n):
+    """Re-run this command as n local ranks under torch.distributed.run."""
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def combine_ranks(tokens, ms_total, per_call_ms, launches, device=None):
+    """Whole-job figures from each rank's own: all ranks' tokens, the slowest
+    rank's elapsed time and main-kernel time, every rank's launches."""
     from bidirectional_mamba_ssm_b200 import replicas
+    tokens, ms_total, _ = replicas.aggregate(tokens, ms_total, device=device)
+    _, per_call_ms, _ = replicas.aggregate(0, per_call_ms, device=device)
+    launches, _, _ = replicas.aggregate(launches, 1.0, device=device)
+    return tokens, ms_total, per_call_ms, int(launches)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream()
-    decode = args.workload == "decode"
-    untied = args.workload == "untied1p3b"
-    w, batch, seqlen = workload_spec(args.workload)
-    if args.batch is not None:
-        batch = args.batch
+
+# --------------------------------------------------------------------------- our arm
+DECODE_SETS = 4   # state/input sets the timed decode steps rotate over (> L2 in all)
+
+
+def build_step(lib, I, w, name, batch, seqlen, rank, dev):
+    """Inputs on the device and the step closure of one workload."""
+    import torch
     H, P, N = w.heads, w.headdim, w.d_state
-
-    # ---- inputs, generated on the device (seeded per rank); untied
-    # directions draw the reverse stream's inputs and parameters separately
-    g = I.make_inputs(w, seed=rank, device=dev, seqlen=seqlen, batch=batch,
-                      conv_bias=decode)
+    decode = name == "decode"
+    untied = name == "untied1p3b"
+    g = I.make_inputs(w, seed=rank, device=dev, seqlen=seqlen, batch=batch, conv_bias=decode)
     gr = I.make_inputs(w, seed=10000 + rank, device=dev, seqlen=seqlen, batch=batch) if untied else None
     y = torch.empty((batch, seqlen, (2 if untied else 1) * H * P), dtype=torch.bfloat16, device=dev)
     dims = lib.make_dims(batch, seqlen, H, P, N, torch.bfloat16)
     ws = lib.new_workspace(dims, device=dev)
+    extra = {}
     if decode:
-        # cached state from a forward scan over a seeded 65536-token prefix
-        state = torch.empty((batch, H, P, N), device=dev)
-        tail = torch.empty((batch, 4, w.channels), dtype=torch.bfloat16, device=dev)
-        pdims = lib.make_dims(1, I.DECODE_PREFIX, H, P, N, torch.bfloat16)
-        pws = lib.new_workspace(pdims, device=dev)
-        py = torch.empty((1, I.DECODE_PREFIX, H * P), dtype=torch.bfloat16, device=dev)
-        for s in range(batch):
-            pre = I.make_inputs(w, seed=1000 + batch * rank + s, device=dev,
-                                seqlen=I.DECODE_PREFIX, batch=1)
-            lib.bimamba_ssd_fwd_rev(pre["xbc"], pre["dt"], g["A"], g["D"], g["conv_w"], g["conv_b"],
-                                    None, state[s:s + 1], py, pws, heads=H, headdim=P, d_state=N)
-            tail[s] = pre["xbc"][0, -4:]
-        del pre, py, pws
+        state, tail = decode_cache(lib, I, w, batch, I.DECODE_PREFIX, g, rank, dev)
+        # Sets of (state, tail, block inputs, y) at distinct addresses: each
+        # timed step reads the set the previous DECODE_SETS - 1 steps did not
+        # touch, ~100 MB each, so its 64 MiB of cached state comes from HBM.
+        sets = [(state, tail, g["xbc"], g["dt"], y)]
+        for _ in range(DECODE_SETS - 1):
+            sets.append((state.clone(), tail.clone(), g["xbc"].clone(), g["dt"].clone(),
+                         torch.empty_like(y)))
+        it = [0]
+        extra.update(state=state, tail=tail)
 
         def step():
-            lib.bimamba_block_decode(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], g["conv_b"],
-                                     state, tail, y, None, None, ws, heads=H, headdim=P, d_state=N)
+            st, tl, xb, dtb, yy = sets[it[0] % DECODE_SETS]
+            it[0] += 1
+            lib.bimamba_block_decode(xb, dtb, g["A"], g["D"], g["conv_w"], g["conv_b"], st, tl, yy,
+                                     None, None, ws, heads=H, headdim=P, d_state=N)
     elif untied:
         def step():
             lib.bimamba_ssd_fwd_rev_untied(g, gr, None, None, y, ws, heads=H, headdim=P,
@@ -246,17 +307,44 @@ def run_ours(args):
         def step():
             lib.bimamba_ssd_fwd_rev(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], None, None,
                                     None, y, ws, heads=H, headdim=P, d_state=N)
+    return step, g, gr, dims, ws, extra
 
+
+def decode_cache(lib, I, w, streams, prefix, g, rank, dev, distinct=None):
+    """The cached forward state and conv tail of `streams` streams, each from
+    a forward scan over a seeded `prefix`-token prefix.  distinct = how many
+    streams get their own prefix (the rest repeat them; the step's cost does
+    not depend on the state's values); default all."""
+    import torch
+    H, P, N = w.heads, w.headdim, w.d_state
+    state = torch.empty((streams, H, P, N), device=dev)
+    tail = torch.empty((streams, 4, w.channels), dtype=torch.bfloat16, device=dev)
+    pdims = lib.make_dims(1, prefix, H, P, N, torch.bfloat16)
+    pws = lib.new_workspace(pdims, device=dev)
+    py = torch.empty((1, prefix, H * P), dtype=torch.bfloat16, device=dev)
+    k = streams if distinct is None else min(distinct, streams)
+    for s in range(k):
+        pre = I.make_inputs(w, seed=1000 + streams * rank + s, device=dev, seqlen=prefix, batch=1)
+        lib.bimamba_ssd_fwd_rev(pre["xbc"], pre["dt"], g["A"], g["D"], g["conv_w"], g["conv_b"],
+                                None, state[s:s + 1], py, pws, heads=H, headdim=P, d_state=N)
+        tail[s] = pre["xbc"][0, -4:]
+        del pre
+    for s in range(k, streams):
+        state[s] = state[s % k]
+        tail[s] = tail[s % k]
     torch.cuda.synchronize()
-    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
-    uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-    sampler = ClockSampler(gpu_id)
+    return state, tail
 
-    # ---- warm-up: at least W steps and at least ~1 s of load for the sampler
+
+def time_steps(args, lib, step, stream, world, dev):
+    """Warm-up, then exactly args.steps timed steps between barriers and
+    synchronisations; CUDA events around the whole region and, through the
+    library's timing hook, around each step's main kernel."""
+    import torch
+    import torch.distributed as dist
     t0 = time.time()
     n = 0
-    while n < args.warmup or time.time() - t0 < 1.0:
+    while n < args.warmup or time.time() - t0 < 1.0:   # and >= ~1 s of load for the sampler
         step()
         n += 1
         if n % 10 == 0:
@@ -264,7 +352,6 @@ def run_ours(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    # events the library records around its main scan kernel in each step
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     for a, b_ in kev:       # materialise the event handles before handing them over
@@ -284,69 +371,103 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     launches = lib.bimamba_launch_count() - launches0
-    clocks = sampler.stop()
     assert lib.bimamba_get_error() == lib.BIMAMBA_OK
-    ms_total = start.elapsed_time(end)
-    per_call_ms = statistics.mean(a.elapsed_time(b_) for a, b_ in kev)
-    tokens = batch * seqlen
-    # whole job: all ranks' tokens over the slowest rank's time
-    _, ms_total, _ = replicas.aggregate(tokens * args.steps, ms_total, device=dev)
-    _, per_call_ms, _ = replicas.aggregate(0, per_call_ms, device=dev)
-    launches, _, _ = replicas.aggregate(launches, 1.0, device=dev)
-    launches = int(launches)
-    ms_step = ms_total / args.steps
-    value = tokens * world / (ms_step / 1e3)
+    return start.elapsed_time(end), statistics.mean(a.elapsed_time(b_) for a, b_ in kev), launches
 
-    # ---- roofline of the dominant kernel (the main scan kernel of each step)
+
+def measure(args, lib, I, name, rank, world, dev, gpu_id, want_e2e=True):
+    """One workload's figures: whole-job tokens/s, the dominant kernel's
+    roofline, clocks during the timed region, launches, and (want_e2e) the
+    end-to-end figure through host buffers."""
+    import torch
+    stream = torch.cuda.current_stream()
+    w, batch, seqlen = workload_spec(name)
+    if args.batch is not None:
+        batch = args.batch
+    decode = name == "decode"
+    untied = name == "untied1p3b"
+    H, P, N = w.heads, w.headdim, w.d_state
+    step, g, gr, dims, ws, extra = build_step(lib, I, w, name, batch, seqlen, rank, dev)
+    torch.cuda.synchronize()
+    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+    sampler = ClockSampler(gpu_id)
+    ms_total, per_call_ms, launches = time_steps(args, lib, step, stream, world, dev)
+    clocks = sampler.stop()
+    tokens = batch * seqlen
+    tok_all, ms_total, per_call_ms, launches = combine_ranks(tokens * args.steps, ms_total,
+                                                             per_call_ms, launches, device=dev)
+    ms_step = ms_total / args.steps
+    value = tok_all / args.steps / (ms_step / 1e3)
     peaks, peak_kind = load_peaks()
     nbytes, flops = algorithmic(w, batch, seqlen, decode, untied)
-    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
-    kernel_s = per_call_ms / 1e3
     kernel_file = "ssd_tc.cu" if (P, N) == (64, 128) else "scan_seq.cu"
-    traffic = kernel_traffic(kernel_file)
-    if decode or t_hbm >= t_tc:
-        roof = {"bound": "hbm", "achieved": nbytes / kernel_s / 1e9, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s"}
+    roof, ctx = roofline(peaks, peak_kind, clocks, nbytes, flops, per_call_ms / 1e3, decode,
+                         kernel_file)
+    if decode:
+        wl = (f"cached block decode: {batch} streams x {seqlen}-token block, H64x64 N128 bf16, "
+              f"65536-token prefix state")
+        l2 = (f"HBM-cold: steps rotate over {DECODE_SETS} sets of state + block inputs + y "
+              f"(~{DECODE_SETS * 100} MB > 126 MB L2)")
     else:
-        roof = {"bound": "tensor", "achieved": flops / kernel_s / 1e12,
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic
-    roof["peak_source"] = f"{peak_kind} ({'sustained' if roof['bound'] == 'tensor' else 'copy'})"
-    roof["kernel"] = kernel_file
-    hbm_ctx = {"achieved_gbs": nbytes / kernel_s / 1e9, "peak_gbs": peaks["hbm_gbs"],
-               "frac": nbytes / kernel_s / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
-               "algorithmic_flops": flops, "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6}
+        wl = w.name + (", untied directions, outputs concatenated" if untied else "")
+        l2 = "inputs larger than L2 (xbc + y per step > 126 MB)"
+    out = {"value": value, "ms_per_step": ms_step, "workload": wl, "batch_per_gpu": batch,
+           "seqlen": seqlen, "l2": l2, "roofline": roof, "roofline_hbm_context": ctx,
+           "clocks": clocks, "gpu_launches": launches, "main_kernel_ms": per_call_ms}
+    if want_e2e:
+        out["e2e"] = run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode,
+                             extra.get("state"), extra.get("tail"), dev, world, gr)
+    del step, g, gr, ws, extra
+    torch.cuda.empty_cache()
+    return out
 
-    # ---- end to end through the public API with host buffers
-    e2e = run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, locals().get("state"),
-                  locals().get("tail"), dev, world, gr)
 
+def run_ours(args, world):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from bidirectional_mamba_ssm_b200 import _lib as lib
+    from bidirectional_mamba_ssm_b200 import inputs as I
+
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+
+    main_name = "long131k" if args.workload == "sweep" else args.workload
+    m = measure(args, lib, I, main_name, rank, world, dev, gpu_id)
+    w, _, _ = workload_spec(main_name)
     result = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "metric": METRIC, "value": m["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": (f"cached block decode: {batch} streams x {seqlen}-token block, "
-                                f"H64x64 N128 bf16, 65536-token prefix state") if decode else
-                   (w.name + ", untied directions, outputs concatenated") if untied else w.name,
-                   "batch_per_gpu": batch, "seqlen": seqlen, "heads": H, "headdim": P,
-                   "d_state": N, "state_dtype": "f32",
-                   "l2": "inputs larger than L2 (xbc + y per step > 126 MB)" if not decode
-                   else "state (64 MiB) + block inputs larger than L2 reuse window",
+        "config": {"workload": m["workload"], "batch_per_gpu": m["batch_per_gpu"],
+                   "seqlen": m["seqlen"], "heads": w.heads, "headdim": w.headdim,
+                   "d_state": w.d_state, "state_dtype": "f32", "l2": m["l2"],
                    "parallelism": f"independent replicas x{world} (no data-path collective)"},
-        "roofline": roof, "roofline_hbm_context": hbm_ctx,
-        "e2e": e2e, "clocks": clocks, "gpu_launches": launches,
+        "roofline": m["roofline"], "roofline_hbm_context": m["roofline_hbm_context"],
+        "e2e": m["e2e"], "clocks": m["clocks"], "gpu_launches": m["gpu_launches"],
     }
+    if args.workload == "long131k" and args.batch is None:
+        # the 1.3B-layer workload (b8 x L4096) measured in the same run
+        lm = measure(args, lib, I, "layer1p3b", rank, world, dev, gpu_id, want_e2e=False)
+        result["layer1p3b"] = {k: lm[k] for k in ("value", "ms_per_step", "workload",
+                                                  "batch_per_gpu", "seqlen", "roofline",
+                                                  "clocks", "gpu_launches")}
     if args.workload == "sweep":
-        del g, y, ws
-        torch.cuda.empty_cache()
-        result["config"]["workload"] = (f"sweep: one sequence, prefill at {SWEEP_LENGTHS[0]}.."
-                                        f"{SWEEP_LENGTHS[-1]} tokens, H64x64 N128 bf16")
-        result["sweep"] = run_sweep(args, lib, w, dev, peaks)
+        result["config"]["workload"] = (m["workload"] + f"; plus a sweep of one sequence, prefill "
+                                        f"and 32-stream 64-token cached decode at "
+                                        f"{SWEEP_LENGTHS[0]}..{SWEEP_LENGTHS[-1]} tokens")
+        result["sweep"] = run_sweep(args, lib, w, dev, rank, gpu_id)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, args.workload)
+        result["cpu_baseline"] = cpu_baseline(w, main_name)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -354,26 +475,29 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_sweep(args, lib, w, dev, peaks):
-    """Prefill time per token of one sequence at each length: the scan's
-    cost should be linear in the length (flat per token).  Every timed call
-    starts with L2 flushed (a 256 MB write between calls, outside the timed
-    region), so the short lengths, whose inputs would fit in L2, are timed
-    cold like the long ones."""
+def run_sweep(args, lib, w, dev, rank, gpu_id):
+    """Per context length L: the prefill (one L-token sequence through
+    bimamba_ssd_fwd_rev) and one cached 64-token block decode step of 32
+    streams whose state came from a forward scan over an L-token prefix.
+    The prefill's cost should grow linearly in L (flat per token), the
+    decode step's not at all (the cached state is O(1) in L).  Every timed
+    call starts with L2 flushed (a 256 MB write between calls, outside the
+    timed region), so the short lengths, whose inputs would fit in L2, are
+    timed cold like the long ones; the figure is the median of the calls."""
     import torch
     from bidirectional_mamba_ssm_b200 import inputs as I
     H, P, N = w.heads, w.headdim, w.d_state
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    out = []
-    for L in SWEEP_LENGTHS:
-        g = I.make_inputs(w, seed=7, device=dev, seqlen=L, batch=1)
-        y = torch.empty((1, L, H * P), dtype=torch.bfloat16, device=dev)
-        ws = lib.new_workspace(lib.make_dims(1, L, H, P, N, torch.bfloat16), device=dev)
+    S, blk = I.DECODE_STREAMS, I.DECODE_BLOCK
+    dw, _, _ = workload_spec("decode")
+    gd = I.make_inputs(dw, seed=rank, device=dev, seqlen=blk, batch=S, conv_bias=True)
+    yd = torch.empty((S, blk, H * P), dtype=torch.bfloat16, device=dev)
+    wsd = lib.new_workspace(lib.make_dims(S, blk, H, P, N, torch.bfloat16), device=dev)
+    peaks, _ = load_peaks()
+    sampler = ClockSampler(gpu_id)
 
-        def call():
-            lib.bimamba_ssd_fwd_rev(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], None, None,
-                                    None, y, ws, heads=H, headdim=P, d_state=N)
+    def cold_median(call):
         for _ in range(max(3, args.warmup)):
             call()
         times = []
@@ -387,16 +511,39 @@ def run_sweep(args, lib, w, dev, peaks):
             b.synchronize()
             times.append(a.elapsed_time(b))
         assert lib.bimamba_get_error() == lib.BIMAMBA_OK
-        ms = statistics.median(times)
-        _, flops = algorithmic(w, 1, L)
-        plan = lib.bimamba_launch_plan(lib.make_dims(1, L, H, P, N, torch.bfloat16))
-        out.append({"seqlen": L, "ms_per_step": ms, "ns_per_token": ms * 1e6 / L,
-                    "tokens_per_s": L / (ms / 1e3),
-                    "tensor_frac": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
-                    "segments": plan["segments"], "state_only_items": plan["items"]})
+        return statistics.median(times)
+
+    rows = []
+    for L in SWEEP_LENGTHS:
+        g = I.make_inputs(w, seed=7, device=dev, seqlen=L, batch=1)
+        y = torch.empty((1, L, H * P), dtype=torch.bfloat16, device=dev)
+        ws = lib.new_workspace(lib.make_dims(1, L, H, P, N, torch.bfloat16), device=dev)
+        ms = cold_median(lambda: lib.bimamba_ssd_fwd_rev(
+            g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], None, None, None, y, ws, heads=H,
+            headdim=P, d_state=N))
         del g, y, ws
         torch.cuda.empty_cache()
-    return out
+        # cached state after an L-token prefix (two distinct prefixes, repeated over the streams)
+        state, tail = decode_cache(lib, I, dw, S, L, gd, rank, dev, distinct=2)
+        dms = cold_median(lambda: lib.bimamba_block_decode(
+            gd["xbc"], gd["dt"], gd["A"], gd["D"], gd["conv_w"], gd["conv_b"], state, tail, yd,
+            None, None, wsd, heads=H, headdim=P, d_state=N))
+        del state, tail
+        torch.cuda.empty_cache()
+        _, flops = algorithmic(w, 1, L)
+        dbytes, _ = algorithmic(dw, S, blk, decode=True)
+        plan = lib.bimamba_launch_plan(lib.make_dims(1, L, H, P, N, torch.bfloat16))
+        rows.append({"seqlen": L, "ms_per_step": ms, "ns_per_token": ms * 1e6 / L,
+                     "tokens_per_s": L / (ms / 1e3), "flops": flops,
+                     "segments": plan["segments"], "state_only_items": plan["items"],
+                     "decode_ms_per_step": dms, "decode_tokens_per_s": S * blk / (dms / 1e3),
+                     "decode_hbm_frac": dbytes / (dms / 1e3) / 1e9 / peaks["hbm_gbs"]})
+    clocks = sampler.stop()
+    tpeak, rule = tensor_peak(peaks, clocks)
+    for r in rows:
+        r["tensor_frac"] = r.pop("flops") / (r["ms_per_step"] / 1e3) / 1e12 / tpeak
+        r["tensor_peak_rule"] = rule
+    return rows
 
 
 def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, world, gr=None):
@@ -554,8 +701,14 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
-    else:
-        run_ours(args)
+        return
+    how, arg = resolve_world(args.gpus, os.environ)
+    if how == "refuse":
+        print(f"bench.py: {arg}", file=sys.stderr)
+        sys.exit(2)
+    if how == "spawn":
+        sys.exit(spawn_ranks(arg))
+    run_ours(args, arg)
 
 
 if __name__ == "__main__":

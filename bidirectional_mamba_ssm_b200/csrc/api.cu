@@ -66,6 +66,30 @@ static int check_dims(const bimamba_dims *d)
 
 static int cuda_status(cudaError_t e) { return e == cudaSuccess ? BIMAMBA_OK : BIMAMBA_ERR_CUDA; }
 
+int check_block_decode(const bimamba_dims *d, const void *xbc_block, const void *dt_block,
+                       const float *A, const float *D, const float *conv_w, const float *conv_b,
+                       const float *state, const void *tail, const void *y, const float *state_out,
+                       const void *tail_out)
+{
+    int st = check_dims(d);
+    if (st != BIMAMBA_OK) return st;
+    if (d->batch == 0) return BIMAMBA_OK;
+    if (d->len == 0) return BIMAMBA_ERR_INVALID;
+    if (!xbc_block || !dt_block || !A || !D || !conv_w || !state || !tail || !y)
+        return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, y, state_out, tail_out};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
+    const size_t esz = d->dtype == BIMAMBA_F32 ? 4 : 2;
+    const int ch = d->heads * d->headdim + 2 * d->ngroups * d->d_state;
+    const size_t tail_bytes = (size_t)d->batch * 4 * ch * esz;
+    if (tail_out) {
+        const char *a = static_cast<const char *>(tail), *b = static_cast<const char *>(tail_out);
+        if (a < b + tail_bytes && b < a + tail_bytes) return BIMAMBA_ERR_INVALID;
+    }
+    return BIMAMBA_OK;
+}
+
 }  // namespace bimamba
 
 using namespace bimamba;
@@ -349,21 +373,11 @@ int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block, const voi
                          float *state_out, void *tail_out, void *workspace,
                          size_t workspace_bytes, bimamba_stream_t stream)
 {
-    int st = check_dims(d);
+    int st = check_block_decode(d, xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, y,
+                                state_out, tail_out);
     if (st != BIMAMBA_OK) return st;
-    if (d->batch == 0 || d->len == 0) return d->len == 0 && d->batch > 0 ? BIMAMBA_ERR_INVALID : BIMAMBA_OK;
-    if (!xbc_block || !dt_block || !A || !D || !conv_w || !state || !tail || !y)
-        return BIMAMBA_ERR_INVALID;
-    const void *ptrs[] = {xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, y, state_out, tail_out};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
-    const size_t esz = d->dtype == BIMAMBA_F32 ? 4 : 2;
+    if (d->batch == 0) return BIMAMBA_OK;
     const int ch = d->heads * d->headdim + 2 * d->ngroups * d->d_state;
-    const size_t tail_bytes = (size_t)d->batch * 4 * ch * esz;
-    if (tail_out) {
-        const char *a = static_cast<const char *>(tail), *b = static_cast<const char *>(tail_out);
-        if (a < b + tail_bytes && b < a + tail_bytes) return BIMAMBA_ERR_INVALID;
-    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     st = run_tied(d, xbc_block, dt_block, A, D, conv_w, conv_b, tail, state, state_out, y,
                   workspace, workspace_bytes, s);

@@ -39,11 +39,19 @@ struct Problem {
 };
 
 size_t workspace_bytes_for(const bimamba_dims &d);
+// argument checks of bimamba_block_decode (nothing launched); BIMAMBA_OK or an error
+int check_block_decode(const bimamba_dims *d, const void *xbc_block, const void *dt_block,
+                       const float *A, const float *D, const float *conv_w, const float *conv_b,
+                       const float *state, const void *tail, const void *y, const float *state_out,
+                       const void *tail_out);
 cudaError_t launch_bimamba(const Problem &p, cudaStream_t stream);
 
 // chunked tensor-core path (bf16, headdim 64, d_state 128)
 bool tc_path_supported(const bimamba_dims &d);
 size_t tc_workspace_bytes(const bimamba_dims &d);
+// leading bytes of that workspace that must be zero when a call starts (the
+// forward/reverse meeting counters); the rest is rewritten by every call
+size_t tc_counter_bytes(const bimamba_dims &d);
 // out[0..2]: segments per direction, chunks per segment, state-only items
 void tc_launch_plan(const bimamba_dims &d, int *out);
 cudaError_t launch_ssd_tc(const Problem &p, cudaStream_t stream);

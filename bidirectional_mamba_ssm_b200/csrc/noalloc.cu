@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "dispatch.h"
 
 namespace bimamba {
 namespace {
@@ -64,17 +65,24 @@ int bimamba_block_decode_noalloc(const bimamba_dims *d, const void *xbc_block,
                                  const void *tail, void *y, float *state_out, void *tail_out,
                                  bimamba_stream_t stream)
 {
-    if (!d) return BIMAMBA_ERR_INVALID;
+    // the same argument checks as bimamba_block_decode, before anything is
+    // queued on the stream: a rejected call launches nothing
+    int st = check_block_decode(d, xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, y,
+                                state_out, tail_out);
+    if (st != BIMAMBA_OK) return st;
+    if (d->batch == 0) return BIMAMBA_OK;
     const size_t need = bimamba_workspace_bytes(d);
     if (need > kScratchBytes) return BIMAMBA_ERR_WORKSPACE;   // beyond the fixed scratch
-    int st = BIMAMBA_OK;
     void *scratch = scratch_address(&st);
     if (st != BIMAMBA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // The decode kernels expect a zeroed workspace.  Every call shares this
-    // array, so clear the part this call uses (a previous call that stopped
-    // early could have left counters set).
-    if (need > 0 && cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    // The decode kernels expect the scratch's meeting counters at zero.
+    // Every call shares this array, so clear them (a previous call that
+    // stopped early, e.g. on a timeout, could have left counters set); the
+    // rest of the scratch is rewritten by every call.
+    const size_t counters = tc_path_supported(*d) ? tc_counter_bytes(*d) : 0;
+    if (counters > 0 && cudaMemsetAsync(scratch, 0, counters, s) != cudaSuccess)
+        return BIMAMBA_ERR_CUDA;
     return bimamba_block_decode(d, xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, y,
                                 state_out, tail_out, scratch, kScratchBytes, stream);
 }

@@ -898,19 +898,26 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             // ---- F: output rows, and the forward + reverse sum
             int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
             const bool first = *flag_slot == 0;
+            bool ready = true;
             if (!first && tid == 0) {
                 // the partner CTA arrived first; wait (bounded) until its
                 // output is visible
-                bool ready = ld_acquire(fl + 1) != 0;
+                ready = ld_acquire(fl + 1) != 0;
                 if (!ready) {
                     const long long w0 = clock64();
                     while (!(ready = ld_acquire(fl + 1) != 0)) {
                         if (clock64() - w0 > kWaitCycles) break;
                     }
                 }
-                if (!ready) record_error(p.status, kStatusTimeout);
             }
-            alu_sync();   // releases the group after thread 0's wait for the partner
+            // releases the group after thread 0's wait for the partner.  A
+            // wait that gave up stops the walk here: the partner's rows are
+            // not added to, and the meeting counters are left as they are
+            // (the caller zero-fills the workspace again after a timeout).
+            if (!alu_sync_and(ready)) {
+                ok = false;
+                break;
+            }
             // the next chunk's wX first, while the partner's rows can be fetched
             if (more) weight_chunk(k + 1);
             // Coalesced output: each thread stages its 32 outputs in shared
@@ -1059,6 +1066,8 @@ void tc_launch_plan(const bimamba_dims &d, int *out)
     out[1] = sp.seg_chunks;
     out[2] = sp.nitems;
 }
+
+size_t tc_counter_bytes(const bimamba_dims &d) { return flags_bytes(d); }
 
 size_t tc_workspace_bytes(const bimamba_dims &d)
 {

@@ -106,7 +106,11 @@ int bimamba_get_error(bimamba_stream_t stream);
 
 /*
  * Depthwise conv1d with `d_conv` taps followed by SiLU (silu != 0) or the
- * identity (silu == 0).  Step "conv + SiLU" of the mixer.
+ * identity (silu == 0).  Step "conv + SiLU" of the mixer: the blog post
+ * "DiffuMamba", network-architecture listing, gives each Mamba mixer a
+ * d_conv = 4 convolution; the reverse stream runs it on the reversed
+ * sequence (same listing: the second module sees the flipped sequence, its
+ * output flipped back), which is the mirrored form below.
  *   u    : (batch, len, ch)    input, dtype
  *   out  : (batch, len, ch)    output, dtype; must not overlap u
  *   w    : (ch, d_conv) fp32   tap j of channel c
@@ -127,11 +131,14 @@ int bimamba_conv_silu(const void *u, void *out, const float *w, const float *bia
  * Bytes of scratch workspace bimamba_ssd_fwd_rev / bimamba_block_decode need
  * for dims `d`.  The caller allocates it once (device memory, 256-byte
  * aligned), zero-fills it before first use, and may reuse it for any later
- * call whose workspace size is not larger.  The kernels return its
- * forward/reverse meeting counters to zero, so it needs no clearing between
- * calls (the rest holds per-call intermediates that every call rewrites).
- * Calls that share one workspace must not run concurrently.
- * Returns 0 for invalid dims.
+ * call whose workspace size is not larger.  A call that completes returns
+ * the workspace's forward/reverse meeting counters to zero, so it needs no
+ * clearing between calls (the rest holds per-call intermediates that every
+ * call rewrites).  After a call whose kernels reported BIMAMBA_ERR_TIMEOUT
+ * (bimamba_get_error), the counters may be left set: zero-fill the workspace
+ * again before reusing it.  Calls that share one workspace must not run
+ * concurrently.  Returns 0 for invalid dims.  This scratch is the library's
+ * own; the pages describe no such buffer.
  */
 size_t bimamba_workspace_bytes(const bimamba_dims *d);
 
@@ -157,7 +164,12 @@ int bimamba_launch_plan(const bimamba_dims *d, int *out);
 /*
  * Full bidirectional mixer core (steps: load, conv+SiLU both ways, decay,
  * intra-chunk contraction, chunk states, state passing, off-diagonal term,
- * fused forward+reverse sum).
+ * fused forward+reverse sum).  Defined by "DiffuMamba: High-Throughput
+ * Diffusion LMs with Mamba Backbone", Japanese technical summary section 2
+ * "Proposed method" and Portuguese technical summary section 2
+ * "Metodologia" (bidirectional Mamba-2 mixer, forward and reverse streams
+ * added), with the Mamba-2 recurrence written at the top of this file and
+ * the blog's network-architecture listing for d_state = 128, d_conv = 4.
  *   xbc         : (batch, len, ch) raw xBC, dtype.  If conv_w == NULL the
  *                 conv and SiLU are skipped and xbc is taken as activated.
  *   dt          : (batch, len, H) dtype, already positive (post-softplus)
@@ -212,6 +224,9 @@ int bimamba_ssd_fwd_rev_untied(const bimamba_dims *d, const void *xbc_f,
 
 /*
  * Sequence shards (one sequence split across ranks, e.g. one GPU each).
+ * The pages describe no sharding; this is the same mixer core as
+ * bimamba_ssd_fwd_rev (same sources), split along the sequence using the
+ * recurrence's linearity in the state.
  * The recurrence is linear in the state, so a shard's effect on the state
  * that crosses it is h -> 2^dec h + S, where S is the state the shard leaves
  * when entered with zero and dec the log2 of the product of its per-token
@@ -277,6 +292,11 @@ int bimamba_ssd_fwd_rev_shard(const bimamba_dims *d, const void *xbc,
  * each with an active block of d->len tokens.  The forward stream resumes
  * from `state` with the conv history `tail`; the reverse stream covers the
  * block only (zero padding past the block end, zero state).  y = sum.
+ * Defined by "Fixed state, long reach: constant-size caches in large-scale
+ * block diffusion", abstract and section 1 (the finished prefix cached as the
+ * forward SSM state, O(1) in the context length; the reverse scan restricted
+ * to the active block; block-causal training makes the cached decode equal
+ * to a full recompute).
  * Result equals a full recompute over prefix + block (forward stream at the
  * block positions) plus the reverse stream over the block alone.
  *   xbc_block : (streams, len, ch) raw xBC of the active block, dtype
@@ -314,9 +334,13 @@ int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block,
  *    for bf16, headdim 64, d_state 128 that is about 16 000 tokens, i.e.
  *    streams x block length, per call).  Nothing is launched then.
  *  - The first call on a device looks up the array's device address, so make
- *    that first call before any stream capture.
- *  - Each call clears the part of the array it uses (asynchronous memset on
- *    `stream`), then runs the same kernels as bimamba_block_decode.
+ *    that first call before any stream capture.  The address is kept for the
+ *    life of the process: do not use the library across cudaDeviceReset.
+ *  - Arguments are checked as bimamba_block_decode checks them, before
+ *    anything is queued.  Each accepted call then clears the array's meeting
+ *    counters (an asynchronous memset on `stream`, so a call that stopped on
+ *    a timeout cannot leave them set for the next) and runs the same kernels
+ *    as bimamba_block_decode.
  *  - All calls share the one array: calls that overlap on the GPU (on
  *    different streams, or from several host threads without ordering) race
  *    and corrupt each other's results.  Serialise them.
