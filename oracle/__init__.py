@@ -270,3 +270,44 @@ def block_decode(block, dt, A, D, conv_w, conv_b, state, tail, *, heads, headdim
                             _ptr(conv_b), _ptr(state), _ptr(tail), S, L, H, P, N,
                             G, K, _ptr(y), _ptr(so), _ptr(to))
     return (y, so, to) if want_commit else y
+
+
+# --------------------------------------------------------------------------
+# The projections on either side of the mixer ("DiffuMamba" blog post,
+# network-architecture listing: d_model = 2048, expand = 2; each mixer maps
+# d_model to its inner width and back, the bidirectional block maps the
+# concatenation of its two streams back to d with a Linear).  Weights are
+# row-major (out_features, in_features), as a Linear layer stores them.
+
+def softplus(x):
+    """softplus(x) = log(1 + exp(x)), evaluated without overflow:
+    max(x, 0) + log1p(exp(-|x|))."""
+    x = _f64(x)
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+
+
+def linear(x, w, bias=None):
+    """A Linear layer: y[..., o] = sum_i x[..., i] w[o, i] (+ bias[o]), in
+    float64 (one library matrix product)."""
+    x, w, bias = _f64(x), _f64(w), _f64(bias)
+    y = np.matmul(x, w.T)
+    return y if bias is None else y + bias
+
+
+def in_proj(u, w_in, dt_bias=None, *, heads, headdim, d_state, ngroups=1):
+    """The mixer's input projection: the first ch = H*P + 2*G*N output rows of
+    w_in give the raw xBC the conv reads, the last H rows the step sizes,
+    dt = softplus(u . w_dt^T + dt_bias).  Returns (xbc, dt)."""
+    ch = heads * headdim + 2 * ngroups * d_state
+    w_in = _f64(w_in)
+    assert w_in.shape[0] == ch + heads
+    xbc = linear(u, w_in[:ch])
+    dt = softplus(linear(u, w_in[ch:], dt_bias))
+    return xbc, dt
+
+
+def out_proj(y, w_out):
+    """The mixer's output projection: out = y . w_out^T (w_out: (d_model,
+    d_inner)); for untied directions with concatenated streams y is
+    (tokens, 2*H*P) and w_out the block's fusion Linear."""
+    return linear(y, w_out)
