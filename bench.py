@@ -54,7 +54,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["long131k", "layer1p3b", "decode", "untied1p3b", "sweep"],
+    ap.add_argument("--workload", choices=["long131k", "layer1p3b", "decode", "decode_pool",
+                                           "untied1p3b", "mixer1p3b", "sweep"],
                     default="long131k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
@@ -73,13 +74,33 @@ def workload_spec(name):
         return I.LAYER_1P3B, I.LAYER_1P3B.batch, I.LAYER_1P3B.seqlen
     if name == "long131k":
         return I.LONG_131K, 1, I.LONG_131K.seqlen
-    if name == "decode":
+    if name in ("decode", "decode_pool"):
         return I.LAYER_1P3B, I.DECODE_STREAMS, I.DECODE_BLOCK
+    if name == "mixer1p3b":   # the layer with its in/out projections around the mixer
+        return I.LAYER_1P3B, I.LAYER_1P3B.batch, I.LAYER_1P3B.seqlen
     if name == "untied1p3b":   # the same layer with untied directions, outputs concatenated
         return I.LAYER_1P3B, I.LAYER_1P3B.batch, I.LAYER_1P3B.seqlen
     if name == "sweep":   # one sequence, prefill at 1k..256k tokens; the line's value at 256k
         return I.LONG_131K, 1, SWEEP_LENGTHS[-1]
     raise ValueError(name)
+
+
+D_MODEL = 2048   # the 1.3B model's width ("DiffuMamba" blog, network-architecture listing)
+POOL_STREAMS = 256   # cached streams held by the pooled-decode workload
+
+
+def gemm_counts(w, tokens, d_model=D_MODEL):
+    """Algorithmic bytes and flops of the two projections of one step:
+    in  [xbc | dt] = u (tokens, d_model) . W_in^T (ch + H, d_model)
+    out out = y (tokens, H*P) . W_out^T (d_model, H*P)
+    bytes: each operand and result once (bf16)."""
+    ch = w.heads * w.headdim + 2 * w.d_state
+    n_in, k_out = ch + w.heads, w.heads * w.headdim
+    f_in = 2 * tokens * n_in * d_model
+    f_out = 2 * tokens * d_model * k_out
+    b_in = 2 * (tokens * d_model + n_in * d_model + tokens * n_in)
+    b_out = 2 * (tokens * k_out + d_model * k_out + tokens * d_model)
+    return (b_in, f_in), (b_out, f_out)
 
 
 def algorithmic(w, batch, seqlen, decode=False, untied=False):
@@ -271,17 +292,25 @@ DECODE_SETS = 4   # state/input sets the timed decode steps rotate over (> L2 in
 
 
 def build_step(lib, I, w, name, batch, seqlen, rank, dev):
-    """Inputs on the device and the step closure of one workload."""
+    """Inputs on the device and the step closure of one workload.  A step
+    takes `ev`, a (start, stop) pair of events (or None), and hands it to the
+    library's timing hook around the call whose main kernel the roofline
+    reports."""
     import torch
     H, P, N = w.heads, w.headdim, w.d_state
     decode = name == "decode"
     untied = name == "untied1p3b"
-    g = I.make_inputs(w, seed=rank, device=dev, seqlen=seqlen, batch=batch, conv_bias=decode)
+    g = I.make_inputs(w, seed=rank, device=dev, seqlen=seqlen, batch=batch,
+                      conv_bias=name in ("decode", "decode_pool"))
     gr = I.make_inputs(w, seed=10000 + rank, device=dev, seqlen=seqlen, batch=batch) if untied else None
     y = torch.empty((batch, seqlen, (2 if untied else 1) * H * P), dtype=torch.bfloat16, device=dev)
     dims = lib.make_dims(batch, seqlen, H, P, N, torch.bfloat16)
     ws = lib.new_workspace(dims, device=dev)
     extra = {}
+
+    def hook(ev):
+        lib.bimamba_set_timing_events(*(ev if ev is not None else (None, None)))
+
     if decode:
         state, tail = decode_cache(lib, I, w, batch, I.DECODE_PREFIX, g, rank, dev)
         # Sets of (state, tail, block inputs, y) at distinct addresses: each
@@ -294,19 +323,61 @@ def build_step(lib, I, w, name, batch, seqlen, rank, dev):
         it = [0]
         extra.update(state=state, tail=tail)
 
-        def step():
+        def step(ev=None):
             st, tl, xb, dtb, yy = sets[it[0] % DECODE_SETS]
             it[0] += 1
+            hook(ev)
             lib.bimamba_block_decode(xb, dtb, g["A"], g["D"], g["conv_w"], g["conv_b"], st, tl, yy,
                                      None, None, ws, heads=H, headdim=P, d_state=N)
+            hook(None)
+    elif name == "decode_pool":
+        # a pool of cached streams; each step decodes the next `batch` of them
+        # (slots rotate through the pool, so the states come from HBM) and
+        # commits every row's state and conv tail back in place
+        pool = I.make_state(POOL_STREAMS, H, P, N, seed=50 + rank, scale=0.05, device=dev)
+        tails = I.make_tail(POOL_STREAMS, 4, w.channels, "bf16", seed=51 + rank, bc_split=H * P,
+                            bc_scale=w.bc_scale, device=dev)
+        groups = POOL_STREAMS // batch
+        slot_sets = [torch.arange(i * batch, (i + 1) * batch, dtype=torch.int32, device=dev)
+                     for i in range(groups)]
+        it = [0]
+
+        def step(ev=None):
+            sl = slot_sets[it[0] % groups]
+            it[0] += 1
+            hook(ev)
+            lib.bimamba_block_decode_pool(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], g["conv_b"],
+                                          pool, tails, sl, None, y, ws, heads=H, headdim=P, d_state=N)
+            hook(None)
+    elif name == "mixer1p3b":
+        tokens = batch * seqlen
+        pr = I.make_projections(D_MODEL, H, P, N, tokens, seed=rank, device=dev)
+        xbc = torch.empty((batch, seqlen, w.channels), dtype=torch.bfloat16, device=dev)
+        dtv = torch.empty((batch, seqlen, H), dtype=torch.bfloat16, device=dev)
+        out = torch.empty((tokens, D_MODEL), dtype=torch.bfloat16, device=dev)
+        del pr["y"]
+        extra.update(proj=pr)
+
+        def step(ev=None):
+            hook(ev)   # the in-projection GEMM is the roofline's kernel
+            lib.bimamba_in_proj(pr["u"], pr["w_in"], pr["dt_bias"], xbc, dtv, heads=H, headdim=P,
+                                d_state=N)
+            hook(None)
+            lib.bimamba_ssd_fwd_rev(xbc, dtv, g["A"], g["D"], g["conv_w"], None, None, None, y, ws,
+                                    heads=H, headdim=P, d_state=N)
+            lib.bimamba_out_proj(y.view(tokens, H * P), pr["w_out"], out)
     elif untied:
-        def step():
+        def step(ev=None):
+            hook(ev)
             lib.bimamba_ssd_fwd_rev_untied(g, gr, None, None, y, ws, heads=H, headdim=P,
                                            d_state=N, concat=True)
+            hook(None)
     else:
-        def step():
+        def step(ev=None):
+            hook(ev)
             lib.bimamba_ssd_fwd_rev(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"], None, None,
                                     None, y, ws, heads=H, headdim=P, d_state=N)
+            hook(None)
     return step, g, gr, dims, ws, extra
 
 
@@ -363,10 +434,8 @@ def time_steps(args, lib, step, stream, world, dev):
     launches0 = lib.bimamba_launch_count()
     start.record(stream)
     for i in range(args.steps):
-        lib.bimamba_set_timing_events(kev[i][0], kev[i][1])
-        step()
+        step(kev[i])
     end.record(stream)
-    lib.bimamba_set_timing_events(None, None)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -384,7 +453,7 @@ def measure(args, lib, I, name, rank, world, dev, gpu_id, want_e2e=True):
     w, batch, seqlen = workload_spec(name)
     if args.batch is not None:
         batch = args.batch
-    decode = name == "decode"
+    decode = name in ("decode", "decode_pool")
     untied = name == "untied1p3b"
     H, P, N = w.heads, w.headdim, w.d_state
     step, g, gr, dims, ws, extra = build_step(lib, I, w, name, batch, seqlen, rank, dev)
@@ -401,13 +470,29 @@ def measure(args, lib, I, name, rank, world, dev, gpu_id, want_e2e=True):
     peaks, peak_kind = load_peaks()
     nbytes, flops = algorithmic(w, batch, seqlen, decode, untied)
     kernel_file = "ssd_tc.cu" if (P, N) == (64, 128) else "scan_seq.cu"
+    if decode:
+        kernel_file = "decode_tc.cu"
+    if name == "decode_pool":   # the commit writes every row's state and conv tail back
+        nbytes += batch * (H * P * N * 4 + 4 * w.channels * 2)
+    if name == "mixer1p3b":
+        (nbytes, flops), _ = gemm_counts(w, batch * seqlen)
+        kernel_file = "gemm_tc.cu"
     roof, ctx = roofline(peaks, peak_kind, clocks, nbytes, flops, per_call_ms / 1e3, decode,
                          kernel_file)
-    if decode:
+    if name == "decode":
         wl = (f"cached block decode: {batch} streams x {seqlen}-token block, H64x64 N128 bf16, "
               f"65536-token prefix state")
         l2 = (f"HBM-cold: steps rotate over {DECODE_SETS} sets of state + block inputs + y "
               f"(~{DECODE_SETS * 100} MB > 126 MB L2)")
+    elif name == "decode_pool":
+        wl = (f"pooled cached decode: {batch} of {POOL_STREAMS} cached streams per step x "
+              f"{seqlen}-token block, H64x64 N128 bf16, every row's state and tail committed")
+        l2 = (f"HBM-cold: consecutive steps take different slots of a {POOL_STREAMS * 2} MiB "
+              f"state pool")
+    elif name == "mixer1p3b":
+        wl = (w.name + f", with its projections: in {D_MODEL}->{w.channels}+{H} (softplus dt), "
+              f"mixer core, out {H * P}->{D_MODEL}")
+        l2 = "inputs larger than L2"
     else:
         wl = w.name + (", untied directions, outputs concatenated" if untied else "")
         l2 = "inputs larger than L2 (xbc + y per step > 126 MB)"
@@ -415,8 +500,7 @@ def measure(args, lib, I, name, rank, world, dev, gpu_id, want_e2e=True):
            "seqlen": seqlen, "l2": l2, "roofline": roof, "roofline_hbm_context": ctx,
            "clocks": clocks, "gpu_launches": launches, "main_kernel_ms": per_call_ms}
     if want_e2e:
-        out["e2e"] = run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode,
-                             extra.get("state"), extra.get("tail"), dev, world, gr)
+        out["e2e"] = run_e2e(args, lib, w, name, g, batch, seqlen, dims, ws, extra, dev, world, gr)
     del step, g, gr, ws, extra
     torch.cuda.empty_cache()
     return out
@@ -546,22 +630,36 @@ def run_sweep(args, lib, w, dev, rank, gpu_id):
     return rows
 
 
-def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, world, gr=None):
+def run_e2e(args, lib, w, name, g, batch, seqlen, dims, ws, extra, dev, world, gr=None):
     """Same metric through the public API from pinned HOST buffers.  Every step
-    copies its inputs (xbc, dt) host->device, runs the call, and copies y back
-    to the host.  Steps are pipelined the way a serving loop would run them:
-    step i+1's upload, step i's kernels and step i-1's download run on three
-    streams with two device buffer sets, ordered by events."""
+    copies its inputs host->device (the raw xbc and dt of each stream; the
+    layer input u for the workload with projections), runs the call(s), and
+    copies the result (y, or the layer output) back to the host.  Steps are
+    pipelined the way a serving loop would run them: step i+1's upload, step
+    i's kernels and step i-1's download run on three streams with two device
+    buffer sets, ordered by events."""
     import torch
     H, P, N = w.heads, w.headdim, w.d_state
     untied = gr is not None
-    # per-step inputs: xbc and dt of each stream (one stream when tied)
-    srcs = [g] + ([gr] if untied else [])
-    hin = [t.cpu().pin_memory() for d in srcs for t in (d["xbc"], d["dt"])]
-    ywidth = (2 if untied else 1) * H * P
-    hy = torch.empty((batch, seqlen, ywidth), dtype=torch.bfloat16).pin_memory()
+    tokens = batch * seqlen
+    if name == "mixer1p3b":
+        pr = extra["proj"]
+        hin = [pr["u"].cpu().pin_memory()]
+        out_shape = (tokens, D_MODEL)
+        mid = [(torch.empty((batch, seqlen, w.channels), dtype=torch.bfloat16, device=dev),
+                torch.empty((batch, seqlen, H), dtype=torch.bfloat16, device=dev),
+                torch.empty((batch, seqlen, H * P), dtype=torch.bfloat16, device=dev)) for _ in range(2)]
+    else:
+        srcs = [g] + ([gr] if untied else [])
+        hin = [t.cpu().pin_memory() for d in srcs for t in (d["xbc"], d["dt"])]
+        out_shape = (batch, seqlen, (2 if untied else 1) * H * P)
+    if name == "decode_pool":
+        pool = I_make_pool(w, dev)
+        slot_sets = [torch.arange(i * batch, (i + 1) * batch, dtype=torch.int32, device=dev)
+                     for i in range(POOL_STREAMS // batch)]
+    hy = torch.empty(out_shape, dtype=torch.bfloat16).pin_memory()
     din = [[torch.empty_like(t, device=dev) for t in hin] for _ in range(2)]
-    dy = [torch.empty((batch, seqlen, ywidth), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dy = [torch.empty(out_shape, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     wss = [ws, lib.new_workspace(dims, device=dev)]
     s_up, s_run, s_down = (torch.cuda.Stream(device=dev) for _ in range(3))
     up_done = [torch.cuda.Event() for _ in range(2)]
@@ -569,6 +667,7 @@ def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, 
     down_done = [torch.cuda.Event() for _ in range(2)]
     for e in run_done + down_done:
         e.record(torch.cuda.current_stream())
+    kw = dict(heads=H, headdim=P, d_state=N, stream=s_run)
 
     def step(i):
         j = i & 1
@@ -578,20 +677,28 @@ def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, 
                 dst.copy_(src, non_blocking=True)
         up_done[j].record(s_up)
         s_run.wait_event(up_done[j])
-        s_run.wait_event(down_done[j])          # y buffer j read back by step i-2
-        dx, ddt = din[j][0], din[j][1]
-        if decode:
-            lib.bimamba_block_decode(dx, ddt, g["A"], g["D"], g["conv_w"], g["conv_b"], state,
-                                     tail, dy[j], None, None, wss[j], heads=H, headdim=P, d_state=N,
-                                     stream=s_run)
+        s_run.wait_event(down_done[j])          # output buffer j read back by step i-2
+        if name == "mixer1p3b":
+            xb, dtb, yb = mid[j]
+            lib.bimamba_in_proj(din[j][0], pr["w_in"], pr["dt_bias"], xb, dtb, heads=H, headdim=P,
+                                d_state=N, stream=s_run)
+            lib.bimamba_ssd_fwd_rev(xb, dtb, g["A"], g["D"], g["conv_w"], None, None, None, yb,
+                                    wss[j], **kw)
+            lib.bimamba_out_proj(yb.view(tokens, H * P), pr["w_out"], dy[j], stream=s_run)
+        elif name == "decode":
+            lib.bimamba_block_decode(din[j][0], din[j][1], g["A"], g["D"], g["conv_w"], g["conv_b"],
+                                     extra["state"], extra["tail"], dy[j], None, None, wss[j], **kw)
+        elif name == "decode_pool":
+            lib.bimamba_block_decode_pool(din[j][0], din[j][1], g["A"], g["D"], g["conv_w"],
+                                          g["conv_b"], pool[0], pool[1],
+                                          slot_sets[i % len(slot_sets)], None, dy[j], wss[j], **kw)
         elif untied:
-            fwd = dict(g, xbc=dx, dt=ddt)
+            fwd = dict(g, xbc=din[j][0], dt=din[j][1])
             rev = dict(gr, xbc=din[j][2], dt=din[j][3])
-            lib.bimamba_ssd_fwd_rev_untied(fwd, rev, None, None, dy[j], wss[j], heads=H, headdim=P,
-                                           d_state=N, concat=True, stream=s_run)
+            lib.bimamba_ssd_fwd_rev_untied(fwd, rev, None, None, dy[j], wss[j], concat=True, **kw)
         else:
-            lib.bimamba_ssd_fwd_rev(dx, ddt, g["A"], g["D"], g["conv_w"], None, None, None,
-                                    dy[j], wss[j], heads=H, headdim=P, d_state=N, stream=s_run)
+            lib.bimamba_ssd_fwd_rev(din[j][0], din[j][1], g["A"], g["D"], g["conv_w"], None, None,
+                                    None, dy[j], wss[j], **kw)
         run_done[j].record(s_run)
         s_down.wait_event(run_done[j])
         with torch.cuda.stream(s_down):
@@ -619,29 +726,45 @@ def run_e2e(args, lib, w, g, batch, seqlen, dims, ws, decode, state, tail, dev, 
             "pipelined": "upload / kernels / download overlapped across steps (3 streams)"}
 
 
+def I_make_pool(w, dev):
+    """A pool of POOL_STREAMS cached streams (seeded states and conv tails)."""
+    from bidirectional_mamba_ssm_b200 import inputs as I
+    pool = I.make_state(POOL_STREAMS, w.heads, w.headdim, w.d_state, seed=60, scale=0.05, device=dev)
+    tails = I.make_tail(POOL_STREAMS, 4, w.channels, "bf16", seed=61, bc_split=w.heads * w.headdim,
+                        bc_scale=w.bc_scale, device=dev)
+    return pool, tails
+
+
 # --------------------------------------------------------------------------- CPU oracle
 def oracle_sample_step(w, workload, seq_tokens, seed=0):
     """Run the oracle once on one sequence prefix of `seq_tokens` tokens of
-    the workload (all heads, both directions, conv fused); return seconds."""
+    the workload (all heads, both directions, conv fused; with the
+    projections for the layer workload); return seconds."""
     import numpy as np
     import oracle
     from bidirectional_mamba_ssm_b200 import inputs as I
-    decode = workload == "decode"
+    decode = workload in ("decode", "decode_pool")
     cpu = I.make_inputs(w, seed=seed, seqlen=seq_tokens, batch=1, conv_bias=decode)
     n = {k: (None if v is None else v.float().double().numpy()) for k, v in cpu.items()}
     kw = dict(heads=w.heads, headdim=w.headdim, d_state=w.d_state)
     if workload == "untied1p3b":
         cr = I.make_inputs(w, seed=seed + 10000, seqlen=seq_tokens, batch=1)
         r = {k: (None if v is None else v.float().double().numpy()) for k, v in cr.items()}
+    if workload == "mixer1p3b":
+        pr = I.make_projections(D_MODEL, w.heads, w.headdim, w.d_state, seq_tokens, seed=seed)
     t0 = time.perf_counter()
     if workload == "untied1p3b":
         oracle.bimamba_untied(n["xbc"], r["xbc"], n["dt"], r["dt"], n["A"], r["A"], n["D"], r["D"],
                               n["conv_w"], r["conv_w"], None, None, concat=True, **kw)
+    elif workload == "mixer1p3b":
+        xbc, dt = oracle.in_proj(pr["u"], pr["w_in"], pr["dt_bias"], **kw)
+        y = oracle.bimamba(xbc[None], dt[None], n["A"], n["D"], n["conv_w"], None, **kw)
+        oracle.out_proj(y[0], pr["w_out"])
     elif decode:
         state = np.zeros((1, w.heads, w.headdim, w.d_state))
         tail = np.zeros((1, 4, w.channels))
         oracle.block_decode(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], n["conv_b"], state,
-                            tail, **kw)
+                            tail, want_commit=workload == "decode_pool", **kw)
     else:
         oracle.bimamba(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], None, **kw)
     return time.perf_counter() - t0
@@ -651,7 +774,7 @@ def cpu_baseline(w, workload):
     """The oracle, as it stands, on host cores: whole sequences of the
     workload's length (capped at 4096 tokens) until ~10 s of CPU time."""
     import oracle
-    seq = 64 if workload == "decode" else 1024
+    seq = 64 if workload in ("decode", "decode_pool") else 1024
     tokens, secs, reps = 0, 0.0, 0
     while secs < 10.0 and reps < 64:
         secs += oracle_sample_step(w, workload, seq, seed=reps)
@@ -669,7 +792,7 @@ def run_reference(args):
         return
     import oracle
     w, batch, seqlen = workload_spec(args.workload)
-    seq = 64 if args.workload == "decode" else 256
+    seq = 64 if args.workload in ("decode", "decode_pool") else 256
     for i in range(args.warmup):
         oracle_sample_step(w, args.workload, seq, seed=i)
     total = 0.0
@@ -686,7 +809,9 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": {"decode": "cached block decode",
-                                "untied1p3b": w.name + ", untied directions, outputs concatenated"}
+                                "decode_pool": "pooled cached decode",
+                                "untied1p3b": w.name + ", untied directions, outputs concatenated",
+                                "mixer1p3b": w.name + ", with its in/out projections"}
                    .get(args.workload, w.name),
                    "batch_per_gpu": batch, "seqlen": seqlen, "heads": w.heads,
                    "headdim": w.headdim, "d_state": w.d_state},

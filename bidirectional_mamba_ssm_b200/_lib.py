@@ -42,6 +42,11 @@ EXPORTED = (
     "bimamba_shard_states",
     "bimamba_ssd_fwd_rev_shard",
     "bimamba_block_decode",
+    "bimamba_block_decode_pool",
+    "bimamba_backward_workspace_bytes",
+    "bimamba_ssd_fwd_rev_backward",
+    "bimamba_in_proj",
+    "bimamba_out_proj",
     "bimamba_noalloc_scratch_bytes",
     "bimamba_block_decode_noalloc",
 )
@@ -92,6 +97,17 @@ def _load() -> ctypes.CDLL:
     lib.bimamba_ssd_fwd_rev_shard.argtypes = [dp] + [vp] * 11 + [i, i, vp, vp, vp, sz, vp]
     lib.bimamba_block_decode.restype = i
     lib.bimamba_block_decode.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.bimamba_block_decode_pool.restype = i
+    lib.bimamba_block_decode_pool.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp,
+                                              sz, vp]
+    lib.bimamba_backward_workspace_bytes.restype = sz
+    lib.bimamba_backward_workspace_bytes.argtypes = [dp]
+    lib.bimamba_ssd_fwd_rev_backward.restype = i
+    lib.bimamba_ssd_fwd_rev_backward.argtypes = [dp] + [vp] * 16 + [sz, vp]
+    lib.bimamba_in_proj.restype = i
+    lib.bimamba_in_proj.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp, vp]
+    lib.bimamba_out_proj.restype = i
+    lib.bimamba_out_proj.argtypes = [i, i, i, vp, vp, vp, vp]
     lib.bimamba_noalloc_scratch_bytes.restype = sz
     lib.bimamba_noalloc_scratch_bytes.argtypes = []
     lib.bimamba_block_decode_noalloc.restype = i
@@ -275,6 +291,76 @@ def bimamba_block_decode(xbc_block, dt_block, A, D, conv_w, conv_b, state, tail,
                                    _stream(stream))
     _check(st, "bimamba_block_decode")
     return y
+
+
+def bimamba_block_decode_pool(xbc_block, dt_block, A, D, conv_w, conv_b, state_pool, tail_pool,
+                              slots, commit, y, workspace, *, heads, headdim, d_state, ngroups=1,
+                              stream=None):
+    """Cached block decode of a batch of streams held in a pool: row s uses
+    pool entry slots[s] (int32 device tensor) and, where commit[s] != 0 (all
+    rows when commit is None), writes its new state and conv tail back there."""
+    S, L, _ = xbc_block.shape
+    dims = make_dims(S, L, heads, headdim, d_state, _dtype_code(xbc_block), ngroups)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.bimamba_block_decode_pool(ctypes.byref(dims), _ptr(xbc_block), _ptr(dt_block), _ptr(A),
+                                        _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(state_pool),
+                                        _ptr(tail_pool), int(state_pool.shape[0]), _ptr(slots),
+                                        _ptr(commit), _ptr(y), _ptr(workspace), wsz, _stream(stream))
+    _check(st, "bimamba_block_decode_pool")
+    return y
+
+
+def bimamba_backward_workspace_bytes(dims: Dims) -> int:
+    return int(_lib.bimamba_backward_workspace_bytes(ctypes.byref(dims)))
+
+
+def bimamba_ssd_fwd_rev_backward(xbc, dt, A, D, conv_w, conv_b, init_state, dy, *, heads, headdim,
+                                 d_state, want_dinit=False, workspace=None, stream=None):
+    """Gradients of sum(dy * y) for y = bimamba_ssd_fwd_rev(...): returns a dict
+    of fp32 tensors xbc, dt, A, D, conv_w, conv_b (None without a bias) and
+    init (None unless want_dinit)."""
+    bsz, L, ch = xbc.shape
+    dims = make_dims(bsz, L, heads, headdim, d_state, _dtype_code(xbc))
+    dev = xbc.device
+    f32 = torch.float32
+    g = {"xbc": torch.empty((bsz, L, ch), dtype=f32, device=dev),
+         "dt": torch.empty((bsz, L, heads), dtype=f32, device=dev),
+         "A": torch.empty((heads,), dtype=f32, device=dev),
+         "D": torch.empty((heads,), dtype=f32, device=dev),
+         "conv_w": torch.empty((ch, 4), dtype=f32, device=dev),
+         "conv_b": None if conv_b is None else torch.empty((ch,), dtype=f32, device=dev),
+         "init": torch.empty((bsz, heads, headdim, d_state), dtype=f32, device=dev)
+         if want_dinit else None}
+    if workspace is None:
+        workspace = torch.empty(max(256, bimamba_backward_workspace_bytes(dims)), dtype=torch.uint8,
+                                device=dev)
+    wsz = workspace.numel() * workspace.element_size()
+    st = _lib.bimamba_ssd_fwd_rev_backward(
+        ctypes.byref(dims), _ptr(xbc), _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b),
+        _ptr(init_state), _ptr(dy), _ptr(g["xbc"]), _ptr(g["dt"]), _ptr(g["A"]), _ptr(g["D"]),
+        _ptr(g["conv_w"]), _ptr(g["conv_b"]), _ptr(g["init"]), _ptr(workspace), wsz, _stream(stream))
+    _check(st, "bimamba_ssd_fwd_rev_backward")
+    return g
+
+
+def bimamba_in_proj(u, w_in, dt_bias, xbc, dt, *, heads, headdim, d_state, stream=None):
+    """[xbc | dt] = u . W_in^T with dt = softplus(. + dt_bias); u (tokens,
+    d_model) bf16, w_in (ch + H, d_model) bf16, xbc (tokens, ch), dt (tokens, H)."""
+    tokens, d_model = u.shape[-2] if u.dim() == 2 else u.shape[0] * u.shape[1], u.shape[-1]
+    st = _lib.bimamba_in_proj(int(tokens), int(d_model), heads, headdim, d_state, _ptr(u), _ptr(w_in),
+                              _ptr(dt_bias), _ptr(xbc), _ptr(dt), _stream(stream))
+    _check(st, "bimamba_in_proj")
+    return xbc, dt
+
+
+def bimamba_out_proj(y, w_out, out, stream=None):
+    """out = y . W_out^T; y (tokens, d_inner) bf16, w_out (d_model, d_inner) bf16."""
+    d_inner = y.shape[-1]
+    tokens = y.numel() // d_inner
+    st = _lib.bimamba_out_proj(int(tokens), int(d_inner), int(w_out.shape[0]), _ptr(y), _ptr(w_out),
+                               _ptr(out), _stream(stream))
+    _check(st, "bimamba_out_proj")
+    return out
 
 
 def bimamba_noalloc_scratch_bytes() -> int:

@@ -135,6 +135,7 @@ int bimamba_get_error(bimamba_stream_t stream)
             return BIMAMBA_ERR_CUDA;
     }
     if (v & kStatusTimeout) return BIMAMBA_ERR_TIMEOUT;
+    if (v & kStatusBadSlot) return BIMAMBA_ERR_INVALID;
     return BIMAMBA_OK;
 }
 
@@ -367,6 +368,25 @@ int bimamba_ssd_fwd_rev_shard(const bimamba_dims *d, const void *xbc, const void
     return cuda_status(launch_bimamba(pr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// The tensor-core decode kernels (blocks of at most 64 tokens): state and
+// tail from pool slots, per-row commit.
+static int run_decode_tc(const bimamba_dims *d, const void *xbc_block, const void *dt_block,
+                         const float *A, const float *D, const float *conv_w, const float *conv_b,
+                         const float *state, const void *tail, const int *slots, int pool,
+                         const int *commit, float *state_out, void *y, void *workspace,
+                         size_t workspace_bytes, cudaStream_t s)
+{
+    const size_t need = workspace_bytes_for(*d);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return BIMAMBA_ERR_WORKSPACE;
+    DecodeProblem q{};
+    q.dims = *d;
+    q.xbc = xbc_block; q.dt = dt_block; q.A = A; q.D = D; q.conv_w = conv_w; q.conv_b = conv_b;
+    q.state = state; q.tail = tail; q.slots = slots; q.pool = pool; q.commit = commit;
+    q.state_out = state_out; q.y = y; q.workspace = workspace;
+    q.status = device_status_word();
+    return cuda_status(launch_decode_tc(q, s));
+}
+
 int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block, const void *dt_block,
                          const float *A, const float *D, const float *conv_w,
                          const float *conv_b, const float *state, const void *tail, void *y,
@@ -379,14 +399,119 @@ int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block, const voi
     if (d->batch == 0) return BIMAMBA_OK;
     const int ch = d->heads * d->headdim + 2 * d->ngroups * d->d_state;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    st = run_tied(d, xbc_block, dt_block, A, D, conv_w, conv_b, tail, state, state_out, y,
-                  workspace, workspace_bytes, s);
+    if (decode_tc_supported(*d))
+        st = run_decode_tc(d, xbc_block, dt_block, A, D, conv_w, conv_b, state, tail, nullptr,
+                           d->batch, nullptr, state_out, y, workspace, workspace_bytes, s);
+    else
+        st = run_tied(d, xbc_block, dt_block, A, D, conv_w, conv_b, tail, state, state_out, y,
+                      workspace, workspace_bytes, s);
     if (st != BIMAMBA_OK || !tail_out) return st;
     cudaError_t e = d->dtype == BIMAMBA_F32
                         ? launch_tail_commit<float>(xbc_block, tail, tail_out, d->batch, d->len, ch, s)
                         : launch_tail_commit<__nv_bfloat16>(xbc_block, tail, tail_out, d->batch,
                                                             d->len, ch, s);
     return cuda_status(e);
+}
+
+int bimamba_block_decode_pool(const bimamba_dims *d, const void *xbc_block, const void *dt_block,
+                              const float *A, const float *D, const float *conv_w,
+                              const float *conv_b, float *state_pool, void *tail_pool,
+                              int pool_size, const int *slots, const int *commit, void *y,
+                              void *workspace, size_t workspace_bytes, bimamba_stream_t stream)
+{
+    int st = check_dims(d);
+    if (st != BIMAMBA_OK) return st;
+    if (d->batch == 0) return BIMAMBA_OK;
+    if (!decode_tc_supported(*d)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (pool_size < 1 || !xbc_block || !dt_block || !A || !D || !conv_w || !state_pool ||
+        !tail_pool || !slots || !y)
+        return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {xbc_block, dt_block, A, D, conv_w, conv_b, state_pool, tail_pool, y};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
+    const int ch = d->heads * d->headdim + 2 * d->ngroups * d->d_state;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = run_decode_tc(d, xbc_block, dt_block, A, D, conv_w, conv_b, state_pool, tail_pool, slots,
+                       pool_size, commit, state_pool, y, workspace, workspace_bytes, s);
+    if (st != BIMAMBA_OK) return st;
+    return cuda_status(launch_tail_commit_pool(xbc_block, tail_pool, slots, commit, pool_size,
+                                               d->batch, d->len, ch, device_status_word(), s));
+}
+
+int bimamba_in_proj(int tokens, int d_model, int heads, int headdim, int d_state, const void *u,
+                    const void *w_in, const float *dt_bias, void *xbc, void *dt,
+                    bimamba_stream_t stream)
+{
+    if (tokens < 0 || d_model <= 0 || heads <= 0 || headdim <= 0 || d_state <= 0)
+        return BIMAMBA_ERR_INVALID;
+    if (d_model % 8 != 0) return BIMAMBA_ERR_UNSUPPORTED;
+    const long long ch = (long long)heads * headdim + 2LL * d_state;
+    if (ch + heads > (1 << 20) || tokens > (1 << 30)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (tokens == 0) return BIMAMBA_OK;
+    if (!u || !w_in || !xbc || !dt) return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {u, w_in, dt_bias, xbc, dt};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
+    GemmProblem g{};
+    g.a = u; g.w = w_in;
+    g.M = tokens; g.N = (int)(ch + heads); g.K = d_model; g.n_split = (int)ch;
+    g.out0 = xbc; g.out1 = dt; g.bias1 = dt_bias;
+    g.status = device_status_word();
+    return cuda_status(launch_gemm_tc(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int bimamba_out_proj(int tokens, int d_inner, int d_model, const void *y, const void *w_out,
+                     void *out, bimamba_stream_t stream)
+{
+    if (tokens < 0 || d_inner <= 0 || d_model <= 0) return BIMAMBA_ERR_INVALID;
+    if (d_inner % 8 != 0) return BIMAMBA_ERR_UNSUPPORTED;
+    if (d_model > (1 << 20) || tokens > (1 << 30)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (tokens == 0) return BIMAMBA_OK;
+    if (!y || !w_out || !out) return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {y, w_out, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return BIMAMBA_ERR_INVALID;
+    GemmProblem g{};
+    g.a = y; g.w = w_out;
+    g.M = tokens; g.N = d_model; g.K = d_inner; g.n_split = d_model;
+    g.out0 = out;
+    g.status = device_status_word();
+    return cuda_status(launch_gemm_tc(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t bimamba_backward_workspace_bytes(const bimamba_dims *d)
+{
+    if (check_dims(d) != BIMAMBA_OK || !backward_supported(*d)) return 0;
+    return backward_workspace_bytes(*d);
+}
+
+int bimamba_ssd_fwd_rev_backward(const bimamba_dims *d, const void *xbc, const void *dt,
+                                 const float *A, const float *D, const float *conv_w,
+                                 const float *conv_b, const float *init_state, const void *dy,
+                                 float *dxbc, float *ddt, float *dA, float *dD, float *dconv_w,
+                                 float *dconv_b, float *dinit, void *workspace,
+                                 size_t workspace_bytes, bimamba_stream_t stream)
+{
+    int st = check_dims(d);
+    if (st != BIMAMBA_OK) return st;
+    if (!backward_supported(*d)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (d->batch == 0 || d->len == 0) return BIMAMBA_ERR_INVALID;
+    if (!xbc || !dt || !A || !D || !conv_w || !dy || !dxbc || !ddt || !dA || !dD || !dconv_w)
+        return BIMAMBA_ERR_INVALID;
+    const void *ptrs[] = {xbc, dt, A, D, conv_w, conv_b, init_state, dy, dxbc, ddt, dA, dD,
+                          dconv_w, dconv_b, dinit};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BIMAMBA_ERR_INVALID;
+    const size_t need = backward_workspace_bytes(*d);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return BIMAMBA_ERR_WORKSPACE;
+    BackwardProblem q{};
+    q.dims = *d;
+    q.xbc = xbc; q.dt = dt; q.dy = dy; q.A = A; q.D = D; q.conv_w = conv_w; q.conv_b = conv_b;
+    q.init = init_state;
+    q.dxbc = dxbc; q.ddt = ddt; q.dA = dA; q.dD = dD; q.dconv_w = dconv_w; q.dconv_b = dconv_b;
+    q.dinit = dinit;
+    q.workspace = workspace;
+    return cuda_status(launch_backward(q, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -14,7 +14,7 @@ namespace bimamba {
 // Kernels that can detect an error at run time (a bounded wait that gave up)
 // OR a bit into the per-device status word whose address the host passes
 // them; bimamba_get_error reads and clears it.
-enum : int { kStatusTimeout = 1 };
+enum : int { kStatusTimeout = 1, kStatusBadSlot = 2 };
 
 __device__ __forceinline__ void record_error(int *status, int bit) {
     if (status) atomicOr(status, bit);

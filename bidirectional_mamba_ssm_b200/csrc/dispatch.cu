@@ -6,7 +6,10 @@ namespace bimamba {
 
 size_t workspace_bytes_for(const bimamba_dims &d)
 {
-    return tc_path_supported(d) ? tc_workspace_bytes(d) : 0;
+    // one size serves both the scan and the cached decode of these dims
+    size_t n = tc_path_supported(d) ? tc_workspace_bytes(d) : 0;
+    if (decode_tc_supported(d)) n = n > decode_tc_workspace_bytes(d) ? n : decode_tc_workspace_bytes(d);
+    return n;
 }
 
 cudaError_t launch_bimamba(const Problem &p, cudaStream_t stream)

@@ -59,6 +59,57 @@ cudaError_t launch_ssd_tc(const Problem &p, cudaStream_t stream);
 // directions; tensor-core path only
 cudaError_t launch_shard_states(const Problem &p, cudaStream_t stream);
 
+// cached block decode on the tensor cores (bf16, headdim 64, d_state 128,
+// blocks of at most 64 tokens): per batch row, the pool slot of its state and
+// conv tail (null: row s uses slot s) and whether it commits (null: every row
+// commits when state_out is given)
+struct DecodeProblem {
+    bimamba_dims dims;            // batch = rows, len = block length
+    const void *xbc, *dt;
+    const float *A, *D, *conv_w, *conv_b;
+    const float *state;           // (pool, H, P, N)
+    const void *tail;             // (pool, 4, ch)
+    const int *slots;             // (batch) or null
+    int pool;                     // pool size: slots must lie in [0, pool)
+    const int *commit;            // (batch) or null
+    float *state_out;             // (pool, H, P, N) or null; may alias state
+    void *y;
+    void *workspace;
+    int *status;
+};
+bool decode_tc_supported(const bimamba_dims &d);
+size_t decode_tc_workspace_bytes(const bimamba_dims &d);
+cudaError_t launch_decode_tc(const DecodeProblem &q, cudaStream_t stream);
+// the new conv tails of committed rows, in place in the pool: tail_pool[slot]
+// <- last 4 raw tokens of (tail_pool[slot], block)
+cudaError_t launch_tail_commit_pool(const void *block, void *tail_pool, const int *slots,
+                                    const int *commit, int pool_size, int rows, int len, int ch,
+                                    int *status, cudaStream_t stream);
+
+// C = A . W^T on the tensor cores (bf16, fp32 accumulation), A (M, K) and W
+// (N, K) row-major; columns [0, n_split) -> out0 (row stride n_split),
+// columns [n_split, N) -> out1 (row stride N - n_split) as softplus(c + bias1)
+struct GemmProblem {
+    const void *a, *w;
+    int M, N, K, n_split;
+    void *out0, *out1;
+    const float *bias1;
+    int *status;
+};
+cudaError_t launch_gemm_tc(const GemmProblem &g, cudaStream_t stream);
+
+// gradients of the mixer core (training path, fp32 results)
+struct BackwardProblem {
+    bimamba_dims dims;
+    const void *xbc, *dt, *dy;
+    const float *A, *D, *conv_w, *conv_b, *init;
+    float *dxbc, *ddt, *dA, *dD, *dconv_w, *dconv_b, *dinit;
+    void *workspace;
+};
+bool backward_supported(const bimamba_dims &d);
+size_t backward_workspace_bytes(const bimamba_dims &d);
+cudaError_t launch_backward(const BackwardProblem &q, cudaStream_t stream);
+
 template <typename T>
 cudaError_t launch_conv_silu(const void *u, void *out, const float *w, const float *bias,
                              const void *tail, int batch, int len, int ch, int rev, int silu,

@@ -69,48 +69,57 @@ constexpr int kP = 64;        // headdim of this kernel
 constexpr int kN = 128;       // d_state of this kernel
 constexpr int kHeads = 2;     // heads per CTA
 constexpr int kPP = kHeads * kP;   // x channels per CTA (128)
-constexpr int kAluThreads = 512;          // compute group (16 warps)
+constexpr int kGroupThreads = 256;        // each of the two compute groups (8 warps)
+constexpr int kTmemWarps = 8;             // warps 0..7: the tensor-memory group
 constexpr int kProducerWarp = 16;         // issues every MMA and TMA load
 constexpr int kProducerTid = 32 * kProducerWarp;
 constexpr int kHelperWarp = 17;           // dt copies, prefix sums, slot factors
-constexpr int kThreads = kAluThreads + 64;
+constexpr int kThreads = 2 * kGroupThreads + 64;
 constexpr int kBC = 2 * kN;   // B and C channels
 constexpr int kRawRows = kQ + 3;   // raw x rows per chunk: 128 slots + 3-token conv halo
 constexpr uint32_t kTmemCols = 512;
 
 // shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t kOffC = 0;          // C      [t][n]   2 x 16 KB (TMA, swizzled)
-constexpr uint32_t kOffB = 32768;      // B      [s][n]   2 x 16 KB (TMA, swizzled)
+constexpr uint32_t kOffZlo = 0;        // 2 KB of zeros (block-diagonal B operand, below the X tiles)
+constexpr uint32_t kOffC = 2048;       // C      [t][n]   2 x 16 KB (TMA, swizzled)
+constexpr uint32_t kOffB = kOffC + 32768;   // B      [s][n]   2 x 16 KB (TMA, swizzled)
 constexpr uint32_t kXbufBytes = 33792; // raw x [131][128] (TMA) -> X [s][p], 16 KB per head
-constexpr uint32_t kOffXbuf0 = 65536;  // x buffer of even walk chunks
+constexpr uint32_t kOffXbuf0 = kOffB + 32768;            // x buffer of even walk chunks
 constexpr uint32_t kOffXbuf1 = kOffXbuf0 + kXbufBytes;   // odd walk chunks
-constexpr uint32_t kOffXw = kOffXbuf1 + kXbufBytes;      // wX [s][p'] 2 x 16 KB
+constexpr uint32_t kOffXw = kOffXbuf1 + kXbufBytes;      // wX [s][p'] 2 x 16 KB; output staging
 constexpr uint32_t kOffS = kOffXw + 32768;               // S^T bf16 [n][p'] 2 x 16 KB
+constexpr uint32_t kOffZhi = kOffS + 32768;              // 2 KB of zeros (above the X tiles)
 constexpr uint32_t kRawBytes = kRawRows * kPP * 2;       // 33536
-constexpr uint32_t kOffCum = kOffS + 32768;      // f32[2][2][128] prefix sums of dt*A (chunk parity, head)
+constexpr uint32_t kOffCum = kOffZhi + 2048;     // f32[2][2][128] prefix sums of dt*A (chunk parity, head)
 constexpr uint32_t kOffDt = kOffCum + 2048;      // f32[2][2][128] dt
 constexpr uint32_t kOffFB = kOffDt + 2048;       // f32[2][2][128] exp(c_R - c_s) dt_s, R = block end
 constexpr uint32_t kOffWgt = kOffFB + 2048;      // f32[2][2][128] exp(c_last - c_s) dt_s
 constexpr uint32_t kOffF4 = kOffWgt + 2048;      // f32[2][2][128] exp(c_R4 - c_s) dt_s, R4 = s | 3
 constexpr uint32_t kOffConvW = kOffF4 + 2048;    // float4[128] conv taps of x
 constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
-constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 x12 + 2 flag pointers (see the kernel)
-constexpr uint32_t kOffTmem = kOffMbar + 112;    // u32 TMEM base
-constexpr uint32_t kOffFlag = kOffTmem + 4;      // i32 handshake result
-constexpr uint32_t kOffDtBuf = kOffFlag + 12;    // [2][128] bf16x2: dt of both heads, by cp.async
+constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 mbarriers (see the kernel)
+constexpr uint32_t kOffTmem = kOffMbar + 128;    // u32 TMEM base
+constexpr uint32_t kOffDtBuf = kOffTmem + 16;    // [2][128] bf16x2: dt of both heads, by cp.async
 constexpr uint32_t kSmemUsed = kOffDtBuf + 2 * kQ * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;   // + alignment slack
 constexpr uint32_t kBCBytes = 4 * kQ * 64 * 2;      // four 128 x 64 bf16 boxes
+static_assert(kOffC % 1024 == 0 && kOffB % 1024 == 0 && kOffXbuf0 % 1024 == 0, "tile alignment");
 static_assert(kOffXbuf1 % 1024 == 0 && kOffXw % 1024 == 0 && kOffS % 1024 == 0, "tile alignment");
+static_assert(kOffZhi % 1024 == 0, "tile alignment");
 static_assert(kRawBytes <= kXbufBytes, "raw x tile must fit its buffer");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory of one CTA");
 
-// TMEM columns: 0..255 hold G/Yd of one chunk and M of the other (the two
-// 128-column regions alternate per chunk); Yo and the state are fixed.
+// TMEM columns.  Region A (0..127) holds G of a chunk, then, in place, its
+// decay-masked M: the 16 columns of G for walk slots 16ks..16ks+15 become
+// M_0 (8 columns of packed bf16 pairs) and M_1 (the next 8), K-step ks of
+// the Yd product's A operand.  Region B (128..255) holds Yd, then Yo and the
+// state are fixed.
+constexpr uint32_t kColG = 0;
+constexpr uint32_t kColYd = 128;   // + 64 * head
 constexpr uint32_t kColYo = 256;   // + 64 * head
 constexpr uint32_t kColS = 384;    // + 64 * head
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
-constexpr int kArriveTid = 480;   // a thread outside warp 0 (which issues the MMAs)
 
 // Per-direction inputs are indexed [0] forward stream, [1] reverse stream
 // (the same pointers when the directions share their parameters); a CTA
@@ -156,22 +165,22 @@ __device__ __forceinline__ void st_release(int *p, int v)
     asm volatile("st.release.gpu.global.b32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
 
-// Barrier over the compute group only (named barrier 1, 512 threads); the
-// producer warp never joins it.
-__device__ __forceinline__ void alu_sync()
+// Barrier over one compute group (named barrier `id`, 256 threads); the
+// producer and helper warps never join it.
+__device__ __forceinline__ void grp_sync(int id)
 {
-    asm volatile("bar.sync 1, 512;" ::: "memory");
+    asm volatile("bar.sync %0, 256;" :: "r"(id) : "memory");
 }
 
-__device__ __forceinline__ bool alu_sync_and(bool pred)
+__device__ __forceinline__ bool grp_sync_and(int id, bool pred)
 {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.b32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 1, 512, p;\n\t"
+        "setp.ne.b32 p, %2, 0;\n\t"
+        "bar.red.and.pred q, %1, 256, p;\n\t"
         "selp.b32 %0, 1, 0, q;\n\t}"
-        : "=r"(r) : "r"((uint32_t)pred) : "memory");
+        : "=r"(r) : "r"(id), "r"((uint32_t)pred) : "memory");
     return r != 0;
 }
 
@@ -280,6 +289,19 @@ bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc_f, const __nv_bfloat16 *
 // zero state; writes the item's end state and its total decay.
 // kConcat: untied directions with concatenated outputs; each direction
 // stores its own half of every output row and the CTAs never meet.
+//
+// Warp roles (all communication through mbarriers; every wait is bounded):
+//   warps 0..7   tensor-memory group: per chunk k, once its MMAs are done,
+//                the output rows (Yd + exp(c) Yo, from TMEM) into a staging
+//                tile; then M(k+1) in place over G(k+1) and the state's
+//                chunk-start scaling with its bf16 copy (the Yo operand).
+//   warps 8..15  shared-memory group: per chunk k, the staged rows to global
+//                memory (the forward/reverse meeting), wX(k+1), and the
+//                in-place conv of chunk k+2's raw rows.
+//   warp 16      producer: every TMA load and every MMA.
+//   warp 17      helper: dt copies, prefix sums and per-slot decay factors.
+// The two compute groups work on different chunks at the same time, and
+// both overlap the tensor core.
 template <bool kStateOnly, bool kConcat>
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant__ CUtensorMap tm_x_r,
@@ -307,32 +329,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     float *f4 = reinterpret_cast<float *>(sm + kOffF4);
     float4 *convw = reinterpret_cast<float4 *>(sm + kOffConvW);
     float *convb = reinterpret_cast<float *>(sm + kOffConvB);
-    int *flag_slot = reinterpret_cast<int *>(sm + kOffFlag);
-    // mbarriers: B/C tiles landed, raw x landed (buffer 0 / 1), G done,
-    // M/state ready for the chunk's MMAs, chunk MMAs done, the dt prefix
-    // sums of an even / odd walk chunk written (one barrier per buffer, so
-    // that the producer may run a chunk ahead without phase aliasing)
-    const uint32_t mb_bc = sbase + kOffMbar;
-    const uint32_t mb_x0 = sbase + kOffMbar + 8;
-    const uint32_t mb_g = sbase + kOffMbar + 24;
-    const uint32_t mb_m = sbase + kOffMbar + 32;
-    const uint32_t mb_e = sbase + kOffMbar + 40;
-    const uint32_t mb_dt0 = sbase + kOffMbar + 48;   // + 8 * (chunk & 1)
-    // a chunk's output rows stored (even / odd walk chunk), and the handshake
-    // flag the producer then raises for it (null: nothing to publish)
-    const uint32_t mb_rows0 = sbase + kOffMbar + 64;
-    int **rel_flag = reinterpret_cast<int **>(sm + kOffMbar + 80);
-    // phase D of an even / odd walk chunk done: its cum/dts/fB buffer is free
-    const uint32_t mb_free0 = sbase + kOffMbar + 96;
-    auto dt_ready = [&](int k, uint32_t &mb, uint32_t &parity) {
-        mb = mb_dt0 + 8 * (k & 1);
-        parity = (k >> 1) & 1;
-    };
+    int *first_slot = reinterpret_cast<int *>(sm + kOffTmem + 4);
+    // mbarriers (each completes once per walk chunk unless noted):
+    const uint32_t mb_bc = sbase + kOffMbar;         // the chunk's B/C tiles landed
+    const uint32_t mb_x0 = sbase + kOffMbar + 8;     // raw x landed in buffer 0 / 1 (+8)
+    const uint32_t mb_g = sbase + kOffMbar + 24;     // G done
+    const uint32_t mb_m = sbase + kOffMbar + 32;     // the chunk's MMA operands ready (one arrival per group)
+    const uint32_t mb_e = sbase + kOffMbar + 40;     // the chunk's MMAs done
+    const uint32_t mb_dt0 = sbase + kOffMbar + 48;   // an even / odd chunk's prefix sums and factors (+8)
+    const uint32_t mb_free0 = sbase + kOffMbar + 64; // an even / odd chunk's factor buffers free (+8)
+    const uint32_t mb_staged = sbase + kOffMbar + 80;   // the chunk's output rows staged
+    const uint32_t mb_bcfree = sbase + kOffMbar + 88;   // the chunk's products that read B/C done
     auto xbuf_off = [](int k) { return (k & 1) ? kOffXbuf1 : kOffXbuf0; };
-    // TMEM regions that alternate between chunks: G(k) and Yd(k) use
-    // columns gcol(k) .. +127, M(k) uses mcol(k) .. +127 (the other region)
-    auto gcol = [](int k) -> uint32_t { return (k & 1) ? 128u : 0u; };
-    auto mcol = [](int k) -> uint32_t { return (k & 1) ? 0u : 128u; };
 
     auto chunk_of = [&](int k, int &t0, int &cnt, int &s0) {
         const int kg = k0 + k;
@@ -446,12 +454,17 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     const float *conv_b = rev ? p.conv_b[1] : p.conv_b[0];
     const bool has_conv = conv_w != nullptr;
     if (tid < kPP && has_conv) {
-        // stored as [q][g] for local channel 8g + q, so that the 16 channel
-        // groups of a warp read 16 consecutive entries (no bank conflicts)
+        // channel c = 4 cq + q of the pair stored at q * 32 + cq, so that
+        // the 32 conv threads of a warp (channel quads cq) read 32
+        // consecutive entries
         const int c = hp * kPP + tid;
-        const int slot = (tid & 7) * (kPP / 8) + (tid >> 3);
+        const int slot = (tid & 3) * 32 + (tid >> 2);
         convw[slot] = *reinterpret_cast<const float4 *>(conv_w + (size_t)c * 4);
         convb[slot] = conv_b ? conv_b[c] : 0.0f;
+    }
+    for (int i = tid; i < 2048 / 16; i += kThreads) {   // zero blocks of the block-diagonal Yd operand
+        reinterpret_cast<uint4 *>(sm + kOffZlo)[i] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4 *>(sm + kOffZhi)[i] = make_uint4(0, 0, 0, 0);
     }
     if (warp == 0) tc::tmem_alloc(sbase + kOffTmem, kTmemCols);
     if (tid == kProducerTid) {
@@ -461,139 +474,124 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         tc::mbar_init(mb_x0, 1);
         tc::mbar_init(mb_x0 + 8, 1);
         tc::mbar_init(mb_g, 1);
-        tc::mbar_init(mb_m, 1);
+        tc::mbar_init(mb_m, 2);          // one arrival from each compute group
         tc::mbar_init(mb_e, 1);
         tc::mbar_init(mb_dt0, 32);       // every helper lane arrives after its part of a scan
         tc::mbar_init(mb_dt0 + 8, 32);
-        tc::mbar_init(mb_free0, 1);
-        tc::mbar_init(mb_free0 + 8, 1);
-        tc::mbar_init(mb_rows0, 1);
-        tc::mbar_init(mb_rows0 + 8, 1);
+        tc::mbar_init(mb_free0, 2);      // both compute groups done with the factors
+        tc::mbar_init(mb_free0 + 8, 2);
+        tc::mbar_init(mb_staged, 1);
+        tc::mbar_init(mb_bcfree, 1);
         issue_x(0);
         if (nk > 1) issue_x(1);
         issue_bc(0);
     }
-    // Global loads that need nothing from the set-up start before its
-    // barrier, so that their latencies overlap (they dominate a CTA that
-    // covers a single chunk, as in block decode): the helper's first dt
-    // copies, and each compute thread's share of the caller's initial state.
     if (warp == kHelperWarp) {
         load_dt_async(0);
         if (nk > 1) load_dt_async(1);
     }
-    float sv_init[32];
-    {
-        const int row = tid & 127, rg = tid >> 7;
-        const size_t sidx0 = ((size_t)b * H + hp * kHeads + (rg >> 1)) * kP * kN;
-        const bool use_init = !kStateOnly && !rev && p.init && tid < kAluThreads;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            sv_init[i] = use_init ? __ldg(p.init + sidx0 + (size_t)(32 * (rg & 1) + i) * kN + row) : 0.0f;
-    }
+    tc::fence_proxy_async();   // the zero blocks, for the tensor core
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kOffTmem);
 
     if (warp == kProducerWarp) {
-        // ================= producer: every MMA and every TMA load, and the
-        // release of each chunk's rows (lane 0)
+        // ================= producer: every MMA and every TMA load (lane 0)
         const uint64_t dC = tc::smem_desc(sbase + kOffC, 16, 1024);       // K-major A (G, Yo)
         const uint64_t dB = tc::smem_desc(sbase + kOffB, 16, 1024);       // K-major B (G)
         const uint64_t dBmn = tc::smem_desc(sbase + kOffB, 16384, 1024);  // MN-major A (state)
-        const uint64_t dX0 = tc::smem_desc(sbase + kOffXbuf0, 1024, 1024);  // MN-major B (Yd)
-        const uint64_t dX1 = tc::smem_desc(sbase + kOffXbuf1, 1024, 1024);
         const uint64_t dS = tc::smem_desc(sbase + kOffS, 16384, 1024);    // MN-major B (Yo)
         const uint64_t dXw = tc::smem_desc(sbase + kOffXw, 16384, 1024);  // MN-major B (state)
         constexpr uint32_t idG = tc::idesc_bf16(128, 128, 0, 0);
-        constexpr uint32_t idYd = tc::idesc_bf16(128, 64, 0, 1);
-        constexpr uint32_t idYo = tc::idesc_bf16(128, 128, 0, 1);
+        constexpr uint32_t idY = tc::idesc_bf16(128, 128, 0, 1);
         constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
-        // lane 0: once chunk j's rows are stored, publish them to the partner
-        // CTA if this CTA arrived first (GPU-scope release; the rows were
-        // made visible to this thread through the group barrier and the
-        // mbarrier).  Done here so that the compute group never waits on it.
-        auto release_rows = [&](int j) -> bool {
-            const bool w = tc::mbar_wait_bounded(mb_rows0 + 8 * (j & 1), (j >> 1) & 1, kWaitCycles);
-            if (w) {
-                int *f = rel_flag[j & 1];
-                if (f) st_release(f, 1);
+        auto issue_g = [&]() {
+#pragma unroll
+            for (int ks = 0; ks < kN / 16; ++ks) {
+                const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                tc::mma_bf16(tmem + kColG, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
             }
-            return w;
+            tc::mma_commit(mb_g);
         };
         bool pok = true;
-        for (int k = 0; k < nk && pok; ++k) {
-            const uint32_t g = tmem + gcol(k);
-            if (lane == 0) {
-                // G(k) overwrites region gcol(k), last used by M(k-1): wait
-                // for the MMAs of chunk k-1, and for this chunk's B/C tiles
-                if (!kStateOnly && k > 0) pok = tc::mbar_wait_bounded(mb_e, (k - 1) & 1, kWaitCycles);
-                if (pok) pok = tc::mbar_wait_bounded(mb_bc, k & 1, kWaitCycles);
+        if (lane == 0) {
+            if (!kStateOnly) {
+                pok = tc::mbar_wait_bounded(mb_bc, 0, kWaitCycles);
                 if (pok) {
                     tc::fence_after_sync();
-                    if constexpr (!kStateOnly) {
-#pragma unroll
-                        for (int ks = 0; ks < kN / 16; ++ks) {
-                            const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            tc::mma_bf16(g, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
-                        }
-                        tc::mma_commit(mb_g);
-                    }
+                    issue_g();
                 }
             }
-            if (lane == 0) {
-                if (!kStateOnly && k > 0 && pok) pok = release_rows(k - 1);
-                // Yd_h = M_h X_h, Yo = C S_in^T, S^T += B^T (wX)
-                if (pok) pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
-                if (pok) {
-                    tc::fence_after_sync();
-                    if constexpr (!kStateOnly) {
-                        const uint64_t dX = (k & 1) ? dX1 : dX0;
-                        const uint32_t mc = tmem + mcol(k);
+            for (int k = 0; k < nk && pok; ++k) {
+                pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
+                if (pok && kStateOnly) pok = tc::mbar_wait_bounded(mb_bc, k & 1, kWaitCycles);
+                if (!pok) break;
+                tc::fence_after_sync();
+                // the state product first: the next chunk's state scaling waits for it
 #pragma unroll
-                        for (int ks = 0; ks < kQ / 16; ++ks) {
-#pragma unroll
-                            for (int hd = 0; hd < kHeads; ++hd)
-                                tc::mma_bf16_tmemA(g + 64 * hd, mc + 64 * hd + 8 * ks,
-                                                   tc::desc_add(dX, hd * 16384 + ks * 2048), idYd, ks > 0);
-                        }
-                    }
+                for (int ks = 0; ks < kQ / 16; ++ks)
+                    tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048), tc::desc_add(dXw, ks * 2048),
+                                 idS, 1);
+                if constexpr (!kStateOnly) {
+                    // Yo = C S_in^T (both heads)
 #pragma unroll
                     for (int ks = 0; ks < kN / 16; ++ks) {
                         const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        if constexpr (!kStateOnly)
-                            tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048),
-                                         idYo, ks > 0);
-                        tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048),
-                                     tc::desc_add(dXw, ks * 2048), idS, 1);
+                        tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048), idY,
+                                     ks > 0);
                     }
-                    tc::mma_commit(mb_e);
+                    // the B/C tiles are free once the state product and Yo are
+                    // done: the next chunk's tiles load while Yd runs
+                    tc::mma_commit(mb_bcfree);
+                    // Yd = [M_0 | M_1] . [[X_0, 0], [0, X_1]]: one N = 128 product over
+                    // K = 256.  K-steps 0..7 take X_0's rows as N block 0 and the
+                    // zeros above the tiles as N block 1 (leading offset = the
+                    // distance to them); K-steps 8..15 the zeros below as N block 0
+                    // and X_1's rows as N block 1.
+                    const uint32_t xb = sbase + xbuf_off(k);
+                    const uint64_t d0 = tc::smem_desc(xb, sbase + kOffZhi - xb, 1024);
+                    const uint64_t d1 = tc::smem_desc(sbase + kOffZlo, xb + 16384 - (sbase + kOffZlo), 1024);
+                    constexpr uint64_t kStep0 = 128ull - (128ull << 16);   // start += 2 KB, offset -= 2 KB
+                    constexpr uint64_t kStep1 = 128ull << 16;              // offset += 2 KB
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        tc::mma_bf16_tmemA(tmem + kColYd, tmem + kColG + 16 * ks, d0 + ks * kStep0, idY, ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        tc::mma_bf16_tmemA(tmem + kColYd, tmem + kColG + 16 * ks + 8, d1 + ks * kStep1, idY, 1);
                 }
-            }
-            pok = __shfl_sync(0xffffffffu, pok, 0);
-            if (!pok || k + 1 >= nk) break;
-            // once they complete, the B/C tiles and this chunk's x buffer
-            // are free: load the next chunk's tiles and the chunk after
-            // next's raw x rows
-            if (lane == 0) {
-                pok = tc::mbar_wait_bounded(mb_e, k & 1, kWaitCycles);
-                if (pok) {
+                tc::mma_commit(mb_e);
+                if (k + 1 >= nk) break;
+                if constexpr (!kStateOnly) {
+                    pok = tc::mbar_wait_bounded(mb_bcfree, k & 1, kWaitCycles);
+                    if (!pok) break;
                     issue_bc(k + 1);
-                    if (k + 2 < nk) issue_x(k + 2);
+                }
+                // once all of them complete: this chunk's x buffer and TMEM
+                // region A are free
+                pok = tc::mbar_wait_bounded(mb_e, k & 1, kWaitCycles);
+                if (!pok) break;
+                if constexpr (kStateOnly) issue_bc(k + 1);
+                if (k + 2 < nk) issue_x(k + 2);
+                if constexpr (!kStateOnly) {
+                    pok = tc::mbar_wait_bounded(mb_bc, (k + 1) & 1, kWaitCycles);
+                    if (!pok) break;
+                    tc::fence_after_sync();
+                    issue_g();
                 }
             }
-            pok = __shfl_sync(0xffffffffu, pok, 0);
+            if (!pok) record_error(p.status, kStatusTimeout);
         }
-        if (!kStateOnly && lane == 0 && pok && nk > 0) pok = release_rows(nk - 1);
-        if (lane == 0 && !pok) record_error(p.status, kStatusTimeout);
+        __syncwarp();
     } else if (warp == kHelperWarp) {
         // ================= helper: dt copies, prefix sums and slot factors
-        // of each chunk, up to two chunks ahead of phase D (the copies of
-        // chunks 0 and 1 were issued before the set-up barrier)
+        // of each chunk, up to two chunks ahead (the copies of chunks 0 and 1
+        // were issued before the set-up barrier)
         bool hok = true;
         for (int j = 0; j < nk; ++j) {
             if (j >= 2) {
-                // buffer j % 2 last held chunk j-2, read up to its phase D
+                // buffer j % 2 last held chunk j-2: wait until both groups are done with it
                 if (lane == 0)
                     hok = tc::mbar_wait_bounded(mb_free0 + 8 * (j & 1), ((j >> 1) - 1) & 1, kWaitCycles);
                 hok = __shfl_sync(0xffffffffu, hok, 0);
@@ -605,79 +603,326 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (lane == 0 && !hok) record_error(p.status, kStatusTimeout);
-    } else {
-        // ================= compute group: 512 threads ======================
-        // thread roles: row = TMEM lane / tile row; rg = 32-column group of
-        // the head pair's 128 columns (head rg >> 1, half rg & 1)
+    } else if (warp < kTmemWarps) {
+        // ================= tensor-memory group (warps 0..7) ================
+        // thread (row, h): TMEM lane `row` (token slot t, or state row n), head h
         const int row = tid & 127;
-        const int rg = tid >> 7;
-        const int hh = rg >> 1;
-        const int hsub = rg & 1;
-        const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        const int h = tid >> 7;
         const int quad = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
+        const int head_g = hp * kHeads + h;
+        auto a_wait = [&](uint32_t mb, uint32_t parity) -> bool {
+            bool w = true;
+            if (tid == 0) w = tc::mbar_wait_bounded(mb, parity, kWaitCycles);
+            return grp_sync_and(1, w);
+        };
+        // ---- the state entering the walk, S^T[n = row][p] of head h ->
+        // TMEM columns kColS + 64 h: the caller's initial state (forward) or
+        // zero, carried through the shards before this one (sequence shards)
+        // and the items before this segment: S <- 2^dec_i S + S_i.
+        {
+            const size_t sidx = ((size_t)b * H + head_g) * kP * kN;
+            const bool use_init = !kStateOnly && !rev && p.init;
+            const int n_sh = (kStateOnly || !p.shard_states) ? 0 : (rev ? p.nranks - 1 - p.rank : p.rank);
+            const int n_in = (kStateOnly || p.item_chunks == 0) ? 0 : k0 / p.item_chunks;
+#pragma unroll 1
+            for (int q16 = 0; q16 < 4; ++q16) {
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    v[i] = use_init ? __ldg(p.init + sidx + (size_t)(16 * q16 + i) * kN + row) : 0.0f;
+                for (int it = 0; it < n_sh; ++it) {
+                    const int q = rev ? p.nranks - 1 - it : it;
+                    const size_t e = (((size_t)q * 2 + dir) * p.batch + b) * H + head_g;
+                    const float *si = p.shard_states + e * kP * kN;
+                    const float a = tc::exp2_approx(p.shard_dec[e]);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = fmaf(v[i], a, si[(size_t)(16 * q16 + i) * kN + row]);
+                }
+                for (int it = 0; it < n_in; ++it) {
+                    const float *si = p.seg_state + ((item_row + it) * kHeads + h) * kP * kN;
+                    const float a = tc::exp2_approx(p.seg_dec[(item_row + it) * kHeads + h]);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = fmaf(v[i], a, si[(size_t)(16 * q16 + i) * kN + row]);
+                }
+                uint32_t r[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(v[i]);
+                tc::tmem_st16(tmem + lane_base + kColS + 64 * h + 16 * q16, r);
+            }
+        }
+        // D of both heads of the pair (M's diagonal; a thread builds both)
+        const float *Dpair = (rev ? p.D[1] : p.D[0]) + hp * kHeads;
+        const float D0 = kStateOnly ? 0.0f : Dpair[0], D1 = kStateOnly ? 0.0f : Dpair[1];
+        float dec = 0.0f;   // state-only: the item's total decay (log2 units)
+
+        // M(k) in place over G(k) (region A): thread (t = row, h) owns the
+        // walk slots of 32-slot blocks 2h, 2h+1 for both heads.  The 16 G
+        // columns of slots 16ks..16ks+15 become [M_0 ks | M_1 ks] (8 + 8
+        // columns of packed bf16 pairs), so no other thread reads them.
+        auto build_m = [&](int k) {
+            const int par = k & 1;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int jb = 2 * h + jj;          // 32-slot block of s
+                const uint32_t col = tmem + lane_base + kColG + 32 * jb;
+                if (jb > quad) {                    // warp-uniform: all s > t
+                    uint32_t z[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) z[i] = 0u;
+                    tc::tmem_st16(col, z);
+                    tc::tmem_st16(col + 16, z);
+                    continue;
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {       // 16-slot unit = K-step 2 jb + u
+                    float g[16];
+                    tc::tmem_ld16(col + 16 * u, g);
+                    uint32_t out[16];               // [head][8 packed pairs]
+#pragma unroll
+                    for (int hd = 0; hd < kHeads; ++hd) {
+                        const float *cm = cum + (par * kHeads + hd) * kQ;
+                        const float ct = cm[row];
+                        const int s0u = 32 * jb + 16 * u;   // first slot of the unit
+                        if (jb < quad) {
+                            // whole block below the diagonal: factorised decay
+                            const float *fbh = fB + (par * kHeads + hd) * kQ + s0u;
+                            const float et = tc::exp2_approx(ct - cm[32 * jb + 31]);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                out[8 * hd + i] = tc::pack_bf16x2(g[2 * i] * et * fbh[2 * i],
+                                                                  g[2 * i + 1] * et * fbh[2 * i + 1]);
+                        } else {
+                            // diagonal block, D on the diagonal; slot s0u + i
+                            // against t's offset r31 in the block
+                            const int r = (row & 31) - 16 * u;
+                            const float Dh = hd ? D1 : D0;
+                            float v[16];
+                            if (cm[32 * jb] - cm[32 * jb + 31] <= 60.0f) {   // warp-uniform (head, block)
+                                // 4-slot sub-blocks: exp(c_t - c_s) = exp(c_t - c_R4)
+                                // exp(c_R4 - c_s), R4 = s | 3.  With the block's whole
+                                // decay at most 2^60 neither factor overflows; for s <= t
+                                // the product is the decay itself
+                                const float *f4h = f4 + (par * kHeads + hd) * kQ + s0u;
+                                float rf[4];
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) rf[j] = tc::exp2_approx(ct - cm[s0u + 4 * j + 3]);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) {
+                                    const float x = fmaf(g[i] * rf[i >> 2], f4h[i], (i == r) ? Dh : 0.0f);
+                                    v[i] = (i <= r) ? x : 0.0f;
+                                }
+                            } else {
+                                // steep decays: one exponential per element, each <= 1
+                                const float *dh_ = dts + (par * kHeads + hd) * kQ + s0u;
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) {
+                                    const float e = tc::exp2_approx(fminf(ct - cm[s0u + i], 0.0f));
+                                    const float x = fmaf(g[i] * e, dh_[i], (i == r) ? Dh : 0.0f);
+                                    v[i] = (i <= r) ? x : 0.0f;
+                                }
+                            }
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) out[8 * hd + i] = tc::pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                        }
+                    }
+                    tc::tmem_st16(col + 16 * u, out);
+                }
+            }
+        };
+        // the state at chunk k's start: bf16 copy of S_in (the Yo operand),
+        // then S <- exp(c_last) S in place
+        auto scale_state = [&](int k) {
+            const float cl = cum[((k & 1) * kHeads + h) * kQ + kQ - 1];
+            const float a_last = tc::exp2_approx(cl);
+            if constexpr (kStateOnly) dec += cl;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float sv[32];
+                const uint32_t col = tmem + lane_base + kColS + 64 * h + 32 * half;
+                tc::tmem_ld32(col, sv);
+                if constexpr (!kStateOnly) {
+#pragma unroll
+                    for (int pc = 0; pc < 4; ++pc)
+                        *reinterpret_cast<uint4 *>(sm + kOffS + h * 16384 + tc::sw128(row, 4 * half + pc)) =
+                            pack8(sv + 8 * pc);
+                }
+#pragma unroll
+                for (int half16 = 0; half16 < 2; ++half16) {
+                    uint32_t r[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sv[16 * half16 + i] * a_last);
+                    tc::tmem_st16(col + 16 * half16, r);
+                }
+            }
+        };
+        // chunk k's output rows, y = Yd + exp(c_t) Yo, into the staging tile
+        // (the wX buffer, free once the chunk's MMAs are done): row t at
+        // t * 256 bytes, 16-byte piece q of it at q ^ (t & 15)
+        auto stage_rows = [&](int k) {
+            const float et = tc::exp2_approx(cum[((k & 1) * kHeads + h) * kQ + row]);
+#pragma unroll
+            for (int qtr = 0; qtr < 4; ++qtr) {
+                float yd[16], yo[16];
+                tc::tmem_ld16(tmem + lane_base + kColYd + 64 * h + 16 * qtr, yd);
+                tc::tmem_ld16(tmem + lane_base + kColYo + 64 * h + 16 * qtr, yo);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) yd[i] = fmaf(et, yo[i], yd[i]);
+#pragma unroll
+                for (int pc = 0; pc < 2; ++pc) {
+                    const int piece = 8 * h + 2 * qtr + pc;
+                    *reinterpret_cast<uint4 *>(sm + kOffXw + row * 256 + ((piece ^ (row & 15)) << 4)) =
+                        pack8(yd + 8 * pc);
+                }
+            }
+        };
+
+        bool ok = a_wait(mb_dt0, 0);   // chunk 0's prefix sums and factors
+        if (ok && !kStateOnly) ok = a_wait(mb_g, 0);
+        if (ok) {
+            tc::fence_after_sync();
+            if constexpr (!kStateOnly) build_m(0);
+            scale_state(0);
+            tc::fence_proxy_async();
+            tc::fence_before_sync();
+            grp_sync(1);
+            if (tid == 0) tc::mbar_arrive(mb_m);
+        }
+        for (int k = 0; k < nk && ok; ++k) {
+            ok = a_wait(mb_e, k & 1);   // chunk k's MMAs done
+            if (!ok) break;
+            tc::fence_after_sync();
+            if constexpr (!kStateOnly) {
+                stage_rows(k);
+                tc::fence_before_sync();   // TMEM reads done before the next chunk's MMAs
+                grp_sync(1);
+                if (tid == 0) tc::mbar_arrive(mb_staged);
+            }
+            if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * (k & 1));
+            if (k + 1 >= nk) break;
+            ok = a_wait(mb_dt0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
+            if (ok && !kStateOnly) ok = a_wait(mb_g, (k + 1) & 1);
+            if (!ok) break;
+            tc::fence_after_sync();
+            if constexpr (!kStateOnly) build_m(k + 1);
+            scale_state(k + 1);
+            tc::fence_proxy_async();   // the bf16 state copy, for the tensor core
+            tc::fence_before_sync();
+            grp_sync(1);
+            if (tid == 0) tc::mbar_arrive(mb_m);
+        }
+        if (ok) {
+            // the last chunk's MMAs are done (waited above)
+            if constexpr (kStateOnly) {
+                // the item's end state and total decay
+                const size_t item = item_row + blockIdx.z;
+                float *so = p.seg_state + (item * kHeads + h) * kP * kN;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float sv[32];
+                    tc::tmem_ld32(tmem + lane_base + kColS + 64 * h + 32 * half, sv);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) so[(size_t)(32 * half + i) * kN + row] = sv[i];
+                }
+                if (row == 0) p.seg_dec[item * kHeads + h] = dec;
+            } else if (!rev && p.fin && k0 + nk == p.nchunks) {
+                const size_t sidx = ((size_t)b * H + head_g) * kP * kN;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float sv[32];
+                    tc::tmem_ld32(tmem + lane_base + kColS + 64 * h + 32 * half, sv);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) p.fin[sidx + (size_t)(32 * half + i) * kN + row] = sv[i];
+                }
+            }
+        }
+        if (!ok && tid == 0) record_error(p.status, kStatusTimeout);
+    } else {
+        // ================= shared-memory group (warps 8..15) ===============
+        const int tb = tid - kGroupThreads;   // 0..255
+        auto b_wait = [&](uint32_t mb, uint32_t parity) -> bool {
+            bool w = true;
+            if (tb == 0) w = tc::mbar_wait_bounded(mb, parity, kWaitCycles);
+            return grp_sync_and(2, w);
+        };
         // conv+SiLU of both heads' x for walk chunk k, in place: the raw
         // rows in x buffer k % 2 become the swizzled X tile of the chunk.
-        // Thread: 8 channels (group g: head g >> 3, piece g & 7) x 4 slots.
-        // Raw row of token u: forward u - (t0 - 3), reverse u - t0.  Every
-        // thread reads its raw rows before the barrier and writes after it.
+        // Thread: channel quad cq (channels 4cq..4cq+3; head cq >> 4) x 16
+        // walk slots 16sg..16sg+15.  Raw row of walk offset j: forward j + 3
+        // (the box starts 3 tokens early), reverse cnt - 1 - j.  Every thread
+        // reads its raw rows before the group barrier and writes after it.
         auto conv_chunk = [&](int k) {
             int t0, cnt, s0;
             chunk_of(k, t0, cnt, s0);
             uint8_t *buf = sm + xbuf_off(k);
-            const __nv_bfloat16 *rawp = reinterpret_cast<const __nv_bfloat16 *>(buf);
-            const int g = tid & 15;
-            const int gh = g >> 3, gp = g & 7;
-            const int j0 = (tid >> 4) * 4;
-            uint4 rr[7];
+            const int cq = tb & 31, sg = tb >> 5;
+            const int j0 = 16 * sg;
+            uint2 rr[19];
 #pragma unroll
-            for (int i = 0; i < 7; ++i) {
+            for (int i = 0; i < 19; ++i) {
                 const int jw = j0 + i - 3;   // walk offset of the raw row
                 const int rrow = rev ? cnt - 1 - jw : jw + 3;
                 rr[i] = (rrow >= 0 && rrow < kRawRows)
-                            ? *reinterpret_cast<const uint4 *>(rawp + rrow * kPP + 8 * g)
-                            : make_uint4(0, 0, 0, 0);
+                            ? *reinterpret_cast<const uint2 *>(buf + rrow * (kPP * 2) + 8 * cq)
+                            : make_uint2(0, 0);
             }
-            alu_sync();
-            float o[4][8];
-            const __nv_bfloat16 *ru = reinterpret_cast<const __nv_bfloat16 *>(rr);
+            grp_sync(2);
+            const int gh = cq >> 4, piece = (cq & 15) >> 1, sub = cq & 1;
+            uint8_t *dst = buf + gh * 16384 + 8 * sub;
+            float u0[4], u1[4], u2[4];
+            auto unpack4 = [](uint2 r, float (&v)[4]) {
+                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
+                const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
+                v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
+            };
+            unpack4(rr[0], u0);
+            unpack4(rr[1], u1);
+            unpack4(rr[2], u2);
+            const bool full = j0 + 16 <= cnt;
             if (has_conv) {
+                float4 w[4];
+                float bq[4];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 w4 = convw[q * (kPP / 8) + g];
-                    const float bq = convb[q * (kPP / 8) + g];
-                    float u[7];
+                for (int q = 0; q < 4; ++q) {
+                    w[q] = convw[q * 32 + cq];
+                    bq[q] = convb[q * 32 + cq];
+                }
 #pragma unroll
-                    for (int r = 0; r < 7; ++r) u[r] = __bfloat162float(ru[8 * r + q]);
+                for (int i = 0; i < 16; ++i) {
+                    float u3[4], o[4];
+                    unpack4(rr[i + 3], u3);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float acc = bq;
-                        acc = fmaf(w4.x, u[i], acc);
-                        acc = fmaf(w4.y, u[i + 1], acc);
-                        acc = fmaf(w4.z, u[i + 2], acc);
-                        acc = fmaf(w4.w, u[i + 3], acc);
-                        o[i][q] = (j0 + i < cnt) ? tc::silu_tanh(acc) : 0.0f;
+                    for (int q = 0; q < 4; ++q) {
+                        float acc = bq[q];
+                        acc = fmaf(w[q].x, u0[q], acc);
+                        acc = fmaf(w[q].y, u1[q], acc);
+                        acc = fmaf(w[q].z, u2[q], acc);
+                        acc = fmaf(w[q].w, u3[q], acc);
+                        o[q] = tc::silu_tanh(acc);
+                        u0[q] = u1[q]; u1[q] = u2[q]; u2[q] = u3[q];
                     }
+                    uint2 pk = make_uint2(tc::pack_bf16x2(o[0], o[1]), tc::pack_bf16x2(o[2], o[3]));
+                    if (!full && j0 + i >= cnt) pk = make_uint2(0, 0);
+                    *reinterpret_cast<uint2 *>(dst + tc::sw128(j0 + i, piece)) = pk;
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        o[i][q] = (j0 + i < cnt) ? __bfloat162float(ru[8 * (i + 3) + q]) : 0.0f;
+                for (int i = 0; i < 16; ++i) {
+                    uint2 pk = rr[i + 3];
+                    if (!full && j0 + i >= cnt) pk = make_uint2(0, 0);
+                    *reinterpret_cast<uint2 *>(dst + tc::sw128(j0 + i, piece)) = pk;
+                }
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<uint4 *>(buf + gh * 16384 + tc::sw128(j0 + i, gp)) = pack8(o[i]);
         };
-        // wX = w_s * X for walk chunk k (X tile in x buffer k % 2)
+        // wX = w_s * X for walk chunk k (X tile in x buffer k % 2): thread
+        // (slot j, head gh), the head's 64 channels
         auto weight_chunk = [&](int k) {
             const uint8_t *xt = sm + xbuf_off(k);
-            const int j = tid & 127, q4 = tid >> 7;   // slot, quarter of the 128 columns
-            const int gh = q4 >> 1;
+            const int j = tb & 127, gh = tb >> 7;
             const float wj = wgt[((k & 1) * kHeads + gh) * kQ + j];
 #pragma unroll
-            for (int pc = 0; pc < 4; ++pc) {
-                const uint32_t off = gh * 16384 + tc::sw128(j, 4 * (q4 & 1) + pc);
+            for (int pc = 0; pc < 8; ++pc) {
+                const uint32_t off = gh * 16384 + tc::sw128(j, pc);
                 float v[8];
                 unpack8(*reinterpret_cast<const uint4 *>(xt + off), v);
 #pragma unroll
@@ -685,317 +930,139 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 *reinterpret_cast<uint4 *>(sm + kOffXw + off) = pack8(v);
             }
         };
-        // one thread polls an mbarrier (two if mb2 != 0); the group barrier
-        // releases the rest
-        auto wait_all = [&](uint32_t mb, uint32_t parity, uint32_t mb2 = 0, uint32_t parity2 = 0) -> bool {
-            bool w = true;
-            if (tid == 0) {
-                w = tc::mbar_wait_bounded(mb, parity, kWaitCycles);
-                if (w && mb2) w = tc::mbar_wait_bounded(mb2, parity2, kWaitCycles);
-            }
-            return alu_sync_and(w);
-        };
 
-        // ---- state S^T[n = row][p' = 32*rg + i] -> TMEM columns kColS + 32*rg.
-        // A segment's entering state: the caller's initial state (forward
-        // stream; loaded before the set-up barrier) or zero, carried through
-        // the items before the segment: S <- 2^dec_i S + S_i, with S_i item
-        // i's end state from zero.
-        const int head_g = hp * kHeads + hh;     // global head of this thread's columns
-        const size_t sidx = ((size_t)b * H + head_g) * kP * kN;
-        {
-            float sv[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] = sv_init[i];
-            // sequence shards: the walk enters this shard with the state the
-            // shards before it in walk order leave (forward: ranks 0..rank-1
-            // from the initial state; reverse: ranks nranks-1..rank+1 from zero)
-            const int n_sh = (kStateOnly || !p.shard_states) ? 0 : (rev ? p.nranks - 1 - p.rank : p.rank);
-            for (int it = 0; it < n_sh; ++it) {
-                const int q = rev ? p.nranks - 1 - it : it;
-                const size_t e = (((size_t)q * 2 + dir) * p.batch + b) * H + head_g;
-                const float *si = p.shard_states + e * kP * kN;
-                const float a = tc::exp2_approx(p.shard_dec[e]);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[i] = fmaf(sv[i], a, si[(size_t)(32 * hsub + i) * kN + row]);
-            }
-            const int n_in = (kStateOnly || p.item_chunks == 0) ? 0 : k0 / p.item_chunks;
-            for (int it = 0; it < n_in; ++it) {
-                const float *si = p.seg_state + ((item_row + it) * kHeads + hh) * kP * kN;
-                const float a = tc::exp2_approx(p.seg_dec[(item_row + it) * kHeads + hh]);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[i] = fmaf(sv[i], a, si[(size_t)(32 * hsub + i) * kN + row]);
-            }
-#pragma unroll
-            for (int half16 = 0; half16 < 2; ++half16) {
-                uint32_t r[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sv[16 * half16 + i]);
-                tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
-            }
-        }
-        uint32_t mbd, pard;
-        dt_ready(0, mbd, pard);
-        bool ok = wait_all(mbd, pard);   // chunk 0's prefix sums and slot factors
-        float dec = 0.0f;   // state-only: total decay of the item (log2 units)
-        const float Dh = kStateOnly ? 0.0f : (rev ? p.D[1] : p.D[0])[head_g];   // no D for states
-
-        int arrival = 0;   // result of this chunk's arrival atomic (thread kArriveTid)
-        ok = ok && wait_all(mb_x0, 0);
+        bool ok = b_wait(mb_x0, 0);
         if (ok) {
             // decode and sequence shards: the conv history before token 0
             // comes from the tail; for sequence shards the reverse stream's
             // conv reads the tokens after the shard from the head (raw rows
             // cnt .. cnt+2 of the walk's first chunk, past the shard end)
             if (!rev && p.tail && k0 == 0) {
-                for (int e = tid; e < 3 * (kPP / 8); e += kAluThreads) {
+                for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
                     const int r = e / (kPP / 8), g = e % (kPP / 8);
                     *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
                         *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
                                                          hp * kPP + 8 * g);
                 }
-                alu_sync();
+                grp_sync(2);
             }
             if (rev && p.head && k0 == 0) {
                 int t0, cnt, s0;
                 chunk_of(0, t0, cnt, s0);
-                for (int e = tid; e < 3 * (kPP / 8); e += kAluThreads) {
+                for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
                     const int r = e / (kPP / 8), g = e % (kPP / 8);
                     *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + (cnt + r) * (kPP * 2) + g * 16) =
                         *reinterpret_cast<const uint4 *>(p.head + ((size_t)b * 4 + r) * ch +
                                                          hp * kPP + 8 * g);
                 }
-                alu_sync();
+                grp_sync(2);
             }
             conv_chunk(0);
-            alu_sync();
-            weight_chunk(0);
+            ok = b_wait(mb_dt0, 0);   // (also the barrier between conv writes and wX reads)
         }
-
+        if (ok) {
+            weight_chunk(0);
+            tc::fence_proxy_async();
+            grp_sync(2);
+            if (tb == 0) {
+                tc::mbar_arrive(mb_m);
+                tc::mbar_arrive(mb_free0);
+            }
+            if (nk > 1) {
+                ok = b_wait(mb_x0 + 8, 0);
+                if (ok) conv_chunk(1);
+            }
+        }
+        int arrival = 0;
         for (int k = 0; k < nk && ok; ++k) {
             int t0, cnt, s0;
             const int c = chunk_of(k, t0, cnt, s0);
-            const bool more = k + 1 < nk;
-
-            // arrive at this chunk's forward/reverse meeting point; the
-            // result is read only after the chunk's MMAs
-            if (!kStateOnly && !kConcat && tid == kArriveTid)
-                arrival = atomicAdd(p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2, 1);
-
-            // ---- D: M_h (both heads, into TMEM) and the state's chunk-start
-            // scaling, once G(k) is done.  Thread (row t, rg): head hh,
-            // s-blocks 2*hsub, 2*hsub+1.
-            tc::fence_proxy_async();          // wX of this chunk (written last iteration)
             if constexpr (!kStateOnly) {
-                ok = wait_all(mb_g, k & 1);
+                // ---- chunk k's rows, and the forward + reverse sum.  The two
+                // CTAs of a (sequence, head pair) meet per token chunk: the
+                // first to arrive stores its rows, the second adds its own to
+                // them (bf16 reductions at L2) once the first has published.
+                int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
+                if (!kConcat && tb == 0) arrival = atomicAdd(fl, 1);
+                ok = b_wait(mb_staged, k & 1);
                 if (!ok) break;
-            }
-            tc::fence_after_sync();
-            const float *cumk = cum + ((k & 1) * kHeads + hh) * kQ;   // this chunk, this head
-            const float *dtsk = dts + ((k & 1) * kHeads + hh) * kQ;
-            const float ct = cumk[row];                     // kept for the epilogue
-            const float a_last = tc::exp2_approx(cumk[kQ - 1]);
-            if constexpr (kStateOnly) dec += cumk[kQ - 1];
-            {
-                const uint32_t gc = gcol(k), mc = mcol(k);
-                if constexpr (!kStateOnly) {
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int jb = 2 * hsub + jj;           // 32-slot block of s
-                        uint32_t packed[16];
-                        if (jb > quad) {                        // warp-uniform: all s > t
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) packed[i] = 0u;
-                        } else {
-                            float gv[32];
-                            tc::tmem_ld32(tmem + lane_base + gc + 32 * jb, gv);
-                            const float *fbh = fB + ((k & 1) * kHeads + hh) * kQ + 32 * jb;
-                            if (jb < quad) {
-                                // whole block below the diagonal: factorised decay
-                                const float et = tc::exp2_approx(ct - cumk[32 * jb + 31]);
-#pragma unroll
-                                for (int i = 0; i < 16; ++i)
-                                    packed[i] = tc::pack_bf16x2(gv[2 * i] * et * fbh[2 * i],
-                                                                gv[2 * i + 1] * et * fbh[2 * i + 1]);
-                            } else {
-                                // diagonal block, D on the diagonal
-                                const float *ch_ = cumk + 32 * jb;
-                                const int r31 = row & 31;
-                                if (ch_[0] - ch_[31] <= 60.0f) {   // warp-uniform (head, block)
-                                    // 4-slot sub-blocks: exp(c_t - c_s) = exp(c_t - c_R4)
-                                    // exp(c_R4 - c_s), R4 = s | 3.  With the block's whole
-                                    // decay at most 2^60 neither factor overflows; for s <= t
-                                    // the product is the decay itself
-                                    const float *f4h = f4 + ((k & 1) * kHeads + hh) * kQ + 32 * jb;
-                                    float rf[8];
-#pragma unroll
-                                    for (int j = 0; j < 8; ++j) rf[j] = tc::exp2_approx(ct - ch_[4 * j + 3]);
-#pragma unroll
-                                    for (int i = 0; i < 32; ++i) {
-                                        const float v = fmaf(gv[i] * rf[i >> 2], f4h[i], (i == r31) ? Dh : 0.0f);
-                                        gv[i] = (i <= r31) ? v : 0.0f;
-                                    }
-                                } else {
-                                    // steep decays: one exponential per element, each <= 1
-                                    const float *dh_ = dtsk + 32 * jb;
-#pragma unroll
-                                    for (int i = 0; i < 32; ++i) {
-                                        const float e = tc::exp2_approx(fminf(ct - ch_[i], 0.0f));
-                                        const float v = fmaf(gv[i] * e, dh_[i], (i == r31) ? Dh : 0.0f);
-                                        gv[i] = (i <= r31) ? v : 0.0f;
-                                    }
-                                }
-#pragma unroll
-                                for (int i = 0; i < 16; ++i) packed[i] = tc::pack_bf16x2(gv[2 * i], gv[2 * i + 1]);
+                bool ready = true;
+                if (tb == 0) {
+                    const bool first = kConcat || arrival == 0;
+                    *first_slot = first;
+                    if (!first) {
+                        // the partner CTA arrived first; wait (bounded) until
+                        // its rows are visible
+                        ready = ld_acquire(fl + 1) != 0;
+                        if (!ready) {
+                            const long long w0 = clock64();
+                            while (!(ready = ld_acquire(fl + 1) != 0)) {
+                                if (clock64() - w0 > kWaitCycles) break;
                             }
                         }
-                        tc::tmem_st16(tmem + lane_base + mc + 64 * hh + 16 * jb, packed);
                     }
                 }
-                // state: bf16 copy of S_in (the Yo operand), then S <- exp(c_last) S
-                float sv[32];
-                tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
-                if constexpr (!kStateOnly) {
-#pragma unroll
-                    for (int pc = 0; pc < 4; ++pc)
-                        *reinterpret_cast<uint4 *>(sm + kOffS + hh * 16384 +
-                                                   tc::sw128(row, 4 * hsub + pc)) = pack8(sv + 8 * pc);
+                // a wait that gave up stops the walk here: the partner's rows
+                // are not added to, and the meeting counters are left as they
+                // are (the caller zero-fills the workspace again after a timeout)
+                if (!grp_sync_and(2, ready)) {
+                    ok = false;
+                    break;
                 }
+                const bool first = *first_slot != 0;
+                const int cp = tb & 15;          // 16-byte piece of a row (8 channels)
+                const int cr = tb >> 4;          // rows cr, cr+16, ..., cr+112
 #pragma unroll
-                for (int half16 = 0; half16 < 2; ++half16) {
-                    uint32_t r[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sv[16 * half16 + i] * a_last);
-                    tc::tmem_st16(tmem + lane_base + kColS + 32 * rg + 16 * half16, r);
-                }
-            }
-            tc::fence_proxy_async();
-            tc::fence_before_sync();
-            alu_sync();
-            if (tid == 0) {
-                tc::mbar_arrive(mb_m);                  // the producer issues the MMAs
-                tc::mbar_arrive(mb_free0 + 8 * (k & 1));   // the helper may reuse this chunk's buffers
-            }
-
-            // ---- while the MMAs run: the next chunk's conv
-            if (more) {
-                ok = wait_all(mb_x0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
-                if (!ok) break;
-                conv_chunk(k + 1);
-            }
-            if (!kStateOnly && tid == kArriveTid) *flag_slot = arrival;
-            // the chunk's MMAs done, and (helper) the next chunk's prefix sums
-            // and slot factors
-            dt_ready(k + 1, mbd, pard);
-            ok = more ? wait_all(mb_e, k & 1, mbd, pard) : wait_all(mb_e, k & 1);
-            if (!ok) break;
-            tc::fence_after_sync();
-            if constexpr (kStateOnly) {
-                if (more) weight_chunk(k + 1);
-                continue;
-            }
-
-            // ---- F: output rows, and the forward + reverse sum
-            int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
-            const bool first = *flag_slot == 0;
-            bool ready = true;
-            if (!first && tid == 0) {
-                // the partner CTA arrived first; wait (bounded) until its
-                // output is visible
-                ready = ld_acquire(fl + 1) != 0;
-                if (!ready) {
-                    const long long w0 = clock64();
-                    while (!(ready = ld_acquire(fl + 1) != 0)) {
-                        if (clock64() - w0 > kWaitCycles) break;
+                for (int jr = 0; jr < 8; ++jr) {
+                    const int r = cr + 16 * jr;
+                    if (r < cnt) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(sm + kOffXw + r * 256 +
+                                                                         ((cp ^ (r & 15)) << 4));
+                        const int tk = rev ? t0 + cnt - 1 - r : t0 + r;
+                        const size_t row0 = kConcat ? ((size_t)b * L + tk) * 2 * H * kP + dir * H * kP
+                                                    : ((size_t)b * L + tk) * H * kP;
+                        uint4 *dstp = reinterpret_cast<uint4 *>(p.y + row0 + hp * kPP) + cp;
+                        if (first) {
+                            *dstp = v;
+                        } else {
+                            asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};"
+                                         :: "l"(dstp), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                                         : "memory");
+                        }
                     }
                 }
-            }
-            // releases the group after thread 0's wait for the partner.  A
-            // wait that gave up stops the walk here: the partner's rows are
-            // not added to, and the meeting counters are left as they are
-            // (the caller zero-fills the workspace again after a timeout).
-            if (!alu_sync_and(ready)) {
-                ok = false;
-                break;
-            }
-            // the next chunk's wX first, while the partner's rows can be fetched
-            if (more) weight_chunk(k + 1);
-            // Coalesced output: each thread stages its 32 outputs in shared
-            // memory (the bf16 state copy's buffer, free until the next
-            // chunk's phase D), then 16 threads per token row move whole
-            // 256-byte rows.  Staging layout: [t][16 pieces of 16 B], piece
-            // q of row t stored at q ^ (t & 15) (conflict-free both ways).
-            const int cp = tid & 15;          // 16-byte piece of a row (8 channels)
-            const int cr = tid >> 4;          // rows cr, cr+32, cr+64, cr+96
-            auto ypiece = [&](int r) -> uint4 * {
-                const int tk = rev ? t0 + cnt - 1 - r : t0 + r;
-                const size_t row0 = kConcat ? ((size_t)b * L + tk) * 2 * H * kP + dir * H * kP
-                                            : ((size_t)b * L + tk) * H * kP;
-                return reinterpret_cast<uint4 *>(p.y + row0 + hp * kPP) + cp;
-            };
-            {
-                float yd[32], yo[32];
-                tc::tmem_ld32(tmem + lane_base + gcol(k) + 64 * hh + 32 * hsub, yd);
-                tc::tmem_ld32(tmem + lane_base + kColYo + 64 * hh + 32 * hsub, yo);
-                const float et = tc::exp2_approx(ct);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) yd[i] = fmaf(et, yo[i], yd[i]);
-#pragma unroll
-                for (int pc = 0; pc < 4; ++pc)
-                    *reinterpret_cast<uint4 *>(sm + kOffS + row * 256 +
-                                               (((4 * rg + pc) ^ (row & 15)) << 4)) = pack8(yd + 8 * pc);
-            }
-            tc::fence_before_sync();
-            alu_sync();
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = cr + 32 * j;
-                if (r < cnt) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(sm + kOffS + r * 256 +
-                                                                     ((cp ^ (r & 15)) << 4));
+                grp_sync(2);   // rows stored; the staging tile is rewritten by wX next
+                if (!kConcat && tb == 0) {
                     if (first) {
-                        *ypiece(r) = v;
+                        st_release(fl + 1, 1);   // publish the rows to the partner
                     } else {
-                        // second to reach the chunk: add to the partner's rows
-                        // at L2 (bf16 reductions, ordered after the partner's
-                        // release through thread 0's acquire and the barrier)
-                        asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};"
-                                     :: "l"(ypiece(r)), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                                     : "memory");
+                        fl[0] = 0;   // leave the workspace zeroed for the next call
+                        fl[1] = 0;
                     }
                 }
+            } else {
+                ok = b_wait(mb_e, k & 1);   // the state product has read wX
+                if (!ok) break;
             }
-            alu_sync();   // rows stored; the staging buffer is rewritten by the next chunk's phase D
-            if (tid == 0) {
-                if (!first) {
-                    fl[0] = 0;   // leave the workspace zeroed for the next call
-                    fl[1] = 0;
-                }
-                rel_flag[k & 1] = (first && !kConcat) ? fl + 1 : nullptr;
-                tc::mbar_arrive(mb_rows0 + 8 * (k & 1));   // the producer publishes them
+            if (k + 1 >= nk) break;
+            // ---- wX of chunk k+1 (its X tile was convolved an iteration ago)
+            ok = b_wait(mb_dt0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
+            if (!ok) break;
+            weight_chunk(k + 1);
+            tc::fence_proxy_async();   // X and wX, for the tensor core
+            grp_sync(2);
+            if (tb == 0) {
+                tc::mbar_arrive(mb_m);
+                tc::mbar_arrive(mb_free0 + 8 * ((k + 1) & 1));
+            }
+            // ---- conv of chunk k+2 (its raw rows were loaded once chunk k's MMAs completed)
+            if (k + 2 < nk) {
+                ok = b_wait(mb_x0 + 8 * ((k + 2) & 1), ((k + 2) >> 1) & 1);
+                if (!ok) break;
+                conv_chunk(k + 2);
             }
         }
-
-        if constexpr (kStateOnly) {
-            if (ok) {
-                // the item's end state and total decay
-                tc::fence_after_sync();
-                float sv[32];
-                tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
-                const size_t item = item_row + blockIdx.z;
-                float *so = p.seg_state + (item * kHeads + hh) * kP * kN;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) so[(size_t)(32 * hsub + i) * kN + row] = sv[i];
-                if (row == 0 && hsub == 0) p.seg_dec[item * kHeads + hh] = dec;
-            }
-        } else if (ok && !rev && p.fin && k0 + nk == p.nchunks) {
-            tc::fence_after_sync();
-            float sv[32];
-            tc::tmem_ld32(tmem + lane_base + kColS + 32 * rg, sv);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) p.fin[sidx + (size_t)(32 * hsub + i) * kN + row] = sv[i];
-        }
-        if (!ok && tid == 0) record_error(p.status, kStatusTimeout);
+        if (!ok && tb == 0) record_error(p.status, kStatusTimeout);
     }
     tc::fence_before_sync();
     __syncthreads();

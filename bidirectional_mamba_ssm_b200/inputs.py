@@ -123,3 +123,32 @@ def make_tail(batch: int, d_conv: int, channels: int, dtype: str, seed: int = 2,
     if bc_split is not None and bc_scale != 1.0:
         t[..., bc_split:] *= bc_scale
     return t.to(torch_dtype(dtype)).contiguous()
+
+
+def make_projections(d_model: int, heads: int, headdim: int, d_state: int, tokens: int,
+                     seed: int = 0, *, d_inner_out: int | None = None, device="cpu"):
+    """Seeded inputs and weights of the mixer's projections (bf16 storage;
+    draws in fp32 from one torch.Generator, in this order):
+
+      u       (tokens, d_model)          N(0, 1)
+      w_in    (ch + H, d_model)          N(0, 1/d_model)   (rows: xBC, then dt)
+      dt_bias (H)                        N(-2, 0.5)        (dt = softplus(u.w + b))
+      w_out   (d_model, d_inner_out)     N(0, 1/d_inner_out), d_inner_out = H*P
+                                         unless given (2*H*P for concatenated
+                                         untied streams)
+      y       (tokens, d_inner_out)      N(0, 1)           (a mixer output)
+    """
+    ch = heads * headdim + 2 * d_state
+    k_out = heads * headdim if d_inner_out is None else d_inner_out
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    u = torch.randn((tokens, d_model), generator=g, device=dev)
+    w_in = torch.randn((ch + heads, d_model), generator=g, device=dev) / math.sqrt(d_model)
+    dt_bias = torch.randn((heads,), generator=g, device=dev) * math.sqrt(0.5) - 2.0
+    w_out = torch.randn((d_model, k_out), generator=g, device=dev) / math.sqrt(k_out)
+    y = torch.randn((tokens, k_out), generator=g, device=dev)
+    bf = torch.bfloat16
+    return {"u": u.to(bf).contiguous(), "w_in": w_in.to(bf).contiguous(),
+            "dt_bias": dt_bias.float().contiguous(), "w_out": w_out.to(bf).contiguous(),
+            "y": y.to(bf).contiguous()}

@@ -320,6 +320,105 @@ int bimamba_block_decode(const bimamba_dims *d, const void *xbc_block,
                          size_t workspace_bytes, bimamba_stream_t stream);
 
 /*
+ * Cached block decode over a pool of cached streams, with a commit per row:
+ * the batch form a serving loop drives.  Block diffusion keeps one cache
+ * entry per stream -- the forward SSM state after its finished prefix and
+ * its last 4 raw tokens ("Fixed state, long reach: constant-size caches in
+ * large-scale block diffusion", abstract and section 1: an O(1) state per
+ * stream, many streams decoded together, a block committed once finished) --
+ * and each step decodes the active blocks of a batch of streams whose
+ * prefixes may all have different lengths.
+ *   d          : batch = rows decoded in this call, len = block length
+ *                (1..64); bf16, headdim 64, d_state 128 (else
+ *                BIMAMBA_ERR_UNSUPPORTED)
+ *   xbc_block, dt_block, A, D, conv_w, conv_b, y : as in bimamba_block_decode,
+ *                row s of the batch
+ *   state_pool : (pool_size, H, P, N) fp32 -- the cached forward states
+ *   tail_pool  : (pool_size, 4, ch) dtype -- the cached conv tails
+ *   slots      : (batch) int32, device -- the pool entry of each row; entries
+ *                of one call must be distinct.  A slot outside
+ *                [0, pool_size) skips its row and makes bimamba_get_error
+ *                report BIMAMBA_ERR_INVALID.
+ *   commit     : (batch) int32, device, or NULL -- rows with commit[s] != 0
+ *                (every row when NULL) write their state after the block and
+ *                their new conv tail back into their pool entry, in place
+ *   workspace  : bimamba_workspace_bytes(d) bytes
+ * Row s's output equals bimamba_block_decode on state_pool[slots[s]] and
+ * tail_pool[slots[s]].
+ */
+int bimamba_block_decode_pool(const bimamba_dims *d, const void *xbc_block,
+                              const void *dt_block, const float *A, const float *D,
+                              const float *conv_w, const float *conv_b,
+                              float *state_pool, void *tail_pool, int pool_size,
+                              const int *slots, const int *commit, void *y,
+                              void *workspace, size_t workspace_bytes,
+                              bimamba_stream_t stream);
+
+/*
+ * Backward pass of the bidirectional mixer core (training): the gradients of
+ * L = sum(dy * y), y = bimamba_ssd_fwd_rev(xbc, dt, A, D, conv_w, conv_b,
+ * init_state), with respect to every input.  "DiffuMamba: High-Throughput
+ * Diffusion LMs with Mamba Backbone" trains this mixer with the
+ * masked-diffusion objective (Portuguese technical summary, section 2
+ * "Metodologia"); the gradients are those of the recurrence and conv written
+ * at the top of this file, run back through both streams.
+ *   xbc, dt, A, D, conv_w (required), conv_b, init_state : the forward call's
+ *                inputs (init_state NULL = zero)
+ *   dy         : (batch, len, H*P) dtype
+ *   outputs, fp32, written (not accumulated):
+ *   dxbc (batch, len, ch), ddt (batch, len, H), dA (H), dD (H),
+ *   dconv_w (ch, 4), dconv_b (ch) or NULL, dinit (batch, H, P, N) or NULL
+ *   workspace  : bimamba_backward_workspace_bytes(d) bytes (no clearing
+ *                needed); it holds both streams' activations, their fp32
+ *                gradients and the state entering every 64-token chunk
+ * Shapes: headdim <= 64 and d_state <= 128, both multiples of 4 (else
+ * BIMAMBA_ERR_UNSUPPORTED); fp32 or bf16 activations.  The chunked backward
+ * runs its small matrix products on the CUDA cores in fp32.
+ */
+size_t bimamba_backward_workspace_bytes(const bimamba_dims *d);
+
+int bimamba_ssd_fwd_rev_backward(const bimamba_dims *d, const void *xbc, const void *dt,
+                                 const float *A, const float *D, const float *conv_w,
+                                 const float *conv_b, const float *init_state,
+                                 const void *dy, float *dxbc, float *ddt, float *dA,
+                                 float *dD, float *dconv_w, float *dconv_b, float *dinit,
+                                 void *workspace, size_t workspace_bytes,
+                                 bimamba_stream_t stream);
+
+/*
+ * The projections on either side of the mixer, on the tensor cores (bf16
+ * operands, fp32 accumulation, bf16 results).  "DiffuMamba" blog post,
+ * network-architecture listing: d_model = 2048 with expand = 2, so each
+ * mixer maps d_model to its inner width H*P and back, and the bidirectional
+ * block maps the concatenation of its two streams (2 d) back to d with a
+ * Linear.  Weights are row-major (out_features, in_features), as a Linear
+ * layer stores them.
+ *
+ * bimamba_in_proj: u (tokens, d_model) -> the mixer's inputs, written in the
+ * layouts bimamba_ssd_fwd_rev reads:
+ *   xbc (tokens, ch)  = u . W_in[0:ch]^T              ch = H*P + 2*N
+ *   dt  (tokens, H)   = softplus(u . W_in[ch:ch+H]^T + dt_bias)
+ *   w_in : (ch + H, d_model) bf16;  dt_bias : (H) fp32 or NULL (zero)
+ * Requires d_model % 8 == 0.
+ *
+ * bimamba_out_proj: out (tokens, d_model) = y . W_out^T
+ *   y     : (tokens, d_inner) bf16 -- the mixer's output; with untied
+ *           directions and concatenated streams d_inner = 2*H*P and W_out is
+ *           the block's fusion Linear (applied after each stream's own output
+ *           map, which composes into one (d_model, 2*H*P) matrix)
+ *   w_out : (d_model, d_inner) bf16
+ * Requires d_inner % 8 == 0.
+ * Both: pointers 16-byte aligned, outputs must not overlap inputs; a kernel
+ * wait that gives up is reported by bimamba_get_error as BIMAMBA_ERR_TIMEOUT.
+ */
+int bimamba_in_proj(int tokens, int d_model, int heads, int headdim, int d_state,
+                    const void *u, const void *w_in, const float *dt_bias, void *xbc,
+                    void *dt, bimamba_stream_t stream);
+
+int bimamba_out_proj(int tokens, int d_inner, int d_model, const void *y,
+                     const void *w_out, void *out, bimamba_stream_t stream);
+
+/*
  * Cached block decode without a caller workspace.  The paper has no
  * counterpart to this entry point; it exists for callers that cannot
  * allocate device memory: a serving process whose memory pool already holds
