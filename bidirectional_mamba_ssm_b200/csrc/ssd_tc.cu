@@ -334,12 +334,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     const uint32_t mb_bc = sbase + kOffMbar;         // the chunk's B/C tiles landed
     const uint32_t mb_x0 = sbase + kOffMbar + 8;     // raw x landed in buffer 0 / 1 (+8)
     const uint32_t mb_g = sbase + kOffMbar + 24;     // G done
-    const uint32_t mb_m = sbase + kOffMbar + 32;     // the chunk's MMA operands ready (one arrival per group)
+    const uint32_t mb_m = sbase + kOffMbar + 32;     // M ready (tensor-memory group)
     const uint32_t mb_e = sbase + kOffMbar + 40;     // the chunk's MMAs done
     const uint32_t mb_dt0 = sbase + kOffMbar + 48;   // an even / odd chunk's prefix sums and factors (+8)
     const uint32_t mb_free0 = sbase + kOffMbar + 64; // an even / odd chunk's factor buffers free (+8)
     const uint32_t mb_staged = sbase + kOffMbar + 80;   // the chunk's output rows staged
     const uint32_t mb_bcfree = sbase + kOffMbar + 88;   // the chunk's products that read B/C done
+    const uint32_t mb_s = sbase + kOffMbar + 96;     // state, its bf16 copy and wX ready (one arrival per group)
     auto xbuf_off = [](int k) { return (k & 1) ? kOffXbuf1 : kOffXbuf0; };
 
     auto chunk_of = [&](int k, int &t0, int &cnt, int &s0) {
@@ -474,7 +475,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         tc::mbar_init(mb_x0, 1);
         tc::mbar_init(mb_x0 + 8, 1);
         tc::mbar_init(mb_g, 1);
-        tc::mbar_init(mb_m, 2);          // one arrival from each compute group
+        tc::mbar_init(mb_m, 1);
+        tc::mbar_init(mb_s, 2);          // one arrival from each compute group
         tc::mbar_init(mb_e, 1);
         tc::mbar_init(mb_dt0, 32);       // every helper lane arrives after its part of a scan
         tc::mbar_init(mb_dt0 + 8, 32);
@@ -524,7 +526,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 }
             }
             for (int k = 0; k < nk && pok; ++k) {
-                pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
+                // the state scaled for this chunk, its bf16 copy and wX
+                pok = tc::mbar_wait_bounded(mb_s, k & 1, kWaitCycles);
                 if (pok && kStateOnly) pok = tc::mbar_wait_bounded(mb_bc, k & 1, kWaitCycles);
                 if (!pok) break;
                 tc::fence_after_sync();
@@ -544,6 +547,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                     // the B/C tiles are free once the state product and Yo are
                     // done: the next chunk's tiles load while Yd runs
                     tc::mma_commit(mb_bcfree);
+                    // M, built while the two products above run
+                    pok = tc::mbar_wait_bounded(mb_m, k & 1, kWaitCycles);
+                    if (!pok) break;
+                    tc::fence_after_sync();
                     // Yd = [M_0 | M_1] . [[X_0, 0], [0, X_1]]: one N = 128 product over
                     // K = 256.  K-steps 0..7 take X_0's rows as N block 0 and the
                     // zeros above the tiles as N block 1 (leading offset = the
@@ -659,7 +666,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         // M(k) in place over G(k) (region A): thread (t = row, h) owns the
         // walk slots of 32-slot blocks 2h, 2h+1 for both heads.  The 16 G
         // columns of slots 16ks..16ks+15 become [M_0 ks | M_1 ks] (8 + 8
-        // columns of packed bf16 pairs), so no other thread reads them.
+        // columns of packed bf16 pairs), so no other thread reads them.  One
+        // TMEM load per block; the stores are not waited for here (the caller
+        // waits once before publishing M).
         auto build_m = [&](int k) {
             const int par = k & 1;
 #pragma unroll
@@ -670,14 +679,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                     uint32_t z[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) z[i] = 0u;
-                    tc::tmem_st16(col, z);
-                    tc::tmem_st16(col + 16, z);
+                    tc::tmem_st16_nw(col, z);
+                    tc::tmem_st16_nw(col + 16, z);
                     continue;
                 }
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {       // 16-slot unit = K-step 2 jb + u
-                    float g[16];
-                    tc::tmem_ld16(col + 16 * u, g);
+                    uint32_t gu[16];
+                    tc::tmem_ld16_nw(col + 16 * u, gu);
+                    tc::tmem_wait_ld16(gu);
                     uint32_t out[16];               // [head][8 packed pairs]
 #pragma unroll
                     for (int hd = 0; hd < kHeads; ++hd) {
@@ -686,12 +696,16 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                         const int s0u = 32 * jb + 16 * u;   // first slot of the unit
                         if (jb < quad) {
                             // whole block below the diagonal: factorised decay
-                            const float *fbh = fB + (par * kHeads + hd) * kQ + s0u;
+                            const float2 *fbh = reinterpret_cast<const float2 *>(fB + (par * kHeads + hd) * kQ + s0u);
                             const float et = tc::exp2_approx(ct - cm[32 * jb + 31]);
+                            const float2 et2 = make_float2(et, et);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                out[8 * hd + i] = tc::pack_bf16x2(g[2 * i] * et * fbh[2 * i],
-                                                                  g[2 * i + 1] * et * fbh[2 * i + 1]);
+                            for (int i = 0; i < 8; ++i) {
+                                const float2 g2 = make_float2(__uint_as_float(gu[2 * i]),
+                                                              __uint_as_float(gu[2 * i + 1]));
+                                const float2 m = tc::mul2(tc::mul2(g2, et2), fbh[i]);
+                                out[8 * hd + i] = tc::pack_bf16x2(m.x, m.y);
+                            }
                         } else {
                             // diagonal block, D on the diagonal; slot s0u + i
                             // against t's offset r31 in the block
@@ -709,7 +723,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                                 for (int j = 0; j < 4; ++j) rf[j] = tc::exp2_approx(ct - cm[s0u + 4 * j + 3]);
 #pragma unroll
                                 for (int i = 0; i < 16; ++i) {
-                                    const float x = fmaf(g[i] * rf[i >> 2], f4h[i], (i == r) ? Dh : 0.0f);
+                                    const float x = fmaf(__uint_as_float(gu[i]) * rf[i >> 2], f4h[i],
+                                                         (i == r) ? Dh : 0.0f);
                                     v[i] = (i <= r) ? x : 0.0f;
                                 }
                             } else {
@@ -718,7 +733,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
 #pragma unroll
                                 for (int i = 0; i < 16; ++i) {
                                     const float e = tc::exp2_approx(fminf(ct - cm[s0u + i], 0.0f));
-                                    const float x = fmaf(g[i] * e, dh_[i], (i == r) ? Dh : 0.0f);
+                                    const float x = fmaf(__uint_as_float(gu[i]) * e, dh_[i],
+                                                         (i == r) ? Dh : 0.0f);
                                     v[i] = (i <= r) ? x : 0.0f;
                                 }
                             }
@@ -726,33 +742,45 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                             for (int i = 0; i < 8; ++i) out[8 * hd + i] = tc::pack_bf16x2(v[2 * i], v[2 * i + 1]);
                         }
                     }
-                    tc::tmem_st16(col + 16 * u, out);
+                    tc::tmem_st16_nw(col + 16 * u, out);
                 }
             }
         };
         // the state at chunk k's start: bf16 copy of S_in (the Yo operand),
-        // then S <- exp(c_last) S in place
+        // then S <- exp(c_last) S in place (stores not waited for here)
         auto scale_state = [&](int k) {
             const float cl = cum[((k & 1) * kHeads + h) * kQ + kQ - 1];
             const float a_last = tc::exp2_approx(cl);
+            const float2 a2 = make_float2(a_last, a_last);
             if constexpr (kStateOnly) dec += cl;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                float sv[32];
+                uint32_t sr[32];
                 const uint32_t col = tmem + lane_base + kColS + 64 * h + 32 * half;
-                tc::tmem_ld32(col, sv);
+                tc::tmem_ld32_nw(col, sr);
+                tc::tmem_wait_ld(sr);
                 if constexpr (!kStateOnly) {
 #pragma unroll
-                    for (int pc = 0; pc < 4; ++pc)
-                        *reinterpret_cast<uint4 *>(sm + kOffS + h * 16384 + tc::sw128(row, 4 * half + pc)) =
-                            pack8(sv + 8 * pc);
+                    for (int pc = 0; pc < 4; ++pc) {
+                        uint4 w;
+                        w.x = tc::pack_bf16x2(__uint_as_float(sr[8 * pc]), __uint_as_float(sr[8 * pc + 1]));
+                        w.y = tc::pack_bf16x2(__uint_as_float(sr[8 * pc + 2]), __uint_as_float(sr[8 * pc + 3]));
+                        w.z = tc::pack_bf16x2(__uint_as_float(sr[8 * pc + 4]), __uint_as_float(sr[8 * pc + 5]));
+                        w.w = tc::pack_bf16x2(__uint_as_float(sr[8 * pc + 6]), __uint_as_float(sr[8 * pc + 7]));
+                        *reinterpret_cast<uint4 *>(sm + kOffS + h * 16384 + tc::sw128(row, 4 * half + pc)) = w;
+                    }
                 }
 #pragma unroll
                 for (int half16 = 0; half16 < 2; ++half16) {
                     uint32_t r[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(sv[16 * half16 + i] * a_last);
-                    tc::tmem_st16(col + 16 * half16, r);
+                    for (int i = 0; i < 16; i += 2) {
+                        const float2 v = tc::mul2(make_float2(__uint_as_float(sr[16 * half16 + i]),
+                                                              __uint_as_float(sr[16 * half16 + i + 1])), a2);
+                        r[i] = __float_as_uint(v.x);
+                        r[i + 1] = __float_as_uint(v.y);
+                    }
+                    tc::tmem_st16_nw(col + 16 * half16, r);
                 }
             }
         };
@@ -761,32 +789,54 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         // t * 256 bytes, 16-byte piece q of it at q ^ (t & 15)
         auto stage_rows = [&](int k) {
             const float et = tc::exp2_approx(cum[((k & 1) * kHeads + h) * kQ + row]);
+            const float2 et2 = make_float2(et, et);
 #pragma unroll
             for (int qtr = 0; qtr < 4; ++qtr) {
-                float yd[16], yo[16];
-                tc::tmem_ld16(tmem + lane_base + kColYd + 64 * h + 16 * qtr, yd);
-                tc::tmem_ld16(tmem + lane_base + kColYo + 64 * h + 16 * qtr, yo);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) yd[i] = fmaf(et, yo[i], yd[i]);
+                uint32_t yy[32];   // [0, 16): Yd, [16, 32): Yo
+                tc::tmem_ld16_nw(tmem + lane_base + kColYd + 64 * h + 16 * qtr, yy);
+                tc::tmem_ld16_nw(tmem + lane_base + kColYo + 64 * h + 16 * qtr, yy + 16);
+                tc::tmem_wait_ld(yy);
 #pragma unroll
                 for (int pc = 0; pc < 2; ++pc) {
+                    float v[8];
+#pragma unroll
+                    for (int i = 0; i < 8; i += 2) {
+                        const int e = 8 * pc + i;
+                        const float2 y2 = tc::fma2(et2, make_float2(__uint_as_float(yy[16 + e]), __uint_as_float(yy[17 + e])),
+                                                   make_float2(__uint_as_float(yy[e]), __uint_as_float(yy[e + 1])));
+                        v[i] = y2.x;
+                        v[i + 1] = y2.y;
+                    }
                     const int piece = 8 * h + 2 * qtr + pc;
-                    *reinterpret_cast<uint4 *>(sm + kOffXw + row * 256 + ((piece ^ (row & 15)) << 4)) =
-                        pack8(yd + 8 * pc);
+                    *reinterpret_cast<uint4 *>(sm + kOffXw + row * 256 + ((piece ^ (row & 15)) << 4)) = pack8(v);
                 }
             }
         };
-
-        bool ok = a_wait(mb_dt0, 0);   // chunk 0's prefix sums and factors
-        if (ok && !kStateOnly) ok = a_wait(mb_g, 0);
-        if (ok) {
-            tc::fence_after_sync();
-            if constexpr (!kStateOnly) build_m(0);
-            scale_state(0);
-            tc::fence_proxy_async();
+        // publish this group's part of a chunk's MMA operands on mbarrier mb
+        auto publish = [&](uint32_t mb, bool smem_operands) {
+            tc::tmem_wait_st();
+            if (smem_operands) tc::fence_proxy_async();   // the bf16 state copy, for the tensor core
             tc::fence_before_sync();
             grp_sync(1);
-            if (tid == 0) tc::mbar_arrive(mb_m);
+            if (tid == 0) tc::mbar_arrive(mb);
+        };
+
+        // Per chunk k: the state at its start (the operands of the state
+        // product and Yo) first, then M(k) (the operand of Yd), so that the
+        // producer issues the first two products while M is being built.
+        bool ok = a_wait(mb_dt0, 0);   // chunk 0's prefix sums and factors
+        if (ok) {
+            tc::fence_after_sync();
+            scale_state(0);
+            publish(mb_s, !kStateOnly);
+            if constexpr (!kStateOnly) {
+                ok = a_wait(mb_g, 0);
+                if (ok) {
+                    tc::fence_after_sync();
+                    build_m(0);
+                    publish(mb_m, false);
+                }
+            }
         }
         for (int k = 0; k < nk && ok; ++k) {
             ok = a_wait(mb_e, k & 1);   // chunk k's MMAs done
@@ -801,15 +851,16 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * (k & 1));
             if (k + 1 >= nk) break;
             ok = a_wait(mb_dt0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
-            if (ok && !kStateOnly) ok = a_wait(mb_g, (k + 1) & 1);
             if (!ok) break;
-            tc::fence_after_sync();
-            if constexpr (!kStateOnly) build_m(k + 1);
             scale_state(k + 1);
-            tc::fence_proxy_async();   // the bf16 state copy, for the tensor core
-            tc::fence_before_sync();
-            grp_sync(1);
-            if (tid == 0) tc::mbar_arrive(mb_m);
+            publish(mb_s, !kStateOnly);
+            if constexpr (!kStateOnly) {
+                ok = a_wait(mb_g, (k + 1) & 1);
+                if (!ok) break;
+                tc::fence_after_sync();
+                build_m(k + 1);
+                publish(mb_m, false);
+            }
         }
         if (ok) {
             // the last chunk's MMAs are done (waited above)
@@ -847,70 +898,67 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         };
         // conv+SiLU of both heads' x for walk chunk k, in place: the raw
         // rows in x buffer k % 2 become the swizzled X tile of the chunk.
-        // Thread: channel quad cq (channels 4cq..4cq+3; head cq >> 4) x 16
-        // walk slots 16sg..16sg+15.  Raw row of walk offset j: forward j + 3
-        // (the box starts 3 tokens early), reverse cnt - 1 - j.  Every thread
-        // reads its raw rows before the group barrier and writes after it.
+        // Thread: channel pair cp (channels 2cp, 2cp+1; head cp >> 5) x 32
+        // walk slots 32sg..32sg+31, in packed fp32.  Raw row of walk offset j:
+        // forward j + 3 (the box starts 3 tokens early), reverse cnt - 1 - j.
+        // Every thread reads its raw rows before the group barrier and
+        // writes after it.
         auto conv_chunk = [&](int k) {
             int t0, cnt, s0;
             chunk_of(k, t0, cnt, s0);
             uint8_t *buf = sm + xbuf_off(k);
-            const int cq = tb & 31, sg = tb >> 5;
-            const int j0 = 16 * sg;
-            uint2 rr[19];
+            const int cp = tb & 63, sg = tb >> 6;
+            const int j0 = 32 * sg;
+            uint32_t rr[35];
 #pragma unroll
-            for (int i = 0; i < 19; ++i) {
+            for (int i = 0; i < 35; ++i) {
                 const int jw = j0 + i - 3;   // walk offset of the raw row
                 const int rrow = rev ? cnt - 1 - jw : jw + 3;
                 rr[i] = (rrow >= 0 && rrow < kRawRows)
-                            ? *reinterpret_cast<const uint2 *>(buf + rrow * (kPP * 2) + 8 * cq)
-                            : make_uint2(0, 0);
+                            ? *reinterpret_cast<const uint32_t *>(buf + rrow * (kPP * 2) + 4 * cp)
+                            : 0u;
             }
             grp_sync(2);
-            const int gh = cq >> 4, piece = (cq & 15) >> 1, sub = cq & 1;
-            uint8_t *dst = buf + gh * 16384 + 8 * sub;
-            float u0[4], u1[4], u2[4];
-            auto unpack4 = [](uint2 r, float (&v)[4]) {
-                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
-                const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
-                v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
+            const int gh = cp >> 5, piece = (cp & 31) >> 2;
+            uint8_t *dst = buf + gh * 16384 + 4 * (cp & 3);
+            const bool full = j0 + 32 <= cnt;
+            auto upair = [](uint32_t r) {
+                return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r));
             };
-            unpack4(rr[0], u0);
-            unpack4(rr[1], u1);
-            unpack4(rr[2], u2);
-            const bool full = j0 + 16 <= cnt;
             if (has_conv) {
-                float4 w[4];
-                float bq[4];
+                // acc = b + sum_j w_j u_j, SiLU(acc) = h + h tanh(h), h = acc / 2
+                const int c0 = 2 * cp, c1 = 2 * cp + 1;   // channels of the pair
+                const float4 wa = convw[(c0 & 3) * 32 + (c0 >> 2)], wb = convw[(c1 & 3) * 32 + (c1 >> 2)];
+                const float2 w0 = make_float2(wa.x, wb.x), w1 = make_float2(wa.y, wb.y);
+                const float2 w2 = make_float2(wa.z, wb.z), w3 = make_float2(wa.w, wb.w);
+                const float2 bp = make_float2(convb[(c0 & 3) * 32 + (c0 >> 2)], convb[(c1 & 3) * 32 + (c1 >> 2)]);
+                const float2 half2 = make_float2(0.5f, 0.5f);
+                float2 u0 = upair(rr[0]), u1 = upair(rr[1]), u2 = upair(rr[2]);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    w[q] = convw[q * 32 + cq];
-                    bq[q] = convb[q * 32 + cq];
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float u3[4], o[4];
-                    unpack4(rr[i + 3], u3);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float acc = bq[q];
-                        acc = fmaf(w[q].x, u0[q], acc);
-                        acc = fmaf(w[q].y, u1[q], acc);
-                        acc = fmaf(w[q].z, u2[q], acc);
-                        acc = fmaf(w[q].w, u3[q], acc);
-                        o[q] = tc::silu_tanh(acc);
-                        u0[q] = u1[q]; u1[q] = u2[q]; u2[q] = u3[q];
-                    }
-                    uint2 pk = make_uint2(tc::pack_bf16x2(o[0], o[1]), tc::pack_bf16x2(o[2], o[3]));
-                    if (!full && j0 + i >= cnt) pk = make_uint2(0, 0);
-                    *reinterpret_cast<uint2 *>(dst + tc::sw128(j0 + i, piece)) = pk;
+                for (int i = 0; i < 32; ++i) {
+                    const float2 u3 = upair(rr[i + 3]);
+                    float2 acc = tc::fma2(w0, u0, bp);
+                    acc = tc::fma2(w1, u1, acc);
+                    acc = tc::fma2(w2, u2, acc);
+                    acc = tc::fma2(w3, u3, acc);
+                    const float2 hh = tc::mul2(acc, half2);
+                    float tx, ty;
+                    asm("tanh.approx.f32 %0, %1;" : "=f"(tx) : "f"(hh.x));
+                    asm("tanh.approx.f32 %0, %1;" : "=f"(ty) : "f"(hh.y));
+                    const float2 o = tc::fma2(hh, make_float2(tx, ty), hh);
+                    uint32_t pk = tc::pack_bf16x2(o.x, o.y);
+                    if (!full && j0 + i >= cnt) pk = 0u;
+                    *reinterpret_cast<uint32_t *>(dst + tc::sw128(j0 + i, piece)) = pk;
+                    u0 = u1;
+                    u1 = u2;
+                    u2 = u3;
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    uint2 pk = rr[i + 3];
-                    if (!full && j0 + i >= cnt) pk = make_uint2(0, 0);
-                    *reinterpret_cast<uint2 *>(dst + tc::sw128(j0 + i, piece)) = pk;
+                for (int i = 0; i < 32; ++i) {
+                    uint32_t pk = rr[i + 3];
+                    if (!full && j0 + i >= cnt) pk = 0u;
+                    *reinterpret_cast<uint32_t *>(dst + tc::sw128(j0 + i, piece)) = pk;
                 }
             }
         };
@@ -965,7 +1013,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             tc::fence_proxy_async();
             grp_sync(2);
             if (tb == 0) {
-                tc::mbar_arrive(mb_m);
+                tc::mbar_arrive(mb_s);
                 tc::mbar_arrive(mb_free0);
             }
             if (nk > 1) {
@@ -1052,7 +1100,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             tc::fence_proxy_async();   // X and wX, for the tensor core
             grp_sync(2);
             if (tb == 0) {
-                tc::mbar_arrive(mb_m);
+                tc::mbar_arrive(mb_s);
                 tc::mbar_arrive(mb_free0 + 8 * ((k + 1) & 1));
             }
             // ---- conv of chunk k+2 (its raw rows were loaded once chunk k's MMAs completed)
