@@ -142,17 +142,6 @@ decode_prep_kernel(const __nv_bfloat16 *__restrict__ xbc, const __nv_bfloat16 *_
         const int c = cbase + 8 * g;
         const __nv_bfloat16 *xb = xbc + (size_t)s * len * ch + c;
         const __nv_bfloat16 *tb = tail + (size_t)slot * 4 * ch + c;
-        auto raw = [&](int j, float (&v)[8]) {   // raw value at walk offset j of this direction
-            const int tok = rev ? len - 1 - j : j;
-            if (tok >= 0 && tok < len) {
-                unpack8f(*reinterpret_cast<const uint4 *>(xb + (size_t)tok * ch), v);
-            } else if (!rev && tok < 0 && tok >= -4) {
-                unpack8f(*reinterpret_cast<const uint4 *>(tb + (size_t)(4 + tok) * ch), v);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] = 0.0f;
-            }
-        };
         float w0[8], w1[8], w2[8], w3[8], bb[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -160,17 +149,27 @@ decode_prep_kernel(const __nv_bfloat16 *__restrict__ xbc, const __nv_bfloat16 *_
             w0[q] = t4.x; w1[q] = t4.y; w2[q] = t4.z; w3[q] = t4.w;
             bb[q] = conv_b ? conv_b[c + q] : 0.0f;
         }
-        float r0[8], r1[8], r2[8];
-        raw(j0 - 3, r0);
-        raw(j0 - 2, r1);
-        raw(j0 - 1, r2);
+        // the 19 raw rows of this thread's 16 slots (3 before), loaded first
+        uint4 rw[19];
+#pragma unroll
+        for (int i = 0; i < 19; ++i) {
+            const int j = j0 + i - 3;
+            const int tok = rev ? len - 1 - j : j;
+            rw[i] = (tok >= 0 && tok < len) ? __ldg(reinterpret_cast<const uint4 *>(xb + (size_t)tok * ch))
+                    : (!rev && tok < 0 && tok >= -4) ? __ldg(reinterpret_cast<const uint4 *>(tb + (size_t)(4 + tok) * ch))
+                                                      : make_uint4(0, 0, 0, 0);
+        }
         const int cc = (8 * g) & 127;                    // channel within B or C
         uint8_t *tile = sm + ((8 * g < 128) ? kPOffB : kPOffC) + (cc >> 6) * 16384;
         const int piece = (cc & 63) >> 3;
+#pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int j = j0 + i;
-            float r3[8], o[8];
-            raw(j, r3);
+            float r0[8], r1[8], r2[8], r3[8], o[8];
+            unpack8f(rw[i], r0);
+            unpack8f(rw[i + 1], r1);
+            unpack8f(rw[i + 2], r2);
+            unpack8f(rw[i + 3], r3);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 float acc = bb[q];
@@ -179,7 +178,6 @@ decode_prep_kernel(const __nv_bfloat16 *__restrict__ xbc, const __nv_bfloat16 *_
                 acc = fmaf(w2[q], r2[q], acc);
                 acc = fmaf(w3[q], r3[q], acc);
                 o[q] = (j < len) ? tc::silu_tanh(acc) : 0.0f;
-                r0[q] = r1[q]; r1[q] = r2[q]; r2[q] = r3[q];
             }
             const int row = 16 * rg + i;
             *reinterpret_cast<uint4 *>(tile + tc::sw128(row, piece)) = pack8f(o);
@@ -351,52 +349,61 @@ decode_tc_kernel(const DecodeParams p)
     const float *dtdir = d ? dtr : dtf;
 
     // ---- conv+SiLU of the head's x into [X_f; X_r] (row r, channels
-    // 32 half .. 32 half + 31), and w o X_f for the commit
+    // 32 half .. 32 half + 31), and w o X_f for the commit.  The four taps'
+    // rows are loaded before any arithmetic (two halves of 16 channels).
     {
-        const int c0 = 32 * half;
-        float acc[32];
+        const int tok = d ? len - 1 - t : t;
+        const float w_commit =
+            (do_commit && d == 0 && t < len) ? tc::exp2_approx(cf[len - 1] - cf[t]) * dtf[t] : 0.0f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = convb[c0 + i];
-        if (t < len) {
-            const int tok = d ? len - 1 - t : t;
+        for (int hc = 0; hc < 2; ++hc) {
+            const int c0 = 32 * half + 16 * hc;
+            uint4 raw[4][2];
 #pragma unroll
             for (int tap = 0; tap < 4; ++tap) {
                 const int u = d ? tok + 3 - tap : tok - 3 + tap;
                 const __nv_bfloat16 *srcp = nullptr;
-                if (u >= 0 && u < len)
-                    srcp = p.xbc + ((size_t)s * len + u) * ch + h * kDP + c0;
-                else if (!d && u < 0)
-                    srcp = p.tail + ((size_t)slot * 4 + 4 + u) * ch + h * kDP + c0;
-                if (srcp) {
+                if (t < len) {
+                    if (u >= 0 && u < len)
+                        srcp = p.xbc + ((size_t)s * len + u) * ch + h * kDP + c0;
+                    else if (!d && u < 0)
+                        srcp = p.tail + ((size_t)slot * 4 + 4 + u) * ch + h * kDP + c0;
+                }
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        float v[8];
-                        unpack8f(__ldg(reinterpret_cast<const uint4 *>(srcp) + v4), v);
+                for (int v4 = 0; v4 < 2; ++v4)
+                    raw[tap][v4] = srcp ? __ldg(reinterpret_cast<const uint4 *>(srcp) + v4) : make_uint4(0, 0, 0, 0);
+            }
+            float acc[16];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 w4 = convw[c0 + 8 * v4 + q];
-                            const float wt = tap == 0 ? w4.x : tap == 1 ? w4.y : tap == 2 ? w4.z : w4.w;
-                            acc[8 * v4 + q] = fmaf(wt, v[q], acc[8 * v4 + q]);
-                        }
+            for (int i = 0; i < 16; ++i) acc[i] = convb[c0 + i];
+#pragma unroll
+            for (int tap = 0; tap < 4; ++tap) {
+#pragma unroll
+                for (int v4 = 0; v4 < 2; ++v4) {
+                    float v[8];
+                    unpack8f(raw[tap][v4], v);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 w4 = convw[c0 + 8 * v4 + q];
+                        const float wt = tap == 0 ? w4.x : tap == 1 ? w4.y : tap == 2 ? w4.z : w4.w;
+                        acc[8 * v4 + q] = fmaf(wt, v[q], acc[8 * v4 + q]);
                     }
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = tc::silu_tanh(acc[i]);
-        } else {
+            for (int i = 0; i < 16; ++i) acc[i] = t < len ? tc::silu_tanh(acc[i]) : 0.0f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-        }
+            for (int pc = 0; pc < 2; ++pc)
+                *reinterpret_cast<uint4 *>(sm + kDOffX + tc::sw128(r, 4 * half + 2 * hc + pc)) =
+                    pack8f(acc + 8 * pc);
+            if (do_commit && d == 0) {
 #pragma unroll
-        for (int pc = 0; pc < 4; ++pc)
-            *reinterpret_cast<uint4 *>(sm + kDOffX + tc::sw128(r, 4 * half + pc)) = pack8f(acc + 8 * pc);
-        if (do_commit && d == 0) {
-            const float w = t < len ? tc::exp2_approx(cf[len - 1] - cf[t]) * dtf[t] : 0.0f;
+                for (int i = 0; i < 16; ++i) acc[i] *= w_commit;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] *= w;
-#pragma unroll
-            for (int pc = 0; pc < 4; ++pc)
-                *reinterpret_cast<uint4 *>(sm + kDOffXw + tc::sw128(t, 4 * half + pc)) = pack8f(acc + 8 * pc);
+                for (int pc = 0; pc < 2; ++pc)
+                    *reinterpret_cast<uint4 *>(sm + kDOffXw + tc::sw128(t, 4 * half + 2 * hc + pc)) =
+                        pack8f(acc + 8 * pc);
+            }
         }
     }
     // ---- M: row r holds its direction's 64 K columns [64 d, 64 d + 64)
@@ -404,7 +411,14 @@ decode_tc_kernel(const DecodeParams p)
     // direction's; D on the diagonal
     {
         const float Dh = p.D[h];
-        const float *grow = reinterpret_cast<const float *>(rec) + ((size_t)d * kDQ + t) * kDQ + 32 * half;
+        const float4 *grow4 = reinterpret_cast<const float4 *>(
+            reinterpret_cast<const float *>(rec) + ((size_t)d * kDQ + t) * kDQ + 32 * half);
+        float g[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldg(grow4 + i);
+            g[4 * i] = v.x; g[4 * i + 1] = v.y; g[4 * i + 2] = v.z; g[4 * i + 3] = v.w;
+        }
         const float ct = cdir[t];
         uint32_t packed[16], zero[16];
 #pragma unroll
@@ -413,13 +427,10 @@ decode_tc_kernel(const DecodeParams p)
 #pragma unroll
             for (int e2 = 0; e2 < 2; ++e2) {
                 const int sl = 32 * half + 2 * i + e2;
-                float m = 0.0f;
-                if (sl <= t && t < len) {
-                    const float g = __ldg(grow + 2 * i + e2);
-                    m = (sl < t) ? g * tc::exp2_approx(fminf(ct - cdir[sl], 0.0f)) * dtdir[sl]
-                                 : fmaf(g, dtdir[t], Dh);
-                }
-                m2[e2] = m;
+                const float gv = g[2 * i + e2];
+                const float m = (sl < t) ? gv * tc::exp2_approx(fminf(ct - cdir[sl], 0.0f)) * dtdir[sl]
+                                         : fmaf(gv, dtdir[t], Dh);
+                m2[e2] = (sl <= t && t < len) ? m : 0.0f;
             }
             packed[i] = tc::pack_bf16x2(m2[0], m2[1]);
             zero[i] = 0u;

@@ -979,12 +979,32 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             }
         };
 
+        // sequence shards: the reverse stream's conv reads the 3 tokens
+        // after the shard (L .. L+2) from the head.  Raw row i of a reverse
+        // chunk buffer is token t0 + i, so they land in the walk's first
+        // chunk and, when that chunk holds fewer than 3 tokens, also in the
+        // second (whose TMA box ran past the shard end and read zeros).
+        auto head_rows = [&](int k) {
+            if (!rev || !p.head) return;
+            int t0, cnt, s0;
+            chunk_of(k, t0, cnt, s0);
+            if (L - t0 >= kRawRows) return;
+            const uint32_t buf = xbuf_off(k);
+            for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
+                const int r = e / (kPP / 8), g = e % (kPP / 8);
+                const int row = L - t0 + r;
+                if (row < kRawRows)
+                    *reinterpret_cast<uint4 *>(sm + buf + row * (kPP * 2) + g * 16) =
+                        *reinterpret_cast<const uint4 *>(p.head + ((size_t)b * 4 + r) * ch +
+                                                         hp * kPP + 8 * g);
+            }
+            grp_sync(2);
+        };
+
         bool ok = b_wait(mb_x0, 0);
         if (ok) {
             // decode and sequence shards: the conv history before token 0
-            // comes from the tail; for sequence shards the reverse stream's
-            // conv reads the tokens after the shard from the head (raw rows
-            // cnt .. cnt+2 of the walk's first chunk, past the shard end)
+            // comes from the tail
             if (!rev && p.tail && k0 == 0) {
                 for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
                     const int r = e / (kPP / 8), g = e % (kPP / 8);
@@ -994,17 +1014,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 }
                 grp_sync(2);
             }
-            if (rev && p.head && k0 == 0) {
-                int t0, cnt, s0;
-                chunk_of(0, t0, cnt, s0);
-                for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
-                    const int r = e / (kPP / 8), g = e % (kPP / 8);
-                    *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + (cnt + r) * (kPP * 2) + g * 16) =
-                        *reinterpret_cast<const uint4 *>(p.head + ((size_t)b * 4 + r) * ch +
-                                                         hp * kPP + 8 * g);
-                }
-                grp_sync(2);
-            }
+            head_rows(0);
             conv_chunk(0);
             ok = b_wait(mb_dt0, 0);   // (also the barrier between conv writes and wX reads)
         }
@@ -1018,7 +1028,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             }
             if (nk > 1) {
                 ok = b_wait(mb_x0 + 8, 0);
-                if (ok) conv_chunk(1);
+                if (ok) {
+                    head_rows(1);
+                    conv_chunk(1);
+                }
             }
         }
         int arrival = 0;
