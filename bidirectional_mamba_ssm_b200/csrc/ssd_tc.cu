@@ -74,7 +74,8 @@ constexpr int kTmemWarps = 8;             // warps 0..7: the tensor-memory group
 constexpr int kProducerWarp = 16;         // issues every MMA and TMA load
 constexpr int kProducerTid = 32 * kProducerWarp;
 constexpr int kHelperWarp = 17;           // dt copies, prefix sums, slot factors
-constexpr int kThreads = 2 * kGroupThreads + 64;
+constexpr int kPublisherWarp = 18;        // sets the meeting flags of stored rows
+constexpr int kThreads = 2 * kGroupThreads + 96;
 constexpr int kBC = 2 * kN;   // B and C channels
 constexpr int kRawRows = kQ + 3;   // raw x rows per chunk: 128 slots + 3-token conv halo
 constexpr uint32_t kTmemCols = 512;
@@ -83,10 +84,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOffZlo = 0;        // 2 KB of zeros (block-diagonal B operand, below the X tiles)
 constexpr uint32_t kOffC = 2048;       // C      [t][n]   2 x 16 KB (TMA, swizzled)
 constexpr uint32_t kOffB = kOffC + 32768;   // B      [s][n]   2 x 16 KB (TMA, swizzled)
-constexpr uint32_t kXbufBytes = 33792; // raw x [131][128] (TMA) -> X [s][p], 16 KB per head
+constexpr uint32_t kXbufBytes = 33792; // raw x [131][128] (TMA) -> X [s][p], 16 KB per head -> output rows
 constexpr uint32_t kOffXbuf0 = kOffB + 32768;            // x buffer of even walk chunks
 constexpr uint32_t kOffXbuf1 = kOffXbuf0 + kXbufBytes;   // odd walk chunks
-constexpr uint32_t kOffXw = kOffXbuf1 + kXbufBytes;      // wX [s][p'] 2 x 16 KB; output staging
+constexpr uint32_t kOffXw = kOffXbuf1 + kXbufBytes;      // wX [s][p'] 2 x 16 KB
 constexpr uint32_t kOffS = kOffXw + 32768;               // S^T bf16 [n][p'] 2 x 16 KB
 constexpr uint32_t kOffZhi = kOffS + 32768;              // 2 KB of zeros (above the X tiles)
 constexpr uint32_t kRawBytes = kRawRows * kPP * 2;       // 33536
@@ -292,20 +293,25 @@ bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc_f, const __nv_bfloat16 *
 //
 // Warp roles (all communication through mbarriers; every wait is bounded):
 //   warps 0..7   tensor-memory group: per chunk k, once its MMAs are done,
-//                the output rows (Yd + exp(c) Yo, from TMEM) into a staging
-//                tile; then M(k+1) in place over G(k+1) and the state's
-//                chunk-start scaling with its bf16 copy (the Yo operand).
-//   warps 8..15  shared-memory group: per chunk k, the staged rows to global
-//                memory (the forward/reverse meeting), wX(k+1), and the
-//                in-place conv of chunk k+2's raw rows.
-//   warp 16      producer: every TMA load and every MMA.
+//                the output rows (Yd + exp(c) Yo, from TMEM) into the
+//                chunk's x buffer (X is no longer needed); then M(k+1) in
+//                place over G(k+1) and the state's chunk-start scaling with
+//                its bf16 copy (the Yo operand).
+//   warps 8..15  shared-memory group: per chunk k, wX(k+1) once the state
+//                product of chunk k has read wX(k), and the in-place conv of
+//                chunk k+2's raw rows.
+//   warp 16      producer: every MMA, and the B/C tile loads.
 //   warp 17      helper: dt copies, prefix sums and per-slot decay factors.
+//   warp 18      publisher: per chunk k, the staged rows to y (the
+//                forward/reverse meeting), then the raw rows of chunk k+2
+//                into the freed x buffer.
 // The two compute groups work on different chunks at the same time, and
 // both overlap the tensor core.
 template <bool kStateOnly, bool kConcat>
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant__ CUtensorMap tm_x_r,
-              const __grid_constant__ CUtensorMap tm_bc, const TcParams p)
+              const __grid_constant__ CUtensorMap tm_bc, const __grid_constant__ CUtensorMap tm_y,
+              const TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -329,7 +335,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     float *f4 = reinterpret_cast<float *>(sm + kOffF4);
     float4 *convw = reinterpret_cast<float4 *>(sm + kOffConvW);
     float *convb = reinterpret_cast<float *>(sm + kOffConvB);
-    int *first_slot = reinterpret_cast<int *>(sm + kOffTmem + 4);
     // mbarriers (each completes once per walk chunk unless noted):
     const uint32_t mb_bc = sbase + kOffMbar;         // the chunk's B/C tiles landed
     const uint32_t mb_x0 = sbase + kOffMbar + 8;     // raw x landed in buffer 0 / 1 (+8)
@@ -471,6 +476,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     if (tid == kProducerTid) {
         tc::prefetch_tmap(rev ? &tm_x_r : &tm_x_f);
         tc::prefetch_tmap(&tm_bc);
+        if (!kStateOnly) tc::prefetch_tmap(&tm_y);
         tc::mbar_init(mb_bc, 1);
         tc::mbar_init(mb_x0, 1);
         tc::mbar_init(mb_x0 + 8, 1);
@@ -579,8 +585,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 // region A are free
                 pok = tc::mbar_wait_bounded(mb_e, k & 1, kWaitCycles);
                 if (!pok) break;
-                if constexpr (kStateOnly) issue_bc(k + 1);
-                if (k + 2 < nk) issue_x(k + 2);
+                if constexpr (kStateOnly) {
+                    issue_bc(k + 1);
+                    if (k + 2 < nk) issue_x(k + 2);   // (the publisher issues them in the full kernel)
+                }
                 if constexpr (!kStateOnly) {
                     pok = tc::mbar_wait_bounded(mb_bc, (k + 1) & 1, kWaitCycles);
                     if (!pok) break;
@@ -589,6 +597,66 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 }
             }
             if (!pok) record_error(p.status, kStatusTimeout);
+        }
+        __syncwarp();
+    } else if (warp == kPublisherWarp) {
+        // ================= publisher: chunk k's output rows, staged by the
+        // tensor-memory group in x buffer k % 2 (free once the chunk's MMAs
+        // are done), to y, and the forward + reverse sum.  The two CTAs of a
+        // (sequence, head pair) meet per token chunk: the first to arrive
+        // stores its rows, the second adds its own to them (bf16 reductions
+        // at L2) once the first has set the chunk's ready flag.  Then x
+        // buffer k % 2 takes chunk k+2's raw rows (TMA, issued here).
+        if constexpr (!kStateOnly) {
+            bool qok = true;
+            const int col0 = (kConcat ? dir * H * kP : 0) + hp * kPP;   // the head pair's first y column
+            for (int k = 0; k < nk && qok && lane == 0; ++k) {
+                int t0, cnt, s0;
+                const int c = chunk_of(k, t0, cnt, s0);
+                int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
+                const int arrival = kConcat ? 0 : atomicAdd(fl, 1);
+                qok = tc::mbar_wait_bounded(mb_staged, k & 1, kWaitCycles);
+                if (!qok) break;
+                const bool first = arrival == 0;
+                const uint32_t stg = sbase + xbuf_off(k);
+                if (first) {
+                    tc::tma_store_3d(&tm_y, stg, col0, t0, b);
+                    tc::tma_store_3d(&tm_y, stg + 16384, col0 + kP, t0, b);
+                } else {
+                    // the partner CTA arrived first; wait (bounded) until its
+                    // rows are visible, then add this CTA's to them at L2.  A
+                    // wait that gave up stops the walk here: the partner's rows
+                    // are not added to, and the meeting counters are left as
+                    // they are (the caller zero-fills the workspace again
+                    // after a timeout).
+                    bool ready;
+                    const long long w0 = clock64();
+                    while (!(ready = ld_acquire(fl + 1) != 0)) {
+                        if (clock64() - w0 > kWaitCycles) break;
+                    }
+                    qok = ready;
+                    if (!qok) break;
+                    tc::fence_proxy_async_global();   // the acquire before the reductions
+                    tc::tma_reduce_add_3d(&tm_y, stg, col0, t0, b);
+                    tc::tma_reduce_add_3d(&tm_y, stg + 16384, col0 + kP, t0, b);
+                }
+                tc::bulk_commit();
+                tc::bulk_wait_read0();   // the staged rows have been read
+                if (k + 2 < nk) issue_x(k + 2);
+                if (!kConcat) {
+                    if (first) {
+                        // publish the rows to the partner once written
+                        tc::bulk_wait0();
+                        tc::fence_proxy_async_global();
+                        st_release(fl + 1, 1);
+                    } else {
+                        fl[0] = 0;   // leave the workspace zeroed for the next call
+                        fl[1] = 0;
+                    }
+                }
+            }
+            if (lane == 0) tc::bulk_wait0();
+            if (lane == 0 && !qok) record_error(p.status, kStatusTimeout);
         }
         __syncwarp();
     } else if (warp == kHelperWarp) {
@@ -670,6 +738,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         // TMEM load per block; the stores are not waited for here (the caller
         // waits once before publishing M).
         auto build_m = [&](int k) {
+            const int row = tc::no_hoist(tid & 127);   // (see no_hoist)
             const int par = k & 1;
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
@@ -688,12 +757,12 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                     uint32_t gu[16];
                     tc::tmem_ld16_nw(col + 16 * u, gu);
                     tc::tmem_wait_ld16(gu);
-                    uint32_t out[16];               // [head][8 packed pairs]
+                    const int s0u = 32 * jb + 16 * u;   // first slot of the unit
 #pragma unroll
                     for (int hd = 0; hd < kHeads; ++hd) {
                         const float *cm = cum + (par * kHeads + hd) * kQ;
                         const float ct = cm[row];
-                        const int s0u = 32 * jb + 16 * u;   // first slot of the unit
+                        uint32_t out[8];            // head hd's 8 packed pairs
                         if (jb < quad) {
                             // whole block below the diagonal: factorised decay
                             const float2 *fbh = reinterpret_cast<const float2 *>(fB + (par * kHeads + hd) * kQ + s0u);
@@ -704,51 +773,60 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                                 const float2 g2 = make_float2(__uint_as_float(gu[2 * i]),
                                                               __uint_as_float(gu[2 * i + 1]));
                                 const float2 m = tc::mul2(tc::mul2(g2, et2), fbh[i]);
-                                out[8 * hd + i] = tc::pack_bf16x2(m.x, m.y);
+                                out[i] = tc::pack_bf16x2(m.x, m.y);
                             }
                         } else {
                             // diagonal block, D on the diagonal; slot s0u + i
-                            // against t's offset r31 in the block
+                            // against t's offset r in the unit
                             const int r = (row & 31) - 16 * u;
                             const float Dh = hd ? D1 : D0;
-                            float v[16];
                             if (cm[32 * jb] - cm[32 * jb + 31] <= 60.0f) {   // warp-uniform (head, block)
                                 // 4-slot sub-blocks: exp(c_t - c_s) = exp(c_t - c_R4)
                                 // exp(c_R4 - c_s), R4 = s | 3.  With the block's whole
                                 // decay at most 2^60 neither factor overflows; for s <= t
                                 // the product is the decay itself
                                 const float *f4h = f4 + (par * kHeads + hd) * kQ + s0u;
-                                float rf[4];
 #pragma unroll
-                                for (int j = 0; j < 4; ++j) rf[j] = tc::exp2_approx(ct - cm[s0u + 4 * j + 3]);
+                                for (int q4 = 0; q4 < 4; ++q4) {
+                                    const float rf = tc::exp2_approx(ct - cm[s0u + 4 * q4 + 3]);
+                                    float v[4];
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) {
-                                    const float x = fmaf(__uint_as_float(gu[i]) * rf[i >> 2], f4h[i],
-                                                         (i == r) ? Dh : 0.0f);
-                                    v[i] = (i <= r) ? x : 0.0f;
+                                    for (int e = 0; e < 4; ++e) {
+                                        const int i = 4 * q4 + e;
+                                        const float x = fmaf(__uint_as_float(gu[i]) * rf, f4h[i],
+                                                             (i == r) ? Dh : 0.0f);
+                                        v[e] = (i <= r) ? x : 0.0f;
+                                    }
+                                    out[2 * q4] = tc::pack_bf16x2(v[0], v[1]);
+                                    out[2 * q4 + 1] = tc::pack_bf16x2(v[2], v[3]);
                                 }
                             } else {
                                 // steep decays: one exponential per element, each <= 1
                                 const float *dh_ = dts + (par * kHeads + hd) * kQ + s0u;
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) {
-                                    const float e = tc::exp2_approx(fminf(ct - cm[s0u + i], 0.0f));
-                                    const float x = fmaf(__uint_as_float(gu[i]) * e, dh_[i],
-                                                         (i == r) ? Dh : 0.0f);
-                                    v[i] = (i <= r) ? x : 0.0f;
+                                for (int i2 = 0; i2 < 8; ++i2) {
+                                    float v[2];
+#pragma unroll
+                                    for (int e = 0; e < 2; ++e) {
+                                        const int i = 2 * i2 + e;
+                                        const float ex = tc::exp2_approx(fminf(ct - cm[s0u + i], 0.0f));
+                                        const float x = fmaf(__uint_as_float(gu[i]) * ex, dh_[i],
+                                                             (i == r) ? Dh : 0.0f);
+                                        v[e] = (i <= r) ? x : 0.0f;
+                                    }
+                                    out[i2] = tc::pack_bf16x2(v[0], v[1]);
                                 }
                             }
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) out[8 * hd + i] = tc::pack_bf16x2(v[2 * i], v[2 * i + 1]);
                         }
+                        tc::tmem_st8_nw(col + 16 * u + 8 * hd, out);
                     }
-                    tc::tmem_st16_nw(col + 16 * u, out);
                 }
             }
         };
         // the state at chunk k's start: bf16 copy of S_in (the Yo operand),
         // then S <- exp(c_last) S in place (stores not waited for here)
         auto scale_state = [&](int k) {
+            const int row = tc::no_hoist(tid & 127);   // (see no_hoist)
             const float cl = cum[((k & 1) * kHeads + h) * kQ + kQ - 1];
             const float a_last = tc::exp2_approx(cl);
             const float2 a2 = make_float2(a_last, a_last);
@@ -784,10 +862,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 }
             }
         };
-        // chunk k's output rows, y = Yd + exp(c_t) Yo, into the staging tile
-        // (the wX buffer, free once the chunk's MMAs are done): row t at
-        // t * 256 bytes, 16-byte piece q of it at q ^ (t & 15)
+        // chunk k's output rows, y = Yd + exp(c_t) Yo, into the chunk's x
+        // buffer (free once its MMAs are done) as two TMA store boxes, one
+        // per head: [token row of the chunk][64 channels], 128-byte rows,
+        // 16-byte piece j of row q at j ^ (q & 7).  The reverse stream's
+        // walk slot r is token row cnt - 1 - r; slots past the chunk end are
+        // not written (the box rows past the sequence end are not stored).
         auto stage_rows = [&](int k) {
+            const int row = tc::no_hoist(tid & 127);   // (see no_hoist)
+            int t0, cnt, s0;
+            chunk_of(k, t0, cnt, s0);
+            const int q = rev ? cnt - 1 - row : row;   // token row in the box
+            uint8_t *box = sm + xbuf_off(k) + h * 16384 + q * 128;
             const float et = tc::exp2_approx(cum[((k & 1) * kHeads + h) * kQ + row]);
             const float2 et2 = make_float2(et, et);
 #pragma unroll
@@ -807,8 +893,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                         v[i] = y2.x;
                         v[i + 1] = y2.y;
                     }
-                    const int piece = 8 * h + 2 * qtr + pc;
-                    *reinterpret_cast<uint4 *>(sm + kOffXw + row * 256 + ((piece ^ (row & 15)) << 4)) = pack8(v);
+                    const int piece = 2 * qtr + pc;
+                    if (q >= 0) *reinterpret_cast<uint4 *>(box + ((piece ^ (q & 7)) << 4)) = pack8(v);
                 }
             }
         };
@@ -844,6 +930,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             tc::fence_after_sync();
             if constexpr (!kStateOnly) {
                 stage_rows(k);
+                tc::fence_proxy_async();   // the staged rows, for the publisher's bulk copies
                 tc::fence_before_sync();   // TMEM reads done before the next chunk's MMAs
                 grp_sync(1);
                 if (tid == 0) tc::mbar_arrive(mb_staged);
@@ -1034,78 +1121,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 }
             }
         }
-        int arrival = 0;
-        for (int k = 0; k < nk && ok; ++k) {
-            int t0, cnt, s0;
-            const int c = chunk_of(k, t0, cnt, s0);
-            if constexpr (!kStateOnly) {
-                // ---- chunk k's rows, and the forward + reverse sum.  The two
-                // CTAs of a (sequence, head pair) meet per token chunk: the
-                // first to arrive stores its rows, the second adds its own to
-                // them (bf16 reductions at L2) once the first has published.
-                int *fl = p.flags + (((size_t)b * HP + hp) * p.nchunks + c) * 2;
-                if (!kConcat && tb == 0) arrival = atomicAdd(fl, 1);
-                ok = b_wait(mb_staged, k & 1);
-                if (!ok) break;
-                bool ready = true;
-                if (tb == 0) {
-                    const bool first = kConcat || arrival == 0;
-                    *first_slot = first;
-                    if (!first) {
-                        // the partner CTA arrived first; wait (bounded) until
-                        // its rows are visible
-                        ready = ld_acquire(fl + 1) != 0;
-                        if (!ready) {
-                            const long long w0 = clock64();
-                            while (!(ready = ld_acquire(fl + 1) != 0)) {
-                                if (clock64() - w0 > kWaitCycles) break;
-                            }
-                        }
-                    }
-                }
-                // a wait that gave up stops the walk here: the partner's rows
-                // are not added to, and the meeting counters are left as they
-                // are (the caller zero-fills the workspace again after a timeout)
-                if (!grp_sync_and(2, ready)) {
-                    ok = false;
-                    break;
-                }
-                const bool first = *first_slot != 0;
-                const int cp = tb & 15;          // 16-byte piece of a row (8 channels)
-                const int cr = tb >> 4;          // rows cr, cr+16, ..., cr+112
-#pragma unroll
-                for (int jr = 0; jr < 8; ++jr) {
-                    const int r = cr + 16 * jr;
-                    if (r < cnt) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(sm + kOffXw + r * 256 +
-                                                                         ((cp ^ (r & 15)) << 4));
-                        const int tk = rev ? t0 + cnt - 1 - r : t0 + r;
-                        const size_t row0 = kConcat ? ((size_t)b * L + tk) * 2 * H * kP + dir * H * kP
-                                                    : ((size_t)b * L + tk) * H * kP;
-                        uint4 *dstp = reinterpret_cast<uint4 *>(p.y + row0 + hp * kPP) + cp;
-                        if (first) {
-                            *dstp = v;
-                        } else {
-                            asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};"
-                                         :: "l"(dstp), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                                         : "memory");
-                        }
-                    }
-                }
-                grp_sync(2);   // rows stored; the staging tile is rewritten by wX next
-                if (!kConcat && tb == 0) {
-                    if (first) {
-                        st_release(fl + 1, 1);   // publish the rows to the partner
-                    } else {
-                        fl[0] = 0;   // leave the workspace zeroed for the next call
-                        fl[1] = 0;
-                    }
-                }
-            } else {
-                ok = b_wait(mb_e, k & 1);   // the state product has read wX
-                if (!ok) break;
-            }
-            if (k + 1 >= nk) break;
+        for (int k = 0; k + 1 < nk && ok; ++k) {
+            // the state product of chunk k has read wX (its commit also
+            // covers Yo in the full kernel)
+            ok = b_wait(kStateOnly ? mb_e : mb_bcfree, k & 1);
+            if (!ok) break;
             // ---- wX of chunk k+1 (its X tile was convolved an iteration ago)
             ok = b_wait(mb_dt0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
             if (!ok) break;
@@ -1289,12 +1309,18 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
     if (e != cudaSuccess) return e;
     count_launch();
 
-    CUtensorMap tm_x_f, tm_x_r, tm_bc;
+    CUtensorMap tm_x_f, tm_x_r, tm_bc, tm_y;
+    // y: (batch, len, H*P) summed, or (batch, len, 2*H*P) concatenated, stored by
+    // 64-channel x 128-token boxes (the states-only launch stores nothing: its
+    // map is a placeholder over the activations)
+    const uint64_t ycols = (uint64_t)(pr.concat ? 2 : 1) * d.heads * kP;
     if (!make_map(&tm_x_f, xbc[0], (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, kPP, kRawRows,
                   false) ||
         !make_map(&tm_x_r, xbc[1], (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, kPP, kRawRows,
                   false) ||
-        !make_map(&tm_bc, act, (uint64_t)kBC, (uint64_t)d.len, (uint64_t)2 * d.batch, 64, kQ, true))
+        !make_map(&tm_bc, act, (uint64_t)kBC, (uint64_t)d.len, (uint64_t)2 * d.batch, 64, kQ, true) ||
+        !(p.y ? make_map(&tm_y, p.y, ycols, (uint64_t)d.len, (uint64_t)d.batch, kP, kQ, true)
+              : make_map(&tm_y, act, (uint64_t)kBC, (uint64_t)d.len, (uint64_t)2 * d.batch, 64, kQ, true)))
         return cudaErrorInvalidValue;
     auto main_kernel = pr.concat ? ssd_tc_kernel<false, true> : ssd_tc_kernel<false, false>;
     e = cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
@@ -1313,7 +1339,7 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
         q.nitems = 1;
         q.item_chunks = q.seg_chunks = p.nchunks;
         ssd_tc_kernel<true, false><<<dim3(d.heads, d.batch, 1), kThreads, kSmemBytes, stream>>>(
-            tm_x_f, tm_x_r, tm_bc, q);
+            tm_x_f, tm_x_r, tm_bc, tm_y, q);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         count_launch();
@@ -1324,13 +1350,13 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
         TcParams q = p;
         q.seg_chunks = sp.item_chunks;   // one CTA per item
         ssd_tc_kernel<true, false><<<dim3(d.heads, d.batch, sp.nitems), kThreads, kSmemBytes, stream>>>(
-            tm_x_f, tm_x_r, tm_bc, q);
+            tm_x_f, tm_x_r, tm_bc, tm_y, q);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         count_launch();
     }
     main_kernel<<<dim3(d.heads, d.batch, sp.nseg), kThreads, kSmemBytes, stream>>>(tm_x_f, tm_x_r, tm_bc,
-                                                                                 p);
+                                                                                 tm_y, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();

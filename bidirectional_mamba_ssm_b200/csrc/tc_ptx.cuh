@@ -223,9 +223,54 @@ __device__ __forceinline__ void tmem_st16_nw(uint32_t taddr, const uint32_t (&r)
         : "memory");
 }
 
+// Store 8 consecutive 32-bit columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_st8_nw(uint32_t taddr, const uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+        :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+           "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st()
 {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// The value itself, through an opaque move: address arithmetic derived from
+// it stays where it is written instead of being hoisted out of the loop
+// around it, which in a kernel near its register limit turns hoisted
+// loop-invariant addresses into spills.
+__device__ __forceinline__ int no_hoist(int v)
+{
+    asm volatile("mov.b32 %0, %0;" : "+r"(v));
+    return v;
+}
+
+// Bulk async-group completion (TMA stores and reductions issued by this thread).
+__device__ __forceinline__ void bulk_commit()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// This thread's bulk copies have finished reading their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read0()
+{
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// This thread's bulk copies are complete (written).
+__device__ __forceinline__ void bulk_wait0()
+{
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Orders this thread's generic-proxy global accesses against its
+// async-proxy (bulk copy) ones.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Packed fp32 pairs (sm_100): two multiplies / fused multiply-adds per
@@ -329,6 +374,24 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int 
         "[%0], [%1, {%2, %3, %4}], [%5];"
         :: "r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
         : "memory");
+}
+
+// Tiled 3-D TMA store of one box from shared memory (c0 innermost),
+// completed through this thread's bulk async-groups.
+__device__ __forceinline__ void tma_store_3d(const void *tmap, uint32_t src, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 :: "l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
+// The same, adding the box's elements to the tensor's at L2 (element type
+// from the tensor map).
+__device__ __forceinline__ void tma_reduce_add_3d(const void *tmap, uint32_t src, int c0, int c1, int c2)
+{
+    asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 :: "l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
 }
 
 // Tiled 2-D TMA load of one box into shared memory (c0 innermost).
