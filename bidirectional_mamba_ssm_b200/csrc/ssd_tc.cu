@@ -740,7 +740,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         auto build_m = [&](int k) {
             const int row = tc::no_hoist(tid & 127);   // (see no_hoist)
             const int par = k & 1;
-#pragma unroll
+#pragma unroll 1
             for (int jj = 0; jj < 2; ++jj) {
                 const int jb = 2 * h + jj;          // 32-slot block of s
                 const uint32_t col = tmem + lane_base + kColG + 32 * jb;
@@ -752,7 +752,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                     tc::tmem_st16_nw(col + 16, z);
                     continue;
                 }
-#pragma unroll
+#pragma unroll 1
                 for (int u = 0; u < 2; ++u) {       // 16-slot unit = K-step 2 jb + u
                     uint32_t gu[16];
                     tc::tmem_ld16_nw(col + 16 * u, gu);
@@ -910,42 +910,37 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         // Per chunk k: the state at its start (the operands of the state
         // product and Yo) first, then M(k) (the operand of Yd), so that the
         // producer issues the first two products while M is being built.
-        bool ok = a_wait(mb_dt0, 0);   // chunk 0's prefix sums and factors
-        if (ok) {
-            tc::fence_after_sync();
-            scale_state(0);
-            publish(mb_s, !kStateOnly);
-            if constexpr (!kStateOnly) {
-                ok = a_wait(mb_g, 0);
-                if (ok) {
-                    tc::fence_after_sync();
-                    build_m(0);
-                    publish(mb_m, false);
-                }
-            }
-        }
-        for (int k = 0; k < nk && ok; ++k) {
-            ok = a_wait(mb_e, k & 1);   // chunk k's MMAs done
-            if (!ok) break;
-            tc::fence_after_sync();
-            if constexpr (!kStateOnly) {
-                stage_rows(k);
-                tc::fence_proxy_async();   // the staged rows, for the publisher's bulk copies
-                tc::fence_before_sync();   // TMEM reads done before the next chunk's MMAs
-                grp_sync(1);
-                if (tid == 0) tc::mbar_arrive(mb_staged);
-            }
-            if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * (k & 1));
-            if (k + 1 >= nk) break;
-            ok = a_wait(mb_dt0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
-            if (!ok) break;
-            scale_state(k + 1);
-            publish(mb_s, !kStateOnly);
-            if constexpr (!kStateOnly) {
-                ok = a_wait(mb_g, (k + 1) & 1);
+        // Per walk chunk j: once chunk j-1's MMAs are done, its output rows;
+        // then the state at chunk j's start (the operands of the state
+        // product and Yo) first, and M(j) (the operand of Yd), so that the
+        // producer issues the first two products while M is being built.
+        // (Every phase has one call site.)
+        bool ok = true;
+        for (int j = 0; j <= nk && ok; ++j) {
+            if (j >= 1) {
+                ok = a_wait(mb_e, (j - 1) & 1);   // chunk j-1's MMAs done
                 if (!ok) break;
                 tc::fence_after_sync();
-                build_m(k + 1);
+                if constexpr (!kStateOnly) {
+                    stage_rows(j - 1);
+                    tc::fence_proxy_async();   // the staged rows, for the publisher's TMA stores
+                    tc::fence_before_sync();   // TMEM reads done before the next chunk's MMAs
+                    grp_sync(1);
+                    if (tid == 0) tc::mbar_arrive(mb_staged);
+                }
+                if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * ((j - 1) & 1));
+                if (j >= nk) break;
+            }
+            ok = a_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);   // chunk j's prefix sums and factors
+            if (!ok) break;
+            tc::fence_after_sync();
+            scale_state(j);
+            publish(mb_s, !kStateOnly);
+            if constexpr (!kStateOnly) {
+                ok = a_wait(mb_g, j & 1);
+                if (!ok) break;
+                tc::fence_after_sync();
+                build_m(j);
                 publish(mb_m, false);
             }
         }
@@ -1088,11 +1083,17 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             grp_sync(2);
         };
 
-        bool ok = b_wait(mb_x0, 0);
-        if (ok) {
-            // decode and sequence shards: the conv history before token 0
-            // comes from the tail
-            if (!rev && p.tail && k0 == 0) {
+        // Per walk chunk j: the conv of its raw rows (x buffer j % 2), then
+        // wX(j) = w o X(j) once the state product of chunk j-1 has read
+        // wX(j-1).  (Every phase has one call site: the kernel's code stays
+        // small enough for the instruction caches.)
+        bool ok = true;
+        for (int j = 0; j < nk && ok; ++j) {
+            ok = b_wait(mb_x0 + 8 * (j & 1), (j >> 1) & 1);
+            if (!ok) break;
+            if (j == 0 && !rev && p.tail && k0 == 0) {
+                // decode and sequence shards: the conv history before token 0
+                // comes from the tail
                 for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
                     const int r = e / (kPP / 8), g = e % (kPP / 8);
                     *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
@@ -1101,46 +1102,23 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 }
                 grp_sync(2);
             }
-            head_rows(0);
-            conv_chunk(0);
-            ok = b_wait(mb_dt0, 0);   // (also the barrier between conv writes and wX reads)
-        }
-        if (ok) {
-            weight_chunk(0);
-            tc::fence_proxy_async();
-            grp_sync(2);
-            if (tb == 0) {
-                tc::mbar_arrive(mb_s);
-                tc::mbar_arrive(mb_free0);
+            if (j < 2) head_rows(j);
+            conv_chunk(j);
+            if (j >= 1) {
+                // the state product of chunk j-1 has read wX (its commit also
+                // covers Yo in the full kernel)
+                ok = b_wait(kStateOnly ? mb_e : mb_bcfree, (j - 1) & 1);
+                if (!ok) break;
             }
-            if (nk > 1) {
-                ok = b_wait(mb_x0 + 8, 0);
-                if (ok) {
-                    head_rows(1);
-                    conv_chunk(1);
-                }
-            }
-        }
-        for (int k = 0; k + 1 < nk && ok; ++k) {
-            // the state product of chunk k has read wX (its commit also
-            // covers Yo in the full kernel)
-            ok = b_wait(kStateOnly ? mb_e : mb_bcfree, k & 1);
+            // (also the barrier between the conv's writes and wX's reads)
+            ok = b_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);
             if (!ok) break;
-            // ---- wX of chunk k+1 (its X tile was convolved an iteration ago)
-            ok = b_wait(mb_dt0 + 8 * ((k + 1) & 1), ((k + 1) >> 1) & 1);
-            if (!ok) break;
-            weight_chunk(k + 1);
+            weight_chunk(j);
             tc::fence_proxy_async();   // X and wX, for the tensor core
             grp_sync(2);
             if (tb == 0) {
                 tc::mbar_arrive(mb_s);
-                tc::mbar_arrive(mb_free0 + 8 * ((k + 1) & 1));
-            }
-            // ---- conv of chunk k+2 (its raw rows were loaded once chunk k's MMAs completed)
-            if (k + 2 < nk) {
-                ok = b_wait(mb_x0 + 8 * ((k + 2) & 1), ((k + 2) >> 1) & 1);
-                if (!ok) break;
-                conv_chunk(k + 2);
+                tc::mbar_arrive(mb_free0 + 8 * (j & 1));
             }
         }
         if (!ok && tb == 0) record_error(p.status, kStatusTimeout);
