@@ -57,6 +57,7 @@
 #include "tc_ptx.cuh"
 
 #include <algorithm>
+#include <type_traits>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -465,8 +466,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         // consecutive entries
         const int c = hp * kPP + tid;
         const int slot = (tid & 3) * 32 + (tid >> 2);
-        convw[slot] = *reinterpret_cast<const float4 *>(conv_w + (size_t)c * 4);
-        convb[slot] = conv_b ? conv_b[c] : 0.0f;
+        const float4 w = *reinterpret_cast<const float4 *>(conv_w + (size_t)c * 4);
+        convw[slot] = make_float4(0.5f * w.x, 0.5f * w.y, 0.5f * w.z, 0.5f * w.w);   // halved (see the conv)
+        convb[slot] = conv_b ? 0.5f * conv_b[c] : 0.0f;
     }
     for (int i = tid; i < 2048 / 16; i += kThreads) {   // zero blocks of the block-diagonal Yd operand
         reinterpret_cast<uint4 *>(sm + kOffZlo)[i] = make_uint4(0, 0, 0, 0);
@@ -515,7 +517,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         constexpr uint32_t idY = tc::idesc_bf16(128, 128, 0, 1);
         constexpr uint32_t idS = tc::idesc_bf16(128, 128, 1, 1);
         auto issue_g = [&]() {
-#pragma unroll
+#pragma unroll 1
             for (int ks = 0; ks < kN / 16; ++ks) {
                 const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
                 tc::mma_bf16(tmem + kColG, tc::desc_add(dC, koff), tc::desc_add(dB, koff), idG, ks > 0);
@@ -538,13 +540,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 if (!pok) break;
                 tc::fence_after_sync();
                 // the state product first: the next chunk's state scaling waits for it
-#pragma unroll
+#pragma unroll 1
                 for (int ks = 0; ks < kQ / 16; ++ks)
                     tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048), tc::desc_add(dXw, ks * 2048),
                                  idS, 1);
                 if constexpr (!kStateOnly) {
                     // Yo = C S_in^T (both heads)
-#pragma unroll
+#pragma unroll 1
                     for (int ks = 0; ks < kN / 16; ++ks) {
                         const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
                         tc::mma_bf16(tmem + kColYo, tc::desc_add(dC, koff), tc::desc_add(dS, ks * 2048), idY,
@@ -567,10 +569,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                     const uint64_t d1 = tc::smem_desc(sbase + kOffZlo, xb + 16384 - (sbase + kOffZlo), 1024);
                     constexpr uint64_t kStep0 = 128ull - (128ull << 16);   // start += 2 KB, offset -= 2 KB
                     constexpr uint64_t kStep1 = 128ull << 16;              // offset += 2 KB
-#pragma unroll
+#pragma unroll 1
                     for (int ks = 0; ks < 8; ++ks)
                         tc::mma_bf16_tmemA(tmem + kColYd, tmem + kColG + 16 * ks, d0 + ks * kStep0, idY, ks > 0);
-#pragma unroll
+#pragma unroll 1
                     for (int ks = 0; ks < 8; ++ks)
                         tc::mma_bf16_tmemA(tmem + kColYd, tmem + kColG + 16 * ks + 8, d1 + ks * kStep1, idY, 1);
                 }
@@ -758,7 +760,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                     tc::tmem_ld16_nw(col + 16 * u, gu);
                     tc::tmem_wait_ld16(gu);
                     const int s0u = 32 * jb + 16 * u;   // first slot of the unit
-#pragma unroll
+#pragma unroll 1
                     for (int hd = 0; hd < kHeads; ++hd) {
                         const float *cm = cum + (par * kHeads + hd) * kQ;
                         const float ct = cm[row];
@@ -831,7 +833,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             const float a_last = tc::exp2_approx(cl);
             const float2 a2 = make_float2(a_last, a_last);
             if constexpr (kStateOnly) dec += cl;
-#pragma unroll
+#pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 uint32_t sr[32];
                 const uint32_t col = tmem + lane_base + kColS + 64 * h + 32 * half;
@@ -876,7 +878,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             uint8_t *box = sm + xbuf_off(k) + h * 16384 + q * 128;
             const float et = tc::exp2_approx(cum[((k & 1) * kHeads + h) * kQ + row]);
             const float2 et2 = make_float2(et, et);
-#pragma unroll
+#pragma unroll 1
             for (int qtr = 0; qtr < 4; ++qtr) {
                 uint32_t yy[32];   // [0, 16): Yd, [16, 32): Yo
                 tc::tmem_ld16_nw(tmem + lane_base + kColYd + 64 * h + 16 * qtr, yy);
@@ -980,69 +982,88 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         };
         // conv+SiLU of both heads' x for walk chunk k, in place: the raw
         // rows in x buffer k % 2 become the swizzled X tile of the chunk.
-        // Thread: channel pair cp (channels 2cp, 2cp+1; head cp >> 5) x 32
-        // walk slots 32sg..32sg+31, in packed fp32.  Raw row of walk offset j:
-        // forward j + 3 (the box starts 3 tokens early), reverse cnt - 1 - j.
-        // Every thread reads its raw rows before the group barrier and
-        // writes after it.
-        auto conv_chunk = [&](int k) {
+        // Thread: channel quad cq (channels 4cq .. 4cq+3, head cq >> 4) x 16
+        // walk slots 16sg .. 16sg+15, in packed fp32 pairs.  The raw row of
+        // slot s's tap j is s + j forward (the box starts 3 tokens early)
+        // and cnt + 2 - s - j reverse (the mirror image); the direction is a
+        // compile-time constant of each instance.  Every thread reads its
+        // raw rows before the group barrier and writes after it.  The taps
+        // and bias are stored halved: SiLU(a) = h + h tanh(h) with h = a / 2.
+        auto conv_impl = [&](auto rev_c, int k) {
+            constexpr bool kR = decltype(rev_c)::value;
             int t0, cnt, s0;
             chunk_of(k, t0, cnt, s0);
             uint8_t *buf = sm + xbuf_off(k);
-            const int cp = tb & 63, sg = tb >> 6;
-            const int j0 = 32 * sg;
-            uint32_t rr[35];
+            const int cq = tb & 31, sg = tb >> 5;
+            const int j0 = 16 * sg;
+            // reverse rows below 0 (slots past a short chunk's end) read other
+            // shared memory of this CTA; those slots are written as zeros
+            const uint8_t *src = buf + (kR ? cnt + 2 - j0 : j0) * (kPP * 2) + 8 * cq;
+            uint2 rr[19];
 #pragma unroll
-            for (int i = 0; i < 35; ++i) {
-                const int jw = j0 + i - 3;   // walk offset of the raw row
-                const int rrow = rev ? cnt - 1 - jw : jw + 3;
-                rr[i] = (rrow >= 0 && rrow < kRawRows)
-                            ? *reinterpret_cast<const uint32_t *>(buf + rrow * (kPP * 2) + 4 * cp)
-                            : 0u;
-            }
+            for (int i = 0; i < 19; ++i)
+                rr[i] = *reinterpret_cast<const uint2 *>(src + (kR ? -i : i) * (kPP * 2));
             grp_sync(2);
-            const int gh = cp >> 5, piece = (cp & 31) >> 2;
-            uint8_t *dst = buf + gh * 16384 + 4 * (cp & 3);
-            const bool full = j0 + 32 <= cnt;
-            auto upair = [](uint32_t r) {
+            uint8_t *dst = buf + (cq >> 4) * 16384 + j0 * 128 + 8 * (cq & 1);
+            const uint32_t pbase = static_cast<uint32_t>((cq & 15) >> 1) << 4;   // piece, before the swizzle
+            const bool full = j0 + 16 <= cnt;
+            auto up = [](uint32_t r) {
                 return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r));
             };
             if (has_conv) {
-                // acc = b + sum_j w_j u_j, SiLU(acc) = h + h tanh(h), h = acc / 2
-                const int c0 = 2 * cp, c1 = 2 * cp + 1;   // channels of the pair
-                const float4 wa = convw[(c0 & 3) * 32 + (c0 >> 2)], wb = convw[(c1 & 3) * 32 + (c1 >> 2)];
-                const float2 w0 = make_float2(wa.x, wb.x), w1 = make_float2(wa.y, wb.y);
-                const float2 w2 = make_float2(wa.z, wb.z), w3 = make_float2(wa.w, wb.w);
-                const float2 bp = make_float2(convb[(c0 & 3) * 32 + (c0 >> 2)], convb[(c1 & 3) * 32 + (c1 >> 2)]);
-                const float2 half2 = make_float2(0.5f, 0.5f);
-                float2 u0 = upair(rr[0]), u1 = upair(rr[1]), u2 = upair(rr[2]);
+                float4 wq[4];
+                float bq[4];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float2 u3 = upair(rr[i + 3]);
-                    float2 acc = tc::fma2(w0, u0, bp);
-                    acc = tc::fma2(w1, u1, acc);
-                    acc = tc::fma2(w2, u2, acc);
-                    acc = tc::fma2(w3, u3, acc);
-                    const float2 hh = tc::mul2(acc, half2);
-                    float tx, ty;
-                    asm("tanh.approx.f32 %0, %1;" : "=f"(tx) : "f"(hh.x));
-                    asm("tanh.approx.f32 %0, %1;" : "=f"(ty) : "f"(hh.y));
-                    const float2 o = tc::fma2(hh, make_float2(tx, ty), hh);
-                    uint32_t pk = tc::pack_bf16x2(o.x, o.y);
-                    if (!full && j0 + i >= cnt) pk = 0u;
-                    *reinterpret_cast<uint32_t *>(dst + tc::sw128(j0 + i, piece)) = pk;
-                    u0 = u1;
-                    u1 = u2;
-                    u2 = u3;
+                for (int q = 0; q < 4; ++q) {
+                    wq[q] = convw[q * 32 + cq];
+                    bq[q] = convb[q * 32 + cq];
+                }
+                // channel pairs (0, 1) and (2, 3) of the quad, per tap
+                const float2 wa0 = make_float2(wq[0].x, wq[1].x), wa1 = make_float2(wq[0].y, wq[1].y);
+                const float2 wa2 = make_float2(wq[0].z, wq[1].z), wa3 = make_float2(wq[0].w, wq[1].w);
+                const float2 wb0 = make_float2(wq[2].x, wq[3].x), wb1 = make_float2(wq[2].y, wq[3].y);
+                const float2 wb2 = make_float2(wq[2].z, wq[3].z), wb3 = make_float2(wq[2].w, wq[3].w);
+                const float2 ba = make_float2(bq[0], bq[1]), bb = make_float2(bq[2], bq[3]);
+                float2 a0 = up(rr[0].x), a1 = up(rr[1].x), a2 = up(rr[2].x);
+                float2 b0 = up(rr[0].y), b1 = up(rr[1].y), b2 = up(rr[2].y);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 a3 = up(rr[i + 3].x), b3 = up(rr[i + 3].y);
+                    float2 ha = tc::fma2(wa0, a0, ba);
+                    float2 hb = tc::fma2(wb0, b0, bb);
+                    ha = tc::fma2(wa1, a1, ha);
+                    hb = tc::fma2(wb1, b1, hb);
+                    ha = tc::fma2(wa2, a2, ha);
+                    hb = tc::fma2(wb2, b2, hb);
+                    ha = tc::fma2(wa3, a3, ha);
+                    hb = tc::fma2(wb3, b3, hb);
+                    float t[4];
+                    asm("tanh.approx.f32 %0, %1;" : "=f"(t[0]) : "f"(ha.x));
+                    asm("tanh.approx.f32 %0, %1;" : "=f"(t[1]) : "f"(ha.y));
+                    asm("tanh.approx.f32 %0, %1;" : "=f"(t[2]) : "f"(hb.x));
+                    asm("tanh.approx.f32 %0, %1;" : "=f"(t[3]) : "f"(hb.y));
+                    const float2 oa = tc::fma2(ha, make_float2(t[0], t[1]), ha);
+                    const float2 ob = tc::fma2(hb, make_float2(t[2], t[3]), hb);
+                    uint2 pk = make_uint2(tc::pack_bf16x2(oa.x, oa.y), tc::pack_bf16x2(ob.x, ob.y));
+                    if (!full && j0 + i >= cnt) pk = make_uint2(0u, 0u);
+                    *reinterpret_cast<uint2 *>(dst + i * 128 + (pbase ^ ((i & 7) << 4))) = pk;
+                    a0 = a1; a1 = a2; a2 = a3;
+                    b0 = b1; b1 = b2; b2 = b3;
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    uint32_t pk = rr[i + 3];
-                    if (!full && j0 + i >= cnt) pk = 0u;
-                    *reinterpret_cast<uint32_t *>(dst + tc::sw128(j0 + i, piece)) = pk;
+                for (int i = 0; i < 16; ++i) {
+                    uint2 pk = rr[i + 3];
+                    if (!full && j0 + i >= cnt) pk = make_uint2(0u, 0u);
+                    *reinterpret_cast<uint2 *>(dst + i * 128 + (pbase ^ ((i & 7) << 4))) = pk;
                 }
             }
+        };
+        auto conv_chunk = [&](int k) {
+            if (rev)
+                conv_impl(std::true_type{}, k);
+            else
+                conv_impl(std::false_type{}, k);
         };
         // wX = w_s * X for walk chunk k (X tile in x buffer k % 2): thread
         // (slot j, head gh), the head's 64 channels
@@ -1050,7 +1071,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             const uint8_t *xt = sm + xbuf_off(k);
             const int j = tb & 127, gh = tb >> 7;
             const float wj = wgt[((k & 1) * kHeads + gh) * kQ + j];
-#pragma unroll
+#pragma unroll 2
             for (int pc = 0; pc < 8; ++pc) {
                 const uint32_t off = gh * 16384 + tc::sw128(j, pc);
                 float v[8];
