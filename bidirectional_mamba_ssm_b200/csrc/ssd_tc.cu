@@ -346,6 +346,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     const uint32_t mb_free0 = sbase + kOffMbar + 64; // an even / odd chunk's factor buffers free (+8)
     const uint32_t mb_staged = sbase + kOffMbar + 80;   // the chunk's output rows staged
     const uint32_t mb_bcfree = sbase + kOffMbar + 88;   // the chunk's products that read B/C done
+    const uint32_t mb_sdone = sbase + kOffMbar + 104;   // the chunk's state product done (wX read)
     const uint32_t mb_s = sbase + kOffMbar + 96;     // state, its bf16 copy and wX ready (one arrival per group)
     auto xbuf_off = [](int k) { return (k & 1) ? kOffXbuf1 : kOffXbuf0; };
 
@@ -492,6 +493,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         tc::mbar_init(mb_free0 + 8, 2);
         tc::mbar_init(mb_staged, 1);
         tc::mbar_init(mb_bcfree, 1);
+        tc::mbar_init(mb_sdone, 1);
         issue_x(0);
         if (nk > 1) issue_x(1);
         issue_bc(0);
@@ -545,6 +547,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                     tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048), tc::desc_add(dXw, ks * 2048),
                                  idS, 1);
                 if constexpr (!kStateOnly) {
+                    tc::mma_commit(mb_sdone);   // wX may be rewritten once it completes
                     // Yo = C S_in^T (both heads)
 #pragma unroll 1
                     for (int ks = 0; ks < kN / 16; ++ks) {
@@ -1068,17 +1071,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         // wX = w_s * X for walk chunk k (X tile in x buffer k % 2): thread
         // (slot j, head gh), the head's 64 channels
         auto weight_chunk = [&](int k) {
+            // in bf16 pairs: w_s rounded to bf16, each product rounded once
             const uint8_t *xt = sm + xbuf_off(k);
             const int j = tb & 127, gh = tb >> 7;
-            const float wj = wgt[((k & 1) * kHeads + gh) * kQ + j];
-#pragma unroll 2
+            const __nv_bfloat162 w2 = __float2bfloat162_rn(wgt[((k & 1) * kHeads + gh) * kQ + j]);
+#pragma unroll
             for (int pc = 0; pc < 8; ++pc) {
                 const uint32_t off = gh * 16384 + tc::sw128(j, pc);
-                float v[8];
-                unpack8(*reinterpret_cast<const uint4 *>(xt + off), v);
+                uint4 v = *reinterpret_cast<const uint4 *>(xt + off);
+                __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&v);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] *= wj;
-                *reinterpret_cast<uint4 *>(sm + kOffXw + off) = pack8(v);
+                for (int q = 0; q < 4; ++q) h2[q] = __hmul2(h2[q], w2);
+                *reinterpret_cast<uint4 *>(sm + kOffXw + off) = v;
             }
         };
 
@@ -1126,9 +1130,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             if (j < 2) head_rows(j);
             conv_chunk(j);
             if (j >= 1) {
-                // the state product of chunk j-1 has read wX (its commit also
-                // covers Yo in the full kernel)
-                ok = b_wait(kStateOnly ? mb_e : mb_bcfree, (j - 1) & 1);
+                // the state product of chunk j-1 has read wX
+                ok = b_wait(kStateOnly ? mb_e : mb_sdone, (j - 1) & 1);
                 if (!ok) break;
             }
             // (also the barrier between the conv's writes and wX's reads)
