@@ -40,6 +40,9 @@
 #include "dispatch.h"
 #include "tc_ptx.cuh"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 namespace bimamba {
 
 namespace {
@@ -70,13 +73,22 @@ constexpr uint32_t kDOffC = 16384;      // C_f image (the Yo operand reads 128 r
 constexpr uint32_t kDOffB = 24576 + 8192;   // B_f image
 constexpr uint32_t kDOffX = 49152;      // [X_f; X_r] MN-major [128 slots][64 p]
 constexpr uint32_t kDOffXw = 65536;     // w o X_f [64 slots][64 p]
-constexpr uint32_t kDOffCum = 73728;    // f32 cf[64], cr[64], dtf[64], dtr[64]
+// the cached fp32 state [64 p][128 n], landed by one bulk copy where X and
+// wX go later (it is converted to the bf16 tile before the conv writes X)
+constexpr uint32_t kDOffSf = kDOffX;
+// raw x rows, rho = token rho - 3, 128 bytes each with the 128-byte swizzle
+// keyed on (rho + 5) & 7: the 3 conv-tail rows, then the TMA box of the
+// block's 64 tokens (1024-aligned; rows past the block end read zeros)
+constexpr uint32_t kDOffRawBox = 82944;
+constexpr uint32_t kDOffRaw = kDOffRawBox - 3 * 128;
+constexpr uint32_t kDOffCum = kDOffRawBox + kDQ * 128;   // f32 cf[64], cr[64], dtf[64], dtr[64]
 constexpr uint32_t kDOffConvW = kDOffCum + 1024;   // float4[64]
 constexpr uint32_t kDOffConvB = kDOffConvW + 1024; // f32[64]
 constexpr uint32_t kDOffMbar = kDOffConvB + 256;   // 2 mbarriers
 constexpr uint32_t kDOffTmem = kDOffMbar + 16;
 constexpr uint32_t kDSmem = kDOffTmem + 16 + 1024;
 static_assert(kDOffB == kDOffC + 16384, "C_f and B_f images are one contiguous copy");
+static_assert(kDOffSf + kDP * kDN * 4 <= kDOffRaw && kDOffRawBox % 1024 == 0, "decode shared-memory map");
 
 constexpr uint32_t kDColM = 0, kDColYd = 64, kDColYo = 128, kDColS = 192;
 
@@ -253,7 +265,7 @@ struct DecodeParams {
 
 // One CTA per (stream, head): both directions of one head over the block.
 __global__ void __launch_bounds__(kDThreads, 2)
-decode_tc_kernel(const DecodeParams p)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -276,12 +288,25 @@ decode_tc_kernel(const DecodeParams p)
     const uint8_t *rec = p.prep + (size_t)s * kPrepBytes;
     const float *state = p.state + ((size_t)slot * H + h) * kDP * kDN;
 
+    // Every global input is requested up front, so that one memory latency
+    // covers them all: the C_f / B_f images, the cached state and the
+    // block's raw x rows by bulk / TMA copies onto one mbarrier, the conv
+    // tail and G rows by plain loads.
     if (warp == 0) tc::tmem_alloc(sbase + kDOffTmem, 256);
     if (tid == 0) {
         tc::mbar_init(mb_ld, 1);
         tc::mbar_init(mb_mma, 1);
-        tc::mbar_expect_tx(mb_ld, 32768);
-        bulk_g2s(sbase + kDOffC, rec + kPrepG, 32768, mb_ld);   // C_f and B_f images
+        tc::prefetch_tmap(&tm_x);
+        tc::mbar_expect_tx(mb_ld, 32768 + kDP * kDN * 4 + kDQ * 128);
+        bulk_g2s(sbase + kDOffC, rec + kPrepG, 32768, mb_ld);          // C_f and B_f images
+        bulk_g2s(sbase + kDOffSf, state, kDP * kDN * 4, mb_ld);        // the cached state
+        tc::tma_load_3d(sbase + kDOffRawBox, &tm_x, h * kDP, 0, s, mb_ld);   // tokens 0..63 (zeros past len)
+    }
+    if (tid >= 64 && tid < 64 + 24) {
+        // conv tail: the 3 newest tokens before the block, raw rows 0..2
+        const int e = tid - 64, rr = e >> 3, c = e & 7;
+        const uint4 v = *reinterpret_cast<const uint4 *>(p.tail + ((size_t)slot * 4 + 1 + rr) * ch + h * kDP + 8 * c);
+        *reinterpret_cast<uint4 *>(sm + kDOffRaw + rr * 128 + ((c ^ ((rr + 5) & 7)) << 4)) = v;
     }
     if (tid < kDP) {
         const int c = h * kDP + tid;
@@ -322,17 +347,36 @@ decode_tc_kernel(const DecodeParams p)
         dtr[2 * lane] = e[0];
         dtr[2 * lane + 1] = e[1];
     }
+    // thread (r, half): stacked row r (TMEM lane) -- direction d = r >> 6,
+    // walk slot t = r & 63 -- and the half of the 64 channels / slots it owns
+    const int r = tid & 127, half = tid >> 7;
+    const int d = r >> 6, t = r & 63;
+    // this thread's G row (L2-resident prep record), loaded while the copies fly
+    float4 grow[8];
     {
-        // the cached state S[p][n] -> bf16 K-major tile (N = p rows, K = n):
-        // thread (p, quarter q of n): 32 values, 4 pieces of one atom
-        const int pr = tid >> 2, q = tid & 3;
-        const float4 *src = reinterpret_cast<const float4 *>(state + (size_t)pr * kDN + 32 * q);
-        uint8_t *atom = sm + kDOffS + (q >> 1) * 8192;
+        const float4 *grow4 = reinterpret_cast<const float4 *>(
+            reinterpret_cast<const float *>(rec) + ((size_t)d * kDQ + t) * kDQ + 32 * half);
 #pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
-            const float4 a = __ldg(src + 2 * pc), b4 = __ldg(src + 2 * pc + 1);
+        for (int i = 0; i < 8; ++i) grow[i] = __ldg(grow4 + i);
+    }
+    tc::fence_before_sync();
+    __syncthreads();   // mbarrier initialised; taps, prefix sums and tail rows written
+    bool ok = tc::mbar_wait_bounded(mb_ld, 0, kDWait);
+    if (!ok && tid == 0) record_error(p.status, kStatusTimeout);
+    ok = __syncthreads_and(ok);
+    if (ok) {
+        // the cached state S[p][n] (fp32, shared) -> bf16 K-major tile (N = p
+        // rows, K = n): 1024 pieces of 8 n; thread: pieces tid + 256 i (a
+        // warp reads two contiguous 512-byte rows per step)
+        const float *sf = reinterpret_cast<const float *>(sm + kDOffSf);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + kDThreads * i;
+            const int pr = e >> 4, pc = e & 15;
+            const float4 a = *reinterpret_cast<const float4 *>(sf + pr * kDN + 8 * pc);
+            const float4 b4 = *reinterpret_cast<const float4 *>(sf + pr * kDN + 8 * pc + 4);
             const float v[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
-            *reinterpret_cast<uint4 *>(atom + tc::sw128(pr, 4 * (q & 1) + pc)) = pack8f(v);
+            *reinterpret_cast<uint4 *>(sm + kDOffS + (pc >> 3) * 8192 + tc::sw128(pr, pc & 7)) = pack8f(v);
         }
     }
     tc::fence_before_sync();
@@ -340,18 +384,14 @@ decode_tc_kernel(const DecodeParams p)
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kDOffTmem);
 
-    // thread (r, half): stacked row r (TMEM lane) -- direction d = r >> 6,
-    // walk slot t = r & 63 -- and the half of the 64 channels / slots it owns
-    const int r = tid & 127, half = tid >> 7;
-    const int d = r >> 6, t = r & 63;
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const float *cdir = d ? cr : cf;
     const float *dtdir = d ? dtr : dtf;
 
     // ---- conv+SiLU of the head's x into [X_f; X_r] (row r, channels
-    // 32 half .. 32 half + 31), and w o X_f for the commit.  The four taps'
-    // rows are loaded before any arithmetic (two halves of 16 channels).
-    {
+    // 32 half .. 32 half + 31), and w o X_f for the commit, from the raw rows
+    // in shared memory (two halves of 16 channels)
+    if (ok) {
         const int tok = d ? len - 1 - t : t;
         const float w_commit =
             (do_commit && d == 0 && t < len) ? tc::exp2_approx(cf[len - 1] - cf[t]) * dtf[t] : 0.0f;
@@ -361,17 +401,16 @@ decode_tc_kernel(const DecodeParams p)
             uint4 raw[4][2];
 #pragma unroll
             for (int tap = 0; tap < 4; ++tap) {
-                const int u = d ? tok + 3 - tap : tok - 3 + tap;
-                const __nv_bfloat16 *srcp = nullptr;
-                if (t < len) {
-                    if (u >= 0 && u < len)
-                        srcp = p.xbc + ((size_t)s * len + u) * ch + h * kDP + c0;
-                    else if (!d && u < 0)
-                        srcp = p.tail + ((size_t)slot * 4 + 4 + u) * ch + h * kDP + c0;
-                }
+                const int u = d ? tok + 3 - tap : tok - 3 + tap;   // token; -3..-1: the tail
+                const int rho = u + 3;
+                const bool valid = t < len && u < len;
 #pragma unroll
-                for (int v4 = 0; v4 < 2; ++v4)
-                    raw[tap][v4] = srcp ? __ldg(reinterpret_cast<const uint4 *>(srcp) + v4) : make_uint4(0, 0, 0, 0);
+                for (int v4 = 0; v4 < 2; ++v4) {
+                    const int chunk = (c0 >> 3) + v4;
+                    raw[tap][v4] = valid ? *reinterpret_cast<const uint4 *>(
+                                               sm + kDOffRaw + rho * 128 + ((chunk ^ ((rho + 5) & 7)) << 4))
+                                         : make_uint4(0, 0, 0, 0);
+                }
             }
             float acc[16];
 #pragma unroll
@@ -409,14 +448,12 @@ decode_tc_kernel(const DecodeParams p)
     // ---- M: row r holds its direction's 64 K columns [64 d, 64 d + 64)
     // (this thread: slots 32 half .. 32 half + 31) and zeros in the other
     // direction's; D on the diagonal
-    {
+    if (ok) {
         const float Dh = p.D[h];
-        const float4 *grow4 = reinterpret_cast<const float4 *>(
-            reinterpret_cast<const float *>(rec) + ((size_t)d * kDQ + t) * kDQ + 32 * half);
         float g[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float4 v = __ldg(grow4 + i);
+            const float4 v = grow[i];
             g[4 * i] = v.x; g[4 * i + 1] = v.y; g[4 * i + 2] = v.z; g[4 * i + 3] = v.w;
         }
         const float ct = cdir[t];
@@ -441,11 +478,9 @@ decode_tc_kernel(const DecodeParams p)
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
-    bool ok = true;
-    if (tid == 0) {
+    if (ok && tid == 0) {
         tc::fence_after_sync();
-        ok = tc::mbar_wait_bounded(mb_ld, 0, kDWait);   // C_f / B_f images landed
-        if (ok) {
+        {
             const uint64_t dX = tc::smem_desc(sbase + kDOffX, 1024, 1024);     // MN-major, N = 64
             const uint64_t dC = tc::smem_desc(sbase + kDOffC, 16, 1024);       // K-major A
             const uint64_t dS = tc::smem_desc(sbase + kDOffS, 16, 1024);       // K-major B (N = p)
@@ -583,6 +618,29 @@ bool decode_tc_supported(const bimamba_dims &d)
 
 size_t decode_tc_workspace_bytes(const bimamba_dims &d) { return (size_t)d.batch * kPrepBytes; }
 
+// The block's raw xBC as a 3-D bf16 tensor map (ch, len, streams), read by
+// 64-channel x 64-token boxes with the 128-byte swizzle (tokens past len
+// read zeros).
+static bool make_block_map(CUtensorMap *m, const void *base, int ch, int len, int streams)
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult qr;
+        void *f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qr) != cudaSuccess ||
+            qr != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)ch, (cuuint64_t)len, (cuuint64_t)streams};
+    const cuuint64_t strides[2] = {(cuuint64_t)ch * 2, (cuuint64_t)ch * len * 2};
+    const cuuint32_t box[3] = {kDP, kDQ, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_decode_tc(const DecodeProblem &q, cudaStream_t stream)
 {
     const bimamba_dims &d = q.dims;
@@ -619,7 +677,9 @@ cudaError_t launch_decode_tc(const DecodeProblem &q, cudaStream_t stream)
     p.ch = ch;
     const TimingEvents ev = timing_events();
     if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
-    decode_tc_kernel<<<dim3(d.heads, d.batch), kDThreads, kDSmem, stream>>>(p);
+    CUtensorMap tm_x;
+    if ((ch * 2) % 16 != 0 || !make_block_map(&tm_x, q.xbc, ch, d.len, d.batch)) return cudaErrorInvalidValue;
+    decode_tc_kernel<<<dim3(d.heads, d.batch), kDThreads, kDSmem, stream>>>(tm_x, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launch();
     if (ev.stop) e = cudaEventRecord(ev.stop, stream);
