@@ -310,8 +310,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
     }
     if (tid < kDP) {
         const int c = h * kDP + tid;
-        convw[tid] = *reinterpret_cast<const float4 *>(p.conv_w + (size_t)c * 4);
-        convb[tid] = p.conv_b ? p.conv_b[c] : 0.0f;
+        const float4 w = *reinterpret_cast<const float4 *>(p.conv_w + (size_t)c * 4);
+        convw[tid] = make_float4(0.5f * w.x, 0.5f * w.y, 0.5f * w.z, 0.5f * w.w);   // halved (see the conv)
+        convb[tid] = p.conv_b ? 0.5f * p.conv_b[c] : 0.0f;
     }
     if (warp == 7) {
         // dt of the head, prefix sums of dt*A in log2 units: forward in token
@@ -388,61 +389,78 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
     const float *cdir = d ? cr : cf;
     const float *dtdir = d ? dtr : dtf;
 
-    // ---- conv+SiLU of the head's x into [X_f; X_r] (row r, channels
-    // 32 half .. 32 half + 31), and w o X_f for the commit, from the raw rows
-    // in shared memory (two halves of 16 channels)
+    // ---- conv+SiLU of the head's x into [X_f; X_r], and w o X_f for the
+    // commit, from the raw rows in shared memory.  Thread: channel quad cq
+    // (channels 4cq .. 4cq+3) x 8 stacked rows 8g .. 8g+7 (direction
+    // g >> 3), in packed fp32 pairs with halved taps and bias: SiLU(a) =
+    // h + h tanh(h), h = a / 2.  Raw row of slot t's tap j: t + j forward,
+    // len + 5 - t - j reverse (token len-1-t, mirrored taps); tokens past
+    // the block end read zeros.
     if (ok) {
-        const int tok = d ? len - 1 - t : t;
-        const float w_commit =
-            (do_commit && d == 0 && t < len) ? tc::exp2_approx(cf[len - 1] - cf[t]) * dtf[t] : 0.0f;
+        const int cq = tid & 15, g = tid >> 4;
+        const int dg = g >> 3, t0 = 8 * (g & 7);
+        uint2 rr[11];
 #pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-            const int c0 = 32 * half + 16 * hc;
-            uint4 raw[4][2];
+        for (int i = 0; i < 11; ++i) {
+            const int rho = dg ? len + 5 - t0 - i : t0 + i;
+            const int chunk = cq >> 1;
+            rr[i] = (rho >= 0 && rho < len + 3)
+                        ? *reinterpret_cast<const uint2 *>(sm + kDOffRaw + rho * 128 +
+                                                           ((chunk ^ ((rho + 5) & 7)) << 4) + 8 * (cq & 1))
+                        : make_uint2(0u, 0u);
+        }
+        float4 wq[4];
+        float bq[4];
 #pragma unroll
-            for (int tap = 0; tap < 4; ++tap) {
-                const int u = d ? tok + 3 - tap : tok - 3 + tap;   // token; -3..-1: the tail
-                const int rho = u + 3;
-                const bool valid = t < len && u < len;
+        for (int q = 0; q < 4; ++q) {
+            wq[q] = convw[4 * cq + q];
+            bq[q] = convb[4 * cq + q];
+        }
+        const float2 wa0 = make_float2(wq[0].x, wq[1].x), wa1 = make_float2(wq[0].y, wq[1].y);
+        const float2 wa2 = make_float2(wq[0].z, wq[1].z), wa3 = make_float2(wq[0].w, wq[1].w);
+        const float2 wb0 = make_float2(wq[2].x, wq[3].x), wb1 = make_float2(wq[2].y, wq[3].y);
+        const float2 wb2 = make_float2(wq[2].z, wq[3].z), wb3 = make_float2(wq[2].w, wq[3].w);
+        const float2 ba = make_float2(bq[0], bq[1]), bb = make_float2(bq[2], bq[3]);
+        auto up = [](uint32_t v) { return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v)); };
+        float2 a0 = up(rr[0].x), a1 = up(rr[1].x), a2 = up(rr[2].x);
+        float2 b0 = up(rr[0].y), b1 = up(rr[1].y), b2 = up(rr[2].y);
+        const bool commit_rows = do_commit && dg == 0;
+        const float c_last = cf[len - 1];
 #pragma unroll
-                for (int v4 = 0; v4 < 2; ++v4) {
-                    const int chunk = (c0 >> 3) + v4;
-                    raw[tap][v4] = valid ? *reinterpret_cast<const uint4 *>(
-                                               sm + kDOffRaw + rho * 128 + ((chunk ^ ((rho + 5) & 7)) << 4))
-                                         : make_uint4(0, 0, 0, 0);
-                }
+        for (int i = 0; i < 8; ++i) {
+            const int tt = t0 + i;
+            const float2 a3 = up(rr[i + 3].x), b3 = up(rr[i + 3].y);
+            float2 ha = tc::fma2(wa0, a0, ba);
+            float2 hb = tc::fma2(wb0, b0, bb);
+            ha = tc::fma2(wa1, a1, ha);
+            hb = tc::fma2(wb1, b1, hb);
+            ha = tc::fma2(wa2, a2, ha);
+            hb = tc::fma2(wb2, b2, hb);
+            ha = tc::fma2(wa3, a3, ha);
+            hb = tc::fma2(wb3, b3, hb);
+            float th[4];
+            asm("tanh.approx.f32 %0, %1;" : "=f"(th[0]) : "f"(ha.x));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(th[1]) : "f"(ha.y));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(th[2]) : "f"(hb.x));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(th[3]) : "f"(hb.y));
+            float2 oa = tc::fma2(ha, make_float2(th[0], th[1]), ha);
+            float2 ob = tc::fma2(hb, make_float2(th[2], th[3]), hb);
+            if (tt >= len) {
+                oa = make_float2(0.0f, 0.0f);
+                ob = oa;
             }
-            float acc[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc[i] = convb[c0 + i];
-#pragma unroll
-            for (int tap = 0; tap < 4; ++tap) {
-#pragma unroll
-                for (int v4 = 0; v4 < 2; ++v4) {
-                    float v[8];
-                    unpack8f(raw[tap][v4], v);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 w4 = convw[c0 + 8 * v4 + q];
-                        const float wt = tap == 0 ? w4.x : tap == 1 ? w4.y : tap == 2 ? w4.z : w4.w;
-                        acc[8 * v4 + q] = fmaf(wt, v[q], acc[8 * v4 + q]);
-                    }
-                }
+            const uint32_t off = tc::sw128(8 * g + i, cq >> 1) + 8 * (cq & 1);
+            *reinterpret_cast<uint2 *>(sm + kDOffX + off) =
+                make_uint2(tc::pack_bf16x2(oa.x, oa.y), tc::pack_bf16x2(ob.x, ob.y));
+            if (commit_rows) {
+                const float wc = tt < len ? tc::exp2_approx(c_last - cf[tt]) * dtf[tt] : 0.0f;
+                const float2 w2 = make_float2(wc, wc);
+                const float2 xa = tc::mul2(oa, w2), xb = tc::mul2(ob, w2);
+                *reinterpret_cast<uint2 *>(sm + kDOffXw + off) =
+                    make_uint2(tc::pack_bf16x2(xa.x, xa.y), tc::pack_bf16x2(xb.x, xb.y));
             }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc[i] = t < len ? tc::silu_tanh(acc[i]) : 0.0f;
-#pragma unroll
-            for (int pc = 0; pc < 2; ++pc)
-                *reinterpret_cast<uint4 *>(sm + kDOffX + tc::sw128(r, 4 * half + 2 * hc + pc)) =
-                    pack8f(acc + 8 * pc);
-            if (do_commit && d == 0) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] *= w_commit;
-#pragma unroll
-                for (int pc = 0; pc < 2; ++pc)
-                    *reinterpret_cast<uint4 *>(sm + kDOffXw + tc::sw128(t, 4 * half + 2 * hc + pc)) =
-                        pack8f(acc + 8 * pc);
-            }
+            a0 = a1; a1 = a2; a2 = a3;
+            b0 = b1; b1 = b2; b2 = b3;
         }
     }
     // ---- M: row r holds its direction's 64 K columns [64 d, 64 d + 64)
