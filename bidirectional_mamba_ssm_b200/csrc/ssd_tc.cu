@@ -100,7 +100,7 @@ constexpr uint32_t kOffF4 = kOffWgt + 2048;      // f32[2][2][128] exp(c_R4 - c_
 constexpr uint32_t kOffConvW = kOffF4 + 2048;    // float4[128] conv taps of x
 constexpr uint32_t kOffConvB = kOffConvW + 16 * kPP;   // f32[128]
 constexpr uint32_t kOffMbar = kOffConvB + 4 * kPP;     // u64 mbarriers (see the kernel)
-constexpr uint32_t kOffTmem = kOffMbar + 128;    // u32 TMEM base
+constexpr uint32_t kOffTmem = kOffMbar + 192;    // u32 TMEM base
 constexpr uint32_t kOffDtBuf = kOffTmem + 16;    // [2][128] bf16x2: dt of both heads, by cp.async
 constexpr uint32_t kSmemUsed = kOffDtBuf + 2 * kQ * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;   // + alignment slack
@@ -348,6 +348,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     const uint32_t mb_bcfree = sbase + kOffMbar + 88;   // the chunk's products that read B/C done
     const uint32_t mb_sdone = sbase + kOffMbar + 104;   // the chunk's state product done (wX read)
     const uint32_t mb_s = sbase + kOffMbar + 96;     // state, its bf16 copy and wX ready (one arrival per group)
+    const uint32_t mb_yfree = sbase + kOffMbar + 112;   // Yd / Yo columns free for the chunk (last rows staged)
     auto xbuf_off = [](int k) { return (k & 1) ? kOffXbuf1 : kOffXbuf0; };
 
     auto chunk_of = [&](int k, int &t0, int &cnt, int &s0) {
@@ -494,6 +495,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         tc::mbar_init(mb_staged, 1);
         tc::mbar_init(mb_bcfree, 1);
         tc::mbar_init(mb_sdone, 1);
+        tc::mbar_init(mb_yfree, 1);
         issue_x(0);
         if (nk > 1) issue_x(1);
         issue_bc(0);
@@ -548,7 +550,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                                  idS, 1);
                 if constexpr (!kStateOnly) {
                     tc::mma_commit(mb_sdone);   // wX may be rewritten once it completes
-                    // Yo = C S_in^T (both heads)
+                    // Yo = C S_in^T (both heads), once the last chunk's rows are out of TMEM
+                    pok = tc::mbar_wait_bounded(mb_yfree, k & 1, kWaitCycles);
+                    if (!pok) break;
+                    tc::fence_after_sync();
 #pragma unroll 1
                     for (int ks = 0; ks < kN / 16; ++ks) {
                         const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -926,21 +931,32 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 ok = a_wait(mb_e, (j - 1) & 1);   // chunk j-1's MMAs done
                 if (!ok) break;
                 tc::fence_after_sync();
+            }
+            if (j < nk) {
+                // the state for chunk j first: its product runs while the rows
+                // of chunk j-1 are read out
+                ok = a_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);   // chunk j's prefix sums and factors
+                if (!ok) break;
+                tc::fence_after_sync();
+                scale_state(j);
+                publish(mb_s, !kStateOnly);
+            }
+            if (j >= 1) {
                 if constexpr (!kStateOnly) {
                     stage_rows(j - 1);
                     tc::fence_proxy_async();   // the staged rows, for the publisher's TMA stores
-                    tc::fence_before_sync();   // TMEM reads done before the next chunk's MMAs
+                    tc::fence_before_sync();   // TMEM reads done before the next chunk's products
                     grp_sync(1);
-                    if (tid == 0) tc::mbar_arrive(mb_staged);
+                    if (tid == 0) {
+                        tc::mbar_arrive(mb_staged);
+                        if (j < nk) tc::mbar_arrive(mb_yfree);
+                    }
                 }
                 if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * ((j - 1) & 1));
                 if (j >= nk) break;
+            } else if (!kStateOnly && tid == 0) {
+                tc::mbar_arrive(mb_yfree);   // nothing staged before chunk 0
             }
-            ok = a_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);   // chunk j's prefix sums and factors
-            if (!ok) break;
-            tc::fence_after_sync();
-            scale_state(j);
-            publish(mb_s, !kStateOnly);
             if constexpr (!kStateOnly) {
                 ok = a_wait(mb_g, j & 1);
                 if (!ok) break;
