@@ -750,20 +750,24 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         auto build_m = [&](int k) {
             const int row = tc::no_hoist(tid & 127);   // (see no_hoist)
             const int par = k & 1;
-#pragma unroll 1
-            for (int jj = 0; jj < 2; ++jj) {
-                const int jb = 2 * h + jj;          // 32-slot block of s
-                const uint32_t col = tmem + lane_base + kColG + 32 * jb;
-                if (jb > quad) {                    // warp-uniform: all s > t
-                    uint32_t z[16];
+            // 16-slot units U = 2 jb + u (K-steps of Yd) of this quarter's rows:
+            // units past the quarter's own block are all zero (s > t); of the
+            // others, warp h takes factorised units h*quad .. h*quad+quad-1 and
+            // diagonal unit 2 quad + h, so both warps of a quarter carry the same
+            // load
+            {
+                uint32_t z[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) z[i] = 0u;
-                    tc::tmem_st16_nw(col, z);
-                    tc::tmem_st16_nw(col + 16, z);
-                    continue;
-                }
+                for (int i = 0; i < 16; ++i) z[i] = 0u;
 #pragma unroll 1
-                for (int u = 0; u < 2; ++u) {       // 16-slot unit = K-step 2 jb + u
+                for (int U = 2 * quad + 2 + h; U < 8; U += 2) tc::tmem_st16_nw(tmem + lane_base + kColG + 16 * U, z);
+            }
+#pragma unroll 1
+            for (int iu = 0; iu <= quad; ++iu) {
+                const int U = iu < quad ? h * quad + iu : 2 * quad + h;
+                const int jb = U >> 1, u = U & 1;   // 32-slot block of s, half of it
+                const uint32_t col = tmem + lane_base + kColG + 32 * jb;
+                {
                     uint32_t gu[16];
                     tc::tmem_ld16_nw(col + 16 * u, gu);
                     tc::tmem_wait_ld16(gu);
