@@ -145,16 +145,18 @@ def code_sha(text):
     return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
-def kernel_traffic(kernel_file):
-    """dram bytes per launch from the committed ncu summary, if it was taken
-    on the current code of the kernel (code_sha recorded there); else None."""
+def kernel_traffic(kernel_file, workload):
+    """dram bytes per timed call (the launches the kernel events bracket) of
+    this workload from the committed ncu summary, if it was taken on the
+    current code of the kernel (code_sha recorded there); else None."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     src = os.path.join(ROOT, "bidirectional_mamba_ssm_b200", "csrc", kernel_file)
     try:
         sha = code_sha(open(src).read())
         for line in open(path):
             parts = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
-            if parts.get("file") == kernel_file and parts.get("code_sha") == sha:
+            if (parts.get("file") == kernel_file and parts.get("workload") == workload
+                    and parts.get("code_sha") == sha):
                 return float(parts["dram_bytes_per_launch"])
     except OSError:
         pass
@@ -229,7 +231,7 @@ def tensor_peak(peaks, clocks):
     return burst, "burst: no sw_power_cap in the clock samples"
 
 
-def roofline(peaks, peak_kind, clocks, nbytes, flops, kernel_s, decode, kernel_file):
+def roofline(peaks, peak_kind, clocks, nbytes, flops, kernel_s, decode, kernel_file, workload=None):
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     tpeak, rule = tensor_peak(peaks, clocks)
     t_tc = flops / (tpeak * 1e12)
@@ -240,7 +242,7 @@ def roofline(peaks, peak_kind, clocks, nbytes, flops, kernel_s, decode, kernel_f
         roof = {"bound": "tensor", "achieved": flops / kernel_s / 1e12, "peak": tpeak,
                 "unit": "TFLOP/s", "peak_source": f"{peak_kind} ({rule})"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = kernel_traffic(kernel_file)
+    roof["traffic"] = kernel_traffic(kernel_file, workload)
     roof["kernel"] = kernel_file
     ctx = {"achieved_gbs": nbytes / kernel_s / 1e9, "peak_gbs": peaks["hbm_gbs"],
            "frac": nbytes / kernel_s / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
@@ -478,7 +480,7 @@ def measure(args, lib, I, name, rank, world, dev, gpu_id, want_e2e=True):
         (nbytes, flops), _ = gemm_counts(w, batch * seqlen)
         kernel_file = "gemm_tc.cu"
     roof, ctx = roofline(peaks, peak_kind, clocks, nbytes, flops, per_call_ms / 1e3, decode,
-                         kernel_file)
+                         kernel_file, name)
     if name == "decode":
         wl = (f"cached block decode: {batch} streams x {seqlen}-token block, H64x64 N128 bf16, "
               f"65536-token prefix state")

@@ -33,15 +33,18 @@ def test_code_hash_ignores_comments_and_whitespace_only():
 
 
 def test_traffic_record_applies_only_to_the_code_it_was_taken_on():
-    """The bench reports the committed DRAM traffic only while the kernel's
-    code (comments aside) is the one the capture was taken on; otherwise
-    traffic is null."""
-    src = open(os.path.join(ROOT, "bidirectional_mamba_ssm_b200", "csrc", "ssd_tc.cu")).read()
-    line = open(os.path.join(ROOT, "profiles", "traffic.txt")).read()
-    parts = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
-    want = float(parts["dram_bytes_per_launch"]) if parts["code_sha"] == bench.code_sha(src) else None
-    assert bench.kernel_traffic("ssd_tc.cu") == want
-    assert bench.kernel_traffic("no_such_kernel.cu") is None
+    """The bench reports the committed DRAM traffic of a workload only while
+    the kernel's code (comments aside) is the one the capture was taken on;
+    otherwise traffic is null."""
+    lines = [l for l in open(os.path.join(ROOT, "profiles", "traffic.txt")) if l.strip()]
+    assert lines
+    for line in lines:
+        parts = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        src = open(os.path.join(ROOT, "bidirectional_mamba_ssm_b200", "csrc", parts["file"])).read()
+        want = float(parts["dram_bytes_per_launch"]) if parts["code_sha"] == bench.code_sha(src) else None
+        assert bench.kernel_traffic(parts["file"], parts["workload"]) == want
+        assert bench.kernel_traffic(parts["file"], "no_such_workload") is None
+    assert bench.kernel_traffic("no_such_kernel.cu", "layer1p3b") is None
 
 
 def test_tensor_peak_follows_the_sampled_clocks():
