@@ -37,15 +37,18 @@ namespace {
 constexpr int kBQ = 64;          // chunk length of the backward
 constexpr int kBThreads = 256;
 
-// C (M x N) = sum_k a(m, k) b(k, n) over the CTA's 256 threads, TM x TN
-// output tiles per thread; `put(m0, n0, acc)` stores a tile.
+// C (M x N) = sum_k a(m, k) b(k, n) over the CTA's 256 threads.  A thread
+// owns rows m0 .. m0+TM-1 and the TN columns n0 + j cs (cs = N / TN), so
+// that the threads of a warp read consecutive columns of b (no bank
+// conflicts on a row-major b); `put(m0, n0, cs, acc)` stores the tile,
+// acc[i][j] being element (m0 + i, n0 + j cs).
 template <int TM, int TN, typename FA, typename FB, typename FP>
 __device__ __forceinline__ void mm(int M, int N, int K, FA a, FB b, FP put)
 {
-    const int tn = N / TN;
-    const int ntiles = (M / TM) * tn;
+    const int cs = N / TN;
+    const int ntiles = (M / TM) * cs;
     for (int tile = threadIdx.x; tile < ntiles; tile += kBThreads) {
-        const int m0 = (tile / tn) * TM, n0 = (tile % tn) * TN;
+        const int m0 = (tile / cs) * TM, n0 = tile % cs;
         float acc[TM][TN];
 #pragma unroll
         for (int i = 0; i < TM; ++i)
@@ -56,13 +59,13 @@ __device__ __forceinline__ void mm(int M, int N, int K, FA a, FB b, FP put)
 #pragma unroll
             for (int i = 0; i < TM; ++i) av[i] = a(m0 + i, k);
 #pragma unroll
-            for (int j = 0; j < TN; ++j) bv[j] = b(k, n0 + j);
+            for (int j = 0; j < TN; ++j) bv[j] = b(k, n0 + j * cs);
 #pragma unroll
             for (int i = 0; i < TM; ++i)
 #pragma unroll
                 for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
-        put(m0, n0, acc);
+        put(m0, n0, cs, acc);
     }
 }
 
@@ -106,7 +109,7 @@ static size_t bwd_smem_floats(int P, int N)
            + (size_t)P * N          // dS
            + 2 * kBQ * kBQ          // W, T
            + 2 * kBQ * N            // X dS, dY S_in
-           + 8 * kBQ + 64;          // per-slot vectors, reductions
+           + 9 * kBQ + 64;          // per-slot vectors, reductions
 }
 
 static size_t bwd_state_smem_floats(int P, int N)
@@ -179,10 +182,10 @@ bwd_state_kernel(const BwdParams p)
         // S = e^{c_last} S + X^T B  (P x N, K = Q)
         mm<4, 4>(P, N, kBQ, [&](int m, int kk) { return X[kk * P + m]; },
                  [&](int kk, int n) { return Bs[kk * N + n]; },
-                 [&](int m0, int n0, float (&acc)[4][4]) {
+                 [&](int m0, int n0, int cs, float (&acc)[4][4]) {
                      for (int i = 0; i < 4; ++i)
                          for (int j = 0; j < 4; ++j) {
-                             float &s = S[(m0 + i) * N + n0 + j];
+                             float &s = S[(m0 + i) * N + n0 + j * cs];
                              s = fmaf(al, s, acc[i][j]);
                          }
                  });
@@ -215,7 +218,16 @@ bwd_scan_kernel(const BwdParams p)
     float *ddt = csum + kBQ;          // [Q] direct dt terms
     float *dc = ddt + kBQ;            // [Q] dL/dc
     float *U = dc + kBQ;              // [Q]
-    float *red = U + kBQ;             // reductions (+ 2 * kBQ spare)
+    float *ecv = U + kBQ;             // [Q] e^{c_t} (0 past the chunk end)
+    float *red = ecv + kBQ;           // reductions (+ 2 * kBQ spare)
+    // X, B and dS are also read down their columns (by consecutive threads):
+    // element (r, c) of each is stored at column c ^ (r & m) of row r, m + 1
+    // = the largest power of two (at most 32) dividing the row length, so
+    // that the column stays in its row and both rows and columns spread over
+    // the banks
+    const int mP = min(P & -P, 32) - 1, mN = min(N & -N, 32) - 1;
+    auto swx = [mP](int r, int c) { return c ^ (r & mP); };   // X [Q][P]
+    auto sw = [mN](int r, int c) { return c ^ (r & mN); };    // B [Q][N], dS [P][N]
     const void *act = rev ? p.act[1] : p.act[0];
     float *dact = rev ? p.dact[1] : p.dact[0];
     const size_t pn = (size_t)P * N;
@@ -223,7 +235,7 @@ bwd_scan_kernel(const BwdParams p)
     const float Ah = p.A[h], Dh = p.D[h];
     const int tid = threadIdx.x, lane = tid & 31;
     float dA_acc = 0.0f, dD_acc = 0.0f;
-    for (int i = tid; i < P * N; i += kBThreads) dS[i] = 0.0f;
+    for (int i = tid; i < P * N; i += kBThreads) dS[i] = 0.0f;   // (zero in any layout)
     for (int k = p.nchunks - 1; k >= 0; --k) {
         const int s0 = k * kBQ, cnt = min(kBQ, L - s0);
         const float *Sin = states + (size_t)k * pn;   // read from L2
@@ -237,7 +249,7 @@ bwd_scan_kernel(const BwdParams p)
                 xv = ldv<T>(act, ti * ch + h * P + q);
                 gv = ldv<T>(p.dy, ti * (size_t)H * P + h * P + q);
             }
-            X[i] = xv;
+            X[j * P + swx(j, q)] = xv;
             dY[i] = gv;
         }
         for (int i = tid; i < kBQ * N; i += kBThreads) {
@@ -248,7 +260,7 @@ bwd_scan_kernel(const BwdParams p)
                 bv = ldv<T>(act, ti * ch + H * P + n);
                 cv = ldv<T>(act, ti * ch + H * P + N + n);
             }
-            Bs[i] = bv;
+            Bs[j * N + sw(j, n)] = bv;
             Cs[i] = cv;
         }
         if (tid < kBQ) {
@@ -276,29 +288,29 @@ bwd_scan_kernel(const BwdParams p)
         const float clast = cvec[cnt - 1];
         // ---- CB = C B^T, DYX = dY X^T (Q x Q), then W, T and the sums of their products
         mm<4, 4>(kBQ, kBQ, N, [&](int t, int n) { return Cs[t * N + n]; },
-                 [&](int n, int s) { return Bs[s * N + n]; },
-                 [&](int t0, int u0, float (&acc)[4][4]) {
+                 [&](int n, int s) { return Bs[s * N + sw(s, n)]; },
+                 [&](int t0, int u0, int cs, float (&acc)[4][4]) {
                      for (int i = 0; i < 4; ++i)
-                         for (int j = 0; j < 4; ++j) Wm[(t0 + i) * kBQ + u0 + j] = acc[i][j];
+                         for (int j = 0; j < 4; ++j) Wm[(t0 + i) * kBQ + u0 + j * cs] = acc[i][j];
                  });
         mm<4, 4>(kBQ, kBQ, P, [&](int t, int q) { return dY[t * P + q]; },
-                 [&](int q, int s) { return X[s * P + q]; },
-                 [&](int t0, int u0, float (&acc)[4][4]) {
+                 [&](int q, int s) { return X[s * P + swx(s, q)]; },
+                 [&](int t0, int u0, int cs, float (&acc)[4][4]) {
                      for (int i = 0; i < 4; ++i)
-                         for (int j = 0; j < 4; ++j) Tm[(t0 + i) * kBQ + u0 + j] = acc[i][j];
+                         for (int j = 0; j < 4; ++j) Tm[(t0 + i) * kBQ + u0 + j * cs] = acc[i][j];
                  });
         // ---- X dS and dY S_in (Q x N, K = P)
-        mm<2, 4>(kBQ, N, P, [&](int s, int q) { return X[s * P + q]; },
-                 [&](int q, int n) { return dS[q * N + n]; },
-                 [&](int m0, int n0, float (&acc)[2][4]) {
+        mm<2, 4>(kBQ, N, P, [&](int s, int q) { return X[s * P + swx(s, q)]; },
+                 [&](int q, int n) { return dS[q * N + sw(q, n)]; },
+                 [&](int m0, int n0, int cs, float (&acc)[2][4]) {
                      for (int i = 0; i < 2; ++i)
-                         for (int j = 0; j < 4; ++j) XdS[(m0 + i) * N + n0 + j] = acc[i][j];
+                         for (int j = 0; j < 4; ++j) XdS[(m0 + i) * N + n0 + j * cs] = acc[i][j];
                  });
         mm<2, 4>(kBQ, N, P, [&](int t, int q) { return dY[t * P + q]; },
                  [&](int q, int n) { return Sin[q * N + n]; },
-                 [&](int m0, int n0, float (&acc)[2][4]) {
+                 [&](int m0, int n0, int cs, float (&acc)[2][4]) {
                      for (int i = 0; i < 2; ++i)
-                         for (int j = 0; j < 4; ++j) dYS[(m0 + i) * N + n0 + j] = acc[i][j];
+                         for (int j = 0; j < 4; ++j) dYS[(m0 + i) * N + n0 + j * cs] = acc[i][j];
                  });
         __syncthreads();
         // element (t, s), s <= t: e = e^{c_t - c_s}, W = CB e dt_s, T = DYX e dt_s;
@@ -327,11 +339,12 @@ bwd_scan_kernel(const BwdParams p)
         for (int j = tid; j < kBQ; j += kBThreads) {
             float xb = 0.0f, cs = 0.0f;
             for (int n = 0; n < N; ++n) {
-                xb = fmaf(XdS[j * N + n], Bs[j * N + n], xb);
+                xb = fmaf(XdS[j * N + n], Bs[j * N + sw(j, n)], xb);
                 cs = fmaf(Cs[j * N + n], dYS[j * N + n], cs);
             }
             const bool in = j < cnt;
             const float el = in ? expf(clast - cvec[j]) : 0.0f;
+            ecv[j] = in ? expf(cvec[j]) : 0.0f;
             U[j] = el * dtv[j] * xb;
             dc[j] = in ? expf(cvec[j]) * cs - U[j] : 0.0f;
             red[kBQ + j] = el * xb;   // direct dt term of the state
@@ -340,20 +353,23 @@ bwd_scan_kernel(const BwdParams p)
         // ---- dX = W^T dY + D dY + w o (B dS^T)   (Q x P)
         mm<2, 4>(kBQ, P, kBQ, [&](int s, int t) { return Wm[t * kBQ + s]; },
                  [&](int t, int q) { return dY[t * P + q]; },
-                 [&](int m0, int q0, float (&acc)[2][4]) {
+                 [&](int m0, int q0, int cs, float (&acc)[2][4]) {
                      for (int i = 0; i < 2; ++i) {
                          const int s = m0 + i;
                          if (s >= cnt) continue;
                          float bds[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                          for (int n = 0; n < N; ++n) {
-                             const float bv = Bs[s * N + n];
+                             const float bv = Bs[s * N + sw(s, n)];
 #pragma unroll
-                             for (int j = 0; j < 4; ++j) bds[j] = fmaf(bv, dS[(q0 + j) * N + n], bds[j]);
+                             for (int j = 0; j < 4; ++j) {
+                                 const int q = q0 + j * cs;
+                                 bds[j] = fmaf(bv, dS[q * N + sw(q, n)], bds[j]);
+                             }
                          }
                          const float wl = expf(clast - cvec[s]) * dtv[s];
                          const size_t ti = (size_t)b * L + tok_of(s);
                          for (int j = 0; j < 4; ++j) {
-                             const int q = q0 + j;
+                             const int q = q0 + j * cs;
                              dact[ti * ch + h * P + q] = acc[i][j] + Dh * dY[s * P + q] + wl * bds[j];
                          }
                      }
@@ -361,34 +377,38 @@ bwd_scan_kernel(const BwdParams p)
         // ---- dB = T^T C + w o (X dS);  dC = T B + e^c o (dY S_in)   (Q x N, summed over heads)
         mm<2, 4>(kBQ, N, kBQ, [&](int s, int t) { return Tm[t * kBQ + s]; },
                  [&](int t, int n) { return Cs[t * N + n]; },
-                 [&](int m0, int n0, float (&acc)[2][4]) {
+                 [&](int m0, int n0, int cs, float (&acc)[2][4]) {
                      for (int i = 0; i < 2; ++i) {
                          const int s = m0 + i;
                          if (s >= cnt) continue;
                          const float wl = expf(clast - cvec[s]) * dtv[s];
                          const size_t ti = (size_t)b * L + tok_of(s);
-                         for (int j = 0; j < 4; ++j)
-                             atomicAdd(dact + ti * ch + H * P + n0 + j, acc[i][j] + wl * XdS[s * N + n0 + j]);
+                         for (int j = 0; j < 4; ++j) {
+                             const int n = n0 + j * cs;
+                             atomicAdd(dact + ti * ch + H * P + n, acc[i][j] + wl * XdS[s * N + n]);
+                         }
                      }
                  });
         mm<2, 4>(kBQ, N, kBQ, [&](int t, int s) { return Tm[t * kBQ + s]; },
-                 [&](int s, int n) { return Bs[s * N + n]; },
-                 [&](int m0, int n0, float (&acc)[2][4]) {
+                 [&](int s, int n) { return Bs[s * N + sw(s, n)]; },
+                 [&](int m0, int n0, int cs, float (&acc)[2][4]) {
                      for (int i = 0; i < 2; ++i) {
                          const int t = m0 + i;
                          if (t >= cnt) continue;
-                         const float ec = expf(cvec[t]);
+                         const float ec = ecv[t];
                          const size_t ti = (size_t)b * L + tok_of(t);
-                         for (int j = 0; j < 4; ++j)
-                             atomicAdd(dact + ti * ch + H * P + N + n0 + j, acc[i][j] + ec * dYS[t * N + n0 + j]);
+                         for (int j = 0; j < 4; ++j) {
+                             const int n = n0 + j * cs;
+                             atomicAdd(dact + ti * ch + H * P + N + n, acc[i][j] + ec * dYS[t * N + n]);
+                         }
                      }
                  });
         // ---- dL/dc, then dt (suffix sums), A and D
         float sdS = 0.0f;   // <dS, S_in>
-        for (int i = tid; i < P * N; i += kBThreads) sdS = fmaf(dS[i], Sin[i], sdS);
+        for (int i = tid; i < P * N; i += kBThreads) sdS = fmaf(dS[(i / N) * N + sw(i / N, i % N)], Sin[i], sdS);
         sdS = block_sum(sdS, red);
         float dd = 0.0f;
-        for (int i = tid; i < cnt * P; i += kBThreads) dd = fmaf(dY[i], X[i], dd);
+        for (int i = tid; i < cnt * P; i += kBThreads) dd = fmaf(dY[i], X[(i / P) * P + swx(i / P, i % P)], dd);
         dD_acc += block_sum(dd, red);
         if (tid == 0) {
             float usum = 0.0f;
@@ -409,12 +429,13 @@ bwd_scan_kernel(const BwdParams p)
         __syncthreads();   // every product that reads dS is done
         // ---- dS_in = e^{c_last} dS + (e^c o dY)^T C   (P x N, K = Q), in place
         const float al = expf(clast);
-        mm<4, 4>(P, N, kBQ, [&](int q, int t) { return t < cnt ? expf(cvec[t]) * dY[t * P + q] : 0.0f; },
+        mm<4, 4>(P, N, kBQ, [&](int q, int t) { return ecv[t] * dY[t * P + q]; },
                  [&](int t, int n) { return Cs[t * N + n]; },
-                 [&](int q0, int n0, float (&acc)[4][4]) {
+                 [&](int q0, int n0, int cs, float (&acc)[4][4]) {
                      for (int i = 0; i < 4; ++i)
                          for (int j = 0; j < 4; ++j) {
-                             float &v = dS[(q0 + i) * N + n0 + j];
+                             const int q = q0 + i, n = n0 + j * cs;
+                             float &v = dS[q * N + sw(q, n)];
                              v = fmaf(al, v, acc[i][j]);
                          }
                  });
@@ -425,7 +446,8 @@ bwd_scan_kernel(const BwdParams p)
         atomicAdd(p.dD + h, dD_acc);
     }
     if (!rev && p.dinit)
-        for (int i = tid; i < P * N; i += kBThreads) p.dinit[((size_t)b * H + h) * pn + i] = dS[i];
+        for (int i = tid; i < P * N; i += kBThreads)
+            p.dinit[((size_t)b * H + h) * pn + i] = dS[(i / N) * N + sw(i / N, i % N)];
 }
 
 // Conv backward of both streams for one (sequence, channel, token tile):
