@@ -55,7 +55,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["long131k", "layer1p3b", "decode", "decode_pool",
-                                           "untied1p3b", "mixer1p3b", "sweep"],
+                                           "untied1p3b", "mixer1p3b", "sweep", "tiny",
+                                           "backward1p3b"],
                     default="long131k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
@@ -82,6 +83,10 @@ def workload_spec(name):
         return I.LAYER_1P3B, I.LAYER_1P3B.batch, I.LAYER_1P3B.seqlen
     if name == "sweep":   # one sequence, prefill at 1k..256k tokens; the line's value at 256k
         return I.LONG_131K, 1, SWEEP_LENGTHS[-1]
+    if name == "backward1p3b":   # gradients of the mixer core at the 1.3B-layer shape
+        return I.LAYER_1P3B, I.LAYER_1P3B.batch, I.LAYER_1P3B.seqlen
+    if name == "tiny":   # the small fp32 case (b1 L256 H4x32 N16): launch-bound, latency is the figure
+        return I.TINY_F32, 1, I.TINY_F32.seqlen
     raise ValueError(name)
 
 
@@ -123,6 +128,21 @@ def algorithmic(w, batch, seqlen, decode=False, untied=False):
         nbytes += batch * (H * P * N * 4 + 4 * (H * P + 2 * N) * esz)
     Q = 64
     flops = 2 * (2 * Q * N + H * (Q * P + 4 * P * N)) * tokens
+    return nbytes, flops
+
+
+def backward_counts(w, tokens):
+    """Algorithmic bytes and flops of one backward call of the mixer core.
+    bytes: raw xBC, dt and dy read (bf16), d(xBC) and d(dt) written (fp32).
+    flops: the adjoint's products per chunk of Q = 64 and per direction and
+    head -- C.B^T, dY.X^T (Q^2 N, Q^2 P), X.dS, dY.S_in (Q P N each), W^T.dY
+    (Q^2 P), B.dS^T (Q N P), T^T.C, T.B (Q^2 N each), the state adjoint (P N Q)
+    -- i.e. Q(3N + 2P) + 5PN multiply-adds per token, head and direction."""
+    H, P, N = w.heads, w.headdim, w.d_state
+    Q = 64
+    ch = H * P + 2 * N
+    nbytes = tokens * (2 * (ch + H + H * P) + 4 * (ch + H))
+    flops = tokens * 2 * 2 * H * (Q * (3 * N + 2 * P) + 5 * P * N)
     return nbytes, flops
 
 
@@ -303,10 +323,11 @@ def build_step(lib, I, w, name, batch, seqlen, rank, dev):
     decode = name == "decode"
     untied = name == "untied1p3b"
     g = I.make_inputs(w, seed=rank, device=dev, seqlen=seqlen, batch=batch,
-                      conv_bias=name in ("decode", "decode_pool"))
+                      conv_bias=name in ("decode", "decode_pool", "backward1p3b"))
     gr = I.make_inputs(w, seed=10000 + rank, device=dev, seqlen=seqlen, batch=batch) if untied else None
-    y = torch.empty((batch, seqlen, (2 if untied else 1) * H * P), dtype=torch.bfloat16, device=dev)
-    dims = lib.make_dims(batch, seqlen, H, P, N, torch.bfloat16)
+    adt = I.torch_dtype(w.dtype)
+    y = torch.empty((batch, seqlen, (2 if untied else 1) * H * P), dtype=adt, device=dev)
+    dims = lib.make_dims(batch, seqlen, H, P, N, adt)
     ws = lib.new_workspace(dims, device=dev)
     extra = {}
 
@@ -368,6 +389,20 @@ def build_step(lib, I, w, name, batch, seqlen, rank, dev):
             lib.bimamba_ssd_fwd_rev(xbc, dtv, g["A"], g["D"], g["conv_w"], None, None, None, y, ws,
                                     heads=H, headdim=P, d_state=N)
             lib.bimamba_out_proj(y.view(tokens, H * P), pr["w_out"], out)
+    elif name == "backward1p3b":
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(7 + rank)
+        dyv = torch.randn((batch, seqlen, H * P), generator=gen, device=dev).to(torch.bfloat16)
+        bws = torch.empty(max(256, lib.bimamba_backward_workspace_bytes(dims)), dtype=torch.uint8,
+                          device=dev)
+        extra.update(dy=dyv, bws=bws)
+
+        def step(ev=None):
+            hook(ev)   # the chunked adjoint kernel is the roofline's kernel
+            lib.bimamba_ssd_fwd_rev_backward(g["xbc"], g["dt"], g["A"], g["D"], g["conv_w"],
+                                             g["conv_b"], None, dyv, heads=H, headdim=P,
+                                             d_state=N, workspace=bws)
+            hook(None)
     elif untied:
         def step(ev=None):
             hook(ev)
@@ -481,6 +516,18 @@ def measure(args, lib, I, name, rank, world, dev, gpu_id, want_e2e=True):
         kernel_file = "gemm_tc.cu"
     roof, ctx = roofline(peaks, peak_kind, clocks, nbytes, flops, per_call_ms / 1e3, decode,
                          kernel_file, name)
+    if name == "backward1p3b":
+        # CUDA-core fp32 products: held against the fp32 FMA peak at the sampled clock
+        nbytes, flops = backward_counts(w, batch * seqlen)
+        mhz = clocks["sm_mhz"] if clocks else 1965.0
+        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        ach = flops / (per_call_ms / 1e3) / 1e12
+        roof = {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "peak_source": f"fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x {mhz:.0f} MHz "
+                               f"(sampled SM clock)", "frac": ach / peak, "traffic": None,
+                "kernel": "backward.cu"}
+        ctx = {"achieved_gbs": nbytes / (per_call_ms / 1e3) / 1e9, "algorithmic_bytes": nbytes,
+               "algorithmic_flops": flops, "note": "whole call: conv, state pass, adjoint, conv backward"}
     if name == "decode":
         wl = (f"cached block decode: {batch} streams x {seqlen}-token block, H64x64 N128 bf16, "
               f"65536-token prefix state")
@@ -495,13 +542,25 @@ def measure(args, lib, I, name, rank, world, dev, gpu_id, want_e2e=True):
         wl = (w.name + f", with its projections: in {D_MODEL}->{w.channels}+{H} (softplus dt), "
               f"mixer core, out {H * P}->{D_MODEL}")
         l2 = "inputs larger than L2"
+    elif name == "backward1p3b":
+        wl = (w.name + ", backward of the mixer core: gradients of xBC, dt, A, D, conv taps and "
+              "bias from dy")
+        l2 = "inputs larger than L2"
+    elif name == "tiny":
+        wl = w.name + " (launch-bound: the figure is the call's latency, not a roofline fraction)"
+        l2 = "L2-resident (0.3 MB per call)"
+        roof["note"] = "launch-bound small case: report latency (latency_us), no roofline claim"
     else:
         wl = w.name + (", untied directions, outputs concatenated" if untied else "")
         l2 = "inputs larger than L2 (xbc + y per step > 126 MB)"
     out = {"value": value, "ms_per_step": ms_step, "workload": wl, "batch_per_gpu": batch,
            "seqlen": seqlen, "l2": l2, "roofline": roof, "roofline_hbm_context": ctx,
            "clocks": clocks, "gpu_launches": launches, "main_kernel_ms": per_call_ms}
-    if want_e2e:
+    if name == "tiny":
+        out["latency_us"] = {"call": ms_step * 1e3, "kernel": per_call_ms * 1e3}
+    if want_e2e and name == "backward1p3b":
+        out["e2e"] = run_e2e_backward(args, lib, w, g, extra, dev)
+    elif want_e2e:
         out["e2e"] = run_e2e(args, lib, w, name, g, batch, seqlen, dims, ws, extra, dev, world, gr)
     del step, g, gr, ws, extra
     torch.cuda.empty_cache()
@@ -532,7 +591,7 @@ def run_ours(args, world):
     result = {
         "metric": METRIC, "value": m["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_per_step"],
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic",
         "config": {"workload": m["workload"], "batch_per_gpu": m["batch_per_gpu"],
                    "seqlen": m["seqlen"], "heads": w.heads, "headdim": w.headdim,
@@ -541,6 +600,8 @@ def run_ours(args, world):
         "roofline": m["roofline"], "roofline_hbm_context": m["roofline_hbm_context"],
         "e2e": m["e2e"], "clocks": m["clocks"], "gpu_launches": m["gpu_launches"],
     }
+    if "latency_us" in m:
+        result["latency_us"] = m["latency_us"]
     if args.workload == "long131k" and args.batch is None:
         # the 1.3B-layer workload (b8 x L4096) measured in the same run
         lm = measure(args, lib, I, "layer1p3b", rank, world, dev, gpu_id, want_e2e=False)
@@ -632,6 +693,41 @@ def run_sweep(args, lib, w, dev, rank, gpu_id):
     return rows
 
 
+def run_e2e_backward(args, lib, w, g, extra, dev):
+    """The backward through the public API from pinned host buffers: every
+    step uploads xBC, dt and dy, runs the call and reads d(xBC) back (one
+    stream, not pipelined)."""
+    import torch
+    H, P, N = w.heads, w.headdim, w.d_state
+    hin = [t.cpu().pin_memory() for t in (g["xbc"], g["dt"], extra["dy"])]
+    din = [torch.empty_like(t, device=dev) for t in hin]
+    hout = torch.empty(g["xbc"].shape, dtype=torch.float32).pin_memory()
+
+    def step():
+        for dst, src in zip(din, hin):
+            dst.copy_(src, non_blocking=True)
+        gr = lib.bimamba_ssd_fwd_rev_backward(din[0], din[1], g["A"], g["D"], g["conv_w"], g["conv_b"],
+                                              None, din[2], heads=H, headdim=P, d_state=N,
+                                              workspace=extra["bws"])
+        hout.copy_(gr["xbc"], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, args.e2e_steps)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    tokens = g["xbc"].shape[0] * g["xbc"].shape[1]
+    return {"value": tokens / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
+            "d2h_bytes_per_step": hout.numel() * hout.element_size(), "ms_per_step": ms}
+
+
 def run_e2e(args, lib, w, name, g, batch, seqlen, dims, ws, extra, dev, world, gr=None):
     """Same metric through the public API from pinned HOST buffers.  Every step
     copies its inputs host->device (the raw xbc and dt of each stream; the
@@ -659,9 +755,10 @@ def run_e2e(args, lib, w, name, g, batch, seqlen, dims, ws, extra, dev, world, g
         pool = I_make_pool(w, dev)
         slot_sets = [torch.arange(i * batch, (i + 1) * batch, dtype=torch.int32, device=dev)
                      for i in range(POOL_STREAMS // batch)]
-    hy = torch.empty(out_shape, dtype=torch.bfloat16).pin_memory()
+    odt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    hy = torch.empty(out_shape, dtype=odt).pin_memory()
     din = [[torch.empty_like(t, device=dev) for t in hin] for _ in range(2)]
-    dy = [torch.empty(out_shape, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dy = [torch.empty(out_shape, dtype=odt, device=dev) for _ in range(2)]
     wss = [ws, lib.new_workspace(dims, device=dev)]
     s_up, s_run, s_down = (torch.cuda.Stream(device=dev) for _ in range(3))
     up_done = [torch.cuda.Event() for _ in range(2)]
@@ -746,7 +843,8 @@ def oracle_sample_step(w, workload, seq_tokens, seed=0):
     import oracle
     from bidirectional_mamba_ssm_b200 import inputs as I
     decode = workload in ("decode", "decode_pool")
-    cpu = I.make_inputs(w, seed=seed, seqlen=seq_tokens, batch=1, conv_bias=decode)
+    cpu = I.make_inputs(w, seed=seed, seqlen=seq_tokens, batch=1,
+                        conv_bias=decode or workload == "backward1p3b")
     n = {k: (None if v is None else v.float().double().numpy()) for k, v in cpu.items()}
     kw = dict(heads=w.heads, headdim=w.headdim, d_state=w.d_state)
     if workload == "untied1p3b":
@@ -762,6 +860,10 @@ def oracle_sample_step(w, workload, seq_tokens, seed=0):
         xbc, dt = oracle.in_proj(pr["u"], pr["w_in"], pr["dt_bias"], **kw)
         y = oracle.bimamba(xbc[None], dt[None], n["A"], n["D"], n["conv_w"], None, **kw)
         oracle.out_proj(y[0], pr["w_out"])
+    elif workload == "backward1p3b":
+        dy = np.random.default_rng(seed).standard_normal((1, seq_tokens, w.heads * w.headdim))
+        oracle.bimamba_mixer_backward(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], n["conv_b"], dy,
+                                      **kw)
     elif decode:
         state = np.zeros((1, w.heads, w.headdim, w.d_state))
         tail = np.zeros((1, 4, w.channels))
@@ -776,7 +878,8 @@ def cpu_baseline(w, workload):
     """The oracle, as it stands, on host cores: whole sequences of the
     workload's length (capped at 4096 tokens) until ~10 s of CPU time."""
     import oracle
-    seq = 64 if workload in ("decode", "decode_pool") else 1024
+    seq = (64 if workload in ("decode", "decode_pool", "backward1p3b")
+           else (256 if workload == "tiny" else 1024))
     tokens, secs, reps = 0, 0.0, 0
     while secs < 10.0 and reps < 64:
         secs += oracle_sample_step(w, workload, seq, seed=reps)
@@ -794,7 +897,7 @@ def run_reference(args):
         return
     import oracle
     w, batch, seqlen = workload_spec(args.workload)
-    seq = 64 if args.workload in ("decode", "decode_pool") else 256
+    seq = 64 if args.workload in ("decode", "decode_pool", "backward1p3b") else 256
     for i in range(args.warmup):
         oracle_sample_step(w, args.workload, seq, seed=i)
     total = 0.0
@@ -813,7 +916,8 @@ def run_reference(args):
         "config": {"workload": {"decode": "cached block decode",
                                 "decode_pool": "pooled cached decode",
                                 "untied1p3b": w.name + ", untied directions, outputs concatenated",
-                                "mixer1p3b": w.name + ", with its in/out projections"}
+                                "mixer1p3b": w.name + ", with its in/out projections",
+                                "backward1p3b": w.name + ", backward of the mixer core"}
                    .get(args.workload, w.name),
                    "batch_per_gpu": batch, "seqlen": seqlen, "heads": w.heads,
                    "headdim": w.headdim, "d_state": w.d_state},
