@@ -2,7 +2,8 @@
 """Throughput of the bidirectional Mamba-2 mixer core on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload layer1p3b|long131k|decode|untied1p3b|sweep]
+                    [--workload long131k|layer1p3b|decode|decode_pool|untied1p3b|mixer1p3b|
+                                sweep|tiny|backward1p3b]
                     [--no-cpu-baseline]
 
 One step = one bimamba_ssd_fwd_rev call over one batch of the workload
