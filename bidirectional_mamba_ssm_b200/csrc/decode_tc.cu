@@ -82,7 +82,8 @@ constexpr uint32_t kDOffSf = kDOffX;
 constexpr uint32_t kDOffRawBox = 82944;
 constexpr uint32_t kDOffRaw = kDOffRawBox - 3 * 128;
 constexpr uint32_t kDOffCum = kDOffRawBox + kDQ * 128;   // f32 cf[64], cr[64], dtf[64], dtr[64]
-constexpr uint32_t kDOffConvW = kDOffCum + 1024;   // float4[64]
+constexpr uint32_t kDOffF8 = kDOffCum + 1024;     // f32 f8f[64], f8r[64]: exp(c_R - c_s) dt_s, R = s | 7
+constexpr uint32_t kDOffConvW = kDOffF8 + 512;     // float4[64]
 constexpr uint32_t kDOffConvB = kDOffConvW + 1024; // f32[64]
 constexpr uint32_t kDOffMbar = kDOffConvB + 256;   // 2 mbarriers
 constexpr uint32_t kDOffTmem = kDOffMbar + 16;
@@ -282,6 +283,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
     const bool do_commit = p.state_out && (!p.commit || p.commit[s] != 0);
     float *cf = reinterpret_cast<float *>(sm + kDOffCum);
     float *cr = cf + 64, *dtf = cf + 128, *dtr = cf + 192;
+    float *f8f = reinterpret_cast<float *>(sm + kDOffF8), *f8r = f8f + 64;
     float4 *convw = reinterpret_cast<float4 *>(sm + kDOffConvW);
     float *convb = reinterpret_cast<float *>(sm + kDOffConvB);
     const uint32_t mb_ld = sbase + kDOffMbar, mb_mma = mb_ld + 8;
@@ -347,6 +349,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
         dtf[2 * lane + 1] = d[1];
         dtr[2 * lane] = e[0];
         dtr[2 * lane + 1] = e[1];
+        __syncwarp();
+        // per-slot factors of the 8-slot groups (from the sums the other lanes wrote)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int j = 2 * lane + i;
+            f8f[j] = tc::exp2_approx(cf[j | 7] - cf[j]) * d[i];
+            f8r[j] = tc::exp2_approx(cr[j | 7] - cr[j]) * e[i];
+        }
     }
     // thread (r, half): stacked row r (TMEM lane) -- direction d = r >> 6,
     // walk slot t = r & 63 -- and the half of the 64 channels / slots it owns
@@ -474,21 +484,37 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
             const float4 v = grow[i];
             g[4 * i] = v.x; g[4 * i + 1] = v.y; g[4 * i + 2] = v.z; g[4 * i + 3] = v.w;
         }
+        // groups of 8 slots: exp(c_t - c_s) dt_s = exp(c_t - c_R) f8[s], R the group's
+        // last slot.  With the group's own decay at most 2^60 neither factor
+        // overflows where the element is kept (s <= t); else one exponential
+        // per element, each <= 1.  (The direction is uniform over a warp.)
         const float ct = cdir[t];
+        const float *f8dir = d ? f8r : f8f;
         uint32_t packed[16], zero[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float m2[2];
+        for (int g8 = 0; g8 < 4; ++g8) {
+            const int sb = 32 * half + 8 * g8;
+            float m[8];
+            if (cdir[sb] - cdir[sb + 7] <= 60.0f) {
+                const float et = tc::exp2_approx(ct - cdir[sb + 7]);
 #pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2) {
-                const int sl = 32 * half + 2 * i + e2;
-                const float gv = g[2 * i + e2];
-                const float m = (sl < t) ? gv * tc::exp2_approx(fminf(ct - cdir[sl], 0.0f)) * dtdir[sl]
-                                         : fmaf(gv, dtdir[t], Dh);
-                m2[e2] = (sl <= t && t < len) ? m : 0.0f;
+                for (int e = 0; e < 8; ++e) m[e] = g[8 * g8 + e] * et * f8dir[sb + e];
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    m[e] = g[8 * g8 + e] * tc::exp2_approx(fminf(ct - cdir[sb + e], 0.0f)) * dtdir[sb + e];
             }
-            packed[i] = tc::pack_bf16x2(m2[0], m2[1]);
-            zero[i] = 0u;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int sl = sb + e;
+                const float me = (sl == t) ? fmaf(g[8 * g8 + e], dtdir[t], Dh) : m[e];
+                m[e] = (sl <= t && t < len) ? me : 0.0f;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                packed[4 * g8 + q] = tc::pack_bf16x2(m[2 * q], m[2 * q + 1]);
+                zero[4 * g8 + q] = 0u;
+            }
         }
         tc::tmem_st16(tmem + lane_base + kDColM + 32 * d + 16 * half, packed);
         tc::tmem_st16(tmem + lane_base + kDColM + 32 * (1 - d) + 16 * half, zero);
