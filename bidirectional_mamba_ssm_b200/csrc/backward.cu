@@ -27,6 +27,8 @@
 //     on the CUDA cores out of shared memory;
 //  4. bwd_conv_kernel: each stream's dact through SiLU' and the transposed
 //     taps to d(xbc), plus the tap and bias gradients, both streams at once.
+#include <algorithm>
+
 #include "common.cuh"
 #include "dispatch.h"
 
@@ -518,7 +520,7 @@ size_t backward_workspace_bytes(const bimamba_dims &d)
     const size_t act = (2 * tokens * ch * esz + 255) & ~(size_t)255;
     const size_t dact = 2 * tokens * ch * sizeof(float);
     const size_t states = 2 * (size_t)d.batch * d.heads * nchunks * d.headdim * d.d_state * sizeof(float);
-    return act + dact + states;
+    return act + dact + std::max(states, backward_tc_supported(d) ? backward_tc_state_bytes(d) : (size_t)0);
 }
 
 template <typename T>
@@ -566,23 +568,44 @@ cudaError_t launch_backward_t(const BackwardProblem &q, cudaStream_t s)
                                      d.batch, d.len, ch, dir, 1, s)) != cudaSuccess)
             return e;
     }
-    const size_t smem = bwd_smem_floats(d.headdim, d.d_state) * sizeof(float);
-    const size_t smem_st = bwd_state_smem_floats(d.headdim, d.d_state) * sizeof(float);
-    if ((e = cudaFuncSetAttribute(bwd_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem_st)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(bwd_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem)) != cudaSuccess)
-        return e;
-    const dim3 grid(d.heads, d.batch, 2);
-    bwd_state_kernel<T><<<grid, kBThreads, smem_st, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    count_launch();
-    const TimingEvents ev = timing_events();
-    if (ev.start && (e = cudaEventRecord(ev.start, s)) != cudaSuccess) return e;
-    bwd_scan_kernel<T><<<grid, kBThreads, smem, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    count_launch();
-    if (ev.stop && (e = cudaEventRecord(ev.stop, s)) != cudaSuccess) return e;
+    if (backward_tc_supported(d)) {
+        // the state and adjoint passes on the tensor cores
+        BackwardTcProblem t{};
+        t.dims = d;
+        t.act[0] = p.act[0];
+        t.act[1] = p.act[1];
+        t.dt = q.dt;
+        t.dy = q.dy;
+        t.A = q.A;
+        t.D = q.D;
+        t.init = q.init;
+        t.dact[0] = p.dact[0];
+        t.dact[1] = p.dact[1];
+        t.ddt = q.ddt;
+        t.dA = q.dA;
+        t.dD = q.dD;
+        t.dinit = q.dinit;
+        t.states = p.states;
+        if ((e = launch_backward_tc(t, s)) != cudaSuccess) return e;
+    } else {
+        const size_t smem = bwd_smem_floats(d.headdim, d.d_state) * sizeof(float);
+        const size_t smem_st = bwd_state_smem_floats(d.headdim, d.d_state) * sizeof(float);
+        if ((e = cudaFuncSetAttribute(bwd_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem_st)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(bwd_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        const dim3 grid(d.heads, d.batch, 2);
+        bwd_state_kernel<T><<<grid, kBThreads, smem_st, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        count_launch();
+        const TimingEvents ev = timing_events();
+        if (ev.start && (e = cudaEventRecord(ev.start, s)) != cudaSuccess) return e;
+        bwd_scan_kernel<T><<<grid, kBThreads, smem, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        count_launch();
+        if (ev.stop && (e = cudaEventRecord(ev.stop, s)) != cudaSuccess) return e;
+    }
     bwd_conv_kernel<T><<<dim3((ch + 127) / 128, (d.len + 63) / 64, d.batch), 128, 0, s>>>(
         static_cast<const T *>(q.xbc), q.conv_w, q.conv_b, p.dact[0], p.dact[1], q.dxbc, q.dconv_w,
         q.dconv_b, d.len, ch);

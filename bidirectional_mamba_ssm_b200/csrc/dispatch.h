@@ -110,6 +110,23 @@ bool backward_supported(const bimamba_dims &d);
 size_t backward_workspace_bytes(const bimamba_dims &d);
 cudaError_t launch_backward(const BackwardProblem &q, cudaStream_t stream);
 
+// the state and adjoint passes of the backward on the tensor cores (bf16,
+// headdim 64, d_state 128): act = each stream's activated xBC, dact = its
+// fp32 gradient (x part written, B/C parts added; zeroed by the caller),
+// states = backward_tc_state_bytes of workspace
+struct BackwardTcProblem {
+    bimamba_dims dims;
+    const void *act[2];
+    const void *dt, *dy;
+    const float *A, *D, *init;
+    float *dact[2];
+    float *ddt, *dA, *dD, *dinit;
+    void *states;
+};
+bool backward_tc_supported(const bimamba_dims &d);
+size_t backward_tc_state_bytes(const bimamba_dims &d);
+cudaError_t launch_backward_tc(const BackwardTcProblem &q, cudaStream_t stream);
+
 template <typename T>
 cudaError_t launch_conv_silu(const void *u, void *out, const float *w, const float *bias,
                              const void *tail, int batch, int len, int ch, int rev, int silu,

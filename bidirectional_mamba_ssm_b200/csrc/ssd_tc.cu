@@ -150,6 +150,11 @@ struct TcParams {
     int seg_chunks;     // walk chunks per CTA
     int item_chunks;    // walk chunks per state-only item (0: no items)
     int nitems;
+    // whole walks of tied directions: the partner CTA reads x chunk c and adds
+    // to its y rows d = nchunks - 1 - 2k walk steps after this CTA (walk step
+    // k); the first touches with 0 < d <= keep_dist stay in L2 (evict_last),
+    // every other touch of x and y goes first (evict_first).  0: no hints.
+    int keep_dist;
     int len, H, ch, nchunks, batch;
 };
 
@@ -365,8 +370,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         chunk_of(k, t0, cnt, s0);
         const uint32_t mb = mb_x0 + 8 * (k & 1);
         tc::mbar_expect_tx(mb, kRawBytes);
-        tc::tma_load_3d(sbase + xbuf_off(k), rev ? &tm_x_r : &tm_x_f, hp * kPP, rev ? t0 : t0 - 3, b,
-                        mb);
+        const void *tm = rev ? &tm_x_r : &tm_x_f;
+        if (p.keep_dist == 0) {
+            tc::tma_load_3d(sbase + xbuf_off(k), tm, hp * kPP, rev ? t0 : t0 - 3, b, mb);
+        } else {
+            const int d = nk - 1 - 2 * k;   // walk steps until the partner reads the chunk
+            const uint64_t pol = (d > 0 && d <= p.keep_dist) ? tc::policy_evict_last() : tc::policy_evict_first();
+            tc::tma_load_3d_hint(sbase + xbuf_off(k), tm, hp * kPP, rev ? t0 : t0 - 3, b, mb, pol);
+        }
     };
     auto issue_bc = [&](int k) {
         int t0, cnt, s0;
@@ -629,9 +640,19 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 if (!qok) break;
                 const bool first = arrival == 0;
                 const uint32_t stg = sbase + xbuf_off(k);
+                // (whole walks) the partner adds to these rows |d| walk steps from now
+                const int d = nk - 1 - 2 * k;
+                const bool hint = p.keep_dist > 0;
+                const uint64_t pol = (first && abs(d) <= p.keep_dist) ? tc::policy_evict_last()
+                                                                      : tc::policy_evict_first();
                 if (first) {
-                    tc::tma_store_3d(&tm_y, stg, col0, t0, b);
-                    tc::tma_store_3d(&tm_y, stg + 16384, col0 + kP, t0, b);
+                    if (hint) {
+                        tc::tma_store_3d_hint(&tm_y, stg, col0, t0, b, pol);
+                        tc::tma_store_3d_hint(&tm_y, stg + 16384, col0 + kP, t0, b, pol);
+                    } else {
+                        tc::tma_store_3d(&tm_y, stg, col0, t0, b);
+                        tc::tma_store_3d(&tm_y, stg + 16384, col0 + kP, t0, b);
+                    }
                 } else {
                     // the partner CTA arrived first; wait (bounded) until its
                     // rows are visible, then add this CTA's to them at L2.  A
@@ -647,8 +668,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                     qok = ready;
                     if (!qok) break;
                     tc::fence_proxy_async_global();   // the acquire before the reductions
-                    tc::tma_reduce_add_3d(&tm_y, stg, col0, t0, b);
-                    tc::tma_reduce_add_3d(&tm_y, stg + 16384, col0 + kP, t0, b);
+                    if (hint) {
+                        tc::tma_reduce_add_3d_hint(&tm_y, stg, col0, t0, b, pol);
+                        tc::tma_reduce_add_3d_hint(&tm_y, stg + 16384, col0 + kP, t0, b, pol);
+                    } else {
+                        tc::tma_reduce_add_3d(&tm_y, stg, col0, t0, b);
+                        tc::tma_reduce_add_3d(&tm_y, stg + 16384, col0 + kP, t0, b);
+                    }
                 }
                 tc::bulk_commit();
                 tc::bulk_wait_read0();   // the staged rows have been read
@@ -1322,6 +1348,15 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
     p.seg_chunks = sp.seg_chunks;
     p.item_chunks = sp.item_chunks;
     p.nitems = sp.nitems;
+    // L2 residency between the two directions' touches of a chunk (whole walks,
+    // tied x, summed y): about 64 KB per kept chunk (its raw x and y rows),
+    // kept for at most keep_dist walk steps, by every co-resident head pair,
+    // within 100 MB of the 126 MB L2
+    p.keep_dist = 0;
+    if (sp.nseg == 1 && !pr.concat && xbc[0] == xbc[1]) {
+        const long long pairs = std::min<long long>(kPlanSMs / 2, (long long)d.batch * (d.heads / kHeads));
+        p.keep_dist = (int)std::min<long long>(p.nchunks, (100ll << 20) / (pairs * (64ll << 10)));
+    }
 
     // prepass: B/C conv+SiLU in walk order for both directions
     bc_prepass_kernel<<<dim3((d.len + 31) / 32, d.batch, 2), 128, 0, stream>>>(
@@ -1360,6 +1395,7 @@ cudaError_t launch_ssd_tc(const Problem &pr, cudaStream_t stream)
         q.seg_dec = pr.dec_out;
         q.nitems = 1;
         q.item_chunks = q.seg_chunks = p.nchunks;
+        q.keep_dist = 0;
         ssd_tc_kernel<true, false><<<dim3(d.heads, d.batch, 1), kThreads, kSmemBytes, stream>>>(
             tm_x_f, tm_x_r, tm_bc, tm_y, q);
         e = cudaGetLastError();
