@@ -135,8 +135,9 @@ def algorithmic(w, batch, seqlen, decode=False, untied=False):
 def backward_counts(w, tokens):
     """Algorithmic bytes and flops of one backward call of the mixer core.
     bytes: raw xBC, dt and dy read (bf16), d(xBC) and d(dt) written (fp32).
-    flops: the adjoint's products per chunk of Q = 64 and per direction and
-    head -- C.B^T, dY.X^T (Q^2 N, Q^2 P), X.dS, dY.S_in (Q P N each), W^T.dY
+    flops: the adjoint's products per chunk of Q = 64 (the convention the
+    forward's count uses; the kernel's chunks are 128 long) and per direction
+    and head -- C.B^T, dY.X^T (Q^2 N, Q^2 P), X.dS, dY.S_in (Q P N each), W^T.dY
     (Q^2 P), B.dS^T (Q N P), T^T.C, T.B (Q^2 N each), the state adjoint (P N Q)
     -- i.e. Q(3N + 2P) + 5PN multiply-adds per token, head and direction."""
     H, P, N = w.heads, w.headdim, w.d_state
@@ -518,17 +519,13 @@ def measure(args, lib, I, name, rank, world, dev, gpu_id, want_e2e=True):
     roof, ctx = roofline(peaks, peak_kind, clocks, nbytes, flops, per_call_ms / 1e3, decode,
                          kernel_file, name)
     if name == "backward1p3b":
-        # CUDA-core fp32 products: held against the fp32 FMA peak at the sampled clock
+        # the adjoint's products on tcgen05 (bf16 operands): held against the
+        # bf16 tensor peak over the adjoint kernel's time
         nbytes, flops = backward_counts(w, batch * seqlen)
-        mhz = clocks["sm_mhz"] if clocks else 1965.0
-        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
-        ach = flops / (per_call_ms / 1e3) / 1e12
-        roof = {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "peak_source": f"fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x {mhz:.0f} MHz "
-                               f"(sampled SM clock)", "frac": ach / peak, "traffic": None,
-                "kernel": "backward.cu"}
-        ctx = {"achieved_gbs": nbytes / (per_call_ms / 1e3) / 1e9, "algorithmic_bytes": nbytes,
-               "algorithmic_flops": flops, "note": "whole call: conv, state pass, adjoint, conv backward"}
+        roof, ctx = roofline(peaks, peak_kind, clocks, nbytes, flops, per_call_ms / 1e3, False,
+                             "backward_tc.cu", name)
+        ctx["note"] = ("flops: the adjoint's products at the Q = 64 convention over the adjoint "
+                       "kernel's time; bytes: the whole call (conv, state pass, adjoint, conv backward)")
     if name == "decode":
         wl = (f"cached block decode: {batch} streams x {seqlen}-token block, H64x64 N128 bf16, "
               f"65536-token prefix state")

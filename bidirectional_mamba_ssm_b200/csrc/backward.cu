@@ -454,7 +454,9 @@ bwd_scan_kernel(const BwdParams p)
 
 // Conv backward of both streams for one (sequence, channel, token tile):
 // dpre = dact o SiLU'(pre); d(xbc) = the transposed taps applied to dpre;
-// tap and bias gradients accumulated.
+// tap and bias gradients accumulated.  One pass over the tile and its
+// 3-token halos: each token's raw value, pre-activations and dpre are
+// computed once and kept in sliding windows.
 template <typename T>
 __global__ void __launch_bounds__(128)
 bwd_conv_kernel(const T *__restrict__ u, const float *__restrict__ w, const float *__restrict__ bias,
@@ -466,6 +468,8 @@ bwd_conv_kernel(const T *__restrict__ u, const float *__restrict__ w, const floa
     const int b = blockIdx.z;
     const int t0 = blockIdx.y * 64, t1 = min(t0 + 64, len);
     const T *ub = u + (size_t)b * len * ch + c;
+    const float *af = dact_f + (size_t)b * len * ch + c;
+    const float *ar = dact_r + (size_t)b * len * ch + c;
     const float w0 = w[c * 4], w1 = w[c * 4 + 1], w2 = w[c * 4 + 2], w3 = w[c * 4 + 3];
     const float bb = bias ? bias[c] : 0.0f;
     auto uv = [&](int t) { return (t >= 0 && t < len) ? Elem<T>::load(ub + (size_t)t * ch) : 0.0f; };
@@ -473,30 +477,54 @@ bwd_conv_kernel(const T *__restrict__ u, const float *__restrict__ w, const floa
         const float sg = 1.0f / (1.0f + expf(-x));
         return sg * (1.0f + x * (1.0f - sg));
     };
-    // dpre of the forward stream at token t (pre_f[t] = b + sum_j w_j u[t-3+j])
-    auto dpre_f = [&](int t) {
-        if (t < 0 || t >= len) return 0.0f;
-        const float pre = bb + w0 * uv(t - 3) + w1 * uv(t - 2) + w2 * uv(t - 1) + w3 * uv(t);
-        return dact_f[((size_t)b * len + t) * ch + c] * dsilu(pre);
-    };
-    // the reverse stream (pre_r[t] = b + sum_j w_j u[t+3-j])
-    auto dpre_r = [&](int t) {
-        if (t < 0 || t >= len) return 0.0f;
-        const float pre = bb + w0 * uv(t + 3) + w1 * uv(t + 2) + w2 * uv(t + 1) + w3 * uv(t);
-        return dact_r[((size_t)b * len + t) * ch + c] * dsilu(pre);
-    };
+    // sliding windows, at output token t = tn - 3: uw[k] = u[t - 3 + k],
+    // pf[k] = dpre_f(t - 3 + k) (k = 0..6), pr[k] = dpre_r(t - 3 + k) (k = 0..3).
+    // Every entry an output reads was brought in by the loop (it starts 3
+    // tokens before the tile), so they start at zero
+    float uw[7], pf[7], pr[7];
+#pragma unroll
+    for (int k = 0; k < 7; ++k) uw[k] = pf[k] = pr[k] = 0.0f;
     float gw0 = 0.0f, gw1 = 0.0f, gw2 = 0.0f, gw3 = 0.0f, gb = 0.0f;
-    for (int t = t0; t < t1; ++t) {
-        // d(xbc)[t]: forward taps j read u[t] at pre_f[t+3-j]; reverse at pre_r[t-3+j]
-        const float g = w0 * dpre_f(t + 3) + w1 * dpre_f(t + 2) + w2 * dpre_f(t + 1) + w3 * dpre_f(t) +
-                        w0 * dpre_r(t - 3) + w1 * dpre_r(t - 2) + w2 * dpre_r(t - 1) + w3 * dpre_r(t);
-        du[((size_t)b * len + t) * ch + c] = g;
-        const float pf = dpre_f(t), pr = dpre_r(t);
-        gw0 += pf * uv(t - 3) + pr * uv(t + 3);
-        gw1 += pf * uv(t - 2) + pr * uv(t + 2);
-        gw2 += pf * uv(t - 1) + pr * uv(t + 1);
-        gw3 += (pf + pr) * uv(t);
-        gb += pf + pr;
+    // step tn = t + 3 brings in u[tn], dpre_f(tn) and dpre_r(tn - 3); token t
+    // completes (its du needs dpre_f up to t + 3 and dpre_r down to t - 3)
+    for (int tn = t0 - 3; tn < t1 + 3; ++tn) {
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+            uw[k] = uw[k + 1];
+            pf[k] = pf[k + 1];
+            pr[k] = pr[k + 1];
+        }
+        uw[6] = uv(tn);   // window now u[tn - 6 .. tn]: uw[k] = u[tn - 6 + k]
+        // dpre_f(tn): pre_f[tn] = b + sum_j w_j u[tn - 3 + j]
+        float dfn = 0.0f;
+        if (tn >= 0 && tn < len) {
+            const float pre = bb + w0 * uw[3] + w1 * uw[4] + w2 * uw[5] + w3 * uw[6];
+            dfn = af[(size_t)tn * ch] * dsilu(pre);
+        }
+        pf[6] = dfn;
+        // dpre_r(tn - 3): pre_r[s] = b + sum_j w_j u[s + 3 - j], s = tn - 3
+        const int sr = tn - 3;
+        float drn = 0.0f;
+        if (sr >= 0 && sr < len) {
+            const float pre = bb + w0 * uw[6] + w1 * uw[5] + w2 * uw[4] + w3 * uw[3];
+            drn = ar[(size_t)sr * ch] * dsilu(pre);
+        }
+        // pr[k] = dpre_r(t - 3 + k) with t = tn - 3: the newest is dpre_r(t) = pr[3];
+        // keep pr[0..3] = dpre_r(t - 3 .. t)
+        pr[3] = drn;
+        const int t = tn - 3;
+        if (t >= t0 && t < t1) {
+            // pf[k] = dpre_f(tn - 6 + k) = dpre_f(t - 3 + k); uw[k] = u[t - 3 + k]
+            const float g = w0 * pf[6] + w1 * pf[5] + w2 * pf[4] + w3 * pf[3] +
+                            w0 * pr[0] + w1 * pr[1] + w2 * pr[2] + w3 * pr[3];
+            du[((size_t)b * len + t) * ch + c] = g;
+            const float dpf = pf[3], dpr = pr[3];
+            gw0 += dpf * uw[0] + dpr * uw[6];
+            gw1 += dpf * uw[1] + dpr * uw[5];
+            gw2 += dpf * uw[2] + dpr * uw[4];
+            gw3 += (dpf + dpr) * uw[3];
+            gb += dpf + dpr;
+        }
     }
     atomicAdd(dw + c * 4, gw0);
     atomicAdd(dw + c * 4 + 1, gw1);

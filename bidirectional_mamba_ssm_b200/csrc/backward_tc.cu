@@ -100,12 +100,6 @@ __device__ __forceinline__ float column_sum32(float (&v)[32], int lane)
     return v[0];
 }
 
-__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d)
-{
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
-                 :: "l"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-
 // ---- state pass: shared memory (offsets from a 1024-byte aligned base)
 constexpr uint32_t kSOffX = 0;             // X [row][p]      16 KB (TMA)
 constexpr uint32_t kSOffB = 16384;         // B [row][n]      2 x 16 KB (TMA)
@@ -287,9 +281,9 @@ constexpr uint32_t kAOffSin = 163840;   // S_in^T [n][p] 16 KB (bulk copy)
 constexpr uint32_t kAOffDS = 180224;    // dS^T [n][p] 16 KB (bf16 copy of the TMEM adjoint)
 constexpr uint32_t kAOffVec = 196608;   // f32 vectors (below)
 // f32 vectors (offsets in floats; see the kernel)
-constexpr int kVCv = 0, kVDt = kVCv + kBQ, kVCum = kVDt + kBQ, kVRsp = kVCum + kBQ, kVColp = kVRsp + 2 * kBQ,
-              kVDdp = kVColp + 4 * kBQ, kVCsp = kVDdp + 4 * kBQ, kVXbp = kVCsp + 2 * kBQ, kVSdp = kVXbp + 2 * kBQ,
-              kVDcw = kVSdp + 2 * kBQ, kVGdw = kVDcw + kBQ, kVUw = kVGdw + kBQ, kVRed = kVUw + kBQ;
+constexpr int kVCv = 0, kVDt = kVCv + kBQ, kVCum = kVDt + kBQ, kVRsp = kVCum + kBQ, kVDdp = kVRsp + 2 * kBQ,
+              kVCsp = kVDdp + 4 * kBQ, kVXbp = kVCsp + 2 * kBQ, kVSdp = kVXbp + 2 * kBQ, kVDcw = kVSdp + 2 * kBQ,
+              kVGdw = kVDcw + kBQ, kVUw = kVGdw + kBQ, kVRed = kVUw + kBQ;
 constexpr int kVecFloats = kVRed + 64;
 constexpr uint32_t kAOffMbar = kAOffVec + 4 * kVecFloats;
 constexpr uint32_t kAOffTmem = kAOffMbar + 32;
@@ -317,7 +311,8 @@ constexpr uint32_t kColDS = 448;    // dS^T (n, p), fp32, carried across chunks
 //  P6  dC out
 __global__ void __launch_bounds__(kBThreads, 1)
 bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_constant__ CUtensorMap tm_act_r,
-                   const __grid_constant__ CUtensorMap tm_dy, const BwdTcParams p)
+                   const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_dact_f,
+                   const __grid_constant__ CUtensorMap tm_dact_r, const BwdTcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
@@ -328,13 +323,13 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
     const bool rev = dir != 0;
     const int L = p.len, H = p.H, ch = p.ch, nc = p.nchunks;
     const CUtensorMap *tm = rev ? &tm_act_r : &tm_act_f;
+    const CUtensorMap *tmd = rev ? &tm_dact_r : &tm_dact_f;   // fp32 gradient, for the B/C reductions
     float *dact = rev ? p.dact[1] : p.dact[0];
     float *vec = reinterpret_cast<float *>(sm + kAOffVec);
     float *cv = vec + kVCv;       // [128] c (log2 units) by row
     float *dtv = vec + kVDt;      // [128] dt by row
     float *cumw = vec + kVCum;    // [128] prefix sums of dt by walk slot
     float *rsp = vec + kVRsp;     // [2][128] row sums of dY X^T o W, per column half
-    float *colp = vec + kVColp;   // [4][128] column sums of dY X^T o W, per row quarter
     float *ddp = vec + kVDdp;     // [4][128] column sums of dY X^T o C B^T o e, per row quarter
     float *csp = vec + kVCsp;     // [2][128] dY_t . (C S_in^T)_t per half
     float *xbp = vec + kVXbp;     // [2][128] x_s . (B dS^T)_s per half
@@ -352,6 +347,7 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         tc::mbar_init(mb_p5, 1);
         tc::prefetch_tmap(tm);
         tc::prefetch_tmap(&tm_dy);
+        tc::prefetch_tmap(tmd);
     }
     if (warp == 0) tc::tmem_alloc(sbase + kAOffTmem, 512);
     tc::fence_before_sync();
@@ -379,7 +375,14 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         const int tok = t0 + r;
         const bool tok_ok = tok >= 0 && tok < L;
         // ---- P0: this chunk's tiles, dt, and the bf16 copy of dS^T
+        // staging rows of the fp32 dB / dC tiles: row q is token t0 + off + q
+        // (the reverse walk's last chunk starts before token 0; a tensor
+        // reduction may not start at a negative row, so its box starts at
+        // token 0 and the rows past the chunk are zeros)
+        const int off = t0 < 0 ? -t0 : 0;
+        const int q = (r - off) & (kBQ - 1);
         if (tid == 0) {
+            tc::bulk_wait_read0();   // the last chunk's dB / dC staging is out of shared memory
             tc::mbar_expect_tx(mb_in, 7 * 16384);
             tc::tma_load_3d(sbase + kAOffX, tm, h * kBP, t0, b, mb_in);
             tc::tma_load_3d(sbase + kAOffDY, &tm_dy, h * kBP, t0, b, mb_in);
@@ -455,7 +458,9 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
                 tc::tmem_ld32_nw(trow + kColDYX + s0, yx);
                 tc::tmem_wait_ld(cb);
                 tc::tmem_wait_ld(yx);
-                float pr[32], pd[32];
+                // pd = dY X^T o C B^T o e; its row sums weighted by dt_s (rs) and
+                // its column sums (times dt_s: those of dY X^T o W) feed dL/dc
+                float pd[32];
                 uint32_t wp[16], tp[16];
 #pragma unroll
                 for (int i4 = 0; i4 < 8; ++i4) {
@@ -473,9 +478,8 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
                         const float yxv = __uint_as_float(yx[i]);
                         wv[e] = cbe * ds_[e];
                         tv[e] = yxv * dec * ds_[e];
-                        pr[i] = yxv * wv[e];
                         pd[i] = yxv * cbe;
-                        rs += pr[i];
+                        rs = fmaf(pd[i], ds_[e], rs);
                     }
                     wp[2 * i4] = tc::pack_bf16x2(wv[0], wv[1]);
                     wp[2 * i4 + 1] = tc::pack_bf16x2(wv[2], wv[3]);
@@ -490,7 +494,6 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
                     *reinterpret_cast<uint4 *>(sm + kAOffT + off) =
                         make_uint4(tp[4 * pc], tp[4 * pc + 1], tp[4 * pc + 2], tp[4 * pc + 3]);
                 }
-                colp[quarter * kBQ + s0 + lane] = column_sum32(pr, lane);
                 ddp[quarter * kBQ + s0 + lane] = column_sum32(pd, lane);
             }
             rsp[hw * kBQ + r] = rs;
@@ -595,18 +598,18 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
                 *reinterpret_cast<uint4 *>(sm + kAOffDY + off) = pack8(yv);
             }
         }
+        // dB rows staged as four 32-column fp32 boxes (128-byte swizzle) in the
+        // W and T tiles, which the products above have finished with
 #pragma unroll 1
         for (int g = 0; g < 2; ++g) {
             uint32_t v[32];
             tc::tmem_ld32_nw(trow + kColCB + 64 * hw + 32 * g, v);
             tc::tmem_wait_ld(v);
-            if (tok_ok) {
-                float *dst = dact + ((size_t)b * L + tok) * ch + H * kBP + 64 * hw + 32 * g;
+            uint8_t *box = sm + (hw ? kAOffT : kAOffW) + 16384 * g;
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    red_add_v4(dst + 4 * i, __uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-            }
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(box + tc::sw128(q, c)) =
+                    r >= off ? make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]) : make_uint4(0u, 0u, 0u, 0u);
         }
         {
             // dS^T <- e^{c_last} dS^T (its bf16 copy was taken in P0)
@@ -628,8 +631,8 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
             const float xb = xbp[r] + xbp[kBQ + r];
             const float el = tc::exp2_approx(fminf(clast - ct, 0.0f));
             const float u = el * dtv[r] * xb;
-            const float csum = colp[r] + colp[kBQ + r] + colp[2 * kBQ + r] + colp[3 * kBQ + r];
             const float dsum = ddp[r] + ddp[kBQ + r] + ddp[2 * kBQ + r] + ddp[3 * kBQ + r];
+            const float csum = dsum * dtv[r];   // column sum of dY X^T o W
             dcw[j] = tc::exp2_approx(fminf(ct, 0.0f)) * (csp[r] + csp[kBQ + r]) - u + (rsp[r] + rsp[kBQ + r]) - csum;
             gdw[j] = dsum + el * xb;
             uw[r] = u;
@@ -638,6 +641,14 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         tc::tmem_wait_st();
         tc::fence_before_sync();
         __syncthreads();
+        if (tid == 0) {
+            // dB += this head's rows (fp32 reductions at L2)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                tc::tma_reduce_add_3d(tmd, sbase + (j < 2 ? kAOffW : kAOffT) + 16384 * (j & 1), H * kBP + 32 * j,
+                                      t0 + off, b);
+            tc::bulk_commit();
+        }
         if (warp == 0) {
             // the chunk's last walk slot also carries e^{c_last} <dS, S_in> + sum_s U_s;
             // then dt gets A times the suffix sums of dL/dc (walk order), A the
@@ -702,23 +713,33 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         ok = __syncthreads_and(ok);
         if (!ok) break;
         tc::fence_after_sync();
-        // ---- P6: dC of row t = r (64 n)
+        // ---- P6: dC of row t = r (64 n), staged like dB in the X, B and S_in
+        // tiles (every product that reads them is done; the next chunk's
+        // loads into them wait for the reductions to read them)
 #pragma unroll 1
         for (int g = 0; g < 2; ++g) {
             uint32_t v[32];
             tc::tmem_ld32_nw(trow + kColDYX + 64 * hw + 32 * g, v);
             tc::tmem_wait_ld(v);
-            if (tok_ok) {
-                float *dst = dact + ((size_t)b * L + tok) * ch + H * kBP + kBN + 64 * hw + 32 * g;
+            const int j = 2 * hw + g;
+            uint8_t *box = sm + (j == 0 ? kAOffX : j == 3 ? kAOffSin : kAOffB + 16384 * (j - 1));
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    red_add_v4(dst + 4 * i, __uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-            }
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(box + tc::sw128(q, c)) =
+                    r >= off ? make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]) : make_uint4(0u, 0u, 0u, 0u);
         }
+        tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                tc::tma_reduce_add_3d(tmd, sbase + (j == 0 ? kAOffX : j == 3 ? kAOffSin : kAOffB + 16384 * (j - 1)),
+                                      H * kBP + kBN + 32 * j, t0 + off, b);
+            tc::bulk_commit();
+        }
     }
+    if (tid == 0) tc::bulk_wait0();   // every reduction written
     if (ok) {
         if (!rev && p.dinit) {
             // the adjoint of the caller's initial state: dinit[p][n] = dS^T[n][p]
@@ -767,17 +788,20 @@ PFN_cuTensorMapEncodeTiled_v12000 bwd_encode_fn()
     return fn;
 }
 
-// (batch, len, cols) bf16, boxes of 64 columns x 128 rows, 128-byte swizzle
-bool make_tile_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t len, uint64_t batch)
+// (batch, len, cols) bf16 or fp32, boxes of 128 bytes x 128 rows, 128-byte swizzle
+bool make_tile_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t len, uint64_t batch,
+                   bool f32 = false)
 {
     auto fn = bwd_encode_fn();
     if (!fn) return false;
+    const uint64_t esz = f32 ? 4 : 2;
     const cuuint64_t dims[3] = {cols, len, batch};
-    const cuuint64_t strides[2] = {cols * 2, cols * len * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)kBQ, 1};
+    const cuuint64_t strides[2] = {cols * esz, cols * len * esz};
+    const cuuint32_t box[3] = {(cuuint32_t)(128 / esz), (cuuint32_t)kBQ, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -815,10 +839,12 @@ cudaError_t launch_backward_tc(const BackwardTcProblem &q, cudaStream_t s)
     p.H = d.heads;
     p.ch = d.heads * kBP + 2 * kBN;
     p.nchunks = (d.len + kBQ - 1) / kBQ;
-    CUtensorMap tm_f, tm_r, tm_dy;
+    CUtensorMap tm_f, tm_r, tm_dy, tm_df, tm_dr;
     if (!make_tile_map(&tm_f, q.act[0], (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch) ||
         !make_tile_map(&tm_r, q.act[1], (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch) ||
-        !make_tile_map(&tm_dy, q.dy, (uint64_t)d.heads * kBP, (uint64_t)d.len, (uint64_t)d.batch))
+        !make_tile_map(&tm_dy, q.dy, (uint64_t)d.heads * kBP, (uint64_t)d.len, (uint64_t)d.batch) ||
+        !make_tile_map(&tm_df, q.dact[0], (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, true) ||
+        !make_tile_map(&tm_dr, q.dact[1], (uint64_t)p.ch, (uint64_t)d.len, (uint64_t)d.batch, true))
         return cudaErrorInvalidValue;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(bwd_tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -832,7 +858,7 @@ cudaError_t launch_backward_tc(const BackwardTcProblem &q, cudaStream_t s)
     count_launch();
     const TimingEvents ev = timing_events();
     if (ev.start && (e = cudaEventRecord(ev.start, s)) != cudaSuccess) return e;
-    bwd_tc_scan_kernel<<<grid, kBThreads, kASmem, s>>>(tm_f, tm_r, tm_dy, p);
+    bwd_tc_scan_kernel<<<grid, kBThreads, kASmem, s>>>(tm_f, tm_r, tm_dy, tm_df, tm_dr, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launch();
     if (ev.stop && (e = cudaEventRecord(ev.stop, s)) != cudaSuccess) return e;

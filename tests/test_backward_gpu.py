@@ -6,7 +6,9 @@ for bf16.  Shapes span several 64-token chunks with ragged tails, with short-
 and long-memory decays, a conv bias and an initial state.  The 64-head case
 checks the per-head gradients (x channels, dt, A, D, x conv taps, initial
 state) of sampled heads; the B and C gradients sum over all heads and are
-checked in full on the small shapes."""
+checked in full on the small shapes.  The bf16 shapes with headdim 64 and
+d_state 128 run the tensor-core kernels (128-token chunks), the others the
+CUDA-core kernels (64-token chunks)."""
 import math
 
 import numpy as np
@@ -89,3 +91,50 @@ def test_backward_64_heads_sampled(lib):
     assert rel_err(to_np(got["D"])[heads], ref["D"]) <= tol
     assert rel_err(to_np(got["conv_w"])[xcols], ref["conv_w"][:hp]) <= tol
     assert rel_err(to_np(got["init"])[:, heads], ref["init"]) <= tol
+
+
+TC_EDGES = [
+    # batch, L, decay: shapes of the tensor-core backward (bf16, headdim 64,
+    # d_state 128): one token, one full 128-token chunk, one chunk plus one
+    # token, several chunks with a ragged tail, and the closed-form decays
+    (1, 1, "short"),
+    (1, 128, "long"),
+    (1, 129, "long"),
+    (3, 257, "short"),
+    (2, 384, "zero"),
+    (1, 200, "steep"),
+]
+
+
+@pytest.mark.parametrize("case", TC_EDGES, ids=lambda c: "-".join(map(str, c)))
+def test_backward_tensor_core_edges(lib, case):
+    """The tensor-core backward against the oracle's adjoint on its edge
+    shapes: chunk boundaries at 1, 128 and 129 tokens, a ragged tail with
+    batch 3, A = 0 (every decay exactly 1: the state adjoint never shrinks)
+    and A = -50 (decays of ~1e-3 per step)."""
+    bsz, L, decay = case
+    H, P, N = 2, 64, 128
+    w = inp_mod.Workload("bwdtc", bsz, L, H, P, N, dtype="bf16", bc_scale=1.0 / math.sqrt(N))
+    a = {"short": (1.0, 16.0), "long": (1e-3, 1e-2), "zero": (1.0, 2.0), "steep": (1.0, 2.0)}[decay]
+    cpu = inp_mod.make_inputs(w, seed=7 * L + bsz, a_range=a, conv_bias=True)
+    if decay == "zero":
+        cpu["A"] = torch.zeros_like(cpu["A"])
+    elif decay == "steep":
+        # a decay of ~e^-6.5 per step; steeper, dL/dA itself underflows (the
+        # oracle's is ~1e-74 at A = -1e4) and a relative metric has nothing
+        # left to compare
+        cpu["A"] = torch.full_like(cpu["A"], -50.0)
+    init = inp_mod.make_state(bsz, H, P, N, seed=9, scale=0.3)
+    g = torch.Generator().manual_seed(L + 1)
+    dy = torch.randn((bsz, L, H * P), generator=g).to(torch.bfloat16)
+    d = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
+    got = lib.bimamba_ssd_fwd_rev_backward(d["xbc"], d["dt"], d["A"], d["D"], d["conv_w"], d["conv_b"],
+                                           init.cuda(), dy.cuda(), heads=H, headdim=P, d_state=N,
+                                           want_dinit=True)
+    assert lib.bimamba_get_error() == lib.BIMAMBA_OK
+    n = {k: to_np(v) for k, v in cpu.items()}
+    ref = oracle.bimamba_mixer_backward(n["xbc"], n["dt"], n["A"], n["D"], n["conv_w"], n["conv_b"],
+                                        to_np(dy), heads=H, headdim=P, d_state=N, init=to_np(init))
+    tol = TOL["bf16"]
+    for k in ("xbc", "dt", "A", "D", "conv_w", "conv_b", "init"):
+        assert rel_err(to_np(got[k]), ref[k]) <= tol, (k, rel_err(to_np(got[k]), ref[k]))
