@@ -379,6 +379,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             tc::tma_load_3d_hint(sbase + xbuf_off(k), tm, hp * kPP, rev ? t0 : t0 - 3, b, mb, pol);
         }
     };
+    // chunk k's raw rows into L2 ahead of their load (the load of the chunk
+    // after next is issued once the current one's buffer is free: by then its
+    // rows come from L2, not HBM)
+    auto prefetch_x = [&](int k) {
+        int t0, cnt, s0;
+        chunk_of(k, t0, cnt, s0);
+        tc::tma_prefetch_l2_3d(rev ? &tm_x_r : &tm_x_f, hp * kPP, rev ? t0 : t0 - 3, b);
+    };
     auto issue_bc = [&](int k) {
         int t0, cnt, s0;
         chunk_of(k, t0, cnt, s0);
@@ -509,6 +517,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         tc::mbar_init(mb_yfree, 1);
         issue_x(0);
         if (nk > 1) issue_x(1);
+        if (!kStateOnly && nk > 2) prefetch_x(2);
         issue_bc(0);
     }
     if (warp == kHelperWarp) {
@@ -679,6 +688,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 tc::bulk_commit();
                 tc::bulk_wait_read0();   // the staged rows have been read
                 if (k + 2 < nk) issue_x(k + 2);
+                if (k + 3 < nk) prefetch_x(k + 3);
                 if (!kConcat) {
                     if (first) {
                         // publish the rows to the partner once written

@@ -394,6 +394,14 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void *tmap, uint32_t src
                  : "memory");
 }
 
+// Prefetch one tiled 3-D box of the tensor into L2 (no shared memory, no
+// completion to wait for; boxes out of the tensor's range fetch nothing there).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void *tmap, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 :: "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+
 // L2 eviction-priority policies for the cache-hinted copies below: data
 // that another CTA reads again soon is kept (evict_last), data read or
 // written for the last time goes first (evict_first).
