@@ -195,6 +195,12 @@ bwd_tc_state_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_c
             tc::tma_load_3d(sbase + kSOffX, tm, h * kBP, t0, b, mb_in);
             tc::tma_load_3d(sbase + kSOffB, tm, H * kBP, t0, b, mb_in);
             tc::tma_load_3d(sbase + kSOffB + 16384, tm, H * kBP + 64, t0, b, mb_in);
+            if (k + 1 < p.nchunks) {
+                const int tn = max(rev ? L - kBQ * (k + 2) : kBQ * (k + 1), 0);   // the next chunk, into L2
+                tc::tma_prefetch_l2_3d(tm, h * kBP, tn, b);
+                tc::tma_prefetch_l2_3d(tm, H * kBP, tn, b);
+                tc::tma_prefetch_l2_3d(tm, H * kBP + 64, tn, b);
+            }
         }
         if (tid < kBQ) {
             const int tok = t0 + r;
@@ -391,6 +397,16 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
             tc::tma_load_3d(sbase + kAOffC, tm, H * kBP + kBN, t0, b, mb_in);
             tc::tma_load_3d(sbase + kAOffC + 16384, tm, H * kBP + kBN + 64, t0, b, mb_in);
             tc::bulk_load(sbase + kAOffSin, tiles + (size_t)k * (kTileBytes / 2), kTileBytes, mb_in);
+            if (k > 0) {
+                // the next chunk's tiles into L2 (its loads are issued only once
+                // this chunk is done with the buffers)
+                const int tn = rev ? L - kBQ * k : kBQ * (k - 1);
+                tc::tma_prefetch_l2_3d(tm, h * kBP, tn, b);
+                tc::tma_prefetch_l2_3d(&tm_dy, h * kBP, tn, b);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tc::tma_prefetch_l2_3d(tm, H * kBP + 64 * j, tn, b);
+                tc::bulk_prefetch_l2(tiles + (size_t)(k - 1) * (kTileBytes / 2), kTileBytes);
+            }
         }
         if (tid < kBQ) dtv[r] = tok_ok ? __bfloat162float(p.dt[((size_t)b * L + tok) * H + h]) : 0.0f;
         {

@@ -402,6 +402,12 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const void *tmap, int c0, int
                  :: "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2) : "memory");
 }
 
+// Prefetch `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(src), "r"(bytes) : "memory");
+}
+
 // L2 eviction-priority policies for the cache-hinted copies below: data
 // that another CTA reads again soon is kept (evict_last), data read or
 // written for the last time goes first (evict_first).
