@@ -141,6 +141,10 @@ decode_prep_kernel(const __nv_bfloat16 *__restrict__ xbc, const __nv_bfloat16 *_
     const uint32_t sbase = tc::smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5;
     const int s = blockIdx.x;
+    // the decode kernel may start now: it loads its inputs that do not come
+    // from here, then waits for this grid (griddepcontrol.wait) before
+    // reading the records
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int slot = slots ? slots[s] : s;
     if (slot < 0 || slot >= pool) return;   // uniform: the decode kernel records the error
     const uint32_t mb = sbase + kPOffMbar;
@@ -300,9 +304,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
         tc::mbar_init(mb_mma, 1);
         tc::prefetch_tmap(&tm_x);
         tc::mbar_expect_tx(mb_ld, 32768 + kDP * kDN * 4 + kDQ * 128);
-        bulk_g2s(sbase + kDOffC, rec + kPrepG, 32768, mb_ld);          // C_f and B_f images
         bulk_g2s(sbase + kDOffSf, state, kDP * kDN * 4, mb_ld);        // the cached state
         tc::tma_load_3d(sbase + kDOffRawBox, &tm_x, h * kDP, 0, s, mb_ld);   // tokens 0..63 (zeros past len)
+        // the prep records of this step (C_f and B_f images) once their grid is done
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        bulk_g2s(sbase + kDOffC, rec + kPrepG, 32768, mb_ld);
     }
     if (tid >= 64 && tid < 64 + 24) {
         // conv tail: the 3 newest tokens before the block, raw rows 0..2
@@ -364,6 +370,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
     const int d = r >> 6, t = r & 63;
     // this thread's G row (L2-resident prep record), loaded while the copies fly
     float4 grow[8];
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // (the prep grid's records are written)
     {
         const float4 *grow4 = reinterpret_cast<const float4 *>(
             reinterpret_cast<const float *>(rec) + ((size_t)d * kDQ + t) * kDQ + 32 * half);
@@ -695,6 +702,10 @@ cudaError_t launch_decode_tc(const DecodeProblem &q, cudaStream_t stream)
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDSmem);
     if (e != cudaSuccess) return e;
+    // the device time of a step: both kernels (the decode kernel overlaps the
+    // prep kernel's end through a programmatic dependent launch)
+    const TimingEvents ev = timing_events();
+    if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
     decode_prep_kernel<<<d.batch, kDThreads, kPSmem, stream>>>(
         static_cast<const __nv_bfloat16 *>(q.xbc), static_cast<const __nv_bfloat16 *>(q.tail), q.slots,
         q.pool, q.conv_w, q.conv_b, prep, d.len, ch, d.heads * d.headdim, q.status);
@@ -719,12 +730,19 @@ cudaError_t launch_decode_tc(const DecodeProblem &q, cudaStream_t stream)
     p.len = d.len;
     p.H = d.heads;
     p.ch = ch;
-    const TimingEvents ev = timing_events();
-    if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
     CUtensorMap tm_x;
     if ((ch * 2) % 16 != 0 || !make_block_map(&tm_x, q.xbc, ch, d.len, d.batch)) return cudaErrorInvalidValue;
-    decode_tc_kernel<<<dim3(d.heads, d.batch), kDThreads, kDSmem, stream>>>(tm_x, p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(d.heads, d.batch);
+    cfg.blockDim = dim3(kDThreads);
+    cfg.dynamicSmemBytes = kDSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, tm_x, p)) != cudaSuccess) return e;
     count_launch();
     if (ev.stop) e = cudaEventRecord(ev.stop, stream);
     return e;
