@@ -269,13 +269,33 @@ bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc_f, const __nv_bfloat16 *
         w0[q] = t4.x; w1[q] = t4.y; w2[q] = t4.z; w3[q] = t4.w;
         bb[q] = conv_b ? conv_b[c + q] : 0.0f;
     }
-    float r0[8], r1[8], r2[8];
-    raw(s_begin - 3, r0);
-    raw(s_begin - 2, r1);
-    raw(s_begin - 1, r2);
-    for (int s = s_begin; s < s_end; ++s) {
-        float r3[8], o[8];
-        raw(s, r3);
+    // every raw row of the thread's 8 steps (and the 3 before) requested at
+    // once, kept as packed bf16
+    uint4 rw[11];
+#pragma unroll
+    for (int i = 0; i < 11; ++i) {
+        const int s = s_begin - 3 + i;
+        if (s < s_end) {
+            if (s >= 0) {
+                rw[i] = *reinterpret_cast<const uint4 *>(xb + (size_t)(rev ? len - 1 - s : s) * ch);
+            } else {
+                float v[8];
+                raw(s, v);
+                rw[i] = pack8(v);
+            }
+        } else {
+            rw[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int s = s_begin + i;
+        if (s >= s_end) break;
+        float r0[8], r1[8], r2[8], r3[8], o[8];
+        unpack8(rw[i], r0);
+        unpack8(rw[i + 1], r1);
+        unpack8(rw[i + 2], r2);
+        unpack8(rw[i + 3], r3);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             float acc = bb[q];
@@ -284,7 +304,6 @@ bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc_f, const __nv_bfloat16 *
             acc = fmaf(w2[q], r2[q], acc);
             acc = fmaf(w3[q], r3[q], acc);
             o[q] = tc::silu_tanh(acc);
-            r0[q] = r1[q]; r1[q] = r2[q]; r2[q] = r3[q];
         }
         *reinterpret_cast<uint4 *>(ob + (size_t)s * kBC) = pack8(o);
     }
