@@ -388,14 +388,16 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         const int off = t0 < 0 ? -t0 : 0;
         const int q = (r - off) & (kBQ - 1);
         if (tid == 0) {
-            tc::bulk_wait_read0();   // the last chunk's dB / dC staging is out of shared memory
+            // dY and C first (no staging lives there), then X, B and S_in once
+            // the last chunk's dB / dC staging in them has been read
             tc::mbar_expect_tx(mb_in, 7 * 16384);
-            tc::tma_load_3d(sbase + kAOffX, tm, h * kBP, t0, b, mb_in);
             tc::tma_load_3d(sbase + kAOffDY, &tm_dy, h * kBP, t0, b, mb_in);
-            tc::tma_load_3d(sbase + kAOffB, tm, H * kBP, t0, b, mb_in);
-            tc::tma_load_3d(sbase + kAOffB + 16384, tm, H * kBP + 64, t0, b, mb_in);
             tc::tma_load_3d(sbase + kAOffC, tm, H * kBP + kBN, t0, b, mb_in);
             tc::tma_load_3d(sbase + kAOffC + 16384, tm, H * kBP + kBN + 64, t0, b, mb_in);
+            tc::bulk_wait_read0();
+            tc::tma_load_3d(sbase + kAOffX, tm, h * kBP, t0, b, mb_in);
+            tc::tma_load_3d(sbase + kAOffB, tm, H * kBP, t0, b, mb_in);
+            tc::tma_load_3d(sbase + kAOffB + 16384, tm, H * kBP + 64, t0, b, mb_in);
             tc::bulk_load(sbase + kAOffSin, tiles + (size_t)k * (kTileBytes / 2), kTileBytes, mb_in);
             if (k > 0) {
                 // the next chunk's tiles into L2 (its loads are issued only once
