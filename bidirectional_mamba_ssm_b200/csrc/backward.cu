@@ -583,8 +583,15 @@ cudaError_t launch_backward_t(const BackwardProblem &q, cudaStream_t s)
     p.ch = ch;
     p.nchunks = (d.len + kBQ - 1) / kBQ;
     cudaError_t e;
-    // outputs that are accumulated start at zero
-    if ((e = cudaMemsetAsync(p.dact[0], 0, 2 * tokens * ch * sizeof(float), s)) != cudaSuccess ||
+    // outputs that are accumulated start at zero.  Of the two streams' fp32
+    // activation gradients (contiguous rows of ch), the tensor-core passes
+    // overwrite the x columns of every row and add to the B/C columns: only
+    // those are zeroed there (a strided 2-D fill), the whole rows otherwise
+    const bool tc_path = backward_tc_supported(d);
+    e = tc_path ? cudaMemset2DAsync(p.dact[0] + (size_t)d.heads * d.headdim, ch * sizeof(float), 0,
+                                    (size_t)2 * d.d_state * sizeof(float), 2 * tokens, s)
+                : cudaMemsetAsync(p.dact[0], 0, 2 * tokens * ch * sizeof(float), s);
+    if (e != cudaSuccess ||
         (e = cudaMemsetAsync(q.ddt, 0, tokens * d.heads * sizeof(float), s)) != cudaSuccess ||
         (e = cudaMemsetAsync(q.dA, 0, d.heads * sizeof(float), s)) != cudaSuccess ||
         (e = cudaMemsetAsync(q.dD, 0, d.heads * sizeof(float), s)) != cudaSuccess ||
@@ -596,7 +603,7 @@ cudaError_t launch_backward_t(const BackwardProblem &q, cudaStream_t s)
                                      d.batch, d.len, ch, dir, 1, s)) != cudaSuccess)
             return e;
     }
-    if (backward_tc_supported(d)) {
+    if (tc_path) {
         // the state and adjoint passes on the tensor cores
         BackwardTcProblem t{};
         t.dims = d;
