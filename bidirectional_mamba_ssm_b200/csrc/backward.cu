@@ -598,11 +598,9 @@ cudaError_t launch_backward_t(const BackwardProblem &q, cudaStream_t s)
         (e = cudaMemsetAsync(q.dconv_w, 0, (size_t)ch * 4 * sizeof(float), s)) != cudaSuccess ||
         (q.dconv_b && (e = cudaMemsetAsync(q.dconv_b, 0, (size_t)ch * sizeof(float), s)) != cudaSuccess))
         return e;
-    for (int dir = 0; dir < 2; ++dir) {
-        if ((e = launch_conv_silu<T>(q.xbc, const_cast<void *>(p.act[dir]), q.conv_w, q.conv_b, nullptr,
-                                     d.batch, d.len, ch, dir, 1, s)) != cudaSuccess)
-            return e;
-    }
+    if ((e = launch_conv_silu_both<T>(q.xbc, const_cast<void *>(p.act[0]), const_cast<void *>(p.act[1]),
+                                      q.conv_w, q.conv_b, d.batch, d.len, ch, s)) != cudaSuccess)
+        return e;
     if (tc_path) {
         // the state and adjoint passes on the tensor cores
         BackwardTcProblem t{};

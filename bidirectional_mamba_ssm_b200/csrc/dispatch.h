@@ -132,6 +132,11 @@ cudaError_t launch_conv_silu(const void *u, void *out, const float *w, const flo
                              const void *tail, int batch, int len, int ch, int rev, int silu,
                              cudaStream_t stream);
 
+// both streams' conv + SiLU of one raw input with tied taps, in token order
+template <typename T>
+cudaError_t launch_conv_silu_both(const void *u, void *out_f, void *out_r, const float *w, const float *bias,
+                                  int batch, int len, int ch, cudaStream_t stream);
+
 template <typename T>
 cudaError_t launch_scan_seq(const Problem &p, cudaStream_t stream);
 
