@@ -101,11 +101,10 @@ __device__ __forceinline__ float column_sum32(float (&v)[32], int lane)
 }
 
 // ---- state pass: shared memory (offsets from a 1024-byte aligned base)
-constexpr uint32_t kSOffX = 0;             // X [row][p]      16 KB (TMA)
+constexpr uint32_t kSOffX = 0;             // X [row][p]      16 KB (TMA), then w o X in place
 constexpr uint32_t kSOffB = 16384;         // B [row][n]      2 x 16 KB (TMA)
-constexpr uint32_t kSOffWX = 49152;        // w o X [row][p]  16 KB
-constexpr uint32_t kSOffS = 65536;         // S_in^T [n][p]   16 KB (to the workspace)
-constexpr uint32_t kSOffVec = 81920;       // f32 c[128] (log2 units, by row), dt[128]
+constexpr uint32_t kSOffS = 49152;         // S_in^T [n][p]   16 KB (to the workspace)
+constexpr uint32_t kSOffVec = 65536;       // f32 c[128] (log2 units, by row), dt[128]
 constexpr uint32_t kSOffMbar = kSOffVec + 1024;
 constexpr uint32_t kSOffTmem = kSOffMbar + 16;
 constexpr uint32_t kSSmem = kSOffTmem + 16 + 1024;
@@ -143,7 +142,7 @@ __device__ __forceinline__ void chunk_prefix(const float *dtv, float *cv, float 
 // The state entering every chunk of one (head, sequence, direction) walk,
 // as bf16 S_in^T tiles.  S^T (lane n, 64 columns p) lives in tensor memory;
 // per chunk: S_in^T -> tile, S^T <- e^{c_last} S^T + B^T (w o X).
-__global__ void __launch_bounds__(kBThreads, 2)
+__global__ void __launch_bounds__(kBThreads, 3)
 bwd_tc_state_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_constant__ CUtensorMap tm_act_r,
                     const BwdTcParams p)
 {
@@ -241,7 +240,7 @@ bwd_tc_state_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_c
                 unpack8(*reinterpret_cast<const uint4 *>(sm + kSOffX + off), f);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) f[i] *= ws;
-                *reinterpret_cast<uint4 *>(sm + kSOffWX + off) = pack8(f);
+                *reinterpret_cast<uint4 *>(sm + kSOffX + off) = pack8(f);   // (this thread's half row only)
             }
             tc::tmem_wait_st();
         }
@@ -255,7 +254,7 @@ bwd_tc_state_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_c
             // S^T[n][p] += sum_s B[s][n] (w o X)[s][p]: A = B read MN-major (M = n),
             // B operand = w o X MN-major (N = p)
             const uint64_t dBmn = tc::smem_desc(sbase + kSOffB, 16384, 1024);
-            const uint64_t dWX = tc::smem_desc(sbase + kSOffWX, 1024, 1024);
+            const uint64_t dWX = tc::smem_desc(sbase + kSOffX, 1024, 1024);
             constexpr uint32_t idS = tc::idesc_bf16(128, 64, 1, 1);
 #pragma unroll
             for (int ks = 0; ks < kBQ / 16; ++ks)
