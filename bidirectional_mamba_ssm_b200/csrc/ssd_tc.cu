@@ -373,6 +373,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     const uint32_t mb_sdone = sbase + kOffMbar + 104;   // the chunk's state product done (wX read)
     const uint32_t mb_s = sbase + kOffMbar + 96;     // state, its bf16 copy and wX ready (one arrival per group)
     const uint32_t mb_yfree = sbase + kOffMbar + 112;   // Yd / Yo columns free for the chunk (last rows staged)
+    const uint32_t mb_xr = sbase + kOffMbar + 120;      // (state-only pass) the chunk's X tile converted
     auto xbuf_off = [](int k) { return (k & 1) ? kOffXbuf1 : kOffXbuf0; };
 
     auto chunk_of = [&](int k, int &t0, int &cnt, int &s0) {
@@ -524,7 +525,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         tc::mbar_init(mb_x0 + 8, 1);
         tc::mbar_init(mb_g, 1);
         tc::mbar_init(mb_m, 1);
-        tc::mbar_init(mb_s, 2);          // one arrival from each compute group
+        // one arrival from each compute group (the state-only pass: from the
+        // tensor-memory group, which forms w o X there too)
+        tc::mbar_init(mb_s, kStateOnly ? 1 : 2);
+        tc::mbar_init(mb_xr, 1);
         tc::mbar_init(mb_e, 1);
         tc::mbar_init(mb_dt0, 32);       // every helper lane arrives after its part of a scan
         tc::mbar_init(mb_dt0 + 8, 32);
@@ -548,6 +552,24 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kOffTmem);
+
+    // wX = w_s * X for walk chunk k (X tile in x buffer k % 2): thread
+    // tt (slot j, head gh), the head's 64 channels
+    auto weight_chunk = [&](int k, int tt) {
+        // in bf16 pairs: w_s rounded to bf16, each product rounded once
+        const uint8_t *xt = sm + xbuf_off(k);
+        const int j = tt & 127, gh = tt >> 7;
+        const __nv_bfloat162 w2 = __float2bfloat162_rn(wgt[((k & 1) * kHeads + gh) * kQ + j]);
+#pragma unroll
+        for (int pc = 0; pc < 8; ++pc) {
+            const uint32_t off = gh * 16384 + tc::sw128(j, pc);
+            uint4 v = *reinterpret_cast<const uint4 *>(xt + off);
+            __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) h2[q] = __hmul2(h2[q], w2);
+            *reinterpret_cast<uint4 *>(sm + kOffXw + off) = v;
+        }
+    };
 
     if (warp == kProducerWarp) {
         // ================= producer: every MMA and every TMA load (lane 0)
@@ -985,43 +1007,64 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         // producer issues the first two products while M is being built.
         // (Every phase has one call site.)
         bool ok = true;
-        for (int j = 0; j <= nk && ok; ++j) {
-            if (j >= 1) {
-                ok = a_wait(mb_e, (j - 1) & 1);   // chunk j-1's MMAs done
-                if (!ok) break;
-                tc::fence_after_sync();
-            }
-            if (j < nk) {
-                // the state for chunk j first: its product runs while the rows
-                // of chunk j-1 are read out
-                ok = a_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);   // chunk j's prefix sums and factors
+        if constexpr (kStateOnly) {
+            // per chunk, once the other group has converted its x: the state
+            // scaling and w o X (so that the conv group never waits on the
+            // products)
+            for (int j = 0; j < nk && ok; ++j) {
+                ok = a_wait(mb_xr, j & 1);
+                if (ok && j >= 1) ok = a_wait(mb_e, (j - 1) & 1);   // the last product has read w o X
+                if (ok) ok = a_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);
                 if (!ok) break;
                 tc::fence_after_sync();
                 scale_state(j);
-                publish(mb_s, !kStateOnly);
+                weight_chunk(j, tid);
+                publish(mb_s, true);
+                if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * (j & 1));
             }
-            if (j >= 1) {
-                if constexpr (!kStateOnly) {
-                    stage_rows(j - 1);
-                    tc::fence_proxy_async();   // the staged rows, for the publisher's TMA stores
-                    tc::fence_before_sync();   // TMEM reads done before the next chunk's products
-                    grp_sync(1);
-                    if (tid == 0) {
-                        tc::mbar_arrive(mb_staged);
-                        if (j < nk) tc::mbar_arrive(mb_yfree);
-                    }
-                }
-                if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * ((j - 1) & 1));
-                if (j >= nk) break;
-            } else if (!kStateOnly && tid == 0) {
-                tc::mbar_arrive(mb_yfree);   // nothing staged before chunk 0
-            }
-            if constexpr (!kStateOnly) {
-                ok = a_wait(mb_g, j & 1);
-                if (!ok) break;
+            if (ok) {
+                ok = a_wait(mb_e, (nk - 1) & 1);   // the last chunk's product
                 tc::fence_after_sync();
-                build_m(j);
-                publish(mb_m, false);
+            }
+        } else {
+            for (int j = 0; j <= nk && ok; ++j) {
+                if (j >= 1) {
+                    ok = a_wait(mb_e, (j - 1) & 1);   // chunk j-1's MMAs done
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                }
+                if (j < nk) {
+                    // the state for chunk j first: its product runs while the rows
+                    // of chunk j-1 are read out
+                    ok = a_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);   // chunk j's prefix sums and factors
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    scale_state(j);
+                    publish(mb_s, !kStateOnly);
+                }
+                if (j >= 1) {
+                    if constexpr (!kStateOnly) {
+                        stage_rows(j - 1);
+                        tc::fence_proxy_async();   // the staged rows, for the publisher's TMA stores
+                        tc::fence_before_sync();   // TMEM reads done before the next chunk's products
+                        grp_sync(1);
+                        if (tid == 0) {
+                            tc::mbar_arrive(mb_staged);
+                            if (j < nk) tc::mbar_arrive(mb_yfree);
+                        }
+                    }
+                    if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * ((j - 1) & 1));
+                    if (j >= nk) break;
+                } else if (!kStateOnly && tid == 0) {
+                    tc::mbar_arrive(mb_yfree);   // nothing staged before chunk 0
+                }
+                if constexpr (!kStateOnly) {
+                    ok = a_wait(mb_g, j & 1);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    build_m(j);
+                    publish(mb_m, false);
+                }
             }
         }
         if (ok) {
@@ -1143,24 +1186,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             else
                 conv_impl(std::false_type{}, k);
         };
-        // wX = w_s * X for walk chunk k (X tile in x buffer k % 2): thread
-        // (slot j, head gh), the head's 64 channels
-        auto weight_chunk = [&](int k) {
-            // in bf16 pairs: w_s rounded to bf16, each product rounded once
-            const uint8_t *xt = sm + xbuf_off(k);
-            const int j = tb & 127, gh = tb >> 7;
-            const __nv_bfloat162 w2 = __float2bfloat162_rn(wgt[((k & 1) * kHeads + gh) * kQ + j]);
-#pragma unroll
-            for (int pc = 0; pc < 8; ++pc) {
-                const uint32_t off = gh * 16384 + tc::sw128(j, pc);
-                uint4 v = *reinterpret_cast<const uint4 *>(xt + off);
-                __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&v);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) h2[q] = __hmul2(h2[q], w2);
-                *reinterpret_cast<uint4 *>(sm + kOffXw + off) = v;
-            }
-        };
-
         // sequence shards: the reverse stream's conv reads the 3 tokens
         // after the shard (L .. L+2) from the head.  Raw row i of a reverse
         // chunk buffer is token t0 + i, so they land in the walk's first
@@ -1188,36 +1213,63 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         // wX(j-1).  (Every phase has one call site: the kernel's code stays
         // small enough for the instruction caches.)
         bool ok = true;
-        for (int j = 0; j < nk && ok; ++j) {
-            ok = b_wait(mb_x0 + 8 * (j & 1), (j >> 1) & 1);
-            if (!ok) break;
-            if (j == 0 && !rev && p.tail && k0 == 0) {
-                // decode and sequence shards: the conv history before token 0
-                // comes from the tail
-                for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
-                    const int r = e / (kPP / 8), g = e % (kPP / 8);
-                    *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
-                        *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
-                                                         hp * kPP + 8 * g);
-                }
-                grp_sync(2);
-            }
-            if (j < 2) head_rows(j);
-            conv_chunk(j);
-            if (j >= 1) {
-                // the state product of chunk j-1 has read wX
-                ok = b_wait(kStateOnly ? mb_e : mb_sdone, (j - 1) & 1);
+        if constexpr (kStateOnly) {
+            // per chunk: its raw rows (and halos) converted in place, handed to
+            // the tensor-memory group, which forms w o X
+            for (int j = 0; j < nk && ok; ++j) {
+                ok = b_wait(mb_x0 + 8 * (j & 1), (j >> 1) & 1);
                 if (!ok) break;
+                if (j == 0 && !rev && p.tail && k0 == 0) {
+                    // decode and sequence shards: the conv history before token 0
+                    // comes from the tail
+                    for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
+                        const int r = e / (kPP / 8), g = e % (kPP / 8);
+                        *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
+                            *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
+                                                             hp * kPP + 8 * g);
+                    }
+                    grp_sync(2);
+                }
+                if (j < 2) head_rows(j);
+                conv_chunk(j);
+                grp_sync(2);
+                if (tb == 0) {
+                    tc::mbar_arrive(mb_xr);
+                    tc::mbar_arrive(mb_free0 + 8 * (j & 1));   // (the conv reads no factors)
+                }
             }
-            // (also the barrier between the conv's writes and wX's reads)
-            ok = b_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);
-            if (!ok) break;
-            weight_chunk(j);
-            tc::fence_proxy_async();   // X and wX, for the tensor core
-            grp_sync(2);
-            if (tb == 0) {
-                tc::mbar_arrive(mb_s);
-                tc::mbar_arrive(mb_free0 + 8 * (j & 1));
+        } else {
+            for (int j = 0; j < nk && ok; ++j) {
+                ok = b_wait(mb_x0 + 8 * (j & 1), (j >> 1) & 1);
+                if (!ok) break;
+                if (j == 0 && !rev && p.tail && k0 == 0) {
+                    // decode and sequence shards: the conv history before token 0
+                    // comes from the tail
+                    for (int e = tb; e < 3 * (kPP / 8); e += kGroupThreads) {
+                        const int r = e / (kPP / 8), g = e % (kPP / 8);
+                        *reinterpret_cast<uint4 *>(sm + kOffXbuf0 + r * (kPP * 2) + g * 16) =
+                            *reinterpret_cast<const uint4 *>(p.tail + ((size_t)b * 4 + 1 + r) * ch +
+                                                             hp * kPP + 8 * g);
+                    }
+                    grp_sync(2);
+                }
+                if (j < 2) head_rows(j);
+                conv_chunk(j);
+                if (j >= 1) {
+                    // the state product of chunk j-1 has read wX
+                    ok = b_wait(kStateOnly ? mb_e : mb_sdone, (j - 1) & 1);
+                    if (!ok) break;
+                }
+                // (also the barrier between the conv's writes and wX's reads)
+                ok = b_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);
+                if (!ok) break;
+                weight_chunk(j, tb);
+                tc::fence_proxy_async();   // X and wX, for the tensor core
+                grp_sync(2);
+                if (tb == 0) {
+                    tc::mbar_arrive(mb_s);
+                    tc::mbar_arrive(mb_free0 + 8 * (j & 1));
+                }
             }
         }
         if (!ok && tb == 0) record_error(p.status, kStatusTimeout);
