@@ -370,10 +370,14 @@ int bimamba_block_decode_pool(const bimamba_dims *d, const void *xbc_block,
  *   dconv_w (ch, 4), dconv_b (ch) or NULL, dinit (batch, H, P, N) or NULL
  *   workspace  : bimamba_backward_workspace_bytes(d) bytes (no clearing
  *                needed); it holds both streams' activations, their fp32
- *                gradients and the state entering every 64-token chunk
+ *                gradients and the state entering every chunk
  * Shapes: headdim <= 64 and d_state <= 128, both multiples of 4 (else
- * BIMAMBA_ERR_UNSUPPORTED); fp32 or bf16 activations.  The chunked backward
- * runs its small matrix products on the CUDA cores in fp32.
+ * BIMAMBA_ERR_UNSUPPORTED); fp32 or bf16 activations.  For bf16 with
+ * headdim 64 and d_state 128 the chunked backward (128-token chunks) runs
+ * every matrix product on the tensor cores (bf16 operands, fp32
+ * accumulation); otherwise (64-token chunks) its small products run on the
+ * CUDA cores in fp32.  Errors: as bimamba_ssd_fwd_rev (a bounded wait that
+ * gave up is reported by bimamba_get_error as BIMAMBA_ERR_TIMEOUT).
  */
 size_t bimamba_backward_workspace_bytes(const bimamba_dims *d);
 
