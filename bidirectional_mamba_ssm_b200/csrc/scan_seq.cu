@@ -13,10 +13,11 @@
 // reverse stream (token len-1-s, index reflection, no flip copy); the
 // outputs are added.
 //
-// One CTA owns (batch b, head h) and runs both directions one after the
-// other: the forward pass writes y, the reverse pass adds to it (or, with
-// the concatenating fusion of untied directions, writes its own half of
-// each output row).  Each direction reads its own inputs and parameters.  Thread
+// One CTA owns (batch b, head h, direction): the two directions run side by
+// side and add their rows into y (zero-filled by the launcher; in fp32 a sum
+// of two terms is exact in either order), or, with the concatenating fusion
+// of untied directions, each writes its own half of each output row.  Each
+// direction reads its own inputs and parameters.  Thread
 // (p, q) owns state row p, columns n = q + NS*k (k < NPT), so each thread
 // carries NPT fp32 state values in registers; the y dot product is reduced
 // over the NS threads of a row with warp shuffles.  Activated x, B, C and dt
@@ -48,7 +49,7 @@ __global__ void __launch_bounds__(512)
 scan_seq_kernel(SeqParams p)
 {
     extern __shared__ float smem[];
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int h = blockIdx.x, b = blockIdx.y, dir = blockIdx.z;
     const int P = p.P, N = p.N, H = p.H, len = p.len, ch = p.ch;
     const int NS = N / NPT;
     const int tid = threadIdx.x;
@@ -57,7 +58,8 @@ scan_seq_kernel(SeqParams p)
     float *bs = xs + kSeqChunk * P;      // [kSeqChunk][N]
     float *cs = bs + kSeqChunk * N;      // [kSeqChunk][N]
     float *ys = cs + kSeqChunk * N;      // [kSeqChunk][P]
-    float *dts = ys + kSeqChunk * P;     // [kSeqChunk]
+    float *dts = ys + kSeqChunk * P;     // [kSeqChunk] dt
+    float *as = dts + kSeqChunk;         // [kSeqChunk] exp(dt A)
 
     const T *tail = p.tail ? static_cast<const T *>(p.tail) + (size_t)b * 4 * ch : nullptr;
     const size_t ystride = (size_t)(p.concat ? 2 : 1) * H * P;   // y row length
@@ -68,7 +70,7 @@ scan_seq_kernel(SeqParams p)
     const unsigned lane_mask = nlanes == 32 ? 0xffffffffu : ((1u << nlanes) - 1u);
     const size_t sidx = ((size_t)b * H + h) * P * N;
 
-    for (int dir = 0; dir < 2; ++dir) {
+    {
         const bool rev = dir == 1;
         // selects, not a run-time index into the parameter arrays
         const T *xbc = static_cast<const T *>(rev ? p.xbc[1] : p.xbc[0]) + (size_t)b * len * ch;
@@ -102,29 +104,40 @@ scan_seq_kernel(SeqParams p)
                     const float w0 = conv_w[c * 4 + 0], w1 = conv_w[c * 4 + 1];
                     const float w2 = conv_w[c * 4 + 2], w3 = conv_w[c * 4 + 3];
                     const float bias = conv_b ? conv_b[c] : 0.0f;
+                    // 8 steps at a time, their raw values requested together
                     float r0 = raw(s0 - 3), r1 = raw(s0 - 2), r2 = raw(s0 - 1);
-                    for (int i = 0; i < cnt; ++i) {
-                        float r3 = raw(s0 + i);
-                        float acc = bias;
-                        acc = fmaf(w0, r0, acc);
-                        acc = fmaf(w1, r1, acc);
-                        acc = fmaf(w2, r2, acc);
-                        acc = fmaf(w3, r3, acc);
-                        dst[i * dstride] = silu_f(acc);
-                        r0 = r1; r1 = r2; r2 = r3;
+                    for (int i0 = 0; i0 < cnt; i0 += 8) {
+                        float rv[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) rv[i] = i0 + i < cnt ? raw(s0 + i0 + i) : 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            if (i0 + i >= cnt) break;
+                            float acc = bias;
+                            acc = fmaf(w0, r0, acc);
+                            acc = fmaf(w1, r1, acc);
+                            acc = fmaf(w2, r2, acc);
+                            acc = fmaf(w3, rv[i], acc);
+                            dst[(i0 + i) * dstride] = silu_f(acc);
+                            r0 = r1; r1 = r2; r2 = rv[i];
+                        }
                     }
                 } else {
                     for (int i = 0; i < cnt; ++i) dst[i * dstride] = raw(s0 + i);
                 }
             }
-            for (int i = tid; i < cnt; i += blockDim.x)
-                dts[i] = Elem<T>::load(dtp + (size_t)walk_token(s0 + i, len, rev) * H + h);
+            for (int i = tid; i < cnt; i += blockDim.x) {
+                const float dv = Elem<T>::load(dtp + (size_t)walk_token(s0 + i, len, rev) * H + h);
+                dts[i] = dv;
+                as[i] = expf(dv * Ah);
+            }
             __syncthreads();
 
             // ---- recurrence over the chunk
+#pragma unroll 4
             for (int i = 0; i < cnt; ++i) {
                 const float d = dts[i];
-                const float a = expf(d * Ah);
+                const float a = as[i];
                 const float xv = xs[i * P + row];
                 const float dx = d * xv;
                 const float *bi = bs + i * N + q;
@@ -141,15 +154,15 @@ scan_seq_kernel(SeqParams p)
             }
             __syncthreads();
 
-            // ---- write back; the reverse pass adds to the forward result
-            // (sum fusion).  Visibility of the forward writes to other threads
-            // of this CTA is ordered by the __syncthreads() calls in between.
+            // ---- write back: added into the zero-filled y (sum fusion), or
+            // stored into this direction's half of the row (concatenation)
             for (int e = tid; e < cnt * P; e += blockDim.x) {
                 const int i = e / P, pc = e % P;
                 T *yp = y + (size_t)walk_token(s0 + i, len, rev) * ystride + h * P + pc;
-                float v = ys[e];
-                if (rev && !p.concat) v += Elem<T>::load(yp);
-                Elem<T>::store(yp, v);
+                if (p.concat)
+                    Elem<T>::store(yp, ys[e]);
+                else
+                    atomicAdd(yp, static_cast<T>(ys[e]));
             }
         }
         if (!rev && p.fin) {
@@ -163,13 +176,17 @@ template <typename T, int NPT>
 static cudaError_t launch_seq_t(const SeqParams &p, int batch, cudaStream_t stream)
 {
     const int threads = p.P * (p.N / NPT);
-    const size_t smem = sizeof(float) * (size_t)(kSeqChunk * (2 * p.P + 2 * p.N) + kSeqChunk);
+    const size_t smem = sizeof(float) * (size_t)(kSeqChunk * (2 * p.P + 2 * p.N) + 2 * kSeqChunk);
     cudaError_t e = cudaFuncSetAttribute(scan_seq_kernel<T, NPT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const TimingEvents ev = timing_events();
     if (ev.start && (e = cudaEventRecord(ev.start, stream)) != cudaSuccess) return e;
-    scan_seq_kernel<T, NPT><<<dim3(p.H, batch), threads, smem, stream>>>(p);
+    // the directions add their rows into y
+    if (!p.concat &&
+        (e = cudaMemsetAsync(p.y, 0, (size_t)batch * p.len * p.H * p.P * sizeof(T), stream)) != cudaSuccess)
+        return e;
+    scan_seq_kernel<T, NPT><<<dim3(p.H, batch, 2), threads, smem, stream>>>(p);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     count_launch();
@@ -196,7 +213,7 @@ cudaError_t launch_scan_seq(const Problem &pr, cudaStream_t stream)
     // at most 512 threads per CTA: P * (N / NPT) <= 512 for P <= 128, N <= 256
     if (N >= 64 && P * (N / 32) > 512) return launch_seq_t<T, 64>(p, batch, stream);
     if (N >= 32) return launch_seq_t<T, 32>(p, batch, stream);
-    if (N == 16) return launch_seq_t<T, 16>(p, batch, stream);
+    if (N == 16) return launch_seq_t<T, 4>(p, batch, stream);
     return launch_seq_t<T, 8>(p, batch, stream);
 }
 
