@@ -25,8 +25,9 @@
 //     and dt, A through dL/dc_j of the chunk's prefix sums (suffix sums for
 //     dt, sum_j dL/dc_j sum_{i<=j} dt_i for A); the small matrix products run
 //     on the CUDA cores out of shared memory;
-//  4. bwd_conv_kernel: each stream's dact through SiLU' and the transposed
-//     taps to d(xbc), plus the tap and bias gradients, both streams at once.
+//  4. bwd_conv_staged_kernel (conv_staged.cu): each stream's dact through
+//     SiLU' and the transposed taps to d(xbc), plus the tap and bias
+//     gradients, both streams at once.
 #include <algorithm>
 
 #include "common.cuh"
@@ -452,132 +453,6 @@ bwd_scan_kernel(const BwdParams p)
             p.dinit[((size_t)b * H + h) * pn + i] = dS[(i / N) * N + sw(i / N, i % N)];
 }
 
-// Conv backward of both streams for one (sequence, 4-channel group, token
-// tile): dpre = dact o SiLU'(pre); d(xbc) = the transposed taps applied to
-// dpre; tap and bias gradients accumulated.  One pass over the tile and its
-// 3-token halos: each token's raw values, pre-activations and dpre are
-// computed once and kept in sliding windows; a thread's 4 channels move as
-// one 16-byte access per fp32 tensor.
-template <typename T>
-__device__ __forceinline__ void load4(const T *p, float (&v)[4]);
-template <>
-__device__ __forceinline__ void load4<float>(const float *p, float (&v)[4])
-{
-    const float4 q = *reinterpret_cast<const float4 *>(p);
-    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-}
-template <>
-__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[4])
-{
-    const uint2 q = *reinterpret_cast<const uint2 *>(p);
-    v[0] = __uint_as_float(q.x << 16); v[1] = __uint_as_float(q.x & 0xffff0000u);
-    v[2] = __uint_as_float(q.y << 16); v[3] = __uint_as_float(q.y & 0xffff0000u);
-}
-
-template <typename T>
-__global__ void __launch_bounds__(128)
-bwd_conv_kernel(const T *__restrict__ u, const float *__restrict__ w, const float *__restrict__ bias,
-                const float *__restrict__ dact_f, const float *__restrict__ dact_r, float *__restrict__ du,
-                float *__restrict__ dw, float *__restrict__ db, int len, int ch)
-{
-    const int c0 = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
-    if (c0 >= ch) return;
-    const int b = blockIdx.z;
-    const int t0 = blockIdx.y * 64, t1 = min(t0 + 64, len);
-    const T *ub = u + (size_t)b * len * ch + c0;
-    const float *af = dact_f + (size_t)b * len * ch + c0;
-    const float *ar = dact_r + (size_t)b * len * ch + c0;
-    float wc[4][4], bc[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float4 q = *reinterpret_cast<const float4 *>(w + (size_t)(c0 + k) * 4);
-        wc[k][0] = q.x; wc[k][1] = q.y; wc[k][2] = q.z; wc[k][3] = q.w;
-        bc[k] = bias ? bias[c0 + k] : 0.0f;
-    }
-    auto dsilu = [](float x) {
-        const float sg = 1.0f / (1.0f + expf(-x));
-        return sg * (1.0f + x * (1.0f - sg));
-    };
-    // sliding windows, at output token t = tn - 3: uw[k] = u[t - 3 + k],
-    // pf[k] = dpre_f(t - 3 + k) (k = 0..6), pr[k] = dpre_r(t - 3 + k) (k = 0..3),
-    // per channel.  Every entry an output reads was brought in by the loop (it
-    // starts 3 tokens before the tile), so they start at zero
-    float uw[7][4], pf[7][4], pr[4][4];
-#pragma unroll
-    for (int k = 0; k < 7; ++k)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) uw[k][q] = pf[k][q] = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) pr[k][q] = 0.0f;
-    float g0[4] = {0, 0, 0, 0}, g1[4] = {0, 0, 0, 0}, g2[4] = {0, 0, 0, 0}, g3[4] = {0, 0, 0, 0},
-          gbs[4] = {0, 0, 0, 0};
-    // step tn = t + 3 brings in u[tn], dpre_f(tn) and dpre_r(tn - 3); token t
-    // completes (its du needs dpre_f up to t + 3 and dpre_r down to t - 3)
-    for (int tn = t0 - 3; tn < t1 + 3; ++tn) {
-        const int sr = tn - 3;
-        float un[4], afn[4], arn[4];
-        if (tn >= 0 && tn < len) {
-            load4<T>(ub + (size_t)tn * ch, un);
-            load4<float>(af + (size_t)tn * ch, afn);
-        } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) un[q] = afn[q] = 0.0f;
-        }
-        if (sr >= 0 && sr < len) {
-            load4<float>(ar + (size_t)sr * ch, arn);
-        } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) arn[q] = 0.0f;
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-            for (int k = 0; k < 6; ++k) {
-                uw[k][q] = uw[k + 1][q];
-                pf[k][q] = pf[k + 1][q];
-            }
-#pragma unroll
-            for (int k = 0; k < 3; ++k) pr[k][q] = pr[k + 1][q];
-            uw[6][q] = un[q];   // uw[k] = u[tn - 6 + k]
-            // dpre_f(tn): pre_f[tn] = b + sum_j w_j u[tn - 3 + j]
-            const float pre_f = bc[q] + wc[q][0] * uw[3][q] + wc[q][1] * uw[4][q] + wc[q][2] * uw[5][q] +
-                                wc[q][3] * uw[6][q];
-            pf[6][q] = (tn >= 0 && tn < len) ? afn[q] * dsilu(pre_f) : 0.0f;
-            // dpre_r(tn - 3): pre_r[s] = b + sum_j w_j u[s + 3 - j], s = tn - 3
-            const float pre_r = bc[q] + wc[q][0] * uw[6][q] + wc[q][1] * uw[5][q] + wc[q][2] * uw[4][q] +
-                                wc[q][3] * uw[3][q];
-            pr[3][q] = (sr >= 0 && sr < len) ? arn[q] * dsilu(pre_r) : 0.0f;
-        }
-        const int t = tn - 3;
-        if (t >= t0 && t < t1) {
-            float g[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                // pf[k] = dpre_f(t - 3 + k); uw[k] = u[t - 3 + k]
-                g[q] = wc[q][0] * pf[6][q] + wc[q][1] * pf[5][q] + wc[q][2] * pf[4][q] + wc[q][3] * pf[3][q] +
-                       wc[q][0] * pr[0][q] + wc[q][1] * pr[1][q] + wc[q][2] * pr[2][q] + wc[q][3] * pr[3][q];
-                const float dpf = pf[3][q], dpr = pr[3][q];
-                g0[q] += dpf * uw[0][q] + dpr * uw[6][q];
-                g1[q] += dpf * uw[1][q] + dpr * uw[5][q];
-                g2[q] += dpf * uw[2][q] + dpr * uw[4][q];
-                g3[q] += (dpf + dpr) * uw[3][q];
-                gbs[q] += dpf + dpr;
-            }
-            *reinterpret_cast<float4 *>(du + ((size_t)b * len + t) * ch + c0) = make_float4(g[0], g[1], g[2], g[3]);
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        atomicAdd(dw + (c0 + q) * 4, g0[q]);
-        atomicAdd(dw + (c0 + q) * 4 + 1, g1[q]);
-        atomicAdd(dw + (c0 + q) * 4 + 2, g2[q]);
-        atomicAdd(dw + (c0 + q) * 4 + 3, g3[q]);
-        if (db) atomicAdd(db + c0 + q, gbs[q]);
-    }
-}
-
 bool backward_supported(const bimamba_dims &d)
 {
     return d.ngroups == 1 && d.d_conv == 4 && d.headdim <= 64 && d.d_state <= 128 &&
@@ -643,8 +518,10 @@ cudaError_t launch_backward_t(const BackwardProblem &q, cudaStream_t s)
         (e = cudaMemsetAsync(q.dconv_w, 0, (size_t)ch * 4 * sizeof(float), s)) != cudaSuccess ||
         (q.dconv_b && (e = cudaMemsetAsync(q.dconv_b, 0, (size_t)ch * sizeof(float), s)) != cudaSuccess))
         return e;
-    if ((e = launch_conv_silu_both<T>(q.xbc, const_cast<void *>(p.act[0]), const_cast<void *>(p.act[1]),
-                                      q.conv_w, q.conv_b, d.batch, d.len, ch, s)) != cudaSuccess)
+    // both streams' activations from one pass over the raw rows (TMA-staged
+    // tiles; the entry point has checked the 16-byte alignment they need)
+    if ((e = launch_conv_silu_both_staged<T>(q.xbc, const_cast<void *>(p.act[0]), const_cast<void *>(p.act[1]),
+                                             q.conv_w, q.conv_b, d.batch, d.len, ch, s)) != cudaSuccess)
         return e;
     if (tc_path) {
         // the state and adjoint passes on the tensor cores
@@ -684,12 +561,8 @@ cudaError_t launch_backward_t(const BackwardProblem &q, cudaStream_t s)
         count_launch();
         if (ev.stop && (e = cudaEventRecord(ev.stop, s)) != cudaSuccess) return e;
     }
-    bwd_conv_kernel<T><<<dim3((ch / 4 + 127) / 128, (d.len + 63) / 64, d.batch), 128, 0, s>>>(
-        static_cast<const T *>(q.xbc), q.conv_w, q.conv_b, p.dact[0], p.dact[1], q.dxbc, q.dconv_w,
-        q.dconv_b, d.len, ch);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    count_launch();
-    return cudaSuccess;
+    return launch_bwd_conv_staged<T>(q.xbc, q.conv_w, q.conv_b, p.dact[0], p.dact[1], q.dxbc, q.dconv_w,
+                                     q.dconv_b, d.batch, d.len, ch, s);
 }
 
 cudaError_t launch_backward(const BackwardProblem &q, cudaStream_t s)

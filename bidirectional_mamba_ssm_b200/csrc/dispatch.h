@@ -132,10 +132,17 @@ cudaError_t launch_conv_silu(const void *u, void *out, const float *w, const flo
                              const void *tail, int batch, int len, int ch, int rev, int silu,
                              cudaStream_t stream);
 
-// both streams' conv + SiLU of one raw input with tied taps, in token order
+// both streams' conv + SiLU of one raw input with tied taps, in token order,
+// and the conv backward of both streams, from TMA-staged tiles (raw rows,
+// activations and gradients 16-byte aligned, ch a multiple of 8)
 template <typename T>
-cudaError_t launch_conv_silu_both(const void *u, void *out_f, void *out_r, const float *w, const float *bias,
-                                  int batch, int len, int ch, cudaStream_t stream);
+cudaError_t launch_conv_silu_both_staged(const void *u, void *out_f, void *out_r, const float *w,
+                                         const float *bias, int batch, int len, int ch, cudaStream_t stream);
+// du = d(loss)/d(raw xBC) (fp32), dw / db += the tap and bias gradients
+template <typename T>
+cudaError_t launch_bwd_conv_staged(const void *u, const float *w, const float *bias, const float *dact_f,
+                                   const float *dact_r, float *du, float *dw, float *db, int batch, int len,
+                                   int ch, cudaStream_t stream);
 
 template <typename T>
 cudaError_t launch_scan_seq(const Problem &p, cudaStream_t stream);
