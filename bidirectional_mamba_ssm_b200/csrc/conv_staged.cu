@@ -90,18 +90,41 @@ template <> __device__ __forceinline__ void stg4<__nv_bfloat16>(__nv_bfloat16 *p
     *reinterpret_cast<uint2 *>(p) = make_uint2(tc::pack_bf16x2(v[0], v[1]), tc::pack_bf16x2(v[2], v[3]));
 }
 
-// SiLU and its derivative through the fast exponential and divide
-// intrinsics (relative error ~1e-6, far inside the fp32 and bf16 bounds):
-// with the IEEE expf and division the conv passes were bound by these
-// instructions rather than by HBM.  For x -> -inf, 1 + e^-x overflows to inf
-// and both give (-)0.
-__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
-
-__device__ __forceinline__ float dsilu(float x)
-{
-    const float sg = __fdividef(1.0f, 1.0f + __expf(-x));
-    return sg * (1.0f + x * (1.0f - sg));
-}
+// SiLU and its derivative, by the activation dtype.  fp32: through the fast
+// exponential and divide intrinsics (relative error ~1e-6, inside the fp32
+// bound; for x -> -inf, 1 + e^-x overflows to inf and both give (-)0).
+// bf16: through the hardware tanh, sigma(x) = 1/2 + tanh(x/2)/2 (relative
+// error ~1e-3 in sigma, far inside the bf16 bound), one special-function
+// operation instead of two.  With the IEEE expf and division the conv
+// passes were bound by these instructions rather than by HBM.
+template <typename T> struct Act;
+template <> struct Act<float> {
+    static __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+    static __device__ __forceinline__ float dsilu(float x)
+    {
+        const float sg = __fdividef(1.0f, 1.0f + __expf(-x));
+        return sg * (1.0f + x * (1.0f - sg));
+    }
+};
+template <> struct Act<__nv_bfloat16> {
+    static __device__ __forceinline__ float tanh_approx(float x)
+    {
+        float t;
+        asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
+        return t;
+    }
+    // x sigma(x) = h + h tanh(h), h = x / 2
+    static __device__ __forceinline__ float silu(float x)
+    {
+        const float h = 0.5f * x;
+        return fmaf(h, tanh_approx(h), h);
+    }
+    static __device__ __forceinline__ float dsilu(float x)
+    {
+        const float sg = fmaf(0.5f, tanh_approx(0.5f * x), 0.5f);
+        return sg * (1.0f + x * (1.0f - sg));
+    }
+};
 
 // One thread issues the tile's TMA boxes onto one mbarrier; every thread
 // waits (bounded).  Returns false on timeout (recorded in the status word).
@@ -169,8 +192,8 @@ conv_silu_both_staged_kernel(const __grid_constant__ CUtensorMap tm_u, T *__rest
             ar = fmaf(wt[k][1], x[5][k], ar);
             ar = fmaf(wt[k][2], x[4][k], ar);
             ar = fmaf(wt[k][3], x[3][k], ar);
-            of[k] = silu_fast(af);
-            orr[k] = silu_fast(ar);
+            of[k] = Act<T>::silu(af);
+            orr[k] = Act<T>::silu(ar);
         }
         if (t0 + i0 + i < len && c < ch) {
             stg4<T>(out_f + base + (size_t)(i0 + i) * ch, of);
@@ -238,8 +261,8 @@ bwd_conv_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_co
         for (int k = 0; k < 4; ++k) {
             const float pre_f = bc[k] + wc[k][0] * u0[k] + wc[k][1] * u1[k] + wc[k][2] * u2[k] + wc[k][3] * u3[k];
             const float pre_r = bc[k] + wc[k][0] * u3[k] + wc[k][1] * u2[k] + wc[k][2] * u1[k] + wc[k][3] * u0[k];
-            a[k] *= dsilu(pre_f);
-            e[k] *= dsilu(pre_r);
+            a[k] *= Act<T>::dsilu(pre_f);
+            e[k] *= Act<T>::dsilu(pre_r);
         }
         *reinterpret_cast<float4 *>(pf + r * kTileC + 4 * q) = make_float4(a[0], a[1], a[2], a[3]);
         *reinterpret_cast<float4 *>(pr + r * kTileC + 4 * q) = make_float4(e[0], e[1], e[2], e[3]);
