@@ -43,7 +43,8 @@ namespace {
 constexpr int kBQ = 128;   // chunk length (walk slots)
 constexpr int kBP = 64;    // headdim
 constexpr int kBN = 128;   // d_state
-constexpr int kBThreads = 256;   // thread: tile row r = tid & 127, column half tid >> 7
+constexpr int kBThreads = 256;   // state pass: tile row r = tid & 127, column half tid >> 7
+constexpr int kAThreads = 512;   // adjoint pass: tile row r = tid & 127, column quarter tid >> 7
 constexpr long long kBWait = 4000000000LL;   // ~2 s at 1.9 GHz
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTileBytes = kBN * kBP * 2;   // one S_in^T tile (16 KB)
@@ -98,6 +99,27 @@ __device__ __forceinline__ float column_sum32(float (&v)[32], int lane)
         }
     }
     return v[0];
+}
+
+// Column sums of a 32-row x 16-column block held one row per lane (v[i] =
+// column i): recursive halving keeps, at each step, the half of the columns
+// selected by one lane bit and adds the partner's other half; after four
+// steps lanes l and l ^ 1 hold partial sums of column l >> 1 over the lanes
+// of their parity, and one more exchange completes both (16 shuffles).
+__device__ __forceinline__ float column_sum16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+        const int o = 16 >> st, m = 8 >> st;   // partner distance, columns kept
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < m; ++i) {
+            const float send = up ? v[i] : v[i + m];
+            const float keep = up ? v[i + m] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
 // ---- state pass: shared memory (offsets from a 1024-byte aligned base)
@@ -286,8 +308,8 @@ constexpr uint32_t kAOffSin = 163840;   // S_in^T [n][p] 16 KB (bulk copy)
 constexpr uint32_t kAOffDS = 180224;    // dS^T [n][p] 16 KB (bf16 copy of the TMEM adjoint)
 constexpr uint32_t kAOffVec = 196608;   // f32 vectors (below)
 // f32 vectors (offsets in floats; see the kernel)
-constexpr int kVCv = 0, kVDt = kVCv + kBQ, kVCum = kVDt + kBQ, kVRsp = kVCum + kBQ, kVDdp = kVRsp + 2 * kBQ,
-              kVCsp = kVDdp + 4 * kBQ, kVXbp = kVCsp + 2 * kBQ, kVSdp = kVXbp + 2 * kBQ, kVDcw = kVSdp + 2 * kBQ,
+constexpr int kVCv = 0, kVDt = kVCv + kBQ, kVCum = kVDt + kBQ, kVRsp = kVCum + kBQ, kVDdp = kVRsp + 4 * kBQ,
+              kVCsp = kVDdp + 4 * kBQ, kVXbp = kVCsp + 4 * kBQ, kVSdp = kVXbp + 4 * kBQ, kVDcw = kVSdp + 4 * kBQ,
               kVGdw = kVDcw + kBQ, kVUw = kVGdw + kBQ, kVRed = kVUw + kBQ;
 constexpr int kVecFloats = kVRed + 64;
 constexpr uint32_t kAOffMbar = kAOffVec + 4 * kVecFloats;
@@ -314,7 +336,7 @@ constexpr uint32_t kColDS = 448;    // dS^T (n, p), fp32, carried across chunks
 //  P4  dX and dB out, dt and A, e^c o dY in place, dS^T <- e^{c_last} dS^T
 //  P5  dC += (e^c o dY) S_in, dS^T += C^T (e^c o dY)
 //  P6  dC out
-__global__ void __launch_bounds__(kBThreads, 1)
+__global__ void __launch_bounds__(kAThreads, 1)
 bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_constant__ CUtensorMap tm_act_r,
                    const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_dact_f,
                    const __grid_constant__ CUtensorMap tm_dact_r, const BwdTcParams p)
@@ -323,7 +345,7 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
     uint8_t *sm = align1024(smem_raw);
     const uint32_t sbase = tc::smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r = tid & (kBQ - 1), hw = tid >> 7, quarter = warp & 3;
+    const int r = tid & (kBQ - 1), qc = tid >> 7, quarter = warp & 3;
     const int h = blockIdx.x, b = blockIdx.y, dir = blockIdx.z;
     const bool rev = dir != 0;
     const int L = p.len, H = p.H, ch = p.ch, nc = p.nchunks;
@@ -334,11 +356,11 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
     float *cv = vec + kVCv;       // [128] c (log2 units) by row
     float *dtv = vec + kVDt;      // [128] dt by row
     float *cumw = vec + kVCum;    // [128] prefix sums of dt by walk slot
-    float *rsp = vec + kVRsp;     // [2][128] row sums of dY X^T o W, per column half
+    float *rsp = vec + kVRsp;     // [4][128] row sums of dY X^T o W, per column quarter
     float *ddp = vec + kVDdp;     // [4][128] column sums of dY X^T o C B^T o e, per row quarter
-    float *csp = vec + kVCsp;     // [2][128] dY_t . (C S_in^T)_t per half
-    float *xbp = vec + kVXbp;     // [2][128] x_s . (B dS^T)_s per half
-    float *sdp = vec + kVSdp;     // [2][128] <dS^T, S_in^T> of row n per half
+    float *csp = vec + kVCsp;     // [4][128] dY_t . (C S_in^T)_t per quarter
+    float *xbp = vec + kVXbp;     // [4][128] x_s . (B dS^T)_s per quarter
+    float *sdp = vec + kVSdp;     // [4][128] <dS^T, S_in^T> of row n per quarter
     float *dcw = vec + kVDcw;     // [128] dL/dc by walk slot
     float *gdw = vec + kVGdw;     // [128] direct dt terms by walk slot
     float *uw = vec + kVUw;       // [128] U_s by row
@@ -365,8 +387,7 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         uint32_t z[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) z[i] = 0u;
-        tc::tmem_st16_nw(trow + kColDS + 32 * hw, z);
-        tc::tmem_st16_nw(trow + kColDS + 32 * hw + 16, z);
+        tc::tmem_st16_nw(trow + kColDS + 16 * qc, z);
         tc::tmem_wait_st();
     }
     const float a2 = p.A[h] * kLog2e, Aa = p.A[h], Dh = p.D[h];
@@ -411,15 +432,15 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         }
         if (tid < kBQ) dtv[r] = tok_ok ? __bfloat162float(p.dt[((size_t)b * L + tok) * H + h]) : 0.0f;
         {
-            uint32_t v[32];
-            tc::tmem_ld32_nw(trow + kColDS + 32 * hw, v);
-            tc::tmem_wait_ld(v);
+            uint32_t v[16];
+            tc::tmem_ld16_nw(trow + kColDS + 16 * qc, v);
+            tc::tmem_wait_ld16(v);
 #pragma unroll
-            for (int pc = 0; pc < 4; ++pc) {
+            for (int pc = 0; pc < 2; ++pc) {
                 float f[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(v[8 * pc + i]);
-                *reinterpret_cast<uint4 *>(sm + kAOffDS + tc::sw128(r, 4 * hw + pc)) = pack8(f);
+                *reinterpret_cast<uint4 *>(sm + kAOffDS + tc::sw128(r, 2 * qc + pc)) = pack8(f);
             }
         }
         tc::fence_proxy_async();
@@ -464,23 +485,24 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         tc::fence_after_sync();
         const float ct = cv[r];
         const float clast = cv[rev ? 0 : kBQ - 1];
-        // ---- P2: W and T of row t = r, columns s = 64 hw .. 64 hw + 63
+        // ---- P2: W and T of row t = r, columns s = 32 qc .. 32 qc + 31 (two
+        // passes of 16)
         {
             float rs = 0.0f;
 #pragma unroll 1
             for (int g = 0; g < 2; ++g) {
-                const int s0 = 64 * hw + 32 * g;
-                uint32_t cb[32], yx[32];
-                tc::tmem_ld32_nw(trow + kColCB + s0, cb);
-                tc::tmem_ld32_nw(trow + kColDYX + s0, yx);
-                tc::tmem_wait_ld(cb);
-                tc::tmem_wait_ld(yx);
+                const int s0 = 32 * qc + 16 * g;
+                uint32_t cb[16], yx[16];
+                tc::tmem_ld16_nw(trow + kColCB + s0, cb);
+                tc::tmem_ld16_nw(trow + kColDYX + s0, yx);
+                tc::tmem_wait_ld16(cb);
+                tc::tmem_wait_ld16(yx);
                 // pd = dY X^T o C B^T o e; its row sums weighted by dt_s (rs) and
                 // its column sums (times dt_s: those of dY X^T o W) feed dL/dc
-                float pd[32];
-                uint32_t wp[16], tp[16];
+                float pd[16];
+                uint32_t wp[8], tp[8];
 #pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
+                for (int i4 = 0; i4 < 4; ++i4) {
                     const float4 c4 = *reinterpret_cast<const float4 *>(cv + s0 + 4 * i4);
                     const float4 d4 = *reinterpret_cast<const float4 *>(dtv + s0 + 4 * i4);
                     const float cs_[4] = {c4.x, c4.y, c4.z, c4.w};
@@ -503,33 +525,36 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
                     tp[2 * i4] = tc::pack_bf16x2(tv[0], tv[1]);
                     tp[2 * i4 + 1] = tc::pack_bf16x2(tv[2], tv[3]);
                 }
+                // columns s0 .. s0+15: 64-column panel qc >> 1, 8-column pieces
+                // 4 (qc & 1) + 2 g + pc
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc) {
-                    const uint32_t off = hw * 16384 + tc::sw128(r, 4 * g + pc);
+                for (int pc = 0; pc < 2; ++pc) {
+                    const uint32_t off = (qc >> 1) * 16384 + tc::sw128(r, 4 * (qc & 1) + 2 * g + pc);
                     *reinterpret_cast<uint4 *>(sm + kAOffW + off) =
                         make_uint4(wp[4 * pc], wp[4 * pc + 1], wp[4 * pc + 2], wp[4 * pc + 3]);
                     *reinterpret_cast<uint4 *>(sm + kAOffT + off) =
                         make_uint4(tp[4 * pc], tp[4 * pc + 1], tp[4 * pc + 2], tp[4 * pc + 3]);
                 }
-                ddp[quarter * kBQ + s0 + lane] = column_sum32(pd, lane);
+                const float csum = column_sum16(pd, lane);
+                if ((lane & 1) == 0) ddp[quarter * kBQ + s0 + (lane >> 1)] = csum;
             }
-            rsp[hw * kBQ + r] = rs;
+            rsp[qc * kBQ + r] = rs;
         }
-        // per-row dot products over this half's 32 p: dY_t . (C S_in^T)_t,
+        // per-row dot products over this quarter's 16 p: dY_t . (C S_in^T)_t,
         // x_s . (B dS^T)_s, dY . x (for D), and <dS^T, S_in^T> of row n = r
         {
-            uint32_t cs[32], x2[32], ds[32];
-            tc::tmem_ld32_nw(trow + kColCS + 32 * hw, cs);
-            tc::tmem_ld32_nw(trow + kColDX2 + 32 * hw, x2);
-            tc::tmem_ld32_nw(trow + kColDS + 32 * hw, ds);
-            tc::tmem_wait_ld(cs);
-            tc::tmem_wait_ld(x2);
-            tc::tmem_wait_ld(ds);
+            uint32_t cs[16], x2[16], ds[16];
+            tc::tmem_ld16_nw(trow + kColCS + 16 * qc, cs);
+            tc::tmem_ld16_nw(trow + kColDX2 + 16 * qc, x2);
+            tc::tmem_ld16_nw(trow + kColDS + 16 * qc, ds);
+            tc::tmem_wait_ld16(cs);
+            tc::tmem_wait_ld16(x2);
+            tc::tmem_wait_ld16(ds);
             float a_cs = 0.0f, a_xb = 0.0f, a_dd = 0.0f, a_sd = 0.0f;
             const float ws = tc::exp2_approx(fminf(clast - ct, 0.0f)) * dtv[r];
 #pragma unroll
-            for (int pc = 0; pc < 4; ++pc) {
-                const uint32_t off = tc::sw128(r, 4 * hw + pc);
+            for (int pc = 0; pc < 2; ++pc) {
+                const uint32_t off = tc::sw128(r, 2 * qc + pc);
                 float yv[8], xv[8], sv[8];
                 unpack8(*reinterpret_cast<const uint4 *>(sm + kAOffDY + off), yv);
                 unpack8(*reinterpret_cast<const uint4 *>(sm + kAOffX + off), xv);
@@ -542,12 +567,12 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
                     a_sd = fmaf(__uint_as_float(ds[8 * pc + i]), sv[i], a_sd);
                     xv[i] *= ws;
                 }
-                // w o X in place (this thread is the last reader of its half row)
+                // w o X in place (this thread is the last reader of its quarter row)
                 *reinterpret_cast<uint4 *>(sm + kAOffX + off) = pack8(xv);
             }
-            csp[hw * kBQ + r] = a_cs;
-            xbp[hw * kBQ + r] = a_xb;
-            sdp[hw * kBQ + r] = a_sd;
+            csp[qc * kBQ + r] = a_cs;
+            xbp[qc * kBQ + r] = a_xb;
+            sdp[qc * kBQ + r] = a_sd;
             dD_acc += a_dd;
         }
         tc::fence_proxy_async();
@@ -586,19 +611,19 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         ok = __syncthreads_and(ok);
         if (!ok) break;
         tc::fence_after_sync();
-        // ---- P4: dX of row s = r (this half's 32 p), dB of row s (64 n)
+        // ---- P4: dX of row s = r (this quarter's 16 p), dB of row s (32 n)
         const float ws = tc::exp2_approx(fminf(clast - ct, 0.0f)) * dtv[r];
         {
-            uint32_t a1[32], a2v[32];
-            tc::tmem_ld32_nw(trow + kColDX1 + 32 * hw, a1);
-            tc::tmem_ld32_nw(trow + kColDX2 + 32 * hw, a2v);
-            tc::tmem_wait_ld(a1);
-            tc::tmem_wait_ld(a2v);
+            uint32_t a1[16], a2v[16];
+            tc::tmem_ld16_nw(trow + kColDX1 + 16 * qc, a1);
+            tc::tmem_ld16_nw(trow + kColDX2 + 16 * qc, a2v);
+            tc::tmem_wait_ld16(a1);
+            tc::tmem_wait_ld16(a2v);
             const float ec = tc::exp2_approx(fminf(ct, 0.0f));
-            float4 *dst = reinterpret_cast<float4 *>(dact + ((size_t)b * L + tok) * ch + h * kBP + 32 * hw);
+            float4 *dst = reinterpret_cast<float4 *>(dact + ((size_t)b * L + tok) * ch + h * kBP + 16 * qc);
 #pragma unroll
-            for (int pc = 0; pc < 4; ++pc) {
-                const uint32_t off = tc::sw128(r, 4 * hw + pc);
+            for (int pc = 0; pc < 2; ++pc) {
+                const uint32_t off = tc::sw128(r, 2 * qc + pc);
                 float yv[8], o[8];
                 unpack8(*reinterpret_cast<const uint4 *>(sm + kAOffDY + off), yv);
 #pragma unroll
@@ -611,18 +636,18 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
                     dst[2 * pc] = make_float4(o[0], o[1], o[2], o[3]);
                     dst[2 * pc + 1] = make_float4(o[4], o[5], o[6], o[7]);
                 }
-                // e^c o dY in place (this thread is the last reader of its half row)
+                // e^c o dY in place (this thread is the last reader of its quarter row)
                 *reinterpret_cast<uint4 *>(sm + kAOffDY + off) = pack8(yv);
             }
         }
         // dB rows staged as four 32-column fp32 boxes (128-byte swizzle) in the
         // W and T tiles, which the products above have finished with
-#pragma unroll 1
-        for (int g = 0; g < 2; ++g) {
+        {
+            // box qc: columns 32 qc .. 32 qc + 31
             uint32_t v[32];
-            tc::tmem_ld32_nw(trow + kColCB + 64 * hw + 32 * g, v);
+            tc::tmem_ld32_nw(trow + kColCB + 32 * qc, v);
             tc::tmem_wait_ld(v);
-            uint8_t *box = sm + (hw ? kAOffT : kAOffW) + 16384 * g;
+            uint8_t *box = sm + (qc < 2 ? kAOffW : kAOffT) + 16384 * (qc & 1);
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 *reinterpret_cast<uint4 *>(box + tc::sw128(q, c)) =
@@ -630,27 +655,26 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         }
         {
             // dS^T <- e^{c_last} dS^T (its bf16 copy was taken in P0)
-            uint32_t v[32];
-            tc::tmem_ld32_nw(trow + kColDS + 32 * hw, v);
-            tc::tmem_wait_ld(v);
+            uint32_t v[16];
+            tc::tmem_ld16_nw(trow + kColDS + 16 * qc, v);
+            tc::tmem_wait_ld16(v);
             const float al = tc::exp2_approx(clast);
+            uint32_t u[16];
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                uint32_t u[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(v[16 * g + i]) * al);
-                tc::tmem_st16_nw(trow + kColDS + 32 * hw + 16 * g, u);
-            }
+            for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(v[i]) * al);
+            tc::tmem_st16_nw(trow + kColDS + 16 * qc, u);
         }
-        if (hw == 0) {
+        if (qc == 0) {
             // dL/dc and the direct dt terms of row r, by walk slot
             const int j = rev ? kBQ - 1 - r : r;
-            const float xb = xbp[r] + xbp[kBQ + r];
+            const float xb = (xbp[r] + xbp[kBQ + r]) + (xbp[2 * kBQ + r] + xbp[3 * kBQ + r]);
             const float el = tc::exp2_approx(fminf(clast - ct, 0.0f));
             const float u = el * dtv[r] * xb;
             const float dsum = ddp[r] + ddp[kBQ + r] + ddp[2 * kBQ + r] + ddp[3 * kBQ + r];
             const float csum = dsum * dtv[r];   // column sum of dY X^T o W
-            dcw[j] = tc::exp2_approx(fminf(ct, 0.0f)) * (csp[r] + csp[kBQ + r]) - u + (rsp[r] + rsp[kBQ + r]) - csum;
+            const float cs4 = (csp[r] + csp[kBQ + r]) + (csp[2 * kBQ + r] + csp[3 * kBQ + r]);
+            const float rs4 = (rsp[r] + rsp[kBQ + r]) + (rsp[2 * kBQ + r] + rsp[3 * kBQ + r]);
+            dcw[j] = tc::exp2_approx(fminf(ct, 0.0f)) * cs4 - u + rs4 - csum;
             gdw[j] = dsum + el * xb;
             uw[r] = u;
         }
@@ -673,7 +697,7 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
             float sd = 0.0f, us = 0.0f;
 #pragma unroll
             for (int i = lane; i < kBQ; i += 32) {
-                sd += sdp[i] + sdp[kBQ + i];
+                sd += (sdp[i] + sdp[kBQ + i]) + (sdp[2 * kBQ + i] + sdp[3 * kBQ + i]);
                 us += uw[i];
             }
 #pragma unroll
@@ -733,12 +757,11 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         // ---- P6: dC of row t = r (64 n), staged like dB in the X, B and S_in
         // tiles (every product that reads them is done; the next chunk's
         // loads into them wait for the reductions to read them)
-#pragma unroll 1
-        for (int g = 0; g < 2; ++g) {
+        {
             uint32_t v[32];
-            tc::tmem_ld32_nw(trow + kColDYX + 64 * hw + 32 * g, v);
+            tc::tmem_ld32_nw(trow + kColDYX + 32 * qc, v);
             tc::tmem_wait_ld(v);
-            const int j = 2 * hw + g;
+            const int j = qc;   // box j: columns 32 j .. 32 j + 31
             uint8_t *box = sm + (j == 0 ? kAOffX : j == 3 ? kAOffSin : kAOffB + 16384 * (j - 1));
 #pragma unroll
             for (int c = 0; c < 8; ++c)
@@ -760,12 +783,12 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
     if (ok) {
         if (!rev && p.dinit) {
             // the adjoint of the caller's initial state: dinit[p][n] = dS^T[n][p]
-            uint32_t v[32];
-            tc::tmem_ld32_nw(trow + kColDS + 32 * hw, v);
-            tc::tmem_wait_ld(v);
+            uint32_t v[16];
+            tc::tmem_ld16_nw(trow + kColDS + 16 * qc, v);
+            tc::tmem_wait_ld16(v);
             float *dst = p.dinit + ((size_t)b * H + h) * kBP * kBN;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) dst[(size_t)(32 * hw + i) * kBN + r] = __uint_as_float(v[i]);
+            for (int i = 0; i < 16; ++i) dst[(size_t)(16 * qc + i) * kBN + r] = __uint_as_float(v[i]);
         }
         // D and A of this head
 #pragma unroll
@@ -774,7 +797,7 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         __syncthreads();
         if (tid == 0) {
             float s = 0.0f;
-            for (int i = 0; i < kBThreads / 32; ++i) s += red[i];
+            for (int i = 0; i < kAThreads / 32; ++i) s += red[i];
             atomicAdd(p.dD + h, s);
         }
         if (warp == 0) {
@@ -875,7 +898,7 @@ cudaError_t launch_backward_tc(const BackwardTcProblem &q, cudaStream_t s)
     count_launch();
     const TimingEvents ev = timing_events();
     if (ev.start && (e = cudaEventRecord(ev.start, s)) != cudaSuccess) return e;
-    bwd_tc_scan_kernel<<<grid, kBThreads, kASmem, s>>>(tm_f, tm_r, tm_dy, tm_df, tm_dr, p);
+    bwd_tc_scan_kernel<<<grid, kAThreads, kASmem, s>>>(tm_f, tm_r, tm_dy, tm_df, tm_dr, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launch();
     if (ev.stop && (e = cudaEventRecord(ev.stop, s)) != cudaSuccess) return e;
