@@ -621,23 +621,33 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
             tc::tmem_wait_ld16(a2v);
             const float ec = tc::exp2_approx(fminf(ct, 0.0f));
             float4 *dst = reinterpret_cast<float4 *>(dact + ((size_t)b * L + tok) * ch + h * kBP + 16 * qc);
+            // the rows leave by two TMA stores of 32-column fp32 boxes (128-byte
+            // swizzle) staged in the X and dS tiles, which the products have
+            // finished with; a chunk whose first row lies before token 0 (the
+            // reverse walk's short chunk: a store may not start at a negative
+            // row) by per-thread stores
+            uint8_t *xbox = sm + ((qc >> 1) ? kAOffDS : kAOffX);
 #pragma unroll
             for (int pc = 0; pc < 2; ++pc) {
-                const uint32_t off = tc::sw128(r, 2 * qc + pc);
+                const uint32_t soff = tc::sw128(r, 2 * qc + pc);
                 float yv[8], o[8];
-                unpack8(*reinterpret_cast<const uint4 *>(sm + kAOffDY + off), yv);
+                unpack8(*reinterpret_cast<const uint4 *>(sm + kAOffDY + soff), yv);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int q = 8 * pc + i;
                     o[i] = __uint_as_float(a1[q]) + Dh * yv[i] + ws * __uint_as_float(a2v[q]);
                     yv[i] *= ec;
                 }
-                if (tok_ok) {
+                if (off == 0) {
+                    const int c0 = 4 * (qc & 1) + 2 * pc;
+                    *reinterpret_cast<float4 *>(xbox + tc::sw128(r, c0)) = make_float4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<float4 *>(xbox + tc::sw128(r, c0 + 1)) = make_float4(o[4], o[5], o[6], o[7]);
+                } else if (tok_ok) {
                     dst[2 * pc] = make_float4(o[0], o[1], o[2], o[3]);
                     dst[2 * pc + 1] = make_float4(o[4], o[5], o[6], o[7]);
                 }
                 // e^c o dY in place (this thread is the last reader of its quarter row)
-                *reinterpret_cast<uint4 *>(sm + kAOffDY + off) = pack8(yv);
+                *reinterpret_cast<uint4 *>(sm + kAOffDY + soff) = pack8(yv);
             }
         }
         // dB rows staged as four 32-column fp32 boxes (128-byte swizzle) in the
@@ -683,6 +693,12 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
         tc::fence_before_sync();
         __syncthreads();
         if (tid == 0) {
+            if (off == 0) {
+                // dX of this head's x columns (written: no other pass adds to them)
+                tc::tma_store_3d(tmd, sbase + kAOffX, h * kBP, t0, b);
+                tc::tma_store_3d(tmd, sbase + kAOffDS, h * kBP + 32, t0, b);
+                tc::bulk_commit();
+            }
             // dB += this head's rows (fp32 reductions at L2)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -750,6 +766,7 @@ bwd_tc_scan_kernel(const __grid_constant__ CUtensorMap tm_act_f, const __grid_co
                 tc::mma_bf16(tmem + kColDS, tc::desc_add(dCmn, ks * 2048), tc::desc_add(dYmn, ks * 2048), idS, 1);
             tc::mma_commit(mb_p5);
             ok = tc::mbar_wait_bounded(mb_p5, par, kBWait);
+            tc::bulk_wait_read1();   // the dX stores have read the X tile (dC is staged there)
         }
         ok = __syncthreads_and(ok);
         if (!ok) break;

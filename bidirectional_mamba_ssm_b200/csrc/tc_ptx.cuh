@@ -261,6 +261,13 @@ __device__ __forceinline__ void bulk_wait_read0()
 }
 
 // This thread's bulk copies are complete (written).
+// Wait until at most the most recent bulk async-group of this thread still
+// reads shared memory.
+__device__ __forceinline__ void bulk_wait_read1()
+{
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_wait0()
 {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
