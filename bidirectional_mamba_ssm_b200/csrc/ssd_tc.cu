@@ -407,13 +407,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         chunk_of(k, t0, cnt, s0);
         tc::tma_prefetch_l2_3d(rev ? &tm_x_r : &tm_x_f, hp * kPP, rev ? t0 : t0 - 3, b);
     };
+    // B (and C) tiles of chunk k.  The state-only pass reads no C: there the
+    // B tiles are double-buffered, odd chunks in the C tile on mbarrier mb_g
+    // (no G there either)
+    auto bbuf_off = [](int k) { return (kStateOnly && (k & 1)) ? kOffC : kOffB; };
     auto issue_bc = [&](int k) {
         int t0, cnt, s0;
         chunk_of(k, t0, cnt, s0);
         const int zc = dir * p.batch + b;
-        tc::mbar_expect_tx(mb_bc, kStateOnly ? kBCBytes / 2 : kBCBytes);
-        tc::tma_load_3d(sbase + kOffB, &tm_bc, 0, s0, zc, mb_bc);
-        tc::tma_load_3d(sbase + kOffB + 16384, &tm_bc, 64, s0, zc, mb_bc);
+        const uint32_t mb = (kStateOnly && (k & 1)) ? mb_g : mb_bc;
+        tc::mbar_expect_tx(mb, kStateOnly ? kBCBytes / 2 : kBCBytes);
+        tc::tma_load_3d(sbase + bbuf_off(k), &tm_bc, 0, s0, zc, mb);
+        tc::tma_load_3d(sbase + bbuf_off(k) + 16384, &tm_bc, 64, s0, zc, mb);
         if constexpr (!kStateOnly) {
             tc::tma_load_3d(sbase + kOffC, &tm_bc, 128, s0, zc, mb_bc);
             tc::tma_load_3d(sbase + kOffC + 16384, &tm_bc, 192, s0, zc, mb_bc);
@@ -542,6 +547,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
         if (nk > 1) issue_x(1);
         if (!kStateOnly && nk > 2) prefetch_x(2);
         issue_bc(0);
+        if (kStateOnly && nk > 1) issue_bc(1);
     }
     if (warp == kHelperWarp) {
         load_dt_async(0);
@@ -555,9 +561,12 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
 
     // wX = w_s * X for walk chunk k (X tile in x buffer k % 2): thread
     // tt (slot j, head gh), the head's 64 channels
+    auto wxbuf_off = [](int k) { return (kStateOnly && (k & 1)) ? kOffS : kOffXw; };
     auto weight_chunk = [&](int k, int tt) {
         // in bf16 pairs: w_s rounded to bf16, each product rounded once
+        // (the state-only pass alternates two wX tiles)
         const uint8_t *xt = sm + xbuf_off(k);
+        uint8_t *wx = sm + wxbuf_off(k);
         const int j = tt & 127, gh = tt >> 7;
         const __nv_bfloat162 w2 = __float2bfloat162_rn(wgt[((k & 1) * kHeads + gh) * kQ + j]);
 #pragma unroll
@@ -567,7 +576,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&v);
 #pragma unroll
             for (int q = 0; q < 4; ++q) h2[q] = __hmul2(h2[q], w2);
-            *reinterpret_cast<uint4 *>(sm + kOffXw + off) = v;
+            *reinterpret_cast<uint4 *>(wx + off) = v;
         }
     };
 
@@ -601,13 +610,16 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             for (int k = 0; k < nk && pok; ++k) {
                 // the state scaled for this chunk, its bf16 copy and wX
                 pok = tc::mbar_wait_bounded(mb_s, k & 1, kWaitCycles);
-                if (pok && kStateOnly) pok = tc::mbar_wait_bounded(mb_bc, k & 1, kWaitCycles);
+                if (pok && kStateOnly)
+                    pok = tc::mbar_wait_bounded((k & 1) ? mb_g : mb_bc, (k >> 1) & 1, kWaitCycles);
                 if (!pok) break;
                 tc::fence_after_sync();
                 // the state product first: the next chunk's state scaling waits for it
+                const uint64_t dBk = kStateOnly ? tc::smem_desc(sbase + bbuf_off(k), 16384, 1024) : dBmn;
+                const uint64_t dXwk = kStateOnly ? tc::smem_desc(sbase + wxbuf_off(k), 16384, 1024) : dXw;
 #pragma unroll 1
                 for (int ks = 0; ks < kQ / 16; ++ks)
-                    tc::mma_bf16(tmem + kColS, tc::desc_add(dBmn, ks * 2048), tc::desc_add(dXw, ks * 2048),
+                    tc::mma_bf16(tmem + kColS, tc::desc_add(dBk, ks * 2048), tc::desc_add(dXwk, ks * 2048),
                                  idS, 1);
                 if constexpr (!kStateOnly) {
                     tc::mma_commit(mb_sdone);   // wX may be rewritten once it completes
@@ -657,8 +669,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
                 pok = tc::mbar_wait_bounded(mb_e, k & 1, kWaitCycles);
                 if (!pok) break;
                 if constexpr (kStateOnly) {
-                    issue_bc(k + 1);
-                    if (k + 2 < nk) issue_x(k + 2);   // (the publisher issues them in the full kernel)
+                    // B buffer k % 2 is free (the tensor-memory group issues the x loads)
+                    if (k + 2 < nk) issue_bc(k + 2);
                 }
                 if constexpr (!kStateOnly) {
                     pok = tc::mbar_wait_bounded(mb_bc, (k + 1) & 1, kWaitCycles);
@@ -1012,15 +1024,23 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant_
             // scaling and w o X (so that the conv group never waits on the
             // products)
             for (int j = 0; j < nk && ok; ++j) {
+                // w o X of chunk j into wX tile j % 2 (the product of chunk
+                // j-2 read it: waited for in the last iteration)
                 ok = a_wait(mb_xr, j & 1);
-                if (ok && j >= 1) ok = a_wait(mb_e, (j - 1) & 1);   // the last product has read w o X
                 if (ok) ok = a_wait(mb_dt0 + 8 * (j & 1), (j >> 1) & 1);
                 if (!ok) break;
                 tc::fence_after_sync();
-                scale_state(j);
                 weight_chunk(j, tid);
+                grp_sync(1);   // x buffer j % 2 read: the load of chunk j+2 may overwrite it
+                if (tid == 0) {
+                    tc::mbar_arrive(mb_free0 + 8 * (j & 1));
+                    if (j + 2 < nk) issue_x(j + 2);
+                }
+                if (j >= 1) ok = a_wait(mb_e, (j - 1) & 1);   // the last product has updated the state
+                if (!ok) break;
+                tc::fence_after_sync();
+                scale_state(j);
                 publish(mb_s, true);
-                if (tid == 0) tc::mbar_arrive(mb_free0 + 8 * (j & 1));
             }
             if (ok) {
                 ok = a_wait(mb_e, (nk - 1) & 1);   // the last chunk's product
