@@ -331,7 +331,11 @@ bc_prepass_kernel(const __nv_bfloat16 *__restrict__ xbc_f, const __nv_bfloat16 *
 //                forward/reverse meeting), then the raw rows of chunk k+2
 //                into the freed x buffer.
 // The two compute groups work on different chunks at the same time, and
-// both overlap the tensor core.
+// both overlap the tensor core.  In the state-only pass the shared-memory
+// group only converts each chunk's x and hands it over; the tensor-memory
+// group forms wX (double-buffered there in the unused bf16 state-copy tile,
+// the B tiles in the unused C tile), releases the x buffer for the load of
+// the chunk after next, and scales the state once the last product is done.
 template <bool kStateOnly, bool kConcat>
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x_f, const __grid_constant__ CUtensorMap tm_x_r,

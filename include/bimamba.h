@@ -376,8 +376,10 @@ int bimamba_block_decode_pool(const bimamba_dims *d, const void *xbc_block,
  * headdim 64 and d_state 128 the chunked backward (128-token chunks) runs
  * every matrix product on the tensor cores (bf16 operands, fp32
  * accumulation); otherwise (64-token chunks) its small products run on the
- * CUDA cores in fp32.  Errors: as bimamba_ssd_fwd_rev (a bounded wait that
- * gave up is reported by bimamba_get_error as BIMAMBA_ERR_TIMEOUT).
+ * CUDA cores in fp32.  The conv passes read 64-token x 64-channel tiles by
+ * TMA and evaluate SiLU and its derivative in fp32, through the hardware
+ * tanh for bf16 activations.  Errors: as bimamba_ssd_fwd_rev (a bounded wait
+ * that gave up is reported by bimamba_get_error as BIMAMBA_ERR_TIMEOUT).
  */
 size_t bimamba_backward_workspace_bytes(const bimamba_dims *d);
 
