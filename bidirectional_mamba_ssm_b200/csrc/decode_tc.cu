@@ -384,17 +384,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const DecodeParams p)
     ok = __syncthreads_and(ok);
     if (ok) {
         // the cached state S[p][n] (fp32, shared) -> bf16 K-major tile (N = p
-        // rows, K = n): 1024 pieces of 8 n; thread: pieces tid + 256 i (a
-        // warp reads two contiguous 512-byte rows per step)
+        // rows, K = n; atom n / 64).  Thread (row pr, quad pc) of step i: n =
+        // 4 pc .. 4 pc + 3 of each atom, so that a half-warp reads 256
+        // contiguous bytes per load (no bank conflicts) and writes one row of
+        // each atom in 8-byte halves of its 16-byte pieces
         const float *sf = reinterpret_cast<const float *>(sm + kDOffSf);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int e = tid + kDThreads * i;
             const int pr = e >> 4, pc = e & 15;
-            const float4 a = *reinterpret_cast<const float4 *>(sf + pr * kDN + 8 * pc);
-            const float4 b4 = *reinterpret_cast<const float4 *>(sf + pr * kDN + 8 * pc + 4);
-            const float v[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
-            *reinterpret_cast<uint4 *>(sm + kDOffS + (pc >> 3) * 8192 + tc::sw128(pr, pc & 7)) = pack8f(v);
+            const float4 a = *reinterpret_cast<const float4 *>(sf + pr * kDN + 4 * pc);
+            const float4 b4 = *reinterpret_cast<const float4 *>(sf + pr * kDN + 64 + 4 * pc);
+            const uint32_t off = tc::sw128(pr, pc >> 1) + 8 * (pc & 1);
+            *reinterpret_cast<uint2 *>(sm + kDOffS + off) =
+                make_uint2(tc::pack_bf16x2(a.x, a.y), tc::pack_bf16x2(a.z, a.w));
+            *reinterpret_cast<uint2 *>(sm + kDOffS + 8192 + off) =
+                make_uint2(tc::pack_bf16x2(b4.x, b4.y), tc::pack_bf16x2(b4.z, b4.w));
         }
     }
     tc::fence_before_sync();
