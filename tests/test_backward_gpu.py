@@ -35,6 +35,7 @@ CASES = [
     ("bf16", 2, 200, 4, 64, 128),
     ("bf16", 1, 300, 2, 64, 128),
     ("bf16", 1, 64, 2, 32, 64),
+    ("bf16", 2, 70, 3, 8, 8),   # 40 channels: a partial 64-channel conv tile, rows of 80 bytes
 ]
 
 
